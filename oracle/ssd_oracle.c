@@ -1,0 +1,343 @@
+/*
+ * ssd_oracle.c -- plain, slow, sequential fp64 reference of the Mamba-2 / SSD
+ * selective-state-space mixer scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the bench's
+ * CPU-baseline leg use it.  It shares no code, header, table or helper with
+ * the CUDA library; its one input is plain arrays of numbers.
+ *
+ * What it computes, per (batch row b, head h), one token at a time:
+ *
+ *   1. causal depthwise conv (kernel K, usually 4) over the x|B|C channels,
+ *      then SiLU  -- "Mini-K3-1H-mamba2-n64-g8" model card, Architecture
+ *      ("causal depthwise-convolution kernel 4"); channel order x|B|C and
+ *      conv_dim = d_inner + 2*n_groups*d_state from the codestral_mamba.ts
+ *      weight-port header (tensor list).  K = 1 means "no conv" (the
+ *      mojolearn Mamba3Block description: v is the raw x split, no conv), and
+ *      then no SiLU either.
+ *      Tap order is upstream PyTorch Conv1d order: w[c, K-1] multiplies the
+ *      current token, w[c, 0] the token K-1 steps back (codestral_mamba.ts,
+ *      "conv1d ... taps reversed" is the other engine's order, not ours).
+ *   2. optional B/C RMSNorm (eps 1e-5) times a weight, plus a per-head bias
+ *      -- mojolearn Mamba3Block, class description and Parameters
+ *      (B_norm/C_norm weight (N,), B_bias/C_bias (H, N)).
+ *   3. dt = softplus(dt_raw + dt_bias[h]) with no clamp -- falcon_mamba.ts
+ *      header ("softplus(dt + bias)"), Mamba3Block ("no dt clamp").
+ *   4. a = A[h] (per-head A, given already negative: A = -exp(A_log) per the
+ *      codestral_mamba.ts reconciliation 2), or the per-token per-head
+ *      A[b,t,h] clamped so that |a| >= 1e-4 (Mamba3Block, "A floor 1e-4").
+ *   5. packed-document reset: when seq_idx[t] != seq_idx[t-1] the recurrent
+ *      state restarts from zero and the conv sees no tap from another
+ *      document (model card, "Checkpoint and training": document IDs reset
+ *      convolution history and recurrent state at every boundary).  The
+ *      caller's initial state belongs to the first document of the row.
+ *   6. h[p,n] <- exp(dt*a) * h[p,n] + dt * x[p] * B[n]
+ *   7. y[p] = sum_n C[n] * h[p,n] + D[h] * x[p];  out = y * silu(z[p])
+ *      (the gate is applied in the core: Mamba3Block class description; D is
+ *      the "structural D (skip connection)" of the transplant article).
+ *   8. after the last token: final SSM state h, and the last K-1 raw conv
+ *      inputs, zeroed where they belong to another document than the last
+ *      token's.
+ *
+ * A decode step is this same computation at L = 1 with the state carried
+ * (Mamba3Block.step: "the same computation as forward at L = 1").
+ *
+ * Everything is double precision.  Inputs arrive as float32 arrays holding
+ * exactly the values the GPU receives (bf16 values widen to fp32 exactly).
+ * Work is spread over (b, h) pairs with POSIX threads; each pair is computed
+ * by one thread, in token order, with no blocking or reordering.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* Shapes and switches of one call.  Layouts (row-major, contiguous):
+ *   x, z      (batch, seqlen, nheads*headdim)        float32
+ *   Bm, Cm    (batch, seqlen, ngroups*dstate)        float32
+ *   dt_raw    (batch, seqlen, nheads)                float32
+ *   dt_bias, D (nheads)                              float32
+ *   A         (nheads) or (batch, seqlen, nheads)    float32, already negative
+ *   conv_w    (conv_dim, dconv), conv_b (conv_dim)   float32, x|B|C channel order
+ *   seq_idx   (batch, seqlen) int32 or NULL (one document per row)
+ *   init_ssm  (batch, nheads, headdim, dstate) float32 or NULL (zeros)
+ *   init_conv (batch, dconv-1, conv_dim) float32 or NULL (zeros); index 0 is
+ *             the oldest token
+ *   bn_w, cn_w (dstate) or NULL (ones); bn_bias, cn_bias (nheads, dstate) or
+ *             NULL (zeros) -- only read when bc_norm != 0
+ * Outputs (double):
+ *   out       (batch, seqlen, nheads*headdim)
+ *   fin_ssm   (batch, nheads, headdim, dstate) or NULL
+ *   fin_conv  (batch, dconv-1, conv_dim) or NULL
+ */
+typedef struct {
+    int batch, seqlen, nheads, headdim, dstate, ngroups, dconv;
+    int a_per_token, bc_norm;
+} oracle_dims;
+
+typedef struct {
+    const float *x, *z, *Bm, *Cm, *dt_raw, *dt_bias, *A, *D, *conv_w, *conv_b;
+    const int32_t *seq_idx;
+    const float *init_ssm, *init_conv;
+    const float *bn_w, *cn_w, *bn_bias, *cn_bias;
+} oracle_inputs;
+
+static double softplus_exact(double v)
+{
+    /* log(1 + e^v), written so that neither branch overflows. */
+    if (v > 20.0) return v + log1p(exp(-v));
+    return log1p(exp(v));
+}
+
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+static int conv_dim_of(const oracle_dims *d)
+{
+    return d->nheads * d->headdim + 2 * d->ngroups * d->dstate;
+}
+
+/* Raw (pre-conv) value of channel ch of the x|B|C stream at (b, t). */
+static double xbc_raw(const oracle_dims *d, const oracle_inputs *in, int b, int t, int ch)
+{
+    const int dx = d->nheads * d->headdim, gn = d->ngroups * d->dstate;
+    const size_t row = (size_t)b * d->seqlen + t;
+    if (ch < dx) return in->x[row * dx + ch];
+    if (ch < dx + gn) return in->Bm[row * gn + (ch - dx)];
+    return in->Cm[row * gn + (ch - dx - gn)];
+}
+
+static int same_doc(const oracle_inputs *in, const oracle_dims *d, int b, int t0, int t1)
+{
+    if (!in->seq_idx) return 1;
+    const int32_t *s = in->seq_idx + (size_t)b * d->seqlen;
+    return s[t0] == s[t1];
+}
+
+/* Channel ch of the conv+SiLU output at (b, t); with dconv == 1 the raw value. */
+static double conv_silu(const oracle_dims *d, const oracle_inputs *in, int b, int t, int ch)
+{
+    const int K = d->dconv, cd = conv_dim_of(d);
+    if (K == 1) return xbc_raw(d, in, b, t, ch);
+    double acc = in->conv_b[ch];
+    for (int k = 0; k < K; k++) {
+        const int tau = t - (K - 1) + k;
+        double v = 0.0;
+        if (tau >= 0) {
+            if (same_doc(in, d, b, tau, t)) v = xbc_raw(d, in, b, tau, ch);
+        } else if (in->init_conv && same_doc(in, d, b, 0, t)) {
+            v = in->init_conv[((size_t)b * (K - 1) + (tau + K - 1)) * cd + ch];
+        }
+        acc += (double)in->conv_w[(size_t)ch * K + k] * v;
+    }
+    return silu(acc);
+}
+
+typedef struct {
+    const oracle_dims *d;
+    const oracle_inputs *in;
+    double *out, *fin_ssm;
+    const int32_t *pairs; /* (b, h) pairs, or NULL for all */
+    int npairs;
+    int next;             /* next pair index, taken under the lock */
+    pthread_mutex_t lock;
+} pair_job;
+
+static void run_pair(const oracle_dims *d, const oracle_inputs *in, int b, int h,
+                     double *out, double *fin_ssm)
+{
+    const int L = d->seqlen, P = d->headdim, N = d->dstate, H = d->nheads;
+    const int g = h / (H / d->ngroups);
+    const int dx = H * P, gn = d->ngroups * N;
+    double *hs = calloc((size_t)P * N, sizeof(double));
+    double *ux = malloc(sizeof(double) * P);
+    double *ub = malloc(sizeof(double) * N);
+    double *uc = malloc(sizeof(double) * N);
+    if (!hs || !ux || !ub || !uc) abort();
+
+    if (in->init_ssm) {
+        const float *s0 = in->init_ssm + ((size_t)b * H + h) * P * N;
+        for (int i = 0; i < P * N; i++) hs[i] = s0[i];
+    }
+    for (int t = 0; t < L; t++) {
+        if (t > 0 && !same_doc(in, d, b, t - 1, t)) memset(hs, 0, sizeof(double) * P * N);
+
+        for (int p = 0; p < P; p++) ux[p] = conv_silu(d, in, b, t, h * P + p);
+        for (int n = 0; n < N; n++) {
+            ub[n] = conv_silu(d, in, b, t, dx + g * N + n);
+            uc[n] = conv_silu(d, in, b, t, dx + gn + g * N + n);
+        }
+        if (d->bc_norm) {
+            double sb = 0.0, sc = 0.0;
+            for (int n = 0; n < N; n++) { sb += ub[n] * ub[n]; sc += uc[n] * uc[n]; }
+            const double rb = 1.0 / sqrt(sb / N + 1e-5), rc = 1.0 / sqrt(sc / N + 1e-5);
+            for (int n = 0; n < N; n++) {
+                const double wb = in->bn_w ? in->bn_w[n] : 1.0, wc = in->cn_w ? in->cn_w[n] : 1.0;
+                const double bb = in->bn_bias ? in->bn_bias[(size_t)h * N + n] : 0.0;
+                const double bc = in->cn_bias ? in->cn_bias[(size_t)h * N + n] : 0.0;
+                ub[n] = ub[n] * rb * wb + bb;
+                uc[n] = uc[n] * rc * wc + bc;
+            }
+        }
+
+        const size_t tok = (size_t)b * L + t;
+        const double dt = softplus_exact((double)in->dt_raw[tok * H + h] + in->dt_bias[h]);
+        double a;
+        if (d->a_per_token) {
+            a = in->A[tok * H + h];
+            if (a > -1e-4) a = -1e-4;
+        } else {
+            a = in->A[h];
+        }
+        const double decay = exp(dt * a);
+
+        for (int p = 0; p < P; p++) {
+            double *hp = hs + (size_t)p * N;
+            const double dxp = dt * ux[p];
+            double y = 0.0;
+            for (int n = 0; n < N; n++) {
+                hp[n] = decay * hp[n] + dxp * ub[n];
+                y += uc[n] * hp[n];
+            }
+            y += in->D[h] * ux[p];
+            const double zv = in->z[tok * dx + h * P + p];
+            out[tok * dx + h * P + p] = y * silu(zv);
+        }
+    }
+    if (fin_ssm) memcpy(fin_ssm + ((size_t)b * H + h) * P * N, hs, sizeof(double) * P * N);
+    free(hs); free(ux); free(ub); free(uc);
+}
+
+static void *pair_worker(void *arg)
+{
+    pair_job *j = arg;
+    const int total = j->pairs ? j->npairs : j->d->batch * j->d->nheads;
+    for (;;) {
+        pthread_mutex_lock(&j->lock);
+        const int i = j->next++;
+        pthread_mutex_unlock(&j->lock);
+        if (i >= total) break;
+        int b, h;
+        if (j->pairs) { b = j->pairs[2 * i]; h = j->pairs[2 * i + 1]; }
+        else { b = i / j->d->nheads; h = i % j->d->nheads; }
+        run_pair(j->d, j->in, b, h, j->out, j->fin_ssm);
+    }
+    return NULL;
+}
+
+/* Number of worker threads the oracle uses when asked for 0 (all online cores). */
+int oracle_default_threads(void)
+{
+    long n = sysconf(_SC_NPROCESSORS_ONLN);
+    return n > 0 ? (int)n : 1;
+}
+
+/*
+ * Full forward.  pairs: npairs (b, h) pairs to compute, or NULL for all;
+ * outputs of pairs not computed are left untouched.  fin_conv, when given, is
+ * filled for every batch row.  Returns the number of threads used, or -1 on a
+ * bad argument.
+ */
+int oracle_forward(const oracle_dims *d, const oracle_inputs *in,
+                   const int32_t *pairs, int npairs, int nthreads,
+                   double *out, double *fin_ssm, double *fin_conv)
+{
+    if (!d || !in || !out) return -1;
+    if (d->batch < 0 || d->seqlen < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 ||
+        d->ngroups < 1 || d->nheads % d->ngroups || d->dconv < 1)
+        return -1;
+    if (d->dconv > 1 && (!in->conv_w || !in->conv_b)) return -1;
+
+    pair_job j;
+    j.d = d; j.in = in; j.out = out; j.fin_ssm = fin_ssm;
+    j.pairs = pairs; j.npairs = npairs; j.next = 0;
+    pthread_mutex_init(&j.lock, NULL);
+    if (nthreads <= 0) nthreads = oracle_default_threads();
+    const int total = pairs ? npairs : d->batch * d->nheads;
+    if (nthreads > total) nthreads = total > 0 ? total : 1;
+    pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int i = 1; i < nthreads; i++) pthread_create(&th[i], NULL, pair_worker, &j);
+    pair_worker(&j);
+    for (int i = 1; i < nthreads; i++) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&j.lock);
+
+    if (fin_conv && d->dconv > 1) {
+        const int K = d->dconv, cd = conv_dim_of(d), L = d->seqlen;
+        for (int b = 0; b < d->batch; b++)
+            for (int i = 0; i < K - 1; i++) {
+                const int tau = L - (K - 1) + i;
+                for (int ch = 0; ch < cd; ch++) {
+                    double v = 0.0;
+                    if (tau >= 0) {
+                        if (same_doc(in, d, b, tau, L - 1)) v = xbc_raw(d, in, b, tau, ch);
+                    } else if (in->init_conv && same_doc(in, d, b, 0, L - 1)) {
+                        v = in->init_conv[((size_t)b * (K - 1) + (tau + K - 1)) * cd + ch];
+                    }
+                    fin_conv[((size_t)b * (K - 1) + i) * cd + ch] = v;
+                }
+            }
+    }
+    return nthreads;
+}
+
+/* Stage: conv+SiLU output of every x|B|C channel, (batch, seqlen, conv_dim). */
+int oracle_conv(const oracle_dims *d, const oracle_inputs *in, double *u)
+{
+    if (!d || !in || !u || d->dconv < 1) return -1;
+    const int cd = conv_dim_of(d);
+    for (int b = 0; b < d->batch; b++)
+        for (int t = 0; t < d->seqlen; t++)
+            for (int ch = 0; ch < cd; ch++)
+                u[((size_t)b * d->seqlen + t) * cd + ch] = conv_silu(d, in, b, t, ch);
+    return 0;
+}
+
+/* Stage: dt = softplus(dt_raw + dt_bias) and a (floored when per token), (batch, seqlen, nheads). */
+int oracle_dt(const oracle_dims *d, const oracle_inputs *in, double *dt, double *a)
+{
+    if (!d || !in || !dt) return -1;
+    const int H = d->nheads;
+    for (int b = 0; b < d->batch; b++)
+        for (int t = 0; t < d->seqlen; t++)
+            for (int h = 0; h < H; h++) {
+                const size_t i = ((size_t)b * d->seqlen + t) * H + h;
+                dt[i] = softplus_exact((double)in->dt_raw[i] + in->dt_bias[h]);
+                if (a) {
+                    double av = d->a_per_token ? in->A[i] : in->A[h];
+                    if (d->a_per_token && av > -1e-4) av = -1e-4;
+                    a[i] = av;
+                }
+            }
+    return 0;
+}
+
+/* Stage: normalised, biased B and C per head, (batch, seqlen, nheads, dstate) each,
+ * taken from the raw B and C (the configurations with a B/C norm have no conv). */
+int oracle_bcnorm(const oracle_dims *d, const oracle_inputs *in, double *bh, double *ch_out)
+{
+    if (!d || !in || !bh || !ch_out) return -1;
+    const int H = d->nheads, N = d->dstate, gn = d->ngroups * N;
+    for (int b = 0; b < d->batch; b++)
+        for (int t = 0; t < d->seqlen; t++) {
+            const size_t row = (size_t)b * d->seqlen + t;
+            for (int h = 0; h < H; h++) {
+                const int g = h / (H / d->ngroups);
+                const float *bv = in->Bm + row * gn + (size_t)g * N;
+                const float *cv = in->Cm + row * gn + (size_t)g * N;
+                double sb = 0.0, sc = 0.0;
+                for (int n = 0; n < N; n++) { sb += (double)bv[n] * bv[n]; sc += (double)cv[n] * cv[n]; }
+                const double rb = 1.0 / sqrt(sb / N + 1e-5), rc = 1.0 / sqrt(sc / N + 1e-5);
+                for (int n = 0; n < N; n++) {
+                    const size_t o = (row * H + h) * N + n;
+                    bh[o] = bv[n] * rb * (in->bn_w ? in->bn_w[n] : 1.0) +
+                            (in->bn_bias ? in->bn_bias[(size_t)h * N + n] : 0.0);
+                    ch_out[o] = cv[n] * rc * (in->cn_w ? in->cn_w[n] : 1.0) +
+                                (in->cn_bias ? in->cn_bias[(size_t)h * N + n] : 0.0);
+                }
+            }
+        }
+    return 0;
+}

@@ -1,0 +1,132 @@
+"""The oracle's pins catch plausible mistakes (no GPU needed).
+
+Each case plants one mistake in a temporary copy of oracle/ssd_oracle.c (a
+dropped term, a wrong sign, a wrong index, a missing reset ...), builds it,
+and checks that the pin battery below -- the same independent forms the
+oracle pin tests use -- rejects it, while the unmodified oracle passes.
+"""
+import os
+import shutil
+
+import numpy as np
+import pytest
+
+from brute_force import head_inputs, quadratic_form, silu
+from selective_state_space_forward_b200.synthetic import Workload, make_inputs
+
+import oracle
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle",
+                   "ssd_oracle.c")
+
+MUTANTS = {
+    "drop_D_skip": ("y += in->D[h] * ux[p];", "y += 0.0 * ux[p];"),
+    "decay_sign": ("const double decay = exp(dt * a);", "const double decay = exp(-dt * a);"),
+    "no_document_reset": ("memset(hs, 0, sizeof(double) * P * N);", "(void)0;"),
+    "conv_taps_reversed": ("in->conv_w[(size_t)ch * K + k]", "in->conv_w[(size_t)ch * K + (K - 1 - k)]"),
+    "update_with_C": ("hp[n] = decay * hp[n] + dxp * ub[n];", "hp[n] = decay * hp[n] + dxp * uc[n];"),
+    "no_gate_silu": ("out[tok * dx + h * P + p] = y * silu(zv);", "out[tok * dx + h * P + p] = y * zv;"),
+    "groups_interleaved": ("const int g = h / (H / d->ngroups);\n    const int dx",
+                           "const int g = h % d->ngroups;\n    const int dx"),
+    "dt_bias_dropped": ("softplus_exact((double)in->dt_raw[tok * H + h] + in->dt_bias[h])",
+                        "softplus_exact((double)in->dt_raw[tok * H + h])"),
+    "a_floor_inverted": ("if (a > -1e-4) a = -1e-4;", "if (a < -1e-4) a = -1e-4;"),
+    "init_history_crosses_documents": ("} else if (in->init_conv && same_doc(in, d, b, 0, t)) {",
+                                       "} else if (in->init_conv) {"),
+    "norm_uses_C_bias_for_B": ("ub[n] = ub[n] * rb * wb + bb;", "ub[n] = ub[n] * rb * wb + bc;"),
+    "output_before_update": ("hp[n] = decay * hp[n] + dxp * ub[n];\n                y += uc[n] * hp[n];",
+                             "y += uc[n] * hp[n];\n                hp[n] = decay * hp[n] + dxp * ub[n];"),
+}
+
+
+def _docs(L, cuts):
+    seq = np.zeros(L, dtype=np.int32)
+    for c in cuts:
+        seq[c:] += 1
+    return seq
+
+
+def _battery(lib) -> list:
+    """Run the independent checks; return the names of those that fail."""
+    failed = []
+    # 1. matrix form, with documents, initial state and per-token A
+    w = Workload("m", 2, 90, 4, 4, 5, 2, 1, "f32", a_per_token=True, init_state=True, seed=21)
+    inp = make_inputs(w)
+    inp["seq_idx"] = np.stack([_docs(90, [1, 64, 65]), _docs(90, [])])
+    inp["A"][0, 3:6, 0] = np.array([0.0, -1e-6, -0.3], dtype=np.float32)
+    dims = w.dims()
+    res = oracle.forward(dims, inp, lib=lib)
+    ok = True
+    for b in range(2):
+        for h in range(4):
+            x, z, Bm, Cm, dt, a, D, seq, h0 = head_inputs(inp, dims, b, h)
+            y, hf = quadratic_form(x, z, Bm, Cm, dt, a, D, seq, h0)
+            got = res["out"][b, :, h * 4:(h + 1) * 4]
+            ok &= bool(np.max(np.abs(got - y)) <= 1e-10 * np.max(np.abs(y)))
+            ok &= bool(np.max(np.abs(res["final_ssm"][b, h] - hf)) <= 1e-10 * np.max(np.abs(hf)))
+    if not ok:
+        failed.append("quadratic_form")
+    # 2. conv against a padded correlation, with documents and an initial history
+    w = Workload("c", 1, 30, 2, 4, 3, 1, 4, "f32", seed=22)
+    inp = make_inputs(w)
+    rng = np.random.default_rng(1)
+    inp["init_conv"] = rng.standard_normal((1, 3, w.conv_dim)).astype(np.float32)
+    inp["seq_idx"] = _docs(30, [2, 17])[None]
+    u = oracle.conv_stage(w.dims(), inp, lib=lib)[0]
+    raw = np.concatenate([inp["x"][0], inp["B"][0], inp["C"][0]], axis=1).astype(np.float64)
+    seq = inp["seq_idx"][0]
+    want = np.empty_like(u)
+    for t in range(30):
+        acc = inp["conv_b"].astype(np.float64).copy()
+        for k in range(4):
+            tau = t - 3 + k
+            if tau >= 0:
+                v = raw[tau] if seq[tau] == seq[t] else 0.0
+            else:
+                v = inp["init_conv"][0, tau + 3].astype(np.float64) if seq[t] == seq[0] else 0.0
+            acc = acc + inp["conv_w"][:, k].astype(np.float64) * v
+        want[t] = silu(acc)
+    if not np.allclose(u, want, rtol=1e-13, atol=1e-300):
+        failed.append("conv")
+    # 3. B/C norm closed form: zero bias, unit weight
+    w = Workload("n", 1, 8, 2, 4, 8, 1, 1, "f32", bc_norm=True, seed=23)
+    inp = make_inputs(w)
+    inp["B_bias"] = np.zeros_like(inp["B_bias"])
+    bh, ch = oracle.bcnorm_stage(w.dims(), inp, lib=lib)
+    m = np.mean(inp["B"][0].astype(np.float64) ** 2, axis=1)
+    if not np.allclose(np.sum(bh[0] ** 2, axis=2), (8 * m / (m + 1e-5))[:, None], rtol=1e-12):
+        failed.append("bcnorm_closed_form")
+    # 4. normed scan == un-normed scan fed per-head B_hat / C_hat (G = H)
+    w = Workload("nw", 1, 40, 2, 4, 8, 1, 1, "f32", bc_norm=True, seed=24)
+    inp = make_inputs(w)
+    r = oracle.forward(w.dims(), inp, lib=lib)
+    bh, ch = oracle.bcnorm_stage(w.dims(), inp)   # the unmodified oracle's norm stage
+    flat = dict(inp, B=bh.reshape(1, 40, 16).astype(np.float32),
+                C=ch.reshape(1, 40, 16).astype(np.float32))
+    r2 = oracle.forward(dict(w.dims(), ngroups=2, bc_norm=0), flat)
+    if not np.max(np.abs(r["out"] - r2["out"])) <= 1e-5 * np.max(np.abs(r2["out"])):
+        failed.append("bcnorm_wiring")
+    return failed
+
+
+def _build_variant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    path = tmp_path / (name + ".c")
+    path.write_text(src.replace(old, new))
+    so = str(tmp_path / (name + ".so"))
+    oracle.build(force=True, src=str(path), out=so)
+    return oracle.load_variant(so)
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_unmodified_oracle_passes_the_battery(oracle_mod):
+    assert _battery(None) == []
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(oracle_mod, tmp_path, name):
+    old, new = MUTANTS[name]
+    lib = _build_variant(tmp_path, name, old, new)
+    assert _battery(lib), f"mutant {name} passed every pin"
