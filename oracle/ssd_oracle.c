@@ -109,11 +109,17 @@ static double xbc_raw(const oracle_dims *d, const oracle_inputs *in, int b, int 
     return in->Cm[row * gn + (ch - dx - gn)];
 }
 
+/* 1 when no document boundary lies in (t0, t1], t0 <= t1: a boundary is a
+ * position r > 0 whose id differs from its left neighbour's, so ids are only
+ * ever compared between neighbours (an id may recur later in the row and
+ * still start a new document). */
 static int same_doc(const oracle_inputs *in, const oracle_dims *d, int b, int t0, int t1)
 {
     if (!in->seq_idx) return 1;
     const int32_t *s = in->seq_idx + (size_t)b * d->seqlen;
-    return s[t0] == s[t1];
+    for (int r = t0 + 1; r <= t1; r++)
+        if (s[r] != s[r - 1]) return 0;
+    return 1;
 }
 
 /* Channel ch of the conv+SiLU output at (b, t); with dconv == 1 the raw value. */

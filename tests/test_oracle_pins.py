@@ -387,3 +387,22 @@ def test_generator_rounds_to_bf16_and_is_seeded():
         assert np.all((a[k].view(np.uint32) & 0xFFFF) == 0)
     assert np.array_equal(round_bf16(np.float32(1.0 + 2 ** -8)), np.float32(1.0))  # tie -> even
     assert np.array_equal(round_bf16(np.float32(1.0 + 3 * 2 ** -8)), np.float32(1.0 + 2 ** -6))
+
+
+def test_document_ids_are_compared_between_neighbours(oracle_mod):
+    """A boundary is where the id changes from one token to the next, so an id
+    that recurs later still starts a new document: [0,0,1,1,0,0] behaves like
+    [0,0,1,1,2,2] in both the conv and the scan."""
+    w = _small(dconv=4, seqlen=48, batch=1, init_state=True)
+    inp = make_inputs(w)
+    rng = np.random.default_rng(8)
+    inp["init_conv"] = rng.standard_normal((1, 3, w.conv_dim)).astype(np.float32)
+    a = _docs_with_boundaries(48, [10, 11, 30])
+    recur = np.where(a == 2, 0, a).astype(np.int32)    # [0..,1,2(->0)..,3]
+    inp["seq_idx"] = recur[None]
+    r1 = oracle_mod.forward(w.dims(), inp)
+    inp["seq_idx"] = a[None]
+    r2 = oracle_mod.forward(w.dims(), inp)
+    assert np.array_equal(r1["out"], r2["out"])
+    assert np.array_equal(r1["final_ssm"], r2["final_ssm"])
+    assert np.array_equal(r1["final_conv"], r2["final_conv"])
