@@ -1,0 +1,517 @@
+#!/usr/bin/env python
+"""Throughput of the SSD mixer scan on B200: tokens/s, roofline fraction,
+decode-step GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ssd_forward over the mini_k3_mixer workload (batch 5 x 8192
+tokens, 32 heads x 64, d_state 64, 8 B/C groups, conv 4, packed documents)
+with its inputs resident in HBM; the whole hot path runs in the library's
+kernels (conv, dt/cumsum, chunk scan with state passing, gated output, final
+state).  Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs
+its own batch -- the scan has no cross-row exchange -- so the scaling is weak
+and `value` counts every rank's tokens over the slowest rank's device time.
+
+Extra keys: `roofline` (dominant kernel against measured HBM bandwidth),
+`forward_roofline` (whole forward against its compulsory bytes), `decode`
+(decode_b256 single-token step, GB/s), `e2e` (host buffers, copies inside the
+timed region), `cpu_baseline` (the fp64 oracle on this host's cores),
+`clocks` (SM clock and throttle reasons sampled during the timed region).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD mixer tokens/s (B·L/s) at 1 B200 and % of roofline; decode-step GB/s"
+WORKLOAD = "mini_k3_mixer"
+DECODE_WORKLOAD = "decode_b256"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "kernel_traffic.json")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--path", choices=["auto", "fused", "staged"], default="auto")
+    p.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; also exercised with gloo on CPU by the tests)
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_init(backend: str):
+    import datetime
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+    return rank, world
+
+
+def aggregate(local_ms: float, local_units: float, world: int, device=None):
+    """(max over ranks of the device time, sum over ranks of the units processed)."""
+    if world <= 1:
+        return local_ms, local_units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([local_units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash(path_kind: str) -> str:
+    """Hash of the sources that make up the dominant kernel of a path."""
+    files = {"fused": ["chunk_fused.cu", "ssd_device.cuh"],
+             "staged": ["chunk_staged.cu", "ssd_device.cuh"],
+             "decode": ["decode.cu", "ssd_device.cuh"]}[path_kind]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "selective_state_space_forward_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel_key: str, path_kind: str, scale: float = 1.0):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    summary is missing or was taken on other kernel sources."""
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            d = json.load(f)
+        e = d[kernel_key]
+    except (OSError, KeyError, ValueError):
+        return None
+    if e.get("source_hash") != kernel_source_hash(path_kind):
+        return None
+    return float(e["dram_bytes_per_launch"]) * scale
+
+
+class ClockSampler:
+    """SM clock and throttle reasons, sampled by NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._dev = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._dev = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._dev, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # NVML missing: report that, keep benchmarking
+            self.error = str(e)
+        self._period = period_s
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._dev,
+                                                                    self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._dev)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._dev is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._dev is not None:
+            self._t.join()
+
+    def summary(self):
+        if self._dev is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        s = sorted(self.samples)
+        med = s[len(s) // 2] if s else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(s)}
+
+
+# ---------------------------------------------------------------------------------------
+def _device_inputs(w, inp, torch):
+    at = torch.bfloat16 if w.act_dtype == "bf16" else torch.float32
+    dev = {}
+    for k in ("x", "z", "B", "C", "conv_w", "conv_b"):
+        dev[k] = None if inp.get(k) is None else torch.from_numpy(inp[k]).to(at).cuda()
+    for k in ("dt_raw", "dt_bias", "A", "D", "B_norm_w", "C_norm_w", "B_bias", "C_bias"):
+        dev[k] = None if inp.get(k) is None else torch.from_numpy(inp[k]).cuda()
+    dev["seq_idx"] = None if inp.get("seq_idx") is None else torch.from_numpy(
+        inp["seq_idx"]).cuda()
+    return dev
+
+
+def forward_bytes(w) -> dict:
+    """Compulsory bytes of one forward of workload w (every input read once,
+    every output written once, plus initial and final state)."""
+    a = 2 if w.act_dtype == "bf16" else 4
+    BL = w.batch * w.seqlen
+    HP, GN, H = w.nheads * w.headdim, w.ngroups * w.dstate, w.nheads
+    b = BL * (HP * a * 3 + 2 * GN * a + H * 4)            # x, z, out, B, C, dt_raw
+    if w.a_per_token:
+        b += BL * H * 4
+    if w.documents != "none":
+        b += BL * 4
+    state = w.batch * H * w.headdim * w.dstate * 4
+    b += state * (2 if w.init_state else 1)
+    if w.dconv > 1:
+        b += w.batch * 3 * w.conv_dim * a
+    return {"bytes": b}
+
+
+def main_kernel_bytes(w, path: str) -> int:
+    """Algorithmic bytes of one launch of the dominant kernel of `path`."""
+    a = 2 if w.act_dtype == "bf16" else 4
+    BL = w.batch * w.seqlen
+    HP, GN, H = w.nheads * w.headdim, w.ngroups * w.dstate, w.nheads
+    nc = (w.seqlen + 63) // 64
+    state = w.batch * H * w.headdim * w.dstate * 4
+    seq = BL * 4 if w.documents != "none" else 0
+    if path == "fused":
+        # x (raw, for its conv), z, out, the conv'd B|C (or raw B, C), dt and acs, ids, state
+        b = BL * (3 * HP * a + 2 * GN * a + 2 * H * 4) + seq + state
+        if w.init_state:
+            b += state
+        if w.dconv > 1:
+            b += w.batch * 3 * HP * a          # the x part of the conv history
+        return b
+    # staged chunk-output kernel: conv'd x|B|C (fp32) or raw, z, out, dt/acs, ids, Hin
+    u = BL * (HP + 2 * GN) * (4 if w.dconv > 1 else a)
+    return u + BL * (2 * HP * a + 2 * H * 4) + seq + w.batch * nc * H * w.headdim * w.dstate * 4
+
+
+def bench_forward(args, torch, rank, world, local_rank, peaks):
+    from selective_state_space_forward_b200 import ssd
+    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
+    w = WORKLOADS[WORKLOAD]
+    inp = make_inputs(w)
+    dev = _device_inputs(w, inp, torch)
+    h = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, w.act_dtype,
+                   a_per_token=w.a_per_token, bc_norm=w.bc_norm, max_batch=w.batch,
+                   max_seqlen=w.seqlen, path=args.path)
+    fin = h.new_state(w.batch)
+    out = torch.empty_like(dev["x"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"],
+                  dev["C"], dev["D"], dev["conv_w"], dev["conv_b"], seq_idx=dev["seq_idx"],
+                  out=out, final_state=fin, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    for a_, b_ in ev:   # materialise the events so their handles exist
+        a_.record(stream)
+        b_.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches0 = h.launch_count()
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for i in range(K):
+            h.set_timing_events(*ev[i])
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    launches = h.launch_count() - launches0
+    h.set_timing_events(None, None)
+    barrier(world)
+    local_ms = t0.elapsed_time(t1) / K
+    kern_ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / K
+    h.check()
+    max_ms, total_tokens = aggregate(local_ms, w.tokens, world,
+                                     device=torch.device("cuda", local_rank))
+
+    kb = main_kernel_bytes(w, h.path)
+    achieved = kb / (kern_ms * 1e-3) / 1e9
+    traffic = measured_traffic(f"{h.path}:{WORKLOAD}", h.path)
+    fb = forward_bytes(w)["bytes"]
+    roof_ms = fb / (peaks["hbm_gbs"] * 1e9) * 1e3
+    res = {
+        "value": total_tokens / (max_ms * 1e-3),
+        "ms_per_step": max_ms,
+        "tokens_per_rank": w.tokens,
+        "path": h.path,
+        "launches": launches,
+        "clocks": clk.summary(),
+        "roofline": {"bound": "hbm", "kernel": "ssd_chunk_fused" if h.path == "fused"
+                     else "chunk_output_kernel", "achieved": round(achieved, 1),
+                     "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                     "algorithmic_bytes": kb, "kernel_ms": round(kern_ms, 4)},
+        "forward_roofline": {"compulsory_bytes": fb, "roofline_ms": round(roof_ms, 4),
+                             "roofline_tokens_per_s": w.tokens / (roof_ms * 1e-3),
+                             "frac": round(roof_ms / local_ms, 4)},
+    }
+    return res, (w, inp, h, dev, out, fin)
+
+
+def bench_e2e(args, torch, ctx, world, local_rank):
+    """Same forward through the public call with the step's inputs in pinned host
+    memory: H2D copies, the call, and the D2H read of the output are timed."""
+    w, inp, h, dev, out, fin = ctx
+    stream = torch.cuda.current_stream()
+    keys = ["x", "z", "B", "C", "dt_raw"] + (["seq_idx"] if dev["seq_idx"] is not None else [])
+    host = {k: dev[k].cpu().pin_memory() for k in keys}
+    dbuf = {k: torch.empty_like(dev[k]) for k in keys}
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    bi = sum(t.numel() * t.element_size() for t in host.values())
+    bo = hout.numel() * hout.element_size()
+
+    def step():
+        for k in keys:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        h.forward(dbuf["x"], dbuf["z"], dbuf["dt_raw"], dev["dt_bias"], dev["A"], dbuf["B"],
+                  dbuf["C"], dev["D"], dev["conv_w"], dev["conv_b"],
+                  seq_idx=dbuf.get("seq_idx"), out=out, final_state=fin, stream=stream)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    K = max(3, min(args.steps, 20))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0.record(stream)
+    for _ in range(K):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / K
+    max_ms, tot = aggregate(ms, w.tokens, world, device=torch.device("cuda", local_rank))
+    return {"value": tot / (max_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
+            "d2h_bytes_per_step": bo, "ms_per_step": max_ms, "steps": K}
+
+
+def bench_decode(args, torch, peaks):
+    """decode_b256: a 2048-token prefill, then single-token steps; each step's
+    decode kernel is timed alone with L2 flushed before it (the fp32 state is
+    just above L2's size, so without the flush part of it would be re-read
+    from L2)."""
+    from selective_state_space_forward_b200 import ssd
+    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs, make_step_inputs
+    w = WORKLOADS[DECODE_WORKLOAD]
+    inp = make_inputs(w)
+    dev = _device_inputs(w, inp, torch)
+    h = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, w.act_dtype,
+                   max_batch=w.batch, max_seqlen=w.seqlen, path=args.path)
+    state = h.new_state(w.batch)
+    h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"],
+              dev["D"], dev["conv_w"], dev["conv_b"], final_state=state)
+    del dev["x"], dev["z"], dev["B"], dev["C"], dev["dt_raw"]
+    steps_in = []
+    for i in range(8):
+        si = make_step_inputs(w, i)
+        steps_in.append({k: torch.from_numpy(v).to(torch.bfloat16 if k in "xzBC" else
+                                                     torch.float32).cuda() for k, v in si.items()})
+    out = torch.empty(w.batch, w.nheads * w.headdim, dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = steps_in[i % len(steps_in)]
+        h.step(s["x"], s["z"], s["dt_raw"], dev["dt_bias"], dev["A"], s["B"], s["C"], dev["D"],
+               dev["conv_w"], dev["conv_b"], state=state, out=out, stream=stream)
+
+    for i in range(10):
+        step(i)
+    n = w.decode_steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for a_, b_ in ev:
+        a_.record(stream)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush.fill_(i & 0xFF)
+        h.set_timing_events(*ev[i])
+        step(i)
+    torch.cuda.synchronize()
+    h.set_timing_events(None, None)
+    h.check()
+    times = sorted(a_.elapsed_time(b_) for a_, b_ in ev)
+    med_ms = times[len(times) // 2]
+    state_b = w.batch * w.nheads * w.headdim * w.dstate * 4
+    conv_b = w.batch * 3 * w.conv_dim * 2
+    io_b = w.batch * (3 * w.nheads * w.headdim * 2 + 2 * w.ngroups * w.dstate * 2 + w.nheads * 4)
+    total = 2 * state_b + 2 * conv_b + io_b
+    gbs = total / (med_ms * 1e-3) / 1e9
+    return {"workload": f"{DECODE_WORKLOAD}: batch 256, 32 heads x 64, d_state 64, 8 groups, "
+                        "conv 4, after a 2048-token prefill",
+            "us_per_step_median": round(med_ms * 1e3, 2), "bytes_per_step": total,
+            "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "peak_source": peaks["source"], "steps_timed": n, "l2": "flushed before each step",
+            "traffic": measured_traffic(f"decode:{DECODE_WORKLOAD}", "decode")}
+
+
+# ---------------------------------------------------------------------------------------
+_INPUT_CACHE = {}
+
+
+def cpu_oracle_run(max_seconds: float | None = None):
+    """The fp64 oracle on this host's cores over (part of) the bench workload.
+    Returns (tokens-equivalent per second, description, threads, seconds)."""
+    import oracle
+    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
+    w = WORKLOADS[WORKLOAD]
+    if WORKLOAD not in _INPUT_CACHE:
+        _INPUT_CACHE[WORKLOAD] = make_inputs(w)
+    inp = _INPUT_CACHE[WORKLOAD]
+    cores = oracle.default_threads()
+    pairs = [(b, hh) for b in range(w.batch) for hh in range(w.nheads)]
+    L = w.seqlen
+    if max_seconds is not None:
+        # calibrate one pair on 512 tokens, then size the sample to the budget
+        t0 = time.time()
+        oracle.forward(w.with_(seqlen=512).dims(), _cut(inp, 512), pairs=[(0, 0)], threads=1,
+                       final=False)
+        per_tok = (time.time() - t0) / 512
+        npairs = min(len(pairs), cores)
+        L = int(max(64, min(w.seqlen, max_seconds / max(per_tok, 1e-9))) // 64 * 64)
+        pairs = pairs[:npairs]
+        inp = _cut(inp, L)
+    dims = w.with_(seqlen=L).dims()
+    t0 = time.time()
+    r = oracle.forward(dims, inp, pairs=pairs, threads=0, final=True)
+    dt = time.time() - t0
+    tokens_equiv = len(pairs) * L / w.nheads
+    desc = (f"{len(pairs)} (row, head) pairs of {WORKLOAD} over {L} tokens each "
+            f"(= {tokens_equiv:.0f} full-width tokens of 32 heads), fp64")
+    return tokens_equiv / dt, desc, r["threads"], dt
+
+
+def _cut(inp, L):
+    keys = ("x", "z", "B", "C", "dt_raw", "seq_idx")
+    return {k: (v[:, :L] if (v is not None and k in keys) else v) for k, v in inp.items()}
+
+
+def reference_arm(args):
+    """The oracle, as it stands, timed on the host cores: each step is a
+    bounded sample of the bench workload."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    for _ in range(args.warmup):
+        cpu_oracle_run(budget)
+    vals, descs, threads, wall = [], None, None, 0.0
+    for _ in range(args.steps):
+        v, descs, threads, dt = cpu_oracle_run(budget)
+        vals.append(v)
+        wall += dt
+    value = sum(vals) / len(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": wall / max(1, args.steps) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": descs},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(n):
+    return {"workload": f"{WORKLOAD}: Mamba-2 SSD mixer, batch 5 x 8192 tokens per GPU, "
+                        "32 heads x 64, d_state 64, 8 B/C groups, conv kernel 4, packed documents "
+                        "(geometric lengths, mean 1500), bf16 activations, fp32 dt/A/D/state",
+            "global_batch": 5 * n, "seq_len": 8192, "parallelism": f"dp{n} (independent rows)",
+            "l2": "inputs larger than L2 (595 MB per step), no flush"}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return reference_arm(args)
+    import torch
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    rank, world = dist_init("nccl")
+    peaks = load_peaks()
+    fwd, ctx = bench_forward(args, torch, rank, world, local_rank, peaks)
+    e2e = None if args.no_e2e else bench_e2e(args, torch, ctx, world, local_rank)
+    del ctx
+    decode = None
+    if not args.no_decode and rank == 0:
+        torch.cuda.empty_cache()
+        decode = bench_decode(args, torch, peaks)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        v, desc, threads, _ = cpu_oracle_run(None)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        line = {"metric": METRIC, "value": fwd["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": fwd["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": config_block(world),
+                "path": fwd["path"], "roofline": fwd["roofline"],
+                "forward_roofline": fwd["forward_roofline"], "decode": decode,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": fwd["launches"],
+                "clocks": fwd["clocks"]}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,201 @@
+/*
+ * ssd.h -- C ABI of libssd.so, a B200 (sm_100a) implementation of the
+ * Mamba-2 / SSD selective-state-space mixer scan.
+ *
+ * The operation (per batch row b and head h, tokens t = 0 .. L-1):
+ *
+ *   u        = SiLU(causal depthwise conv, kernel 4, over the x|B|C channels)
+ *              -- "Mini-K3-1H-mamba2-n64-g8" model card, Architecture; the
+ *              channel order x|B|C and conv_dim = H*P + 2*G*N follow the
+ *              codestral_mamba.ts weight-port header.  With dconv = 1 there
+ *              is no conv and no SiLU (mojolearn Mamba3Block: "v is the raw
+ *              x split").
+ *   B_t, C_t = optional RMSNorm (eps 1e-5) * weight + per-head bias
+ *              (mojolearn Mamba3Block, class description and Parameters)
+ *   dt_t     = softplus(dt_raw_t + dt_bias[h]), no clamp (falcon_mamba.ts
+ *              header; Mamba3Block "no dt clamp")
+ *   a_t      = A[h], or per token max-magnitude-floored: min(A[b,t,h], -1e-4)
+ *              (Mamba3Block "A floor 1e-4")
+ *   h_t      = exp(dt_t a_t) h_{t-1} + dt_t x_t (outer) B_t      (P x N, fp32)
+ *   y_t      = C_t . h_t + D[h] x_t ;   out_t = y_t * SiLU(z_t)
+ *
+ * and the state restarts from zero (and the conv sees no earlier token) at
+ * every packed-document boundary: a position whose seq_idx differs from its
+ * left neighbour's (model card, "Checkpoint and training").  The caller's
+ * initial state belongs to the first document of each row.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *    and row-major as described per argument.  Activation tensors (x, z, B,
+ *    C, out, conv_w, conv_b and the conv part of a state buffer) have the
+ *    handle's act_dtype; dt_raw, dt_bias, A, D, norm weights and the SSM
+ *    state are fp32; seq_idx is int32.
+ *  - x, z, B, C, out and state buffers must be 16-byte aligned; the other
+ *    pointers 4-byte aligned.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  A handle serves one stream at a time.
+ *  - Arguments are validated on the host before anything is launched: a call
+ *    that returns an error status launched nothing and touched no memory.
+ *    ssd_last_error() then names the offending argument (the calling thread's
+ *    message).  Errors raised on the device by an accepted call are reported
+ *    by ssd_check().
+ *  - Calls allocate nothing: ssd_create sizes the handle's workspace for
+ *    max_batch x max_seqlen.
+ */
+#ifndef SSD_H
+#define SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                 /* cudaStream_t is struct CUstream_st* */
+typedef struct ssd_handle ssd_handle;
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,        /* null/ill-formed argument, bad shape */
+    SSD_ERR_UNSUPPORTED = 2,        /* well-formed but not implemented (e.g. headdim % 8) */
+    SSD_ERR_ALIGNMENT = 3,          /* pointer not aligned as required */
+    SSD_ERR_SHAPE_EXCEEDS_MAX = 4,  /* batch/seqlen above the handle's maxima */
+    SSD_ERR_CUDA = 5,               /* a CUDA runtime call failed */
+    SSD_ERR_DEVICE = 6              /* ssd_check: the device reported an error */
+} ssd_status;
+
+typedef enum { SSD_DTYPE_F32 = 0, SSD_DTYPE_BF16 = 1 } ssd_dtype;
+typedef enum { SSD_A_PER_HEAD = 0, SSD_A_PER_TOKEN = 1 } ssd_a_mode;
+
+/* Which kernel sequence ssd_forward runs.
+ *  FUSED : one persistent chunk-sweep kernel per (row, head) that keeps the
+ *          running state on chip (tcgen05 tensor-core contractions, bf16
+ *          operands, fp32 accumulation); bf16 activations, headdim 64,
+ *          d_state 64 or 128.
+ *  STAGED: the five-stage pipeline conv -> dt/cumsum -> chunk states ->
+ *          state passing -> chunk outputs, fp32 arithmetic throughout; any
+ *          supported shape and both dtypes.
+ *  AUTO  : FUSED when the shape and dtype allow it, else STAGED. */
+typedef enum { SSD_PATH_AUTO = 0, SSD_PATH_FUSED = 1, SSD_PATH_STAGED = 2 } ssd_path;
+
+typedef struct {
+    int32_t nheads;      /* H >= 1 */
+    int32_t headdim;     /* P, multiple of 8, <= 128 */
+    int32_t dstate;      /* N, multiple of 8, <= 256 */
+    int32_t ngroups;     /* G, divides H; head h uses B/C group h / (H / G) */
+    int32_t dconv;       /* 1 (no conv) or 4 */
+    int32_t chunk;       /* 0 or 64 (the chunk length of the chunked scan) */
+    int32_t act_dtype;   /* ssd_dtype */
+    int32_t a_mode;      /* ssd_a_mode */
+    int32_t bc_norm;     /* 1: B/C RMSNorm + per-head bias, see ssd_set_bc_norm */
+    int32_t max_batch;   /* >= 1 */
+    int32_t max_seqlen;  /* >= 1 */
+    int32_t path;        /* ssd_path */
+} ssd_desc;
+
+/* Create a handle for one layer shape.  Validates d, picks the path, and
+ * allocates (cudaMalloc, on the current device) the workspace every later
+ * call uses.  On success *out owns that memory until ssd_destroy. */
+ssd_status ssd_create(const ssd_desc* d, ssd_handle** out);
+
+/* Free the handle's workspace and the handle; NULL is a no-op.  The caller
+ * must make sure no call on the handle is still running on the GPU. */
+void ssd_destroy(ssd_handle* h);
+
+/* The path ssd_create chose (SSD_PATH_FUSED or SSD_PATH_STAGED), or -1. */
+int32_t ssd_get_path(const ssd_handle* h);
+
+/* B/C normalisation parameters (Mamba3Block Parameters: B_norm.weight,
+ * C_norm.weight (N); B_bias, C_bias (H, N)), device fp32 pointers that must
+ * stay valid while calls run.  NULL weight = ones, NULL bias = zeros.  Only
+ * for handles created with bc_norm = 1. */
+ssd_status ssd_set_bc_norm(ssd_handle* h, const float* B_norm_w, const float* C_norm_w,
+                           const float* B_bias, const float* C_bias);
+
+/* Bytes of one state buffer for `batch` rows: the fp32 SSM state
+ * (batch, H, P, N), then, at ssd_state_conv_offset, the conv history
+ * (batch, dconv-1, conv_dim) in act_dtype, oldest token first (absent when
+ * dconv = 1).  An all-zero buffer is a fresh state (Mamba3Block.allocate_state). */
+size_t ssd_state_bytes(const ssd_handle* h, int32_t batch);
+size_t ssd_state_conv_offset(const ssd_handle* h, int32_t batch);
+
+/*
+ * Forward over `seqlen` tokens of `batch` rows (Mamba3Block.forward with a
+ * state: read at entry, written at exit).
+ *   x, z, out   (batch, seqlen, H*P)   channel h*P + p
+ *   dt_raw      (batch, seqlen, H)     fp32
+ *   dt_bias, D  (H)                    fp32
+ *   A           (H) fp32, already negative (A = -exp(A_log), codestral_mamba.ts
+ *               reconciliation 2), or (batch, seqlen, H) when a_mode = PER_TOKEN
+ *   B, C        (batch, seqlen, G*N)
+ *   conv_w      (conv_dim, dconv), conv_b (conv_dim), x|B|C channel order; w[c, dconv-1]
+ *               multiplies the current token.  NULL iff dconv = 1.
+ *   seq_idx     (batch, seqlen) int32 document ids, or NULL (one document per row)
+ *   init_state  state buffer (ssd_state_bytes) read at entry, or NULL (zeros)
+ *   final_state state buffer written at exit, or NULL; may equal init_state
+ *   out         may not alias any input
+ * Returns SSD_OK or an error before any launch (see above).
+ */
+ssd_status ssd_forward(ssd_handle* h, int32_t batch, int32_t seqlen,
+                       const void* x, const void* z, const float* dt_raw, const float* dt_bias,
+                       const float* A, const void* B, const void* C, const float* D,
+                       const void* conv_w, const void* conv_b, const int32_t* seq_idx,
+                       const void* init_state, void* out, void* final_state,
+                       struct CUstream_st* stream);
+
+/*
+ * One decode token per row (Mamba3Block.step: the same computation as forward
+ * at L = 1 with the state carried).  Inputs are the forward's with seqlen 1:
+ * x, z, out (batch, H*P); B, C (batch, G*N); dt_raw (batch, H); A (H) or
+ * (batch, H).  `state` is required and updated in place.
+ */
+ssd_status ssd_step(ssd_handle* h, int32_t batch,
+                    const void* x, const void* z, const float* dt_raw, const float* dt_bias,
+                    const float* A, const void* B, const void* C, const float* D,
+                    const void* conv_w, const void* conv_b, void* state, void* out,
+                    struct CUstream_st* stream);
+
+/*
+ * Stage entry points: run one stage of the staged path alone, for stage-level
+ * checks and profiling.
+ *   ssd_stage_conv : u (batch, seqlen, conv_dim) fp32 = SiLU(conv) of x|B|C
+ *                    (the first stage; init_state as in ssd_forward).
+ *   ssd_stage_dt   : dt (batch, H, seqlen) fp32 = softplus(dt_raw + dt_bias) and
+ *                    acs (batch, H, seqlen) fp32 = cumulative sum of dt*a restarted
+ *                    at every chunk start (64 tokens).
+ */
+ssd_status ssd_stage_conv(ssd_handle* h, int32_t batch, int32_t seqlen, const void* x,
+                          const void* B, const void* C, const void* conv_w, const void* conv_b,
+                          const int32_t* seq_idx, const void* init_state, float* u,
+                          struct CUstream_st* stream);
+ssd_status ssd_stage_dt(ssd_handle* h, int32_t batch, int32_t seqlen, const float* dt_raw,
+                        const float* dt_bias, const float* A, float* dt, float* acs,
+                        struct CUstream_st* stream);
+
+/* Measurement hook.  When start and stop are cudaEvent_t handles (created by
+ * the caller), every later ssd_forward / ssd_step records `start` on its
+ * stream just before its main kernel (the fused chunk sweep, the staged
+ * chunk-output kernel, or the decode kernel) and `stop` just after it, so
+ * cudaEventElapsedTime gives that kernel's device time.  NULL, NULL turns the
+ * hook off.  The events stay owned by the caller. */
+ssd_status ssd_set_timing_events(ssd_handle* h, void* start, void* stop);
+
+/* Number of kernels this handle has launched since ssd_create. */
+uint64_t ssd_launch_count(const ssd_handle* h);
+
+/* Wait for `stream`, then read and clear the handle's device status word.
+ * SSD_ERR_DEVICE when a kernel reported an error (ssd_last_error says which),
+ * SSD_ERR_CUDA when the stream itself failed. */
+ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream);
+
+/* The calling thread's last error message ("" when none). */
+const char* ssd_last_error(void);
+
+/* A static name for a status code. */
+const char* ssd_status_string(ssd_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSD_H */

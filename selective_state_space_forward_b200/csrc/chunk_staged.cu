@@ -1,0 +1,282 @@
+// chunk_staged.cu -- the staged path's K3 (chunk states), K4 (state passing)
+// and K5 (chunk outputs), in fp32 arithmetic.
+//
+// The chunked evaluation of the selective scan (chunk 64; mojolearn
+// Mamba3Block, "chunk size 64"): within a chunk c of tokens t0 .. t0+Lc-1,
+// with acs_t the chunk-local inclusive sum of dt*a and seg_t the number of
+// document boundaries at positions t0 .. t (a boundary at t0 means the token
+// before the chunk belongs to another document):
+//
+//   chunk state    S_c[p,n]  = sum_{s: seg_s = seg_last} exp(acs_last - acs_s) dt_s x_s[p] B_s[n]
+//   state passing  Hin_0     = initial state;  Hin_{c+1} = k_c Hin_c + S_c,
+//                  k_c = exp(acs_last) if the chunk holds no boundary, else 0
+//   chunk output   y_t[p]    = sum_{s<=t, seg_s = seg_t} (C_t . B_s) exp(acs_t - acs_s) dt_s x_s[p]
+//                            + [seg_t = 0] exp(acs_t) C_t . Hin_c[p, :]  +  D x_t[p]
+//                  out_t     = y_t * SiLU(z_t)
+//
+// which is the recurrence h_t = exp(dt_t a_t) h_{t-1} + dt_t x_t B_t^T,
+// y_t = C_t h_t + D x_t split at chunk boundaries, with the state restarting at
+// every packed-document boundary (model card, "Checkpoint and training").
+// x, B, C are the conv+SiLU outputs when the conv is on (u from K1, fp32),
+// else the raw inputs; B and C are RMS-normalised and given the head's bias
+// when the B/C norm is on (Mamba3Block class description).
+#include "ssd_device.cuh"
+#include "ssd_kernels.h"
+
+namespace ssd {
+
+// Chunk-local segment ids: seg[t] = boundaries at positions t0 .. t0+t.
+__device__ void chunk_segments(const int32_t* seq_row, int t0, int Lc, int* seg, int* flag)
+{
+    const int tid = threadIdx.x;
+    if (tid < kChunk) flag[tid] = (tid < Lc) ? is_boundary(seq_row, t0 + tid) : 0;
+    __syncthreads();
+    if (tid < kChunk) {
+        int acc = 0;
+        for (int j = 0; j <= tid; j++) acc += flag[j];
+        seg[tid] = acc;
+    }
+    __syncthreads();
+}
+
+// Load token rows [t0, t0+64) of the head's x (fp32 result, zero past the end).
+template <typename T>
+__device__ void load_x_rows(const Shape& s, const FwdArgs& a, const float* u, int b, int h,
+                            int t0, int Lc, float* xs, int ld)
+{
+    const int P = s.headdim, HP = s.nheads * P, cd = s.conv_dim();
+    for (int i = threadIdx.x; i < kChunk * P; i += blockDim.x) {
+        const int r = i / P, p = i % P;
+        float v = 0.0f;
+        if (r < Lc) {
+            const int64_t tok = (int64_t)b * s.seqlen + t0 + r;
+            v = u ? u[tok * cd + h * P + p] : to_f(((const T*)a.x)[tok * HP + h * P + p]);
+        }
+        xs[r * ld + p] = v;
+    }
+}
+
+// Load B (which = 0) or C (which = 1) rows of the head's group, then apply the
+// B/C norm and the head's bias when enabled.
+template <typename T>
+__device__ void load_bc_rows(const Shape& s, const FwdArgs& a, const float* u, int b, int h,
+                             int t0, int Lc, int which, float* dst, int ld)
+{
+    const int N = s.dstate, GN = s.ngroups * N, HP = s.nheads * s.headdim, cd = s.conv_dim();
+    const int g = h / (s.nheads / s.ngroups);
+    const T* raw = (const T*)(which ? a.C : a.B);
+    for (int i = threadIdx.x; i < kChunk * N; i += blockDim.x) {
+        const int r = i / N, n = i % N;
+        float v = 0.0f;
+        if (r < Lc) {
+            const int64_t tok = (int64_t)b * s.seqlen + t0 + r;
+            v = u ? u[tok * cd + HP + which * GN + g * N + n] : to_f(raw[tok * GN + g * N + n]);
+        }
+        dst[r * ld + n] = v;
+    }
+    if (!s.bc_norm) return;
+    __syncthreads();
+    const float* wn = which ? a.cn_w : a.bn_w;
+    const float* bias = which ? a.cn_bias : a.bn_bias;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int r = warp; r < Lc; r += nw) {
+        float ss = 0.0f;
+        for (int n = lane; n < N; n += 32) ss += dst[r * ld + n] * dst[r * ld + n];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float rs = rsqrtf(ss / N + kNormEps);
+        for (int n = lane; n < N; n += 32)
+            dst[r * ld + n] = dst[r * ld + n] * rs * (wn ? wn[n] : 1.0f) +
+                              (bias ? bias[(int64_t)h * N + n] : 0.0f);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+chunk_state_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float* __restrict__ dt,
+                   const float* __restrict__ acs, float* __restrict__ states)
+{
+    extern __shared__ float sm[];
+    const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
+    float* xs = sm;                    // [64][P], pre-scaled by the token weight
+    float* bs = xs + kChunk * P;       // [64][N]
+    float* wv = bs + kChunk * N;       // [64]
+    int* seg = (int*)(wv + kChunk);    // [64]
+    int* flag = seg + kChunk;          // [64]
+
+    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, seg, flag);
+    const float* dtr = dt + ((int64_t)b * H + h) * L + t0;
+    const float* acr = acs + ((int64_t)b * H + h) * L + t0;
+    if (threadIdx.x < kChunk) {
+        const int r = threadIdx.x;
+        wv[r] = (r < Lc && seg[r] == seg[Lc - 1]) ? expf(acr[Lc - 1] - acr[r]) * dtr[r] : 0.0f;
+    }
+    load_x_rows<T>(s, a, u, b, h, t0, Lc, xs, P);
+    load_bc_rows<T>(s, a, u, b, h, t0, Lc, 0, bs, N);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kChunk * P; i += blockDim.x) xs[i] *= wv[i / P];
+    __syncthreads();
+
+    float* dst = states + (((int64_t)b * nc + c) * H + h) * P * N;
+    for (int e = threadIdx.x; e < P * N; e += blockDim.x) {
+        const int p = e / N, n = e % N;
+        float acc = 0.0f;
+        for (int r = 0; r < Lc; r++) acc += xs[r * P + p] * bs[r * N + n];
+        dst[e] = acc;
+    }
+}
+
+// One thread per state element (row, head, p, n), walking the chunks in order.
+// Reads the initial state before writing the final one, so they may alias.
+__global__ void __launch_bounds__(256)
+state_passing_kernel(Shape s, const float* __restrict__ cdecay, float* __restrict__ states,
+                     const float* init, float* fin)
+{
+    const int PN = s.headdim * s.dstate, H = s.nheads, nc = s.nchunks();
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)s.batch * H * PN) return;
+    const int e = (int)(gid % PN);
+    const int h = (int)((gid / PN) % H);
+    const int b = (int)(gid / ((int64_t)PN * H));
+    float hv = init ? init[gid] : 0.0f;
+    const float* kd = cdecay + ((int64_t)b * H + h) * nc;
+    for (int c = 0; c < nc; c++) {
+        float* sp = states + (((int64_t)b * nc + c) * H + h) * PN + e;
+        const float sc = *sp;
+        *sp = hv;
+        hv = kd[c] * hv + sc;
+    }
+    if (fin) fin[gid] = hv;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float* __restrict__ dt,
+                    const float* __restrict__ acs, const float* __restrict__ hin)
+{
+    extern __shared__ float sm[];
+    const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
+    const int HP = H * P;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
+    const int NB = N + 1;              // padded row stride (bank spread)
+    float* cs = sm;                    // [64][N]
+    float* bs = cs + kChunk * N;       // [64][N+1]
+    float* xs = bs + kChunk * NB;      // [64][P]
+    float* hs = xs + kChunk * P;       // [P][N+1]
+    float* cb = hs + P * NB;           // [64][65]
+    float* ac = cb + kChunk * 65;      // [64]
+    float* dv = ac + kChunk;           // [64]
+    int* seg = (int*)(dv + kChunk);    // [64]
+    int* flag = seg + kChunk;          // [64]
+
+    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, seg, flag);
+    if (threadIdx.x < kChunk) {
+        const int r = threadIdx.x;
+        const int64_t o = ((int64_t)b * H + h) * L + t0 + r;
+        ac[r] = r < Lc ? acs[o] : 0.0f;
+        dv[r] = r < Lc ? dt[o] : 0.0f;
+    }
+    load_x_rows<T>(s, a, u, b, h, t0, Lc, xs, P);
+    load_bc_rows<T>(s, a, u, b, h, t0, Lc, 1, cs, N);
+    load_bc_rows<T>(s, a, u, b, h, t0, Lc, 0, bs, NB);
+    const float* hp = hin + (((int64_t)b * nc + c) * H + h) * P * N;
+    for (int e = threadIdx.x; e < P * N; e += blockDim.x) hs[(e / N) * NB + e % N] = hp[e];
+    __syncthreads();
+
+    for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
+        const int t = e / kChunk, r = e % kChunk;
+        float v = 0.0f;
+        if (r <= t && t < Lc && seg[r] == seg[t]) {
+            float dot = 0.0f;
+            for (int n = 0; n < N; n++) dot += cs[t * N + n] * bs[r * NB + n];
+            v = dot * expf(ac[t] - ac[r]) * dv[r];
+        }
+        cb[t * 65 + r] = v;
+    }
+    __syncthreads();
+
+    const float Dh = a.D[h];
+    for (int e = threadIdx.x; e < kChunk * P; e += blockDim.x) {
+        const int t = e / P, p = e % P;
+        if (t >= Lc) continue;
+        float y = 0.0f;
+        for (int r = 0; r <= t; r++) y += cb[t * 65 + r] * xs[r * P + p];
+        if (seg[t] == 0) {
+            float off = 0.0f;
+            for (int n = 0; n < N; n++) off += cs[t * N + n] * hs[p * NB + n];
+            y += expf(ac[t]) * off;
+        }
+        y += Dh * xs[t * P + p];
+        const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
+        const float zv = to_f(((const T*)a.z)[o]);
+        ((T*)a.out)[o] = from_f<T>(y * silu_f(zv));
+    }
+}
+
+size_t chunk_state_smem_bytes(const Shape& s)
+{
+    return sizeof(float) * ((size_t)kChunk * s.headdim + (size_t)kChunk * s.dstate + kChunk) +
+           sizeof(int) * 2 * kChunk;
+}
+
+size_t chunk_output_smem_bytes(const Shape& s)
+{
+    const size_t N = s.dstate, P = s.headdim;
+    return sizeof(float) * (kChunk * N + kChunk * (N + 1) + kChunk * P + P * (N + 1) +
+                            kChunk * 65 + 2 * kChunk) + sizeof(int) * 2 * kChunk;
+}
+
+cudaError_t launch_chunk_state(const Shape& s, const FwdArgs& a, const float* u,
+                               const float* dt, const float* acs, float* states, cudaStream_t st)
+{
+    const dim3 grid(s.nchunks(), s.nheads, s.batch);
+    const size_t smem = chunk_state_smem_bytes(s);
+    cudaError_t e;
+    if (s.act_bf16) {
+        e = cudaFuncSetAttribute(chunk_state_kernel<bf16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        chunk_state_kernel<bf16><<<grid, 256, smem, st>>>(s, a, u, dt, acs, states);
+    } else {
+        e = cudaFuncSetAttribute(chunk_state_kernel<float>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        chunk_state_kernel<float><<<grid, 256, smem, st>>>(s, a, u, dt, acs, states);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_passing(const Shape& s, const FwdArgs& a, const float* cdecay,
+                                 float* states, cudaStream_t st)
+{
+    const int64_t total = (int64_t)s.batch * s.nheads * s.headdim * s.dstate;
+    state_passing_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+        s, cdecay, states, a.init_ssm, a.final_ssm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_output(const Shape& s, const FwdArgs& a, const float* u,
+                                const float* dt, const float* acs, const float* hin,
+                                cudaStream_t st)
+{
+    const dim3 grid(s.nchunks(), s.nheads, s.batch);
+    const size_t smem = chunk_output_smem_bytes(s);
+    cudaError_t e;
+    if (s.act_bf16) {
+        e = cudaFuncSetAttribute(chunk_output_kernel<bf16>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        chunk_output_kernel<bf16><<<grid, 256, smem, st>>>(s, a, u, dt, acs, hin);
+    } else {
+        e = cudaFuncSetAttribute(chunk_output_kernel<float>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        chunk_output_kernel<float><<<grid, 256, smem, st>>>(s, a, u, dt, acs, hin);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

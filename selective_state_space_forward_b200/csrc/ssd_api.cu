@@ -1,0 +1,486 @@
+// ssd_api.cu -- host layer of libssd.so: the C ABI declared in include/ssd.h.
+//
+// Every entry point validates its arguments on the host before enqueuing any
+// work, names the bad argument in a thread-local message (the refuse-by-name
+// convention of the mojolearn Mamba3Block docs: wrong inputs "are refused by
+// name rather than converted"), and launches its kernels on the caller's
+// stream.  Workspace is allocated once, at ssd_create, for the handle's
+// maximum batch and sequence length.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "ssd.h"
+#include "ssd_kernels.h"
+
+using namespace ssd;
+
+namespace {
+
+thread_local std::string g_err;
+
+ssd_status fail(ssd_status st, const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+ssd_status cuda_fail(cudaError_t e, const char* what)
+{
+    return fail(SSD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+}  // namespace
+
+struct ssd_handle {
+    ssd_desc d;
+    int path;             // SSD_PATH_FUSED or SSD_PATH_STAGED
+    int device;
+    char* ws;             // one cudaMalloc'd block
+    size_t ws_bytes;
+    float* u;             // staged: conv output (B, L, conv_dim) fp32
+    float* dt;            // (B, H, L)
+    float* acs;           // (B, H, L)
+    float* cdecay;        // staged: (B, H, nc)
+    float* states;        // staged: (B, nc, H, P, N)
+    void* ubc;            // fused: conv'd B|C (B, L, 2GN) bf16
+    int* status;          // device status word
+    const float *bn_w, *cn_w, *bn_bias, *cn_bias;
+    cudaEvent_t ev_start, ev_stop;   // measurement hook (caller-owned), or null
+    uint64_t launches;               // kernels launched since ssd_create
+};
+
+namespace {
+
+int conv_dim(const ssd_desc& d) { return d.nheads * d.headdim + 2 * d.ngroups * d.dstate; }
+size_t act_size(const ssd_desc& d) { return d.act_dtype == SSD_DTYPE_BF16 ? 2 : 4; }
+
+Shape make_shape(const ssd_handle* h, int batch, int seqlen)
+{
+    Shape s;
+    s.batch = batch;
+    s.seqlen = seqlen;
+    s.nheads = h->d.nheads;
+    s.headdim = h->d.headdim;
+    s.dstate = h->d.dstate;
+    s.ngroups = h->d.ngroups;
+    s.dconv = h->d.dconv;
+    s.act_bf16 = h->d.act_dtype == SSD_DTYPE_BF16;
+    s.a_per_token = h->d.a_mode == SSD_A_PER_TOKEN;
+    s.bc_norm = h->d.bc_norm;
+    return s;
+}
+
+size_t conv_offset(const ssd_desc& d, int batch)
+{
+    return align256((size_t)batch * d.nheads * d.headdim * d.dstate * sizeof(float));
+}
+
+bool fused_supported(const ssd_desc& d)
+{
+    return fused_path_available() && d.act_dtype == SSD_DTYPE_BF16 && d.headdim == 64 &&
+           (d.dstate == 64 || d.dstate == 128);
+}
+
+ssd_status validate_desc(const ssd_desc* d)
+{
+    if (!d) return fail(SSD_ERR_INVALID_ARG, "desc is NULL");
+    if (d->nheads < 1) return fail(SSD_ERR_INVALID_ARG, "nheads must be >= 1 (got %d)", d->nheads);
+    if (d->headdim < 8 || d->headdim > 128 || d->headdim % 8)
+        return fail(SSD_ERR_UNSUPPORTED, "headdim must be a multiple of 8 in [8, 128] (got %d)",
+                    d->headdim);
+    if (d->dstate < 8 || d->dstate > 256 || d->dstate % 8)
+        return fail(SSD_ERR_UNSUPPORTED, "dstate must be a multiple of 8 in [8, 256] (got %d)",
+                    d->dstate);
+    if (d->ngroups < 1 || d->nheads % d->ngroups)
+        return fail(SSD_ERR_INVALID_ARG, "ngroups (%d) must divide nheads (%d)", d->ngroups,
+                    d->nheads);
+    if (d->dconv != 1 && d->dconv != 4)
+        return fail(SSD_ERR_UNSUPPORTED, "dconv must be 1 (no conv) or 4 (got %d)", d->dconv);
+    if (d->chunk != 0 && d->chunk != 64)
+        return fail(SSD_ERR_UNSUPPORTED, "chunk must be 0 or 64 (got %d)", d->chunk);
+    if (d->act_dtype != SSD_DTYPE_F32 && d->act_dtype != SSD_DTYPE_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "act_dtype %d is not an ssd_dtype", d->act_dtype);
+    if (d->a_mode != SSD_A_PER_HEAD && d->a_mode != SSD_A_PER_TOKEN)
+        return fail(SSD_ERR_INVALID_ARG, "a_mode %d is not an ssd_a_mode", d->a_mode);
+    if (d->bc_norm != 0 && d->bc_norm != 1)
+        return fail(SSD_ERR_INVALID_ARG, "bc_norm must be 0 or 1 (got %d)", d->bc_norm);
+    if (d->max_batch < 1 || d->max_seqlen < 1)
+        return fail(SSD_ERR_INVALID_ARG, "max_batch and max_seqlen must be >= 1");
+    if (d->path < SSD_PATH_AUTO || d->path > SSD_PATH_STAGED)
+        return fail(SSD_ERR_INVALID_ARG, "path %d is not an ssd_path", d->path);
+    if (d->path == SSD_PATH_FUSED && !fused_supported(*d))
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "the fused path needs bf16 activations, headdim 64 and dstate 64 or 128");
+    return SSD_OK;
+}
+
+ssd_status check_ptr(const void* p, const char* name, size_t align, bool required)
+{
+    if (!p) return required ? fail(SSD_ERR_INVALID_ARG, "%s is NULL", name) : SSD_OK;
+    if (!aligned(p, align))
+        return fail(SSD_ERR_ALIGNMENT, "%s (%p) is not %zu-byte aligned", name, p, align);
+    return SSD_OK;
+}
+
+#define SSD_TRY(expr)                     \
+    do {                                  \
+        ssd_status st_ = (expr);          \
+        if (st_ != SSD_OK) return st_;    \
+    } while (0)
+
+#define SSD_CUDA(expr, what)                          \
+    do {                                              \
+        cudaError_t e_ = (expr);                      \
+        if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+    } while (0)
+
+// A kernel launch: counted, and reported as SSD_ERR_CUDA when it fails.
+#define SSD_LAUNCH(h, expr, what)                     \
+    do {                                              \
+        (h)->launches++;                              \
+        SSD_CUDA(expr, what);                         \
+    } while (0)
+
+// The main kernel of a call, bracketed by the caller's timing events when set.
+#define SSD_MAIN_LAUNCH(h, st, expr, what)                                         \
+    do {                                                                           \
+        if ((h)->ev_start) SSD_CUDA(cudaEventRecord((h)->ev_start, st), "timing event"); \
+        SSD_LAUNCH(h, expr, what);                                                 \
+        if ((h)->ev_stop) SSD_CUDA(cudaEventRecord((h)->ev_stop, st), "timing event");   \
+    } while (0)
+
+ssd_status check_handle_dims(const ssd_handle* h, int batch, int seqlen)
+{
+    if (!h) return fail(SSD_ERR_INVALID_ARG, "handle is NULL");
+    if (batch < 0 || seqlen < 0)
+        return fail(SSD_ERR_INVALID_ARG, "batch (%d) and seqlen (%d) must be >= 0", batch, seqlen);
+    if (batch > h->d.max_batch)
+        return fail(SSD_ERR_SHAPE_EXCEEDS_MAX, "batch %d exceeds max_batch %d", batch,
+                    h->d.max_batch);
+    if (seqlen > h->d.max_seqlen)
+        return fail(SSD_ERR_SHAPE_EXCEEDS_MAX, "seqlen %d exceeds max_seqlen %d", seqlen,
+                    h->d.max_seqlen);
+    return SSD_OK;
+}
+
+// Pointers shared by forward and step.
+ssd_status check_common(const ssd_handle* h, const void* x, const void* z, const float* dt_raw,
+                        const float* dt_bias, const float* A, const void* B, const void* C,
+                        const float* D, const void* conv_w, const void* conv_b, const void* out)
+{
+    SSD_TRY(check_ptr(x, "x", 16, true));
+    SSD_TRY(check_ptr(z, "z", 16, true));
+    SSD_TRY(check_ptr(B, "B", 16, true));
+    SSD_TRY(check_ptr(C, "C", 16, true));
+    SSD_TRY(check_ptr(out, "out", 16, true));
+    SSD_TRY(check_ptr(dt_raw, "dt_raw", 4, true));
+    SSD_TRY(check_ptr(dt_bias, "dt_bias", 4, true));
+    SSD_TRY(check_ptr(A, "A", 4, true));
+    SSD_TRY(check_ptr(D, "D", 4, true));
+    if (h->d.dconv == 4) {
+        SSD_TRY(check_ptr(conv_w, "conv_w", 16, true));
+        SSD_TRY(check_ptr(conv_b, "conv_b", 16, true));
+    } else if (conv_w || conv_b) {
+        return fail(SSD_ERR_INVALID_ARG, "conv_w/conv_b must be NULL when dconv is 1");
+    }
+    if (out == x || out == z || out == B || out == C)
+        return fail(SSD_ERR_INVALID_ARG, "out may not alias an input");
+    return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssd_last_error(void) { return g_err.c_str(); }
+
+const char* ssd_status_string(ssd_status s)
+{
+    switch (s) {
+    case SSD_OK: return "SSD_OK";
+    case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG";
+    case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED";
+    case SSD_ERR_ALIGNMENT: return "SSD_ERR_ALIGNMENT";
+    case SSD_ERR_SHAPE_EXCEEDS_MAX: return "SSD_ERR_SHAPE_EXCEEDS_MAX";
+    case SSD_ERR_CUDA: return "SSD_ERR_CUDA";
+    case SSD_ERR_DEVICE: return "SSD_ERR_DEVICE";
+    }
+    return "SSD_ERR_UNKNOWN";
+}
+
+ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
+{
+    g_err.clear();
+    if (!out) return fail(SSD_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    SSD_TRY(validate_desc(d));
+    int path = d->path;
+    if (path == SSD_PATH_AUTO) path = fused_supported(*d) ? SSD_PATH_FUSED : SSD_PATH_STAGED;
+
+    ssd_desc dd = *d;
+    dd.chunk = 64;
+    dd.path = path;
+    Shape s;
+    s.batch = dd.max_batch; s.seqlen = dd.max_seqlen; s.nheads = dd.nheads;
+    s.headdim = dd.headdim; s.dstate = dd.dstate; s.ngroups = dd.ngroups; s.dconv = dd.dconv;
+    s.act_bf16 = dd.act_dtype == SSD_DTYPE_BF16; s.a_per_token = dd.a_mode; s.bc_norm = dd.bc_norm;
+    if (path == SSD_PATH_STAGED) {
+        const size_t lim = 227 * 1024;
+        if (chunk_output_smem_bytes(s) > lim || chunk_state_smem_bytes(s) > lim)
+            return fail(SSD_ERR_UNSUPPORTED,
+                        "headdim %d x dstate %d needs more shared memory than the staged path has",
+                        dd.headdim, dd.dstate);
+    }
+
+    const size_t BL = (size_t)dd.max_batch * dd.max_seqlen;
+    const size_t nc = (size_t)(dd.max_seqlen + 63) / 64;
+    const size_t H = dd.nheads, P = dd.headdim, N = dd.dstate, G = dd.ngroups;
+    size_t off = 0, o_u = 0, o_dt, o_acs, o_cd = 0, o_st = 0, o_ubc = 0, o_status;
+    auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+    if (path == SSD_PATH_STAGED && dd.dconv == 4) o_u = take(BL * conv_dim(dd) * sizeof(float));
+    o_dt = take((size_t)dd.max_batch * H * dd.max_seqlen * sizeof(float));
+    o_acs = take((size_t)dd.max_batch * H * dd.max_seqlen * sizeof(float));
+    if (path == SSD_PATH_STAGED) {
+        o_cd = take((size_t)dd.max_batch * H * nc * sizeof(float));
+        o_st = take((size_t)dd.max_batch * nc * H * P * N * sizeof(float));
+    }
+    if (path == SSD_PATH_FUSED && dd.dconv == 4) o_ubc = take(BL * 2 * G * N * 2);
+    o_status = take(256);
+
+    ssd_handle* h = new ssd_handle();
+    h->d = dd;
+    h->path = path;
+    cudaGetDevice(&h->device);
+    cudaError_t e = cudaMalloc(&h->ws, off);
+    if (e != cudaSuccess) {
+        delete h;
+        return cuda_fail(e, "cudaMalloc(workspace)");
+    }
+    h->ws_bytes = off;
+    h->u = (path == SSD_PATH_STAGED && dd.dconv == 4) ? (float*)(h->ws + o_u) : nullptr;
+    h->dt = (float*)(h->ws + o_dt);
+    h->acs = (float*)(h->ws + o_acs);
+    h->cdecay = path == SSD_PATH_STAGED ? (float*)(h->ws + o_cd) : nullptr;
+    h->states = path == SSD_PATH_STAGED ? (float*)(h->ws + o_st) : nullptr;
+    h->ubc = (path == SSD_PATH_FUSED && dd.dconv == 4) ? (void*)(h->ws + o_ubc) : nullptr;
+    h->status = (int*)(h->ws + o_status);
+    e = cudaMemset(h->status, 0, 256);
+    if (e != cudaSuccess) {
+        cudaFree(h->ws);
+        delete h;
+        return cuda_fail(e, "cudaMemset(status)");
+    }
+    *out = h;
+    return SSD_OK;
+}
+
+void ssd_destroy(ssd_handle* h)
+{
+    if (!h) return;
+    cudaFree(h->ws);
+    delete h;
+}
+
+int32_t ssd_get_path(const ssd_handle* h) { return h ? h->path : -1; }
+
+ssd_status ssd_set_bc_norm(ssd_handle* h, const float* B_norm_w, const float* C_norm_w,
+                           const float* B_bias, const float* C_bias)
+{
+    g_err.clear();
+    if (!h) return fail(SSD_ERR_INVALID_ARG, "handle is NULL");
+    if (!h->d.bc_norm) return fail(SSD_ERR_INVALID_ARG, "handle was created with bc_norm = 0");
+    SSD_TRY(check_ptr(B_norm_w, "B_norm_w", 4, false));
+    SSD_TRY(check_ptr(C_norm_w, "C_norm_w", 4, false));
+    SSD_TRY(check_ptr(B_bias, "B_bias", 4, false));
+    SSD_TRY(check_ptr(C_bias, "C_bias", 4, false));
+    h->bn_w = B_norm_w;
+    h->cn_w = C_norm_w;
+    h->bn_bias = B_bias;
+    h->cn_bias = C_bias;
+    return SSD_OK;
+}
+
+size_t ssd_state_conv_offset(const ssd_handle* h, int32_t batch)
+{
+    if (!h || batch < 0) return 0;
+    return conv_offset(h->d, batch);
+}
+
+size_t ssd_state_bytes(const ssd_handle* h, int32_t batch)
+{
+    if (!h || batch < 0) return 0;
+    size_t b = conv_offset(h->d, batch);
+    if (h->d.dconv == 4) b += (size_t)batch * 3 * conv_dim(h->d) * act_size(h->d);
+    return align256(b);
+}
+
+ssd_status ssd_forward(ssd_handle* h, int32_t batch, int32_t seqlen, const void* x, const void* z,
+                       const float* dt_raw, const float* dt_bias, const float* A, const void* B,
+                       const void* C, const float* D, const void* conv_w, const void* conv_b,
+                       const int32_t* seq_idx, const void* init_state, void* out,
+                       void* final_state, struct CUstream_st* stream)
+{
+    g_err.clear();
+    SSD_TRY(check_handle_dims(h, batch, seqlen));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (batch == 0) return SSD_OK;
+    SSD_TRY(check_ptr(init_state, "init_state", 16, false));
+    SSD_TRY(check_ptr(final_state, "final_state", 16, false));
+    if (seqlen == 0) {   // no token: the state passes through unchanged
+        if (final_state && final_state != init_state) {
+            const size_t n = ssd_state_bytes(h, batch);
+            SSD_CUDA(init_state ? cudaMemcpyAsync(final_state, init_state, n,
+                                                  cudaMemcpyDeviceToDevice, st)
+                                : cudaMemsetAsync(final_state, 0, n, st),
+                     "empty-sequence state copy");
+        }
+        return SSD_OK;
+    }
+    SSD_TRY(check_common(h, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, out));
+    SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
+    if (out == init_state || out == final_state)
+        return fail(SSD_ERR_INVALID_ARG, "out may not alias a state buffer");
+
+    const Shape s = make_shape(h, batch, seqlen);
+    FwdArgs a;
+    a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
+    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
+    a.init_ssm = (const float*)init_state;
+    a.init_conv = (init_state && s.dconv == 4) ? (const char*)init_state + conv_offset(h->d, batch)
+                                               : nullptr;
+    a.out = out;
+    a.final_ssm = (float*)final_state;
+    a.final_conv = (final_state && s.dconv == 4) ? (char*)final_state + conv_offset(h->d, batch)
+                                                 : nullptr;
+    a.bn_w = h->bn_w; a.cn_w = h->cn_w; a.bn_bias = h->bn_bias; a.cn_bias = h->cn_bias;
+
+    if (h->path == SSD_PATH_STAGED) {
+        if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_all(s, a, h->u, st), "conv kernel");
+        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, h->cdecay, st), "dt/cumsum kernel");
+        SSD_LAUNCH(h, launch_chunk_state(s, a, h->u, h->dt, h->acs, h->states, st),
+                   "chunk-state kernel");
+        SSD_LAUNCH(h, launch_state_passing(s, a, h->cdecay, h->states, st), "state-passing kernel");
+        SSD_MAIN_LAUNCH(h, st, launch_chunk_output(s, a, h->u, h->dt, h->acs, h->states, st),
+                        "chunk-output kernel");
+    } else {
+        if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_bc(s, a, h->ubc, st), "B|C conv kernel");
+        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, nullptr, st), "dt/cumsum kernel");
+        SSD_MAIN_LAUNCH(h, st, launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->status, st),
+                        "fused chunk kernel");
+    }
+    if (a.final_conv) SSD_LAUNCH(h, launch_conv_state(s, a, st), "conv-state kernel");
+    return SSD_OK;
+}
+
+ssd_status ssd_step(ssd_handle* h, int32_t batch, const void* x, const void* z,
+                    const float* dt_raw, const float* dt_bias, const float* A, const void* B,
+                    const void* C, const float* D, const void* conv_w, const void* conv_b,
+                    void* state, void* out, struct CUstream_st* stream)
+{
+    g_err.clear();
+    SSD_TRY(check_handle_dims(h, batch, 1));
+    if (batch == 0) return SSD_OK;
+    SSD_TRY(check_common(h, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, out));
+    SSD_TRY(check_ptr(state, "state", 16, true));
+    if (out == state) return fail(SSD_ERR_INVALID_ARG, "out may not alias the state");
+    const Shape s = make_shape(h, batch, 1);
+    FwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
+    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.out = out;
+    a.bn_w = h->bn_w; a.cn_w = h->cn_w; a.bn_bias = h->bn_bias; a.cn_bias = h->cn_bias;
+    void* hist = s.dconv == 4 ? (char*)state + conv_offset(h->d, batch) : nullptr;
+    SSD_MAIN_LAUNCH(h, (cudaStream_t)stream,
+                    launch_decode_step(s, a, (float*)state, hist, (cudaStream_t)stream),
+                    "decode kernel");
+    return SSD_OK;
+}
+
+ssd_status ssd_stage_conv(ssd_handle* h, int32_t batch, int32_t seqlen, const void* x,
+                          const void* B, const void* C, const void* conv_w, const void* conv_b,
+                          const int32_t* seq_idx, const void* init_state, float* u,
+                          struct CUstream_st* stream)
+{
+    g_err.clear();
+    SSD_TRY(check_handle_dims(h, batch, seqlen));
+    if (h->d.dconv != 4) return fail(SSD_ERR_UNSUPPORTED, "the handle has no conv (dconv is 1)");
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    SSD_TRY(check_ptr(x, "x", 16, true));
+    SSD_TRY(check_ptr(B, "B", 16, true));
+    SSD_TRY(check_ptr(C, "C", 16, true));
+    SSD_TRY(check_ptr(conv_w, "conv_w", 16, true));
+    SSD_TRY(check_ptr(conv_b, "conv_b", 16, true));
+    SSD_TRY(check_ptr(u, "u", 16, true));
+    SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
+    SSD_TRY(check_ptr(init_state, "init_state", 16, false));
+    const Shape s = make_shape(h, batch, seqlen);
+    FwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.x = x; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b; a.seq_idx = seq_idx;
+    a.init_conv = init_state ? (const char*)init_state + conv_offset(h->d, batch) : nullptr;
+    SSD_LAUNCH(h, launch_conv_silu_all(s, a, u, (cudaStream_t)stream), "conv kernel");
+    return SSD_OK;
+}
+
+ssd_status ssd_stage_dt(ssd_handle* h, int32_t batch, int32_t seqlen, const float* dt_raw,
+                        const float* dt_bias, const float* A, float* dt, float* acs,
+                        struct CUstream_st* stream)
+{
+    g_err.clear();
+    SSD_TRY(check_handle_dims(h, batch, seqlen));
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    SSD_TRY(check_ptr(dt_raw, "dt_raw", 4, true));
+    SSD_TRY(check_ptr(dt_bias, "dt_bias", 4, true));
+    SSD_TRY(check_ptr(A, "A", 4, true));
+    SSD_TRY(check_ptr(dt, "dt", 4, true));
+    SSD_TRY(check_ptr(acs, "acs", 4, true));
+    const Shape s = make_shape(h, batch, seqlen);
+    FwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A;
+    SSD_LAUNCH(h, launch_dt_cumsum(s, a, dt, acs, nullptr, (cudaStream_t)stream),
+               "dt/cumsum kernel");
+    return SSD_OK;
+}
+
+ssd_status ssd_set_timing_events(ssd_handle* h, void* start, void* stop)
+{
+    g_err.clear();
+    if (!h) return fail(SSD_ERR_INVALID_ARG, "handle is NULL");
+    if ((start == nullptr) != (stop == nullptr))
+        return fail(SSD_ERR_INVALID_ARG, "start and stop must both be set or both be NULL");
+    h->ev_start = (cudaEvent_t)start;
+    h->ev_stop = (cudaEvent_t)stop;
+    return SSD_OK;
+}
+
+uint64_t ssd_launch_count(const ssd_handle* h) { return h ? h->launches : 0; }
+
+ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream)
+{
+    g_err.clear();
+    if (!h) return fail(SSD_ERR_INVALID_ARG, "handle is NULL");
+    SSD_CUDA(cudaStreamSynchronize((cudaStream_t)stream), "cudaStreamSynchronize");
+    int word = 0;
+    SSD_CUDA(cudaMemcpy(&word, h->status, sizeof word, cudaMemcpyDeviceToHost), "status read");
+    if (word == 0) return SSD_OK;
+    SSD_CUDA(cudaMemset(h->status, 0, sizeof word), "status clear");
+    return fail(SSD_ERR_DEVICE, "device status 0x%x:%s%s", word,
+                (word & kStatusTimeout) ? " a bounded wait timed out;" : "",
+                (word & kStatusBadLaunch) ? " a kernel rejected its launch shape;" : "");
+}
+
+}  // extern "C"

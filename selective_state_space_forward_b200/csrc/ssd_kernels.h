@@ -1,0 +1,73 @@
+// ssd_kernels.h -- host-side launch functions of the libssd kernels (internal).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __CUDACC__
+#define SSD_HD __host__ __device__
+#else
+#define SSD_HD
+#endif
+
+namespace ssd {
+
+// Device status word bits (read and cleared by ssd_check).
+constexpr int kStatusTimeout = 1;   // a bounded wait gave up
+constexpr int kStatusBadLaunch = 2; // a kernel saw a launch shape it cannot serve
+
+// Shapes of one call, resolved by the host layer.
+struct Shape {
+    int batch, seqlen, nheads, headdim, dstate, ngroups, dconv;
+    int act_bf16;     // activations are bf16 (else fp32)
+    int a_per_token;  // A is (batch, seqlen, H)
+    int bc_norm;      // B/C RMSNorm + per-head bias
+    SSD_HD int nchunks() const { return (seqlen + 63) / 64; }
+    SSD_HD int conv_dim() const { return nheads * headdim + 2 * ngroups * dstate; }
+};
+
+// Pointers of one forward call (device memory).
+struct FwdArgs {
+    const void *x, *z, *B, *C, *conv_w, *conv_b;
+    const float *dt_raw, *dt_bias, *A, *D;
+    const int32_t* seq_idx;
+    const float* init_ssm;   // (batch, H, P, N) or null
+    const void* init_conv;   // (batch, dconv-1, conv_dim) act or null
+    void* out;
+    float* final_ssm;        // or null
+    void* final_conv;        // or null
+    const float *bn_w, *cn_w, *bn_bias, *cn_bias;  // B/C norm parameters (nullable)
+};
+
+// K1: conv + SiLU of every x|B|C channel into u (batch, seqlen, conv_dim) fp32.
+cudaError_t launch_conv_silu_all(const Shape& s, const FwdArgs& a, float* u, cudaStream_t st);
+// K1 (fused path): conv + SiLU of the B|C channels only, bf16 (batch, seqlen, 2*G*N).
+cudaError_t launch_conv_silu_bc(const Shape& s, const FwdArgs& a, void* ubc, cudaStream_t st);
+// Final conv history (batch, dconv-1, conv_dim) from the raw inputs / initial history.
+cudaError_t launch_conv_state(const Shape& s, const FwdArgs& a, cudaStream_t st);
+// K2: dt = softplus(dt_raw + dt_bias), acs = per-chunk cumsum of dt*a (batch, H, seqlen),
+// and the per-chunk carry factor cdecay (batch, H, nchunks): exp(sum of the chunk's dt*a)
+// when the chunk holds no document boundary, else 0.  cdecay may be null.
+cudaError_t launch_dt_cumsum(const Shape& s, const FwdArgs& a, float* dt, float* acs,
+                             float* cdecay, cudaStream_t st);
+// K3 (staged): chunk states (batch, nchunks, H, P, N) fp32.
+cudaError_t launch_chunk_state(const Shape& s, const FwdArgs& a, const float* u,
+                               const float* dt, const float* acs, float* states, cudaStream_t st);
+// K4: states -> per-chunk entering states, in place; writes final_ssm.
+cudaError_t launch_state_passing(const Shape& s, const FwdArgs& a, const float* cdecay,
+                                 float* states, cudaStream_t st);
+// K5 (staged): chunk outputs with the D skip and SiLU(z) gate.
+cudaError_t launch_chunk_output(const Shape& s, const FwdArgs& a, const float* u,
+                                const float* dt, const float* acs, const float* hin,
+                                cudaStream_t st);
+size_t chunk_output_smem_bytes(const Shape& s);
+size_t chunk_state_smem_bytes(const Shape& s);
+// KF: the fused chunk sweep (one CTA per row and head; state kept on chip).
+bool fused_path_available();
+cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc, const float* dt,
+                               const float* acs, int* status, cudaStream_t st);
+// K6: one decode token per row, state updated in place.
+cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
+                               cudaStream_t st);
+
+}  // namespace ssd

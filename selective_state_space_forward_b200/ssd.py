@@ -1,0 +1,247 @@
+"""ctypes binding of libssd.so (include/ssd.h): argument marshalling only.
+
+Every step of the scan runs in the library's CUDA kernels; this module turns
+torch tensors into device pointers and ssd_* status codes into exceptions.
+It never computes on the host and has no fallback: if libssd.so is missing it
+raises.
+
+    h = Handle(nheads=32, headdim=64, dstate=64, ngroups=8, dconv=4,
+               act_dtype="bf16", max_batch=5, max_seqlen=8192)
+    out = h.forward(x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, seq_idx=seq)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd.so")
+
+SSD_OK = 0
+STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED",
+                3: "SSD_ERR_ALIGNMENT", 4: "SSD_ERR_SHAPE_EXCEEDS_MAX", 5: "SSD_ERR_CUDA",
+                6: "SSD_ERR_DEVICE"}
+PATHS = {"auto": 0, "fused": 1, "staged": 2}
+PATH_NAMES = {1: "fused", 2: "staged"}
+DTYPES = {"f32": (0, torch.float32), "bf16": (1, torch.bfloat16)}
+
+# Every symbol include/ssd.h declares.
+EXPORTS = ("ssd_create", "ssd_destroy", "ssd_get_path", "ssd_set_bc_norm", "ssd_state_bytes",
+           "ssd_state_conv_offset", "ssd_forward", "ssd_step", "ssd_stage_conv", "ssd_stage_dt",
+           "ssd_set_timing_events", "ssd_launch_count", "ssd_check", "ssd_last_error",
+           "ssd_status_string")
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "nheads", "headdim", "dstate", "ngroups", "dconv", "chunk", "act_dtype", "a_mode",
+        "bc_norm", "max_batch", "max_seqlen", "path")]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Open libssd.so and declare its signatures (raises when it was not built)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m selective_state_space_forward_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.ssd_create.argtypes = [ctypes.POINTER(Desc), ctypes.POINTER(vp)]
+    lib.ssd_destroy.argtypes = [vp]
+    lib.ssd_destroy.restype = None
+    lib.ssd_get_path.argtypes = [vp]
+    lib.ssd_get_path.restype = i32
+    lib.ssd_set_bc_norm.argtypes = [vp, vp, vp, vp, vp]
+    lib.ssd_state_bytes.argtypes = [vp, i32]
+    lib.ssd_state_bytes.restype = sz
+    lib.ssd_state_conv_offset.argtypes = [vp, i32]
+    lib.ssd_state_conv_offset.restype = sz
+    lib.ssd_forward.argtypes = [vp, i32, i32] + [vp] * 15 + [vp]
+    lib.ssd_step.argtypes = [vp, i32] + [vp] * 13
+    lib.ssd_stage_conv.argtypes = [vp, i32, i32] + [vp] * 9
+    lib.ssd_stage_dt.argtypes = [vp, i32, i32] + [vp] * 6
+    lib.ssd_set_timing_events.argtypes = [vp, vp, vp]
+    lib.ssd_launch_count.argtypes = [vp]
+    lib.ssd_launch_count.restype = ctypes.c_uint64
+    lib.ssd_check.argtypes = [vp, vp]
+    lib.ssd_last_error.argtypes = []
+    lib.ssd_last_error.restype = ctypes.c_char_p
+    lib.ssd_status_string.argtypes = [ctypes.c_int]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    for f in ("ssd_create", "ssd_set_bc_norm", "ssd_forward", "ssd_step", "ssd_stage_conv",
+              "ssd_stage_dt", "ssd_set_timing_events", "ssd_check"):
+        getattr(lib, f).restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _raise(lib, st: int):
+    if st != SSD_OK:
+        raise SSDError(st, lib.ssd_last_error().decode())
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() and not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise TypeError(f"{name} must be contiguous")
+    return t.data_ptr() or None
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class Handle:
+    """One layer shape: an ssd_handle plus its (library-owned) workspace."""
+
+    def __init__(self, nheads, headdim, dstate, ngroups=1, dconv=4, act_dtype="bf16",
+                 a_per_token=False, bc_norm=False, max_batch=1, max_seqlen=1, path="auto",
+                 lib=None):
+        self.lib = lib or load_library()
+        self.nheads, self.headdim, self.dstate, self.ngroups = nheads, headdim, dstate, ngroups
+        self.dconv, self.act_dtype = dconv, act_dtype
+        self.a_per_token, self.bc_norm = bool(a_per_token), bool(bc_norm)
+        self.torch_dtype = DTYPES[act_dtype][1]
+        d = Desc(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv,
+                 chunk=64, act_dtype=DTYPES[act_dtype][0], a_mode=int(bool(a_per_token)),
+                 bc_norm=int(bool(bc_norm)), max_batch=max_batch, max_seqlen=max_seqlen,
+                 path=PATHS[path])
+        h = ctypes.c_void_p()
+        _raise(self.lib, self.lib.ssd_create(ctypes.byref(d), ctypes.byref(h)))
+        self._h = h
+        self._keep = ()
+        self.path = PATH_NAMES.get(self.lib.ssd_get_path(h), "?")
+
+    @property
+    def conv_dim(self):
+        return self.nheads * self.headdim + 2 * self.ngroups * self.dstate
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self.lib.ssd_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ---- state buffers -------------------------------------------------------------
+    def state_bytes(self, batch: int) -> int:
+        return int(self.lib.ssd_state_bytes(self._h, batch))
+
+    def conv_offset(self, batch: int) -> int:
+        return int(self.lib.ssd_state_conv_offset(self._h, batch))
+
+    def new_state(self, batch: int, device="cuda") -> torch.Tensor:
+        """A zero (fresh) state buffer for `batch` rows, as raw bytes."""
+        return torch.zeros(self.state_bytes(batch), dtype=torch.uint8, device=device)
+
+    def state_views(self, buf: torch.Tensor, batch: int):
+        """(ssm (batch, H, P, N) fp32, conv history (batch, 3, conv_dim) or None) views of buf."""
+        n = batch * self.nheads * self.headdim * self.dstate
+        ssm = buf[:n * 4].view(torch.float32).view(batch, self.nheads, self.headdim, self.dstate)
+        conv = None
+        if self.dconv == 4:
+            off = self.conv_offset(batch)
+            es = 2 if self.act_dtype == "bf16" else 4
+            conv = buf[off:off + batch * 3 * self.conv_dim * es].view(self.torch_dtype).view(
+                batch, 3, self.conv_dim)
+        return ssm, conv
+
+    # ---- calls -----------------------------------------------------------------------
+    def set_bc_norm(self, B_norm_w=None, C_norm_w=None, B_bias=None, C_bias=None):
+        f = torch.float32
+        self._keep = (B_norm_w, C_norm_w, B_bias, C_bias)
+        _raise(self.lib, self.lib.ssd_set_bc_norm(
+            self._h, _ptr(B_norm_w, f, "B_norm_w"), _ptr(C_norm_w, f, "C_norm_w"),
+            _ptr(B_bias, f, "B_bias"), _ptr(C_bias, f, "C_bias")))
+
+    def forward(self, x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None, seq_idx=None,
+                init_state=None, out=None, final_state=None, stream=None):
+        """ssd_forward; returns `out` (allocated like x when not given)."""
+        at, f = self.torch_dtype, torch.float32
+        batch, seqlen = (x.shape[0], x.shape[1]) if x.dim() == 3 else (0, 0)
+        if out is None:
+            out = torch.empty_like(x)
+        _raise(self.lib, self.lib.ssd_forward(
+            self._h, batch, seqlen, _ptr(x, at, "x"), _ptr(z, at, "z"),
+            _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"), _ptr(A, f, "A"),
+            _ptr(B, at, "B"), _ptr(C, at, "C"), _ptr(D, f, "D"), _ptr(conv_w, at, "conv_w"),
+            _ptr(conv_b, at, "conv_b"), _ptr(seq_idx, torch.int32, "seq_idx"),
+            _ptr(init_state, torch.uint8, "init_state"), _ptr(out, at, "out"),
+            _ptr(final_state, torch.uint8, "final_state"), _stream(stream)))
+        return out
+
+    def step(self, x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None, state=None,
+             out=None, stream=None):
+        """ssd_step: one token per row, `state` updated in place; returns `out`."""
+        at, f = self.torch_dtype, torch.float32
+        if out is None:
+            out = torch.empty_like(x)
+        _raise(self.lib, self.lib.ssd_step(
+            self._h, x.shape[0], _ptr(x, at, "x"), _ptr(z, at, "z"), _ptr(dt_raw, f, "dt_raw"),
+            _ptr(dt_bias, f, "dt_bias"), _ptr(A, f, "A"), _ptr(B, at, "B"), _ptr(C, at, "C"),
+            _ptr(D, f, "D"), _ptr(conv_w, at, "conv_w"), _ptr(conv_b, at, "conv_b"),
+            _ptr(state, torch.uint8, "state"), _ptr(out, at, "out"), _stream(stream)))
+        return out
+
+    def stage_conv(self, x, B, C, conv_w, conv_b, seq_idx=None, init_state=None, u=None,
+                   stream=None):
+        at = self.torch_dtype
+        batch, seqlen = x.shape[0], x.shape[1]
+        if u is None:
+            u = torch.empty(batch, seqlen, self.conv_dim, dtype=torch.float32, device=x.device)
+        _raise(self.lib, self.lib.ssd_stage_conv(
+            self._h, batch, seqlen, _ptr(x, at, "x"), _ptr(B, at, "B"), _ptr(C, at, "C"),
+            _ptr(conv_w, at, "conv_w"), _ptr(conv_b, at, "conv_b"),
+            _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(init_state, torch.uint8, "init_state"),
+            _ptr(u, torch.float32, "u"), _stream(stream)))
+        return u
+
+    def stage_dt(self, dt_raw, dt_bias, A, stream=None):
+        f = torch.float32
+        batch, seqlen = dt_raw.shape[0], dt_raw.shape[1]
+        dt = torch.empty(batch, self.nheads, seqlen, dtype=f, device=dt_raw.device)
+        acs = torch.empty_like(dt)
+        _raise(self.lib, self.lib.ssd_stage_dt(
+            self._h, batch, seqlen, _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"),
+            _ptr(A, f, "A"), _ptr(dt, f, "dt"), _ptr(acs, f, "acs"), _stream(stream)))
+        return dt, acs
+
+    def set_timing_events(self, start=None, stop=None):
+        """Bracket the main kernel of later calls with these torch.cuda.Events."""
+        _raise(self.lib, self.lib.ssd_set_timing_events(
+            self._h, start.cuda_event if start is not None else None,
+            stop.cuda_event if stop is not None else None))
+
+    def launch_count(self) -> int:
+        return int(self.lib.ssd_launch_count(self._h))
+
+    def check(self, stream=None):
+        _raise(self.lib, self.lib.ssd_check(self._h, _stream(stream)))
