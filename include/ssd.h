@@ -163,15 +163,16 @@ ssd_status ssd_step(ssd_handle* h, int32_t batch,
  *                    (the first stage; init_state as in ssd_forward).
  *   ssd_stage_dt   : dt (batch, H, seqlen) fp32 = softplus(dt_raw + dt_bias) and
  *                    acs (batch, H, seqlen) fp32 = cumulative sum of dt*a restarted
- *                    at every chunk start (64 tokens).
+ *                    at every chunk start (64 tokens) and at every document
+ *                    boundary of seq_idx (NULL = none).
  */
 ssd_status ssd_stage_conv(ssd_handle* h, int32_t batch, int32_t seqlen, const void* x,
                           const void* B, const void* C, const void* conv_w, const void* conv_b,
                           const int32_t* seq_idx, const void* init_state, float* u,
                           struct CUstream_st* stream);
 ssd_status ssd_stage_dt(ssd_handle* h, int32_t batch, int32_t seqlen, const float* dt_raw,
-                        const float* dt_bias, const float* A, float* dt, float* acs,
-                        struct CUstream_st* stream);
+                        const float* dt_bias, const float* A, const int32_t* seq_idx, float* dt,
+                        float* acs, struct CUstream_st* stream);
 
 /* Measurement hook.  When start and stop are cudaEvent_t handles (created by
  * the caller), every later ssd_forward / ssd_step records `start` on its

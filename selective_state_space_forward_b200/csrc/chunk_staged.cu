@@ -3,13 +3,15 @@
 //
 // The chunked evaluation of the selective scan (chunk 64; mojolearn
 // Mamba3Block, "chunk size 64"): within a chunk c of tokens t0 .. t0+Lc-1,
-// with acs_t the chunk-local inclusive sum of dt*a and seg_t the number of
-// document boundaries at positions t0 .. t (a boundary at t0 means the token
-// before the chunk belongs to another document):
+// with acs_t the inclusive sum of dt*a from the start of t's segment (the
+// chunk start or the last document boundary) and seg_t the number of document
+// boundaries at positions t0 .. t (a boundary at t0 means the token before the
+// chunk belongs to another document):
 //
 //   chunk state    S_c[p,n]  = sum_{s: seg_s = seg_last} exp(acs_last - acs_s) dt_s x_s[p] B_s[n]
 //   state passing  Hin_0     = initial state;  Hin_{c+1} = k_c Hin_c + S_c,
-//                  k_c = exp(acs_last) if the chunk holds no boundary, else 0
+//                  k_c = exp(acs_last) if the chunk holds no boundary, else Hin_c is
+//                  dropped (Hin_{c+1} = S_c)
 //   chunk output   y_t[p]    = sum_{s<=t, seg_s = seg_t} (C_t . B_s) exp(acs_t - acs_s) dt_s x_s[p]
 //                            + [seg_t = 0] exp(acs_t) C_t . Hin_c[p, :]  +  D x_t[p]
 //                  out_t     = y_t * SiLU(z_t)
@@ -146,7 +148,8 @@ state_passing_kernel(Shape s, const float* __restrict__ cdecay, float* __restric
         float* sp = states + (((int64_t)b * nc + c) * H + h) * PN + e;
         const float sc = *sp;
         *sp = hv;
-        hv = kd[c] * hv + sc;
+        const float k = kd[c];
+        hv = (k == kChunkReset) ? sc : k * hv + sc;   // select: a reset drops hv exactly
     }
     if (fin) fin[gid] = hv;
 }

@@ -1,30 +1,43 @@
 // dt_cumsum.cu -- K2: dt = softplus(dt_raw + dt_bias), dA = dt * a, and the
-// per-chunk (64-token) inclusive cumulative sum of dA.
+// per-chunk (64-token) segmented inclusive cumulative sum of dA.
 //
 // softplus(dt + bias) per head: falcon_mamba.ts header; no dt clamp:
 // mojolearn Mamba3Block.  a = A[h] (A = -exp(A_log), codestral_mamba.ts
 // reconciliation 2), or per token min(A[b,t,h], -1e-4) (Mamba3Block, "A floor
-// 1e-4").  The per-chunk carry factor is exp(sum of the chunk's dA) when no
-// document boundary (model card, "Checkpoint and training") falls inside the
+// 1e-4").
+//
+// The sum restarts at the chunk start and at every packed-document boundary
+// inside the chunk (model card, "Checkpoint and training": state flow resets
+// at every boundary), so acs_t - acs_s for two tokens of one document sums
+// only that document's dA -- a changed document elsewhere in the row cannot
+// even change the rounding of another document's decays.  The per-chunk carry
+// factor is exp(acs of the chunk's last token) when no boundary falls in the
 // chunk -- including one between the chunk's first token and the previous
-// chunk's last -- and 0 otherwise: the state entering such a chunk does not
-// reach its end.
+// chunk's last -- and the reset marker -1 otherwise: the state entering such
+// a chunk does not reach its end.
 //
 // One warp per (row, head, chunk): lane l owns tokens l and l+32 of the chunk;
-// two shuffle scans give the inclusive sums.  Warps are ordered head-fastest,
-// so the warps of one block read neighbouring dt_raw words of the same token
-// rows (dt_raw is (batch, seqlen, H)).
+// two segmented shuffle scans give the inclusive sums.  Warps are ordered
+// head-fastest, so the warps of one block read neighbouring dt_raw words of
+// the same token rows (dt_raw is (batch, seqlen, H)).
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
 
 namespace ssd {
 
-__device__ __forceinline__ float warp_incl_scan(float v, int lane)
+// Segmented inclusive scan across the warp: a lane with start = 1 begins a
+// new segment.  Returns the sum from the lane's segment start to the lane;
+// `start` becomes 1 when a segment start lies at or before the lane.
+__device__ __forceinline__ float warp_seg_scan(float v, int& start, int lane)
 {
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += n;
+        const float nv = __shfl_up_sync(0xffffffffu, v, o);
+        const int nf = __shfl_up_sync(0xffffffffu, start, o);
+        if (lane >= o) {
+            if (!start) v = nv + v;
+            start |= nf;
+        }
     }
     return v;
 }
@@ -45,24 +58,30 @@ dt_cumsum_kernel(Shape s, const float* __restrict__ dt_raw, const float* __restr
     const float bias = dt_bias[h];
     const float a_head = s.a_per_token ? 0.0f : A[h];
 
+    const int32_t* seq_row = seq ? seq + (int64_t)b * L : nullptr;
     float dtv[2], dA[2];
-    int bd = 0;
+    int bd[2];
 #pragma unroll
     for (int half = 0; half < 2; half++) {
         const int t = t0 + half * 32 + lane;
         dtv[half] = 0.0f;
         dA[half] = 0.0f;
+        bd[half] = 0;
         if (t < L) {
             const int64_t i = ((int64_t)b * L + t) * H + h;
             dtv[half] = softplus_f(dt_raw[i] + bias);
             const float av = s.a_per_token ? fminf(A[i], -kAFloor) : a_head;
             dA[half] = dtv[half] * av;
-            bd |= is_boundary(seq ? seq + (int64_t)b * L : nullptr, t);
+            bd[half] = is_boundary(seq_row, t);
         }
     }
-    const float s0 = warp_incl_scan(dA[0], lane);
-    const float tot0 = __shfl_sync(0xffffffffu, s0, 31);
-    const float s1 = warp_incl_scan(dA[1], lane) + tot0;
+    const int any_bd = __any_sync(0xffffffffu, bd[0] | bd[1]);
+    int f0 = bd[0] | (lane == 0);   // the chunk start opens a segment
+    int f1 = bd[1];
+    const float s0 = warp_seg_scan(dA[0], f0, lane);
+    float s1 = warp_seg_scan(dA[1], f1, lane);
+    const float tail0 = __shfl_sync(0xffffffffu, s0, 31);
+    if (!f1) s1 = tail0 + s1;       // no segment start in tokens 32 .. lane+32
 
     const int64_t row = ((int64_t)b * H + h) * L;
     if (t0 + lane < L) {
@@ -74,10 +93,9 @@ dt_cumsum_kernel(Shape s, const float* __restrict__ dt_raw, const float* __restr
         acs_out[row + t0 + 32 + lane] = s1;
     }
     if (cdecay != nullptr) {
-        const int any_bd = __any_sync(0xffffffffu, bd);
         const int last = (L - t0 < kChunk ? L - t0 : kChunk) - 1;   // chunk-local index
         const float acs_last = __shfl_sync(0xffffffffu, last < 32 ? s0 : s1, last & 31);
-        if (lane == 0) cdecay[((int64_t)b * H + h) * nc + c] = any_bd ? 0.0f : expf(acs_last);
+        if (lane == 0) cdecay[((int64_t)b * H + h) * nc + c] = any_bd ? kChunkReset : expf(acs_last);
     }
 }
 

@@ -436,8 +436,8 @@ ssd_status ssd_stage_conv(ssd_handle* h, int32_t batch, int32_t seqlen, const vo
 }
 
 ssd_status ssd_stage_dt(ssd_handle* h, int32_t batch, int32_t seqlen, const float* dt_raw,
-                        const float* dt_bias, const float* A, float* dt, float* acs,
-                        struct CUstream_st* stream)
+                        const float* dt_bias, const float* A, const int32_t* seq_idx, float* dt,
+                        float* acs, struct CUstream_st* stream)
 {
     g_err.clear();
     SSD_TRY(check_handle_dims(h, batch, seqlen));
@@ -445,12 +445,13 @@ ssd_status ssd_stage_dt(ssd_handle* h, int32_t batch, int32_t seqlen, const floa
     SSD_TRY(check_ptr(dt_raw, "dt_raw", 4, true));
     SSD_TRY(check_ptr(dt_bias, "dt_bias", 4, true));
     SSD_TRY(check_ptr(A, "A", 4, true));
+    SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
     SSD_TRY(check_ptr(dt, "dt", 4, true));
     SSD_TRY(check_ptr(acs, "acs", 4, true));
     const Shape s = make_shape(h, batch, seqlen);
     FwdArgs a;
     memset(&a, 0, sizeof a);
-    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A;
+    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.seq_idx = seq_idx;
     SSD_LAUNCH(h, launch_dt_cumsum(s, a, dt, acs, nullptr, (cudaStream_t)stream),
                "dt/cumsum kernel");
     return SSD_OK;

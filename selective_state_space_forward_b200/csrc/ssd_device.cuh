@@ -12,6 +12,7 @@ constexpr int kChunk = 64;        // chunk length of the chunked scan
 constexpr int kConvK = 4;         // causal conv kernel width when the conv is on
 constexpr float kAFloor = 1e-4f;  // per-token |A| floor (Mamba3Block "A floor 1e-4")
 constexpr float kNormEps = 1e-5f; // B/C RMSNorm epsilon (Mamba3Block Parameters)
+constexpr float kChunkReset = -1.0f;  // carry factor of a chunk holding a document boundary
 
 __device__ __forceinline__ float to_f(float v) { return v; }
 __device__ __forceinline__ float to_f(bf16 v) { return __bfloat162float(v); }

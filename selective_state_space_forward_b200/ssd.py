@@ -69,10 +69,10 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_state_bytes.restype = sz
     lib.ssd_state_conv_offset.argtypes = [vp, i32]
     lib.ssd_state_conv_offset.restype = sz
-    lib.ssd_forward.argtypes = [vp, i32, i32] + [vp] * 15 + [vp]
+    lib.ssd_forward.argtypes = [vp, i32, i32] + [vp] * 14 + [vp]
     lib.ssd_step.argtypes = [vp, i32] + [vp] * 13
     lib.ssd_stage_conv.argtypes = [vp, i32, i32] + [vp] * 9
-    lib.ssd_stage_dt.argtypes = [vp, i32, i32] + [vp] * 6
+    lib.ssd_stage_dt.argtypes = [vp, i32, i32] + [vp] * 7
     lib.ssd_set_timing_events.argtypes = [vp, vp, vp]
     lib.ssd_launch_count.argtypes = [vp]
     lib.ssd_launch_count.restype = ctypes.c_uint64
@@ -224,14 +224,15 @@ class Handle:
             _ptr(u, torch.float32, "u"), _stream(stream)))
         return u
 
-    def stage_dt(self, dt_raw, dt_bias, A, stream=None):
+    def stage_dt(self, dt_raw, dt_bias, A, seq_idx=None, stream=None):
         f = torch.float32
         batch, seqlen = dt_raw.shape[0], dt_raw.shape[1]
         dt = torch.empty(batch, self.nheads, seqlen, dtype=f, device=dt_raw.device)
         acs = torch.empty_like(dt)
         _raise(self.lib, self.lib.ssd_stage_dt(
             self._h, batch, seqlen, _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"),
-            _ptr(A, f, "A"), _ptr(dt, f, "dt"), _ptr(acs, f, "acs"), _stream(stream)))
+            _ptr(A, f, "A"), _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(dt, f, "dt"),
+            _ptr(acs, f, "acs"), _stream(stream)))
         return dt, acs
 
     def set_timing_events(self, start=None, stop=None):

@@ -35,6 +35,24 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def _declared_param_counts():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(ssd_[a-z_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    counts = _declared_param_counts()
+    assert sorted(counts) == sorted(ssd.EXPORTS)
+    for name, n in counts.items():
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None and len(argtypes) == n, (name, n, argtypes)
+
+
 def test_status_strings(lib):
     for code, name in ssd.STATUS_NAMES.items():
         assert lib.ssd_status_string(code).decode() == name
@@ -73,9 +91,10 @@ def test_bad_descriptor_is_refused_by_name(lib, kw, status, word):
 
 
 def test_null_handle_is_refused(lib):
-    st = lib.ssd_forward(None, 1, 1, *([None] * 16))
+    st = lib.ssd_forward(None, 1, 1, *([None] * 15))
     assert st == 1 and "handle" in lib.ssd_last_error().decode()
     st = lib.ssd_step(None, 1, *([None] * 13))
+    assert st == 1
     assert st == 1
     assert lib.ssd_check(None, None) == 1
     assert lib.ssd_get_path(None) == -1

@@ -141,21 +141,28 @@ def test_stage_conv_matches_oracle():
 
 
 def test_stage_dt_matches_oracle():
+    """dt and the segmented per-chunk cumsum: the sum of dt*a restarts at each
+    chunk start and each document boundary (from the oracle's dt and a)."""
     w = _small("mamba3_siso", batch=2, seqlen=200)
     inp = make_inputs(w)
     inp["A"][0, 3:7, 5] = np.array([0.0, -1e-6, -1e-4, -2.0], dtype=np.float32)
+    seq = np.stack([_docs_row(200, [1, 30, 64, 65, 100, 199]), _docs_row(200, [])])
     dt_ref, a_ref = oracle.dt_stage(w.dims(), inp)
     h = make_handle(w, "staged")
     dev = to_device(inp, w)
-    dt, acs = h.stage_dt(dev["dt_raw"], dev["dt_bias"], dev["A"])
+    dt, acs = h.stage_dt(dev["dt_raw"], dev["dt_bias"], dev["A"],
+                         seq_idx=torch.from_numpy(seq).cuda())
     dt = dt.double().cpu().numpy()
     acs = acs.double().cpu().numpy()
     assert np.allclose(dt, dt_ref.transpose(0, 2, 1), rtol=2e-6, atol=1e-30)
     da = (dt_ref * a_ref).transpose(0, 2, 1)
-    for c0 in range(0, w.seqlen, 64):
-        ref = np.cumsum(da[:, :, c0:c0 + 64], axis=2)
-        got = acs[:, :, c0:c0 + 64]
-        assert np.allclose(got, ref, rtol=1e-5, atol=1e-5 * np.max(np.abs(ref)))
+    ref = np.empty_like(da)
+    for b in range(2):
+        for t in range(w.seqlen):
+            start = t % 64 == 0 or seq[b, t] != seq[b, t - 1]
+            ref[b, :, t] = da[b, :, t] if start else ref[b, :, t - 1] + da[b, :, t]
+    scale = np.max(np.abs(ref))
+    assert np.allclose(acs, ref, rtol=1e-5, atol=1e-6 * scale)
 
 
 @pytest.mark.parametrize("path", PATHS)
