@@ -91,7 +91,7 @@ size_t conv_offset(const ssd_desc& d, int batch)
 bool fused_supported(const ssd_desc& d)
 {
     return fused_path_available() && d.act_dtype == SSD_DTYPE_BF16 && d.headdim == 64 &&
-           (d.dstate == 64 || d.dstate == 128);
+           (d.dstate == 64 || d.dstate == 128) && !d.bc_norm;
 }
 
 ssd_status validate_desc(const ssd_desc* d)
@@ -123,7 +123,8 @@ ssd_status validate_desc(const ssd_desc* d)
         return fail(SSD_ERR_INVALID_ARG, "path %d is not an ssd_path", d->path);
     if (d->path == SSD_PATH_FUSED && !fused_supported(*d))
         return fail(SSD_ERR_UNSUPPORTED,
-                    "the fused path needs bf16 activations, headdim 64 and dstate 64 or 128");
+                    "the fused path needs bf16 activations, headdim 64, dstate 64 or 128 and "
+                    "no B/C norm");
     return SSD_OK;
 }
 

@@ -96,6 +96,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Teardown wait: like mbar_wait but it does not stop at the abort flag, so an
+// aborting CTA still lets its own copies and MMAs land before it exits.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* status, int status_bit)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; i++) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255) == 0 && global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(status, status_bit);
+            return false;
+        }
+    }
+}
+
 // ---- proxy fences -------------------------------------------------------------------
 // Generic-proxy shared-memory writes become visible to the async proxy (TMA
 // store, tensor core operand reads) after this fence plus a barrier.
