@@ -13,21 +13,23 @@
 //   mask      M[t,s] = S[t,s] exp(acs_t - acs_s)  [s <= t, seg_s = seg_t]
 //   Ydiag     M Xd                           tcgen05, 64 x 64 x 64
 //   Yoff      C h_c^T                        tcgen05, 64 x 64 x N (bf16 copy of h_c)
-//   state     h_{c+1} = k_c h_c + B^T Xs     tcgen05, accumulates in TMEM
-//             (k_c = exp(acs_last), or 0 when the chunk holds a boundary)
+//   chunk     S_c = B^T Xs                   tcgen05, N x 64 x 64
+//   state     h_{c+1} = k_c h_c + S_c        fp32, in registers
+//             (k_c = exp(acs_last), dropped when the chunk holds a boundary)
 //   epilogue  out_t = (Ydiag_t + [seg_t = 0] exp(acs_t) Yoff_t + D u_t) SiLU(z_t)
 //
-// The chunk-state contraction accumulates onto k_c h_c inside the tensor
-// memory, so the fp32 state is carried on chip from the initial state to the
-// final one; only a bf16 copy of it is staged in shared memory as the Yoff
-// operand.  The gate, the D skip and the output cast are fused in the
-// epilogue (spec kernel list items 3-5).
+// The fp32 state is carried in the compute threads' registers from the
+// initial state to the final one; a bf16 copy of it is staged in shared
+// memory each chunk as the Yoff operand.  The gate, the D skip and the output
+// cast are fused in the epilogue.
 //
-// Roles (192 threads): warps 0-3 compute (conv, state hand-off, masks,
-// epilogue; each warp reaches TMEM lanes 32w .. 32w+31), warp 4 produces (TMA
-// tile loads into a 2-stage ring, dt/acs/boundary flags), warp 5 issues the
-// MMAs from one thread.  Every wait is bounded: after 1 s a waiter raises the
-// CTA's abort flag and the device status word, and all roles drain and exit.
+// Roles (320 threads): warps 0-7 compute (state update, conv, masks,
+// epilogue; warp w reaches TMEM lanes 32*(w%4) .. +31 and takes the column
+// half w/4), warp 8 produces (TMA tile loads into a 2-stage ring plus the
+// chunk's per-token scalars: dt, decay weights, segment ids, carry), warp 9
+// issues the MMAs from one thread.  Every wait is bounded: after 1 s a waiter
+// raises the CTA's abort flag and the device status word, and all roles
+// drain and exit.
 //
 // Tile layouts (see tc05.cuh): x, z, B, C, out tiles are [64 tokens][64
 // channels] bf16 with the 128-byte swizzle, as TMA writes them; N = 128
@@ -42,14 +44,18 @@
 namespace ssd {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kComputeThreads = 128;
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = 32 * kComputeWarps;
+constexpr int kProducerWarp = kComputeWarps;
+constexpr int kMmaWarp = kComputeWarps + 1;
+constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr int kTile = 64 * 128;        // one [64][64] bf16 tile
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColCB = 0, kColY = 64, kColYO = 128, kColST = 192;
+constexpr uint32_t kColCB = 0, kColY = 64, kColYO = 128, kColS = 192;
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct FusedParams {
-    int batch, seqlen, nheads, ngroups, conv;
+    int batch, seqlen, nheads, ngroups;
     const float* dt;          // (B, H, L) from K2
     const float* acs;         // (B, H, L) segmented cumsum from K2
     const int32_t* seq;       // (B, L) or null
@@ -62,62 +68,84 @@ struct FusedParams {
     int* status;
 };
 
+// Per-token values of one chunk, written by the producer warp.
+struct ChunkScalars {
+    float dt[64];      // dt_t (0 past the end of the sequence)
+    float wd[64];      // [seg_t = seg_last] exp(acs_last - acs_t) dt_t
+    float f[64];       // [seg_t = 0] exp(acs_t): weight of the carried-state term
+    float a2[64];      // acs_t * log2(e)
+    uint8_t seg[64];   // document boundaries at chunk positions 0 .. t
+    float carry;       // exp(acs_last), or kChunkReset when the chunk holds a boundary
+    uint32_t m0, m1;   // boundary at chunk position r (bit r of m0 | m1 << 32)
+    uint32_t pre;      // bit 0: boundary at t0-2, bit 1: at t0-1
+    uint32_t pad[4];
+};
+
 template <int NS>
 struct Layout {
     static constexpr int kBC = (NS / 64) * kTile;
     static constexpr int kStage = 2 * kTile + 2 * kBC;        // x, z, B, C
     static constexpr int kRing = 2 * kStage;
-    static constexpr int kMop = kRing;                        // mask operand / out tile
+    static constexpr int kMop = kRing;                        // mask operand, then the out tile
     static constexpr int kXd = kMop + kTile;
     static constexpr int kXs = kXd + kTile;
-    static constexpr int kXb = kXs + kTile;
+    static constexpr int kXb = kXs + kTile;                   // u in bf16, [t][p]
     static constexpr int kHt = kXb + kTile;                   // h^T, NS rows x 128 B
-    static constexpr int kSmall = kHt + NS * 128;
-    // small region
-    static constexpr int kDt = kSmall;                        // [2][64] f32
-    static constexpr int kAcs = kDt + 2 * 64 * 4;             // [2][64] f32
-    static constexpr int kBd = kAcs + 2 * 64 * 4;             // [2][4] u32: mask lo, mask hi, pre, pad
-    static constexpr int kHalo = kBd + 2 * 16;                // [2][3][64] bf16
-    static constexpr int kBar = kHalo + 2 * 3 * 64 * 2;       // 7 mbarriers
+    static constexpr int kScal = kHt + NS * 128;              // ChunkScalars[2]
+    static constexpr int kHalo = kScal + 2 * (int)sizeof(ChunkScalars);   // u32 [2][3][32]
+    static constexpr int kBar = kHalo + 2 * 3 * 32 * 4;       // 8 mbarriers
     static constexpr int kMisc = kBar + 8 * 8;                // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
 };
 
-__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void bar_compute()
+{
+    asm volatile("bar.sync 1, %0;" ::"n"(kComputeThreads) : "memory");
+}
 
-// Compute-warp barrier that also returns the OR of v over the 128 threads, so
-// every thread takes the same branch afterwards.
+// Compute-warp barrier that also returns the OR of v over the compute
+// threads, so every one of them takes the same branch afterwards.
 __device__ __forceinline__ int bar_compute_or(int v)
 {
     uint32_t r;
     asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(v)
+        : "r"(v), "n"(kComputeThreads)
         : "memory");
     return (int)r;
 }
 
 __device__ __forceinline__ uint32_t mask_le(int i) { return i >= 31 ? 0xffffffffu : ((2u << i) - 1u); }
 
-// Number of document boundaries at chunk positions 0 .. t.
-__device__ __forceinline__ int seg_of(uint32_t m0, uint32_t m1, int t)
-{
-    return t < 32 ? __popc(m0 & mask_le(t)) : __popc(m0) + __popc(m1 & mask_le(t - 32));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
     const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&v);
 }
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ float fast_silu(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
+// 2^x, hardware approximation (PTX ex2.approx).
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// SiLU(v) = v * (1 + tanh(v/2)) / 2, one hardware tanh (PTX tanh.approx).
+__device__ __forceinline__ float silu_t(float v)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
+    return v * fmaf(0.5f, t, 0.5f);
+}
 
 template <int NS, bool CONV>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, NS == 64 ? 2 : 1)
 ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
                 const __grid_constant__ CUtensorMap tm_out, FusedParams p)
@@ -125,16 +153,15 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     using LY = Layout<NS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float* s_dt = (float*)(sm + LY::kDt);
-    float* s_acs = (float*)(sm + LY::kAcs);
-    uint32_t* s_bd = (uint32_t*)(sm + LY::kBd);
-    bf16* s_halo = (bf16*)(sm + LY::kHalo);
+    ChunkScalars* scal = (ChunkScalars*)(sm + LY::kScal);
+    uint32_t* s_halo = (uint32_t*)(sm + LY::kHalo);
     uint64_t* bar = (uint64_t*)(sm + LY::kBar);
     uint64_t* full = bar;           // [2]
     uint64_t* empty = bar + 2;      // [2]
     uint64_t* cb_done = bar + 4;
     uint64_t* ops_ready = bar + 5;
     uint64_t* mma_done = bar + 6;
+    uint64_t* drain = bar + 7;
     uint32_t* s_tmem = (uint32_t*)(sm + LY::kMisc);
     volatile int* s_abort = (volatile int*)(sm + LY::kMisc + 4);
 
@@ -153,7 +180,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         tc::mbar_init(cb_done, 1);
         tc::mbar_init(ops_ready, kComputeThreads);
         tc::mbar_init(mma_done, 1);
-        tc::mbar_init(&bar[7], 1);           // teardown drain of the MMA pipe
+        tc::mbar_init(drain, 1);
         *s_abort = 0;
         tc::fence_mbar_init();
     }
@@ -161,7 +188,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         tc::tmem_alloc(s_tmem, kTmemCols);
         tc::tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kProducerWarp && lane == 0) {
         tc::tma_prefetch_desc(&tm_x);
         tc::tma_prefetch_desc(&tm_z);
         tc::tma_prefetch_desc(&tm_b);
@@ -173,7 +200,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     tc::tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
         const int32_t* seq_row = p.seq ? p.seq + (int64_t)b * L : nullptr;
         const float* dt_row = p.dt + bh * L;
@@ -192,32 +219,50 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 tc::tma_load_3d(st + kTile, &tm_z, &full[s], h * 64, t0, b);
 #pragma unroll
                 for (int j = 0; j < NS / 64; j++) {
-                    const int bx = CONV ? g * NS + 64 * j : g * NS + 64 * j;
-                    const int cx = CONV ? p.ngroups * NS + g * NS + 64 * j : g * NS + 64 * j;
+                    const int bx = g * NS + 64 * j;
+                    const int cx = (CONV ? p.ngroups * NS : 0) + g * NS + 64 * j;
                     tc::tma_load_3d(st + 2 * kTile + j * kTile, &tm_b, &full[s], bx, t0, b);
                     tc::tma_load_3d(st + 2 * kTile + LY::kBC + j * kTile, &tm_c, &full[s], cx, t0, b);
                 }
             }
-            float* dts = s_dt + s * 64;
-            float* acv = s_acs + s * 64;
+            ChunkScalars* cs = &scal[s];
+            const int Lc = min(64, L - t0);
+            float dtv[2], acv[2];
             int bdv[2];
 #pragma unroll
-            for (int half = 0; half < 2; half++) {
-                const int t = t0 + half * 32 + lane;
+            for (int hf = 0; hf < 2; hf++) {
+                const int t = t0 + hf * 32 + lane;
                 const bool ok = t < L;
-                dts[half * 32 + lane] = ok ? dt_row[t] : 0.0f;
-                acv[half * 32 + lane] = ok ? acs_row[t] : 0.0f;
-                bdv[half] = ok ? is_boundary(seq_row, t) : 0;
+                dtv[hf] = ok ? dt_row[t] : 0.0f;
+                acv[hf] = ok ? acs_row[t] : 0.0f;
+                bdv[hf] = ok ? is_boundary(seq_row, t) : 0;
             }
             const uint32_t m0 = __ballot_sync(0xffffffffu, bdv[0]);
             const uint32_t m1 = __ballot_sync(0xffffffffu, bdv[1]);
+            const int seg0 = __popc(m0 & mask_le(lane));
+            const int seg1 = __popc(m0) + __popc(m1 & mask_le(lane));
+            const int last = Lc - 1;
+            const int seg_last = __shfl_sync(0xffffffffu, last < 32 ? seg0 : seg1, last & 31);
+            const float acs_last = __shfl_sync(0xffffffffu, last < 32 ? acv[0] : acv[1], last & 31);
+            const int segv[2] = {seg0, seg1};
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+                const int r = hf * 32 + lane;
+                const bool ok = r < Lc;
+                cs->dt[r] = dtv[hf];
+                cs->wd[r] = (ok && segv[hf] == seg_last) ? __expf(acs_last - acv[hf]) * dtv[hf] : 0.0f;
+                cs->f[r] = (ok && segv[hf] == 0) ? __expf(acv[hf]) : 0.0f;
+                cs->a2[r] = acv[hf] * kLog2e;
+                cs->seg[r] = (uint8_t)segv[hf];
+            }
             if (lane == 0) {
                 uint32_t pre = 0;
                 if (t0 - 2 >= 1 && is_boundary(seq_row, t0 - 2)) pre |= 1u;
                 if (t0 - 1 >= 1 && is_boundary(seq_row, t0 - 1)) pre |= 2u;
-                s_bd[s * 4 + 0] = m0;
-                s_bd[s * 4 + 1] = m1;
-                s_bd[s * 4 + 2] = pre;
+                cs->carry = (m0 | m1) ? kChunkReset : __expf(acs_last);
+                cs->m0 = m0;
+                cs->m1 = m1;
+                cs->pre = pre;
             }
             __syncwarp();
             tc::mbar_arrive(&full[s]);
@@ -226,10 +271,10 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // an aborting CTA lets its last loads land before the shared memory is released
         for (int k = max(0, issued - 2); k < issued; k++)
             tc::mbar_drain(&full[k & 1], (k >> 1) & 1, p.status, kStatusTimeout);
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
         if (lane == 0) {
-            const uint32_t id_cb = tc::idesc_bf16(64, 64, false, false);
+            const uint32_t id_64 = tc::idesc_bf16(64, 64, false, false);
             const uint32_t id_yo = tc::idesc_bf16(64, 64, false, true);
             const uint32_t id_st = tc::idesc_bf16(NS, 64, true, false);
             const uint32_t a_mop = tc::smem_u32(sm + LY::kMop);
@@ -242,12 +287,12 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 tc::tc_fence_after();
                 const uint32_t a_b = tc::smem_u32(sm + s * LY::kStage + 2 * kTile);
                 const uint32_t a_c = a_b + LY::kBC;
-                // CB = C B^T: both K-major over n
+                // C B^T: both K-major over n
 #pragma unroll
                 for (int kk = 0; kk < NS / 16; kk++) {
                     const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
                     tc::mma_bf16(tmem + kColCB, tc::sdesc_sw128(a_c + off, 16, 1024),
-                                 tc::sdesc_sw128(a_b + off, 16, 1024), id_cb, kk > 0);
+                                 tc::sdesc_sw128(a_b + off, 16, 1024), id_64, kk > 0);
                 }
                 tc::mma_commit(cb_done);
                 if (!tc::mbar_wait(ops_ready, c & 1, s_abort, p.status, kStatusTimeout)) break;
@@ -256,7 +301,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                 for (int kk = 0; kk < 4; kk++)
                     tc::mma_bf16(tmem + kColY, tc::sdesc_sw128(a_mop + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(a_xd + kk * 32, 16, 1024), id_cb, kk > 0);
+                                 tc::sdesc_sw128(a_xd + kk * 32, 16, 1024), id_64, kk > 0);
                 // Yoff = C h^T (K = n; h^T is MN-major: rows n, 64 p per row)
 #pragma unroll
                 for (int kk = 0; kk < NS / 16; kk++) {
@@ -264,193 +309,164 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     tc::mma_bf16(tmem + kColYO, tc::sdesc_sw128(a_c + off, 16, 1024),
                                  tc::sdesc_sw128(a_ht + kk * 2048, 8192, 1024), id_yo, kk > 0);
                 }
-                // state^T[n][p] += B^T Xs (A = B tile as MN-major over n, K = s)
+                // S_c^T[n][p] = B^T Xs (A = the B tile as MN-major over n, K = s)
 #pragma unroll
                 for (int kk = 0; kk < 4; kk++)
-                    tc::mma_bf16(tmem + kColST, tc::sdesc_sw128(a_b + kk * 2048, kTile, 1024),
-                                 tc::sdesc_sw128(a_xs + kk * 32, 16, 1024), id_st, 1);
+                    tc::mma_bf16(tmem + kColS, tc::sdesc_sw128(a_b + kk * 2048, kTile, 1024),
+                                 tc::sdesc_sw128(a_xs + kk * 32, 16, 1024), id_st, kk > 0);
                 tc::mma_commit(mma_done);
             }
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ compute warps 0-3
+        // ------------------------------------------------------------ compute warps 0-7
         const int HP = H * 64;
         const int cdim = HP + 2 * p.ngroups * NS;
-        const int pch = tid & 63;            // conv channel
-        const int tgb = tid >> 6;            // token-group parity for the conv
-        float wk[4] = {0.f, 0.f, 0.f, 1.f}, cbias = 0.f;
+        const int sub = warp & 3;                  // TMEM lane quarter
+        const int half = warp >> 2;                // column half
+        const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
+        // M=64 accumulators: row r16, this thread's 16 columns start at c16
+        const int r16 = 16 * sub + (lane & 15);
+        const int c16 = half * 16 + (lane < 16 ? 0 : 32);
+        // conv: channel pair pp, tokens 8*warp .. 8*warp+7
+        const int pp = lane;
+        const int r0 = 8 * warp;
+        float wk[2][4] = {{0.f, 0.f, 0.f, 1.f}, {0.f, 0.f, 0.f, 1.f}}, cbias[2] = {0.f, 0.f};
         if (CONV) {
-            const int ch = h * 64 + pch;
 #pragma unroll
-            for (int k = 0; k < 4; k++) wk[k] = __bfloat162float(p.conv_w[(int64_t)ch * 4 + k]);
-            cbias = __bfloat162float(p.conv_b[ch]);
-            // halo for chunk 0: the caller's conv history of this channel (zeros when none)
-            if (tid < 64) {
+            for (int e = 0; e < 2; e++) {
+                const int ch = h * 64 + 2 * pp + e;
 #pragma unroll
-                for (int j = 0; j < 3; j++)
-                    s_halo[j * 64 + pch] = p.init_conv
-                        ? p.init_conv[((int64_t)b * 3 + j) * cdim + h * 64 + pch]
-                        : __float2bfloat16(0.0f);
+                for (int k = 0; k < 4; k++) wk[e][k] = __bfloat162float(p.conv_w[(int64_t)ch * 4 + k]);
+                cbias[e] = __bfloat162float(p.conv_b[ch]);
+            }
+            // halo for chunk 0: the caller's conv history of these channels (zeros when none)
+            if (tid < 96) {
+                const int j = tid >> 5;
+                s_halo[j * 32 + pp] = p.init_conv
+                    ? *(const uint32_t*)(p.init_conv + ((int64_t)b * 3 + j) * cdim + h * 64 + 2 * pp)
+                    : 0u;
             }
         }
         const float Dh = p.D[h];
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-        // M=64 accumulator mapping: row r16 = 16*warp + (lane & 15); this thread's
-        // 32 columns start at c16 (0 or 32)
-        const int r16 = 16 * warp + (lane & 15);
-        const int c16 = lane < 16 ? 0 : 32;
 
-        // ---- initial state into TMEM (state^T: rows n, columns p)
-        {
-            const float* s0 = p.init_ssm ? p.init_ssm + bh * 64 * NS : nullptr;
-            if (NS == 128) {
-                const int n = 32 * warp + lane;
+        // ---- the carried state h (fp32, registers): S^T[n][p] layout of the state MMA
+        constexpr int HR = NS == 128 ? 32 : 16;
+        float hs[HR];
+        const float* s0 = p.init_ssm ? p.init_ssm + bh * 64 * NS : nullptr;
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    uint32_t r[16];
-#pragma unroll
-                    for (int j = 0; j < 16; j++)
-                        r[j] = __float_as_uint(s0 ? s0[(int64_t)(q * 16 + j) * NS + n] : 0.0f);
-                    tc::tmem_st16(tmem + lane_base + kColST + q * 16, r);
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    uint32_t r[16];
-#pragma unroll
-                    for (int j = 0; j < 16; j++)
-                        r[j] = __float_as_uint(s0 ? s0[(int64_t)(c16 + q * 16 + j) * NS + r16] : 0.0f);
-                    tc::tmem_st16_x2_32(tmem + lane_base + kColST + q * 16, r);
-                }
-            }
-            tc::tmem_wait_st();
+        for (int j = 0; j < HR; j++) {
+            const int pcol = NS == 128 ? half * 32 + j : c16 + j;
+            const int n = NS == 128 ? 32 * sub + lane : r16;
+            hs[j] = s0 ? s0[(int64_t)pcol * NS + n] : 0.0f;
         }
+        float carry_prev = 0.0f;
         bar_compute();
 
         for (int c = 0; c < nc; c++) {
             const int s = c & 1;
             const int t0 = c * 64;
-            const int Lc = min(64, L - t0);
             // On abort the waits return at once; every thread still runs the same
             // sequence of compute barriers and leaves at the end of the iteration.
             tc::mbar_wait(&full[s], (c >> 1) & 1, s_abort, p.status, kStatusTimeout);
             const uint8_t* st = sm + s * LY::kStage;
-            const float* dts = s_dt + s * 64;
-            const float* acv = s_acs + s * 64;
-            const uint32_t m0 = s_bd[s * 4 + 0], m1 = s_bd[s * 4 + 1], pre = s_bd[s * 4 + 2];
-            const int seg_last = seg_of(m0, m1, Lc - 1);
-            const float acs_last = acv[Lc - 1];
-            const bool reset = (m0 | m1) != 0;
+            const ChunkScalars* cs = &scal[s];
+            const uint32_t m0 = cs->m0, m1 = cs->m1, pre = cs->pre;
+            const float carry = cs->carry;
+            const bool quiet = (m0 | m1 | pre) == 0;      // no boundary near this chunk
 
-            // ---- (A) conv and the operand tiles: channel pch, tokens 8*tg .. 8*tg+7
-            const bf16* halo_in = s_halo + (c & 1) * 192;
-            bf16* halo_out = s_halo + ((c + 1) & 1) * 192;
-#pragma unroll 1
-            for (int i = 0; i < 4; i++) {
-                const int tg = tgb + 2 * i;
-                const int r0 = tg * 8;
-                float raw[11];
+            // ---- (A) state: h_c = k_{c-1} h_{c-1} + S_{c-1}; bf16 h_c^T -> Yoff operand
+            if (c > 0) {
+                uint32_t r[HR];
+                if (NS == 128) {
+                    tc::tmem_ld16(tmem + lane_base + kColS + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                    tc::tmem_ld16(tmem + lane_base + kColS + half * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16 % HR]));
+                } else {
+                    tc::tmem_ld16_x2_32(tmem + lane_base + kColS + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                }
+                tc::tmem_wait_ld();
+                const bool drop = carry_prev == kChunkReset;
+#pragma unroll
+                for (int j = 0; j < HR; j++)
+                    hs[j] = (drop ? 0.0f : carry_prev * hs[j]) + __uint_as_float(r[j]);
+            }
+            {
+                const int n = NS == 128 ? 32 * sub + lane : r16;
+                const int pc = NS == 128 ? half * 32 : c16;
+#pragma unroll
+                for (int q = 0; q < HR / 8; q++) {
+                    const uint4 v = make_uint4(pack_bf16(hs[8 * q], hs[8 * q + 1]),
+                                               pack_bf16(hs[8 * q + 2], hs[8 * q + 3]),
+                                               pack_bf16(hs[8 * q + 4], hs[8 * q + 5]),
+                                               pack_bf16(hs[8 * q + 6], hs[8 * q + 7]));
+                    *(uint4*)(sm + LY::kHt + tc::sw128_offset(n, pc + 8 * q)) = v;
+                }
+            }
+            carry_prev = carry;
+
+            // ---- (B) conv and the operand tiles: channels 2pp, 2pp+1; tokens r0 .. r0+7
+            {
+                const uint32_t* halo_in = s_halo + (c & 1) * 96;
+                uint32_t* halo_out = s_halo + ((c + 1) & 1) * 96;
+                uint32_t raw[11];
 #pragma unroll
                 for (int q = 0; q < 11; q++) {
                     const int row = r0 - 3 + q;
-                    if (row >= 0)
-                        raw[q] = __bfloat162float(*(const bf16*)(st + tc::sw128_offset(row, pch)));
-                    else
-                        raw[q] = CONV ? __bfloat162float(halo_in[(row + 3) * 64 + pch]) : 0.f;
+                    if (row >= 0) raw[q] = *(const uint32_t*)(st + tc::sw128_offset(row, 2 * pp));
+                    else raw[q] = CONV ? halo_in[(row + 3) * 32 + pp] : 0u;
                 }
-                if (CONV && tg == 7) {
+                if (CONV && warp == 7) {
 #pragma unroll
-                    for (int j = 0; j < 3; j++)
-                        halo_out[j * 64 + pch] = *(const bf16*)(st + tc::sw128_offset(61 + j, pch));
+                    for (int j = 0; j < 3; j++) halo_out[j * 32 + pp] = raw[8 + j];
                 }
-                float ud[8], us[8];
+                float ud[2][8], us[2][8];
 #pragma unroll
                 for (int q = 0; q < 8; q++) {
                     const int t = r0 + q;
-                    float u;
+                    float u[2];
                     if (CONV) {
-                        // a boundary at chunk position r (r >= 0 from the masks,
-                        // -2/-1 from the two positions before the chunk)
-                        auto bd = [&](int r) -> bool {
-                            if (r >= 32) return (m1 >> (r - 32)) & 1u;
-                            if (r >= 0) return (m0 >> r) & 1u;
-                            return (pre >> (r + 2)) & 1u;
-                        };
-                        const bool ok2 = !bd(t);
-                        const bool ok1 = ok2 && !bd(t - 1);
-                        const bool ok0 = ok1 && !bd(t - 2);
-                        float acc = cbias + wk[3] * raw[q + 3];
-                        acc += ok2 ? wk[2] * raw[q + 2] : 0.f;
-                        acc += ok1 ? wk[1] * raw[q + 1] : 0.f;
-                        acc += ok0 ? wk[0] * raw[q] : 0.f;
-                        u = fast_silu(acc);
+                        bool ok2 = true, ok1 = true, ok0 = true;
+                        if (!quiet) {
+                            auto bd = [&](int r) -> bool {
+                                if (r >= 32) return (m1 >> (r - 32)) & 1u;
+                                if (r >= 0) return (m0 >> r) & 1u;
+                                return (pre >> (r + 2)) & 1u;
+                            };
+                            ok2 = !bd(t);
+                            ok1 = ok2 && !bd(t - 1);
+                            ok0 = ok1 && !bd(t - 2);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 2; e++) {
+                            auto xv = [&](int qq) { return e ? bf_hi(raw[qq]) : bf_lo(raw[qq]); };
+                            float acc = fmaf(wk[e][3], xv(q + 3), cbias[e]);
+                            acc += ok2 ? wk[e][2] * xv(q + 2) : 0.f;
+                            acc += ok1 ? wk[e][1] * xv(q + 1) : 0.f;
+                            acc += ok0 ? wk[e][0] * xv(q) : 0.f;
+                            u[e] = silu_t(acc);
+                        }
                     } else {
-                        u = raw[q + 3];
+                        u[0] = bf_lo(raw[q + 3]);
+                        u[1] = bf_hi(raw[q + 3]);
                     }
-                    *(bf16*)(sm + LY::kXb + tc::sw128_offset(t, pch)) = __float2bfloat16(u);
-                    const bool valid = t < Lc;
-                    ud[q] = valid ? dts[t] * u : 0.f;
-                    us[q] = (valid && seg_of(m0, m1, t) == seg_last)
-                                ? __expf(acs_last - acv[t]) * ud[q] : 0.f;
+                    *(uint32_t*)(sm + LY::kXb + tc::sw128_offset(t, 2 * pp)) = pack_bf16(u[0], u[1]);
+                    const float dtt = cs->dt[t], wdt = cs->wd[t];
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        ud[e][q] = dtt * u[e];
+                        us[e][q] = wdt * u[e];
+                    }
                 }
-                const uint4 vd = make_uint4(pack_bf16(ud[0], ud[1]), pack_bf16(ud[2], ud[3]),
-                                            pack_bf16(ud[4], ud[5]), pack_bf16(ud[6], ud[7]));
-                const uint4 vs = make_uint4(pack_bf16(us[0], us[1]), pack_bf16(us[2], us[3]),
-                                            pack_bf16(us[4], us[5]), pack_bf16(us[6], us[7]));
-                *(uint4*)(sm + LY::kXd + tc::sw128_offset(pch, r0)) = vd;
-                *(uint4*)(sm + LY::kXs + tc::sw128_offset(pch, r0)) = vs;
-            }
-
-            // ---- (B) state hand-off: h_c -> bf16 h^T operand; TMEM state <- k_c h_c
-            const float carry = reset ? 0.f : __expf(acs_last);
-            if (NS == 128) {
-                const int n = 32 * warp + lane;
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    uint32_t r[16];
-                    tc::tmem_ld16(tmem + lane_base + kColST + q * 16, r);
-                    tc::tmem_wait_ld();
-                    uint4 lo, hi;
-                    lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                    lo.y = pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                    lo.z = pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                    lo.w = pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                    hi.x = pack_bf16(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                    hi.y = pack_bf16(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                    hi.z = pack_bf16(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                    hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                    *(uint4*)(sm + LY::kHt + tc::sw128_offset(n, q * 16)) = lo;
-                    *(uint4*)(sm + LY::kHt + tc::sw128_offset(n, q * 16 + 8)) = hi;
-#pragma unroll
-                    for (int j = 0; j < 16; j++)
-                        r[j] = __float_as_uint(reset ? 0.f : carry * __uint_as_float(r[j]));
-                    tc::tmem_st16(tmem + lane_base + kColST + q * 16, r);
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    uint32_t r[16];
-                    tc::tmem_ld16_x2_32(tmem + lane_base + kColST + q * 16, r);
-                    tc::tmem_wait_ld();
-                    uint4 lo, hi;
-                    lo.x = pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1]));
-                    lo.y = pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3]));
-                    lo.z = pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5]));
-                    lo.w = pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7]));
-                    hi.x = pack_bf16(__uint_as_float(r[8]), __uint_as_float(r[9]));
-                    hi.y = pack_bf16(__uint_as_float(r[10]), __uint_as_float(r[11]));
-                    hi.z = pack_bf16(__uint_as_float(r[12]), __uint_as_float(r[13]));
-                    hi.w = pack_bf16(__uint_as_float(r[14]), __uint_as_float(r[15]));
-                    *(uint4*)(sm + LY::kHt + tc::sw128_offset(r16, c16 + q * 16)) = lo;
-                    *(uint4*)(sm + LY::kHt + tc::sw128_offset(r16, c16 + q * 16 + 8)) = hi;
-#pragma unroll
-                    for (int j = 0; j < 16; j++)
-                        r[j] = __float_as_uint(reset ? 0.f : carry * __uint_as_float(r[j]));
-                    tc::tmem_st16_x2_32(tmem + lane_base + kColST + q * 16, r);
+                for (int e = 0; e < 2; e++) {
+                    const uint4 vd = make_uint4(pack_bf16(ud[e][0], ud[e][1]), pack_bf16(ud[e][2], ud[e][3]),
+                                                pack_bf16(ud[e][4], ud[e][5]), pack_bf16(ud[e][6], ud[e][7]));
+                    const uint4 vs = make_uint4(pack_bf16(us[e][0], us[e][1]), pack_bf16(us[e][2], us[e][3]),
+                                                pack_bf16(us[e][4], us[e][5]), pack_bf16(us[e][6], us[e][7]));
+                    *(uint4*)(sm + LY::kXd + tc::sw128_offset(2 * pp + e, r0)) = vd;
+                    *(uint4*)(sm + LY::kXs + tc::sw128_offset(2 * pp + e, r0)) = vs;
                 }
             }
-            tc::tmem_wait_st();
 
             // ---- (C) mask: M[t][s] from the C B^T accumulator
             if (tid == 0) tc::bulk_wait_read0();     // the previous out tile has left shared memory
@@ -459,27 +475,29 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             tc::tc_fence_after();
             {
                 const int t = r16;
-                const float at = acv[t];
-                const int segt = seg_of(m0, m1, t);
+                uint32_t r[16];
+                tc::tmem_ld16_x2_32(tmem + lane_base + kColCB + half * 16, r);
+                tc::tmem_wait_ld();
+                float mv[16];
+                if (c16 > t) {
 #pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    uint32_t r[16];
-                    tc::tmem_ld16_x2_32(tmem + lane_base + kColCB + q * 16, r);
-                    tc::tmem_wait_ld();
-                    float mv[16];
+                    for (int j = 0; j < 16; j++) mv[j] = 0.f;
+                } else {
+                    const float at = cs->a2[t];
+                    const int segt = cs->seg[t];
 #pragma unroll
                     for (int j = 0; j < 16; j++) {
-                        const int sidx = c16 + q * 16 + j;
-                        const bool keep = sidx <= t && seg_of(m0, m1, sidx) == segt;
-                        mv[j] = keep ? __uint_as_float(r[j]) * __expf(at - acv[sidx]) : 0.f;
+                        const int sidx = c16 + j;
+                        const bool keep = sidx <= t && (quiet || cs->seg[sidx] == segt);
+                        mv[j] = keep ? __uint_as_float(r[j]) * ex2(at - cs->a2[sidx]) : 0.f;
                     }
-                    const uint4 lo = make_uint4(pack_bf16(mv[0], mv[1]), pack_bf16(mv[2], mv[3]),
-                                                pack_bf16(mv[4], mv[5]), pack_bf16(mv[6], mv[7]));
-                    const uint4 hi = make_uint4(pack_bf16(mv[8], mv[9]), pack_bf16(mv[10], mv[11]),
-                                                pack_bf16(mv[12], mv[13]), pack_bf16(mv[14], mv[15]));
-                    *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, c16 + q * 16)) = lo;
-                    *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, c16 + q * 16 + 8)) = hi;
                 }
+                const uint4 lo = make_uint4(pack_bf16(mv[0], mv[1]), pack_bf16(mv[2], mv[3]),
+                                            pack_bf16(mv[4], mv[5]), pack_bf16(mv[6], mv[7]));
+                const uint4 hi = make_uint4(pack_bf16(mv[8], mv[9]), pack_bf16(mv[10], mv[11]),
+                                            pack_bf16(mv[12], mv[13]), pack_bf16(mv[14], mv[15]));
+                *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, c16)) = lo;
+                *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, c16 + 8)) = hi;
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
@@ -490,38 +508,28 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             tc::tc_fence_after();
             {
                 const int t = r16;
-                const float f = (seg_of(m0, m1, t) == 0) ? __expf(acv[t]) : 0.f;
+                const float f = cs->f[t];
                 const uint8_t* zt = st + kTile;
+                uint32_t ry[16], ro[16];
+                tc::tmem_ld16_x2_32(tmem + lane_base + kColY + half * 16, ry);
+                tc::tmem_ld16_x2_32(tmem + lane_base + kColYO + half * 16, ro);
+                tc::tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    uint32_t ry[16], ro[16];
-                    tc::tmem_ld16_x2_32(tmem + lane_base + kColY + q * 16, ry);
-                    tc::tmem_ld16_x2_32(tmem + lane_base + kColYO + q * 16, ro);
-                    tc::tmem_wait_ld();
+                for (int hh = 0; hh < 2; hh++) {
+                    const int col = c16 + hh * 8;
+                    const uint4 xv = *(const uint4*)(sm + LY::kXb + tc::sw128_offset(t, col));
+                    const uint4 zv = *(const uint4*)(zt + tc::sw128_offset(t, col));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+                    uint32_t ow[4];
 #pragma unroll
-                    for (int hh = 0; hh < 2; hh++) {
-                        const int col = c16 + q * 16 + hh * 8;
-                        const uint4 xv = *(const uint4*)(sm + LY::kXb + tc::sw128_offset(t, col));
-                        const uint4 zv = *(const uint4*)(zt + tc::sw128_offset(t, col));
-                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                        const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int e = 0; e < 4; e++) {
-                            float o2[2];
-#pragma unroll
-                            for (int k = 0; k < 2; k++) {
-                                const int j = hh * 8 + e * 2 + k;
-                                const float xu = __uint_as_float(k ? (xw[e] & 0xFFFF0000u) : (xw[e] << 16));
-                                const float zz = __uint_as_float(k ? (zw[e] & 0xFFFF0000u) : (zw[e] << 16));
-                                const float y = __uint_as_float(ry[j]) + f * __uint_as_float(ro[j]) + Dh * xu;
-                                o2[k] = y * fast_silu(zz);
-                            }
-                            ow[e] = pack_bf16(o2[0], o2[1]);
-                        }
-                        *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, col)) =
-                            make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    for (int e = 0; e < 4; e++) {
+                        const int j = hh * 8 + e * 2;
+                        const float y0 = fmaf(f, __uint_as_float(ro[j]), __uint_as_float(ry[j])) + Dh * bf_lo(xw[e]);
+                        const float y1 = fmaf(f, __uint_as_float(ro[j + 1]), __uint_as_float(ry[j + 1])) + Dh * bf_hi(xw[e]);
+                        ow[e] = pack_bf16(y0 * silu_t(bf_lo(zw[e])), y1 * silu_t(bf_hi(zw[e])));
                     }
+                    *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, col)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
             tc::fence_async_smem();
@@ -534,39 +542,32 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if (aborted) break;
         }
 
-        // ---- final state (state^T in TMEM: rows n, columns p) -> (b, h, p, n)
-        if (p.final_ssm != nullptr && !*s_abort) {
-            tc::tc_fence_after();
-            float* fs = p.final_ssm + bh * 64 * NS;
+        // ---- final state: h_L = k_last h + S_last  ->  (b, h, p, n)
+        if (p.final_ssm != nullptr && !*s_abort && nc > 0) {
+            uint32_t r[HR];
             if (NS == 128) {
-                const int n = 32 * warp + lane;
-#pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    uint32_t r[16];
-                    tc::tmem_ld16(tmem + lane_base + kColST + q * 16, r);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; j++) fs[(int64_t)(q * 16 + j) * NS + n] = __uint_as_float(r[j]);
-                }
+                tc::tmem_ld16(tmem + lane_base + kColS + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                tc::tmem_ld16(tmem + lane_base + kColS + half * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16 % HR]));
             } else {
+                tc::tmem_ld16_x2_32(tmem + lane_base + kColS + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            }
+            tc::tmem_wait_ld();
+            const bool drop = carry_prev == kChunkReset;
+            float* fs = p.final_ssm + bh * 64 * NS;
+            const int n = NS == 128 ? 32 * sub + lane : r16;
 #pragma unroll
-                for (int q = 0; q < 2; q++) {
-                    uint32_t r[16];
-                    tc::tmem_ld16_x2_32(tmem + lane_base + kColST + q * 16, r);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; j++)
-                        fs[(int64_t)(c16 + q * 16 + j) * NS + r16] = __uint_as_float(r[j]);
-                }
+            for (int j = 0; j < HR; j++) {
+                const int pcol = NS == 128 ? half * 32 + j : c16 + j;
+                fs[(int64_t)pcol * NS + n] = (drop ? 0.0f : carry_prev * hs[j]) + __uint_as_float(r[j]);
             }
         }
         if (tid == 0) tc::bulk_wait0();
     }
 
     // ---- teardown: no MMA may still be running when the tensor memory is freed
-    if (warp == 5 && lane == 0) {
-        tc::mma_commit(&bar[7]);
-        tc::mbar_drain(&bar[7], 0, p.status, kStatusTimeout);
+    if (warp == kMmaWarp && lane == 0) {
+        tc::mma_commit(drain);
+        tc::mbar_drain(drain, 0, p.status, kStatusTimeout);
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -644,7 +645,6 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.seqlen = s.seqlen;
     fp.nheads = s.nheads;
     fp.ngroups = s.ngroups;
-    fp.conv = s.dconv == 4;
     fp.dt = dt;
     fp.acs = acs;
     fp.seq = a.seq_idx;
@@ -661,4 +661,3 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
 }
 
 }  // namespace ssd
-

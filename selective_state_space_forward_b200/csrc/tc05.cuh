@@ -63,14 +63,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
         : "memory");
 }
 
+// try_wait suspends the thread in hardware (up to the hint, in ns) until the
+// phase completes, so a waiting warp does not spin through issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
         : "memory");
     return ok != 0;
 }
@@ -85,7 +87,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; i++) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255) == 0) {
+        if ((i & 7) == 0) {
             if (*abort) return false;
             if (global_ns() - t0 > kWaitLimitNs) {
                 *abort = 1;
@@ -104,7 +106,7 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* 
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; i++) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255) == 0 && global_ns() - t0 > kWaitLimitNs) {
+        if ((i & 7) == 0 && global_ns() - t0 > kWaitLimitNs) {
             atomicOr(status, status_bit);
             return false;
         }
