@@ -128,22 +128,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// 2^x, hardware approximation (PTX ex2.approx).
-__device__ __forceinline__ float ex2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// SiLU(v) = v * (1 + tanh(v/2)) / 2, one hardware tanh (PTX tanh.approx).
-__device__ __forceinline__ float silu_t(float v)
-{
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
-    return v * fmaf(0.5f, t, 0.5f);
-}
-
 template <int NS, bool CONV>
 __global__ void __launch_bounds__(kThreads, NS == 64 ? 2 : 1)
 ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,

@@ -11,16 +11,16 @@
 // document.
 //
 // Layout: one thread owns 8 consecutive channels (one 16-byte bf16 vector, or
-// two fp32 vectors) of 4 consecutive tokens, so its 7 input rows are loaded
-// once and every load and store is a full 16-byte access; consecutive
-// threads walk the channel axis, so a warp touches contiguous 512-byte
-// (bf16) spans of a token row.
+// two fp32 vectors) of 8 consecutive tokens and slides a 3-row window, so each
+// input row is loaded once per thread and every load and store is a full
+// 16-byte access; consecutive threads walk the channel axis, so a warp touches
+// contiguous 512-byte (bf16) spans of a token row.
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
 
 namespace ssd {
 
-constexpr int kTokPerThread = 4;
+constexpr int kTokPerThread = 8;
 
 template <typename T>
 __device__ __forceinline__ const T* channel_src(const Shape& s, const T* x, const T* B, const T* C,
@@ -32,10 +32,41 @@ __device__ __forceinline__ const T* channel_src(const Shape& s, const T* x, cons
     stride = GN; col = c - HP - GN; return C;
 }
 
-// One thread: channels [c, c+8) of tokens [t0, t0+4) of row b.
-// OutT is float (staged path) or bf16 (fused path's shared B|C operand).
+// Eight consecutive elements kept in their storage form (fewer registers than
+// eight floats for bf16) and widened on use.
+template <typename T> struct Vec8;
+template <> struct Vec8<bf16> {
+    uint4 r;
+    __device__ __forceinline__ void load(const bf16* p) { r = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void zero() { r = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ float operator[](int i) const
+    {
+        const uint32_t w = i < 2 ? r.x : i < 4 ? r.y : i < 6 ? r.z : r.w;
+        return (i & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
+    }
+};
+template <> struct Vec8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p)
+    {
+        a = reinterpret_cast<const float4*>(p)[0];
+        b = reinterpret_cast<const float4*>(p)[1];
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ float operator[](int i) const
+    {
+        const float4& v = i < 4 ? a : b;
+        const int j = i & 3;
+        return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+    }
+};
+
+// One thread: channels [c, c+8) of tokens [t0, t0+8) of row b, with a rolling
+// window of the three previous raw rows.  OutT is float (staged path, exact
+// SiLU) or bf16 (fused path's shared B|C operand, hardware-tanh SiLU: the
+// result is rounded to bf16 anyway).
 template <typename T, typename OutT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 conv_silu_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
                  const T* __restrict__ Cm, const T* __restrict__ w, const T* __restrict__ bias,
                  const int32_t* __restrict__ seq, const T* __restrict__ hist0,
@@ -58,61 +89,53 @@ conv_silu_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
     const T* src = channel_src(s, x, Bm, Cm, c, stride, col);
     src += (int64_t)b * L * stride + col;
 
-    float wk[8][4], bs[8];
-    {
-        float t8[8];
+    Vec8<T> wv[4], bv;          // weight (channel i, tap k) = element 4*i + k
 #pragma unroll
-        for (int q = 0; q < 4; q++) {   // 32 weights: channels c..c+7, taps 0..3
-            load8(w + (int64_t)c * 4 + q * 8, t8);
-#pragma unroll
-            for (int i = 0; i < 8; i++) wk[q * 2 + i / 4][i % 4] = t8[i];
-        }
-        load8(bias + c, bs);
-    }
+    for (int q = 0; q < 4; q++) wv[q].load(w + (int64_t)c * 4 + q * 8);
+    bv.load(bias + c);
 
     const int t0 = tg * kTokPerThread;
     const int32_t* seq_row = seq ? seq + (int64_t)b * L : nullptr;
-    // bd[j] = boundary at position t0 - 2 + j  (j = 0 .. 5)
-    int bd[kTokPerThread + 2];
+    uint32_t bdm = 0;           // bit j: boundary at position t0 - 2 + j
 #pragma unroll
     for (int j = 0; j < kTokPerThread + 2; j++) {
         const int64_t pos = (int64_t)t0 - 2 + j;
-        bd[j] = (pos >= 1 && pos < L) ? is_boundary(seq_row, pos) : 0;
+        if (pos >= 1 && pos < L && is_boundary(seq_row, pos)) bdm |= 1u << j;
     }
-    // rows t0-3 .. t0+3
-    float win[kTokPerThread + 3][8];
+    Vec8<T> win[3];             // rows t-3, t-2, t-1
 #pragma unroll
-    for (int j = 0; j < kTokPerThread + 3; j++) {
+    for (int j = 0; j < 3; j++) {
         const int64_t tau = (int64_t)t0 - 3 + j;
-        if (tau >= 0 && tau < L) {
-            load8(src + tau * stride, win[j]);
-        } else if (tau < 0 && hist0 != nullptr) {
-            load8(hist0 + ((int64_t)b * 3 + (tau + 3)) * cd + c, win[j]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; i++) win[j][i] = 0.0f;
-        }
+        if (tau >= 0 && tau < L) win[j].load(src + tau * stride);
+        else if (tau < 0 && hist0 != nullptr) win[j].load(hist0 + ((int64_t)b * 3 + (tau + 3)) * cd + c);
+        else win[j].zero();
     }
 
     OutT* dst = u + (int64_t)b * L * (cd - cbase) + (c - cbase);
-#pragma unroll
+#pragma unroll 1
     for (int q = 0; q < kTokPerThread; q++) {
         const int64_t t = t0 + q;
         if (t >= L) break;
-        // tap k uses row t-3+k, i.e. win[q+k]; valid when no boundary at t-2+k .. t
-        const int okk2 = !bd[q + 2];
-        const int okk1 = okk2 && !bd[q + 1];
-        const int okk0 = okk1 && !bd[q];
+        Vec8<T> cur;
+        cur.load(src + t * stride);
+        // tap k reads row t-3+k; valid when no boundary at positions t-2+k .. t
+        const bool ok2 = !((bdm >> (q + 2)) & 1u);
+        const bool ok1 = ok2 && !((bdm >> (q + 1)) & 1u);
+        const bool ok0 = ok1 && !((bdm >> q) & 1u);
         float o[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) {
-            float acc = bs[i] + wk[i][3] * win[q + 3][i];
-            acc += okk2 ? wk[i][2] * win[q + 2][i] : 0.0f;
-            acc += okk1 ? wk[i][1] * win[q + 1][i] : 0.0f;
-            acc += okk0 ? wk[i][0] * win[q][i] : 0.0f;
-            o[i] = silu_f(acc);
+            const int e = 4 * i;
+            float acc = fmaf(wv[(e + 3) >> 3][(e + 3) & 7], cur[i], bv[i]);
+            acc += ok2 ? wv[(e + 2) >> 3][(e + 2) & 7] * win[2][i] : 0.0f;
+            acc += ok1 ? wv[(e + 1) >> 3][(e + 1) & 7] * win[1][i] : 0.0f;
+            acc += ok0 ? wv[e >> 3][e & 7] * win[0][i] : 0.0f;
+            o[i] = sizeof(OutT) == 2 ? silu_t(acc) : silu_f(acc);
         }
         store8(dst + t * (cd - cbase), o);
+        win[0] = win[1];
+        win[1] = win[2];
+        win[2] = cur;
     }
 }
 

@@ -10,34 +10,28 @@
 //
 // One block per (row, B/C group): the group's B|C conv channels and its heads'
 // x channels are convolved once, so each conv-history column has exactly one
-// reader/writer.  The state is the traffic (95% of the bytes): each warp owns
-// state rows (head, p) of N floats, loads four rows' vectors before using any
-// (memory-level parallelism), and writes each element back once.
+// reader/writer.  The state is 95% of the bytes and is read and written once:
+// in the main kernel 8 lanes share a state row (each lane a float4 per 32
+// floats of the row, so a row is read in full 128-byte pieces), a warp walks 4
+// rows at a time, the next rows' loads are issued before the current rows are
+// computed, and the row's C.h sum is reduced over its 8 lanes.
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
 
 namespace ssd {
 
-constexpr int kDecodeThreads = 128;
-constexpr int kRowsInFlight = 4;
+constexpr int kDecodeThreads = 256;
 
-template <typename T, int V>
-__global__ void __launch_bounds__(kDecodeThreads)
-decode_step_kernel(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ hist)
+// Conv + SiLU of the new token, dt and decay per head, B/C norm: fills the
+// block's shared arrays ux[hpg*P], ub[N], uc[N], dts[hpg], dec[hpg] and, with
+// the norm, the per-head bh/ch[hpg][N].  Ends with a block barrier.
+template <typename T>
+__device__ void decode_prologue(const Shape& s, const FwdArgs& a, T* hist, float* ux, float* ub,
+                                float* uc, float* dts, float* dec, float* bh, float* ch, int g, int b)
 {
-    extern __shared__ float sm[];
     const int H = s.nheads, P = s.headdim, N = s.dstate, G = s.ngroups;
     const int hpg = H / G, HP = H * P, GN = G * N, cd = s.conv_dim();
-    const int g = blockIdx.x, b = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    float* ux = sm;                 // [hpg*P]
-    float* ub = ux + hpg * P;       // [N]
-    float* uc = ub + N;             // [N]
-    float* dts = uc + N;            // [hpg]
-    float* dec = dts + hpg;         // [hpg]
-    float* bh = dec + hpg;          // [hpg][N] (B/C norm only)
-    float* ch = bh + (s.bc_norm ? hpg * N : 0);
-
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const T* x = (const T*)a.x;
     const T* Bm = (const T*)a.B;
     const T* Cm = (const T*)a.C;
@@ -86,7 +80,7 @@ decode_step_kernel(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ 
     }
     __syncthreads();
     if (s.bc_norm) {
-        // warps 0 / 1 normalise B / C; every warp then adds the heads' biases
+        // warps 0 / 1 normalise B / C; every thread then adds the heads' biases
         if (warp < 2) {
             float* v = warp ? uc : ub;
             float ss = 0.0f;
@@ -106,70 +100,132 @@ decode_step_kernel(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ 
         }
         __syncthreads();
     }
+}
 
-    // state rows (hl, p), kRowsInFlight at a time per warp
+struct DecodeSmem {
+    float *ux, *ub, *uc, *dts, *dec, *bh, *ch;
+    __device__ DecodeSmem(float* sm, const Shape& s)
+    {
+        const int hpg = s.nheads / s.ngroups;
+        const int hp4 = (hpg + 3) & ~3;      // keeps bh/ch 16-byte aligned
+        ux = sm;
+        ub = ux + hpg * s.headdim;
+        uc = ub + s.dstate;
+        dts = uc + s.dstate;
+        dec = dts + hp4;
+        bh = dec + hp4;
+        ch = bh + (s.bc_norm ? hpg * s.dstate : 0);
+    }
+};
+
+// Main kernel: N = 32 * NV.  Lane l8 of a row owns float4 q at floats
+// (q * 8 + l8) * 4 .. +3, so the 8 lanes of a row cover 32 consecutive floats
+// per q.
+template <typename T, int NV>
+__global__ void __launch_bounds__(kDecodeThreads)
+decode_step_vec(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ hist)
+{
+    extern __shared__ float sm[];
+    const int H = s.nheads, P = s.headdim, N = s.dstate;
+    const int hpg = H / s.ngroups, HP = H * P;
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    DecodeSmem sv(sm, s);
+    decode_prologue<T>(s, a, hist, sv.ux, sv.ub, sv.uc, sv.dts, sv.dec, sv.bh, sv.ch, g, b);
+
+    const int sub = lane >> 3, l8 = lane & 7;
+    float4 Bq[NV], Cq[NV];
+    if (!s.bc_norm) {
+#pragma unroll
+        for (int q = 0; q < NV; q++) {
+            Bq[q] = *reinterpret_cast<const float4*>(sv.ub + (q * 8 + l8) * 4);
+            Cq[q] = *reinterpret_cast<const float4*>(sv.uc + (q * 8 + l8) * 4);
+        }
+    }
     const int nrows = hpg * P;
-    for (int r0 = warp * kRowsInFlight; r0 < nrows; r0 += nw * kRowsInFlight) {
-        float st[kRowsInFlight][V];
-        float* rowp[kRowsInFlight];
+    const int step = nw * 4;
+    float* base = ssm + ((int64_t)b * H + (int64_t)g * hpg) * P * N;   // row r at base + r*N
+    auto load_row = [&](int r, float4 (&v)[NV]) {
+        if (r < nrows) {
 #pragma unroll
-        for (int q = 0; q < kRowsInFlight; q++) {
-            const int row = r0 + q;
-            const int hl = row / P, p = row % P;
-            rowp[q] = ssm + (((int64_t)b * H + g * hpg + hl) * P + p) * N;
+            for (int q = 0; q < NV; q++)
+                v[q] = *reinterpret_cast<const float4*>(base + (int64_t)r * N + (q * 8 + l8) * 4);
         }
-        float ysum[kRowsInFlight];
+    };
+    int r = warp * 4 + sub;
+    float4 cur[NV], nxt[NV];
+    load_row(r, cur);
+    for (; r - sub < nrows; r += step) {
+        load_row(r + step, nxt);
+        const bool valid = r < nrows;
+        const int hl = valid ? r / P : 0;
+        const float xdt = valid ? sv.dts[hl] * sv.ux[r] : 0.f;
+        const float d = sv.dec[hl];
+        float y = 0.f;
 #pragma unroll
-        for (int q = 0; q < kRowsInFlight; q++) ysum[q] = 0.0f;
-        for (int n0 = lane * V; n0 < N; n0 += 32 * V) {
-#pragma unroll
-            for (int q = 0; q < kRowsInFlight; q++) {
-                if (V == 4) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(rowp[q] + n0);
-                    st[q][0] = t4.x; st[q][1] = t4.y; st[q][2] = t4.z; st[q][3] = t4.w;
-                } else if (V == 2) {
-                    const float2 t2 = *reinterpret_cast<const float2*>(rowp[q] + n0);
-                    st[q][0] = t2.x; st[q][1] = t2.y;
-                } else {
-                    st[q][0] = rowp[q][n0];
-                }
+        for (int q = 0; q < NV; q++) {
+            float4 bv = Bq[q], cv = Cq[q];
+            if (s.bc_norm) {
+                bv = *reinterpret_cast<const float4*>(sv.bh + hl * N + (q * 8 + l8) * 4);
+                cv = *reinterpret_cast<const float4*>(sv.ch + hl * N + (q * 8 + l8) * 4);
             }
-#pragma unroll
-            for (int q = 0; q < kRowsInFlight; q++) {
-                const int row = r0 + q;
-                const int hl = row / P;
-                const float* Bv = s.bc_norm ? bh + hl * N : ub;
-                const float* Cv = s.bc_norm ? ch + hl * N : uc;
-                const float xdt = dts[hl] * ux[row];
-                const float d = dec[hl];
-#pragma unroll
-                for (int k = 0; k < V; k++) {
-                    const float hv = d * st[q][k] + xdt * Bv[n0 + k];
-                    st[q][k] = hv;
-                    ysum[q] += Cv[n0 + k] * hv;
-                }
-                if (V == 4) {
-                    *reinterpret_cast<float4*>(rowp[q] + n0) =
-                        make_float4(st[q][0], st[q][1], st[q][2], st[q][3]);
-                } else if (V == 2) {
-                    *reinterpret_cast<float2*>(rowp[q] + n0) = make_float2(st[q][0], st[q][1]);
-                } else {
-                    rowp[q][n0] = st[q][0];
-                }
-            }
+            float4 hv;
+            hv.x = fmaf(d, cur[q].x, xdt * bv.x);
+            hv.y = fmaf(d, cur[q].y, xdt * bv.y);
+            hv.z = fmaf(d, cur[q].z, xdt * bv.z);
+            hv.w = fmaf(d, cur[q].w, xdt * bv.w);
+            y = fmaf(cv.x, hv.x, y);
+            y = fmaf(cv.y, hv.y, y);
+            y = fmaf(cv.z, hv.z, y);
+            y = fmaf(cv.w, hv.w, y);
+            if (valid)
+                *reinterpret_cast<float4*>(base + (int64_t)r * N + (q * 8 + l8) * 4) = hv;
+        }
+        y += __shfl_xor_sync(0xffffffffu, y, 1);
+        y += __shfl_xor_sync(0xffffffffu, y, 2);
+        y += __shfl_xor_sync(0xffffffffu, y, 4);
+        if (valid && l8 == 0) {
+            const int hh = g * hpg + hl, p = r % P;
+            const int64_t o = (int64_t)b * HP + hh * P + p;
+            const float zv = to_f(((const T*)a.z)[o]);
+            ((T*)a.out)[o] = from_f<T>((y + a.D[hh] * sv.ux[r]) * silu_f(zv));
         }
 #pragma unroll
-        for (int q = 0; q < kRowsInFlight; q++) {
-            float y = ysum[q];
+        for (int q = 0; q < NV; q++) cur[q] = nxt[q];
+    }
+}
+
+// General kernel for any d_state (a multiple of 8): a warp per state row.
+template <typename T>
+__global__ void __launch_bounds__(kDecodeThreads)
+decode_step_any(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ hist)
+{
+    extern __shared__ float sm[];
+    const int H = s.nheads, P = s.headdim, N = s.dstate;
+    const int hpg = H / s.ngroups, HP = H * P;
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    DecodeSmem sv(sm, s);
+    decode_prologue<T>(s, a, hist, sv.ux, sv.ub, sv.uc, sv.dts, sv.dec, sv.bh, sv.ch, g, b);
+    const int nrows = hpg * P;
+    for (int r = warp; r < nrows; r += nw) {
+        const int hl = r / P;
+        const float* Bv = s.bc_norm ? sv.bh + hl * N : sv.ub;
+        const float* Cv = s.bc_norm ? sv.ch + hl * N : sv.uc;
+        const float xdt = sv.dts[hl] * sv.ux[r], d = sv.dec[hl];
+        float* row = ssm + (((int64_t)b * H + g * hpg + hl) * P + r % P) * N;
+        float y = 0.f;
+        for (int n = lane; n < N; n += 32) {
+            const float hv = fmaf(d, row[n], xdt * Bv[n]);
+            row[n] = hv;
+            y = fmaf(Cv[n], hv, y);
+        }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
-            if (lane == 0) {
-                const int row = r0 + q;
-                const int hl = row / P, p = row % P, h = g * hpg + hl;
-                const int64_t o = (int64_t)b * HP + h * P + p;
-                const float zv = to_f(((const T*)a.z)[o]);
-                ((T*)a.out)[o] = from_f<T>((y + a.D[h] * ux[row]) * silu_f(zv));
-            }
+        for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(0xffffffffu, y, o);
+        if (lane == 0) {
+            const int hh = g * hpg + hl;
+            const int64_t o = (int64_t)b * HP + hh * P + r % P;
+            ((T*)a.out)[o] = from_f<T>((y + a.D[hh] * sv.ux[r]) * silu_f(to_f(((const T*)a.z)[o])));
         }
     }
 }
@@ -179,11 +235,18 @@ static cudaError_t launch_decode_t(const Shape& s, const FwdArgs& a, float* ssm,
                                    cudaStream_t st)
 {
     const int hpg = s.nheads / s.ngroups;
-    const size_t smem = sizeof(float) * ((size_t)hpg * s.headdim + 2 * s.dstate + 2 * hpg +
+    const size_t hp4 = (size_t)((hpg + 3) & ~3);
+    const size_t smem = sizeof(float) * ((size_t)hpg * s.headdim + 2 * s.dstate + 2 * hp4 +
                                          (s.bc_norm ? 2 * (size_t)hpg * s.dstate : 0));
     const dim3 grid(s.ngroups, s.batch);
-    auto kern = (s.dstate % 128 == 0) ? decode_step_kernel<T, 4>
-              : (s.dstate % 64 == 0) ? decode_step_kernel<T, 2> : decode_step_kernel<T, 1>;
+    void (*kern)(Shape, FwdArgs, float*, T*);
+    switch (s.dstate) {
+    case 32: kern = decode_step_vec<T, 1>; break;
+    case 64: kern = decode_step_vec<T, 2>; break;
+    case 128: kern = decode_step_vec<T, 4>; break;
+    case 256: kern = decode_step_vec<T, 8>; break;
+    default: kern = decode_step_any<T>; break;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kDecodeThreads, smem, st>>>(s, a, ssm, (T*)hist);
