@@ -1,9 +1,9 @@
 // chunk_fused.cu -- KF: the fused chunk sweep of the SSD scan on sm_100a.
 //
-// One CTA owns one (batch row, head) and walks its 64-token chunks in order
-// (chunk 64: mojolearn Mamba3Block), so the running state never leaves the
-// SM.  Per chunk c (tokens t0 .. t0+63), with acs the segmented cumsum of
-// dt*a written by K2 and seg_t the number of document boundaries at t0 .. t:
+// Work: every (batch row, head) stream of 64-token chunks (chunk 64: mojolearn
+// Mamba3Block) is cut into segments of consecutive chunks.  Per chunk c, with
+// acs the segmented cumsum of dt*a written by K2 and seg_t the number of
+// document boundaries at t0 .. t:
 //
 //   conv      u_t = SiLU(conv(x)) for the head's 64 channels (K1's arithmetic;
 //             B and C of the group come pre-convolved from K1, or raw)
@@ -18,10 +18,13 @@
 //             (k_c = exp(acs_last), dropped when the chunk holds a boundary)
 //   epilogue  out_t = (Ydiag_t + [seg_t = 0] exp(acs_t) Yoff_t + D u_t) SiLU(z_t)
 //
-// The fp32 state is carried in the compute threads' registers from the
-// initial state to the final one; a bf16 copy of it is staged in shared
-// memory each chunk as the Yoff operand.  The gate, the D skip and the output
-// cast are fused in the epilogue.
+// Schedule: a persistent grid (every CTA resident) takes work items -- segment
+// k of stream s -- in the order j = k * streams + s, CTA i taking i, i + G, ...
+// A segment's entering state is the previous segment's leaving state, handed
+// over through global memory with an epoch-tagged flag; because items are
+// segment-major and every CTA is resident, each dependency points to an item
+// started earlier and the wait ends.  This keeps every SM busy to within one
+// item whatever the number of streams, and lets two CTAs share each SM.
 //
 // Roles (320 threads): warps 0-7 compute (state update, conv, masks,
 // epilogue; warp w reaches TMEM lanes 32*(w%4) .. +31 and takes the column
@@ -53,18 +56,24 @@ constexpr int kTile = 64 * 128;        // one [64][64] bf16 tile
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColCB = 0, kColY = 64, kColYO = 128, kColS = 192;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kItemsPerSm = 16;        // bound on work items per SM (sizes the hand-off buffers)
 
 struct FusedParams {
     int batch, seqlen, nheads, ngroups;
+    int nseg, cps, nitems;    // segments per stream, chunks per segment, items
+    unsigned epoch;           // tag of this call's hand-off flags
     const float* dt;          // (B, H, L) from K2
     const float* acs;         // (B, H, L) segmented cumsum from K2
     const int32_t* seq;       // (B, L) or null
     const float* D;
+    const bf16* x;            // raw x, for the conv history at segment starts
     const bf16* conv_w;       // (conv_dim, 4) or null
     const bf16* conv_b;
     const bf16* init_conv;    // (B, 3, conv_dim) or null
     const float* init_ssm;    // (B, H, 64, N) or null
     float* final_ssm;         // or null
+    float* hseg;              // (streams, nseg, 64, N) segment leaving states
+    unsigned* flags;          // (streams, nseg)
     int* status;
 };
 
@@ -128,6 +137,40 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// The flattened step sequence a CTA walks: its work items in order, each item's
+// chunks in order.  Every role iterates it identically.
+struct StepIter {
+    int j, c, cend, b, h, k;
+    int H, nstr, cps, nc, nitems, G;
+    __device__ StepIter(const FusedParams& p, int nc_)
+    {
+        H = p.nheads; nstr = p.batch * p.nheads; cps = p.cps; nc = nc_;
+        nitems = p.nitems; G = gridDim.x;
+        j = blockIdx.x;
+        load_item();
+    }
+    __device__ void load_item()
+    {
+        if (j >= nitems) return;
+        k = j / nstr;
+        const int s = j % nstr;
+        b = s / H;
+        h = s % H;
+        c = k * cps;
+        cend = min(c + cps, nc);
+    }
+    __device__ bool valid() const { return j < nitems; }
+    __device__ bool first() const { return c == k * cps; }
+    __device__ bool last() const { return c == cend - 1; }
+    __device__ void next()
+    {
+        if (++c >= cend) {
+            j += G;
+            load_item();
+        }
+    }
+};
+
 template <int NS, bool CONV>
 __global__ void __launch_bounds__(kThreads, NS == 64 ? 2 : 1)
 ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
@@ -151,10 +194,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.nheads, L = p.seqlen;
-    const int b = blockIdx.x / H, h = blockIdx.x % H;
-    const int g = h / (H / p.ngroups);
     const int nc = (L + 63) / 64;
-    const int64_t bh = (int64_t)b * H + h;
 
     if (tid == 0) {
         for (int i = 0; i < 2; i++) {
@@ -186,29 +226,31 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
-        const int32_t* seq_row = p.seq ? p.seq + (int64_t)b * L : nullptr;
-        const float* dt_row = p.dt + bh * L;
-        const float* acs_row = p.acs + bh * L;
         const uint32_t tx = (uint32_t)(2 * kTile + 2 * LY::kBC);
-        int issued = 0;
-        for (int c = 0; c < nc; c++) {
-            const int s = c & 1;
-            if (c >= 2 && !tc::mbar_wait(&empty[s], ((c >> 1) & 1) ^ 1, s_abort, p.status, kStatusTimeout))
+        int q = 0;
+        for (StepIter it(p, nc); it.valid(); it.next(), q++) {
+            const int s = q & 1;
+            if (q >= 2 && !tc::mbar_wait(&empty[s], ((q >> 1) & 1) ^ 1, s_abort, p.status, kStatusTimeout))
                 break;
-            const int t0 = c * 64;
+            const int b = it.b, h = it.h, g = h / (H / p.ngroups);
+            const int t0 = it.c * 64;
+            const int64_t bh = (int64_t)b * H + h;
             uint8_t* st = sm + s * LY::kStage;
             if (lane == 0) {
                 tc::mbar_arrive_expect_tx(&full[s], tx);
                 tc::tma_load_3d(st, &tm_x, &full[s], h * 64, t0, b);
                 tc::tma_load_3d(st + kTile, &tm_z, &full[s], h * 64, t0, b);
 #pragma unroll
-                for (int j = 0; j < NS / 64; j++) {
-                    const int bx = g * NS + 64 * j;
-                    const int cx = (CONV ? p.ngroups * NS : 0) + g * NS + 64 * j;
-                    tc::tma_load_3d(st + 2 * kTile + j * kTile, &tm_b, &full[s], bx, t0, b);
-                    tc::tma_load_3d(st + 2 * kTile + LY::kBC + j * kTile, &tm_c, &full[s], cx, t0, b);
+                for (int jj = 0; jj < NS / 64; jj++) {
+                    const int bx = g * NS + 64 * jj;
+                    const int cx = (CONV ? p.ngroups * NS : 0) + g * NS + 64 * jj;
+                    tc::tma_load_3d(st + 2 * kTile + jj * kTile, &tm_b, &full[s], bx, t0, b);
+                    tc::tma_load_3d(st + 2 * kTile + LY::kBC + jj * kTile, &tm_c, &full[s], cx, t0, b);
                 }
             }
+            const int32_t* seq_row = p.seq ? p.seq + (int64_t)b * L : nullptr;
+            const float* dt_row = p.dt + bh * L;
+            const float* acs_row = p.acs + bh * L;
             ChunkScalars* cs = &scal[s];
             const int Lc = min(64, L - t0);
             float dtv[2], acv[2];
@@ -250,11 +292,10 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
             __syncwarp();
             tc::mbar_arrive(&full[s]);
-            issued = c + 1;
         }
         // an aborting CTA lets its last loads land before the shared memory is released
-        for (int k = max(0, issued - 2); k < issued; k++)
-            tc::mbar_drain(&full[k & 1], (k >> 1) & 1, p.status, kStatusTimeout);
+        for (int k2 = max(0, q - 2); k2 < q; k2++)
+            tc::mbar_drain(&full[k2 & 1], (k2 >> 1) & 1, p.status, kStatusTimeout);
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issue
         if (lane == 0) {
@@ -265,9 +306,10 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const uint32_t a_xd = tc::smem_u32(sm + LY::kXd);
             const uint32_t a_xs = tc::smem_u32(sm + LY::kXs);
             const uint32_t a_ht = tc::smem_u32(sm + LY::kHt);
-            for (int c = 0; c < nc; c++) {
-                const int s = c & 1;
-                if (!tc::mbar_wait(&full[s], (c >> 1) & 1, s_abort, p.status, kStatusTimeout)) break;
+            int q = 0;
+            for (StepIter it(p, nc); it.valid(); it.next(), q++) {
+                const int s = q & 1;
+                if (!tc::mbar_wait(&full[s], (q >> 1) & 1, s_abort, p.status, kStatusTimeout)) break;
                 tc::tc_fence_after();
                 const uint32_t a_b = tc::smem_u32(sm + s * LY::kStage + 2 * kTile);
                 const uint32_t a_c = a_b + LY::kBC;
@@ -279,7 +321,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                  tc::sdesc_sw128(a_b + off, 16, 1024), id_64, kk > 0);
                 }
                 tc::mma_commit(cb_done);
-                if (!tc::mbar_wait(ops_ready, c & 1, s_abort, p.status, kStatusTimeout)) break;
+                if (!tc::mbar_wait(ops_ready, q & 1, s_abort, p.status, kStatusTimeout)) break;
                 tc::tc_fence_after();
                 // Ydiag = M Xd (K = s)
 #pragma unroll
@@ -304,8 +346,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         __syncwarp();
     } else {
         // ------------------------------------------------------------ compute warps 0-7
-        const int HP = H * 64;
-        const int cdim = HP + 2 * p.ngroups * NS;
+        const int cdim = H * 64 + 2 * p.ngroups * NS;
         const int sub = warp & 3;                  // TMEM lane quarter
         const int half = warp >> 2;                // column half
         const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
@@ -315,98 +356,133 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         // conv: channel pair pp, tokens 8*warp .. 8*warp+7
         const int pp = lane;
         const int r0 = 8 * warp;
-        float wk[2][4] = {{0.f, 0.f, 0.f, 1.f}, {0.f, 0.f, 0.f, 1.f}}, cbias[2] = {0.f, 0.f};
-        if (CONV) {
-#pragma unroll
-            for (int e = 0; e < 2; e++) {
-                const int ch = h * 64 + 2 * pp + e;
-#pragma unroll
-                for (int k = 0; k < 4; k++) wk[e][k] = __bfloat162float(p.conv_w[(int64_t)ch * 4 + k]);
-                cbias[e] = __bfloat162float(p.conv_b[ch]);
-            }
-            // halo for chunk 0: the caller's conv history of these channels (zeros when none)
-            if (tid < 96) {
-                const int j = tid >> 5;
-                s_halo[j * 32 + pp] = p.init_conv
-                    ? *(const uint32_t*)(p.init_conv + ((int64_t)b * 3 + j) * cdim + h * 64 + 2 * pp)
-                    : 0u;
-            }
-        }
-        const float Dh = p.D[h];
-
-        // ---- the carried state h (fp32, registers): S^T[n][p] layout of the state MMA
+        // the carried state h: S^T[n][p] layout of the state MMA
         constexpr int HR = NS == 128 ? 32 : 16;
+        const int nrow = NS == 128 ? 32 * sub + lane : r16;
+        const int pcol = NS == 128 ? half * 32 : c16;
         float hs[HR];
-        const float* s0 = p.init_ssm ? p.init_ssm + bh * 64 * NS : nullptr;
-#pragma unroll
-        for (int j = 0; j < HR; j++) {
-            const int pcol = NS == 128 ? half * 32 + j : c16 + j;
-            const int n = NS == 128 ? 32 * sub + lane : r16;
-            hs[j] = s0 ? s0[(int64_t)pcol * NS + n] : 0.0f;
-        }
-        float carry_prev = 0.0f;
-        bar_compute();
+        float wk[2][4] = {{0.f, 0.f, 0.f, 1.f}, {0.f, 0.f, 0.f, 1.f}}, cbias[2] = {0.f, 0.f};
+        float Dh = 0.f, carry_prev = 0.f;
+        int cur_h = -1;
+        auto load_S = [&](uint32_t (&r)[HR]) {
+            if (NS == 128) {
+                tc::tmem_ld16(tmem + lane_base + kColS + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                tc::tmem_ld16(tmem + lane_base + kColS + half * 32 + 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(&r[16 % HR]));
+            } else {
+                tc::tmem_ld16_x2_32(tmem + lane_base + kColS + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            }
+            tc::tmem_wait_ld();
+        };
 
-        for (int c = 0; c < nc; c++) {
-            const int s = c & 1;
-            const int t0 = c * 64;
+        int q = 0;
+        for (StepIter it(p, nc); it.valid(); it.next(), q++) {
+            const int s = q & 1;
+            const int b = it.b, h = it.h, t0 = it.c * 64;
+            const int64_t str = (int64_t)b * H + h;
+            const bool first = it.first();
+            // ---- per-head constants
+            if (h != cur_h) {
+                cur_h = h;
+                Dh = p.D[h];
+                if (CONV) {
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const int ch = h * 64 + 2 * pp + e;
+#pragma unroll
+                        for (int kq = 0; kq < 4; kq++) wk[e][kq] = __bfloat162float(p.conv_w[(int64_t)ch * 4 + kq]);
+                        cbias[e] = __bfloat162float(p.conv_b[ch]);
+                    }
+                }
+            }
             // On abort the waits return at once; every thread still runs the same
             // sequence of compute barriers and leaves at the end of the iteration.
-            tc::mbar_wait(&full[s], (c >> 1) & 1, s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(&full[s], (q >> 1) & 1, s_abort, p.status, kStatusTimeout);
             const uint8_t* st = sm + s * LY::kStage;
             const ChunkScalars* cs = &scal[s];
             const uint32_t m0 = cs->m0, m1 = cs->m1, pre = cs->pre;
             const float carry = cs->carry;
             const bool quiet = (m0 | m1 | pre) == 0;      // no boundary near this chunk
 
-            // ---- (A) state: h_c = k_{c-1} h_{c-1} + S_{c-1}; bf16 h_c^T -> Yoff operand
-            if (c > 0) {
-                uint32_t r[HR];
-                if (NS == 128) {
-                    tc::tmem_ld16(tmem + lane_base + kColS + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                    tc::tmem_ld16(tmem + lane_base + kColS + half * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16 % HR]));
+            // ---- (A) state entering this chunk -> bf16 h^T (the Yoff operand)
+            if (first) {
+                const float* src = nullptr;
+                if (it.k == 0) {
+                    src = p.init_ssm ? p.init_ssm + str * 64 * NS : nullptr;
                 } else {
-                    tc::tmem_ld16_x2_32(tmem + lane_base + kColS + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                    // the previous segment's leaving state (an item started earlier)
+                    const unsigned* fl = p.flags + str * p.nseg + (it.k - 1);
+                    if (tid == 0) {
+                        const uint64_t tw = tc::global_ns();
+                        unsigned v;
+                        for (;;) {
+                            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(fl) : "memory");
+                            if (v == p.epoch || *s_abort) break;
+                            if (tc::global_ns() - tw > tc::kWaitLimitNs) {
+                                *s_abort = 1;
+                                atomicOr(p.status, kStatusTimeout);
+                                break;
+                            }
+                            __nanosleep(128);
+                        }
+                    }
+                    bar_compute();
+                    src = p.hseg + (str * p.nseg + (it.k - 1)) * 64 * NS;
                 }
-                tc::tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < HR; jj++) hs[jj] = src ? __ldcg(src + (int64_t)(pcol + jj) * NS + nrow) : 0.f;
+            } else {
+                // h_c = k_{c-1} h_{c-1} + S_{c-1}  (S_{c-1} complete: mma_done of the last step)
+                uint32_t r[HR];
+                load_S(r);
                 const bool drop = carry_prev == kChunkReset;
 #pragma unroll
-                for (int j = 0; j < HR; j++)
-                    hs[j] = (drop ? 0.0f : carry_prev * hs[j]) + __uint_as_float(r[j]);
+                for (int jj = 0; jj < HR; jj++)
+                    hs[jj] = (drop ? 0.0f : carry_prev * hs[jj]) + __uint_as_float(r[jj]);
             }
-            {
-                const int n = NS == 128 ? 32 * sub + lane : r16;
-                const int pc = NS == 128 ? half * 32 : c16;
 #pragma unroll
-                for (int q = 0; q < HR / 8; q++) {
-                    const uint4 v = make_uint4(pack_bf16(hs[8 * q], hs[8 * q + 1]),
-                                               pack_bf16(hs[8 * q + 2], hs[8 * q + 3]),
-                                               pack_bf16(hs[8 * q + 4], hs[8 * q + 5]),
-                                               pack_bf16(hs[8 * q + 6], hs[8 * q + 7]));
-                    *(uint4*)(sm + LY::kHt + tc::sw128_offset(n, pc + 8 * q)) = v;
-                }
+            for (int qq = 0; qq < HR / 8; qq++) {
+                const uint4 v = make_uint4(pack_bf16(hs[8 * qq], hs[8 * qq + 1]),
+                                           pack_bf16(hs[8 * qq + 2], hs[8 * qq + 3]),
+                                           pack_bf16(hs[8 * qq + 4], hs[8 * qq + 5]),
+                                           pack_bf16(hs[8 * qq + 6], hs[8 * qq + 7]));
+                *(uint4*)(sm + LY::kHt + tc::sw128_offset(nrow, pcol + 8 * qq)) = v;
             }
             carry_prev = carry;
 
             // ---- (B) conv and the operand tiles: channels 2pp, 2pp+1; tokens r0 .. r0+7
             {
-                const uint32_t* halo_in = s_halo + (c & 1) * 96;
-                uint32_t* halo_out = s_halo + ((c + 1) & 1) * 96;
+                const uint32_t* halo_in = s_halo + (q & 1) * 96;
+                uint32_t* halo_out = s_halo + ((q + 1) & 1) * 96;
                 uint32_t raw[11];
 #pragma unroll
-                for (int q = 0; q < 11; q++) {
-                    const int row = r0 - 3 + q;
-                    if (row >= 0) raw[q] = *(const uint32_t*)(st + tc::sw128_offset(row, 2 * pp));
-                    else raw[q] = CONV ? halo_in[(row + 3) * 32 + pp] : 0u;
+                for (int qq = 0; qq < 11; qq++) {
+                    const int row = r0 - 3 + qq;
+                    if (row >= 0) {
+                        raw[qq] = *(const uint32_t*)(st + tc::sw128_offset(row, 2 * pp));
+                    } else if (!CONV) {
+                        raw[qq] = 0u;
+                    } else if (!first) {
+                        raw[qq] = halo_in[(row + 3) * 32 + pp];
+                    } else {
+                        // segment start: the three tokens before the chunk from the raw x,
+                        // or the caller's conv history before token 0
+                        const int tok = t0 + row;
+                        raw[qq] = tok >= 0
+                            ? *(const uint32_t*)(p.x + ((int64_t)b * L + tok) * (H * 64) + h * 64 + 2 * pp)
+                            : (p.init_conv ? *(const uint32_t*)(p.init_conv + ((int64_t)b * 3 + (tok + 3)) * cdim +
+                                                               h * 64 + 2 * pp)
+                                           : 0u);
+                    }
                 }
                 if (CONV && warp == 7) {
 #pragma unroll
-                    for (int j = 0; j < 3; j++) halo_out[j * 32 + pp] = raw[8 + j];
+                    for (int jj = 0; jj < 3; jj++) halo_out[jj * 32 + pp] = raw[8 + jj];
                 }
                 float ud[2][8], us[2][8];
 #pragma unroll
-                for (int q = 0; q < 8; q++) {
-                    const int t = r0 + q;
+                for (int qq = 0; qq < 8; qq++) {
+                    const int t = r0 + qq;
                     float u[2];
                     if (CONV) {
                         bool ok2 = true, ok1 = true, ok0 = true;
@@ -422,23 +498,23 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         }
 #pragma unroll
                         for (int e = 0; e < 2; e++) {
-                            auto xv = [&](int qq) { return e ? bf_hi(raw[qq]) : bf_lo(raw[qq]); };
-                            float acc = fmaf(wk[e][3], xv(q + 3), cbias[e]);
-                            acc += ok2 ? wk[e][2] * xv(q + 2) : 0.f;
-                            acc += ok1 ? wk[e][1] * xv(q + 1) : 0.f;
-                            acc += ok0 ? wk[e][0] * xv(q) : 0.f;
+                            auto xv = [&](int k3) { return e ? bf_hi(raw[k3]) : bf_lo(raw[k3]); };
+                            float acc = fmaf(wk[e][3], xv(qq + 3), cbias[e]);
+                            acc += ok2 ? wk[e][2] * xv(qq + 2) : 0.f;
+                            acc += ok1 ? wk[e][1] * xv(qq + 1) : 0.f;
+                            acc += ok0 ? wk[e][0] * xv(qq) : 0.f;
                             u[e] = silu_t(acc);
                         }
                     } else {
-                        u[0] = bf_lo(raw[q + 3]);
-                        u[1] = bf_hi(raw[q + 3]);
+                        u[0] = bf_lo(raw[qq + 3]);
+                        u[1] = bf_hi(raw[qq + 3]);
                     }
                     *(uint32_t*)(sm + LY::kXb + tc::sw128_offset(t, 2 * pp)) = pack_bf16(u[0], u[1]);
                     const float dtt = cs->dt[t], wdt = cs->wd[t];
 #pragma unroll
                     for (int e = 0; e < 2; e++) {
-                        ud[e][q] = dtt * u[e];
-                        us[e][q] = wdt * u[e];
+                        ud[e][qq] = dtt * u[e];
+                        us[e][qq] = wdt * u[e];
                     }
                 }
 #pragma unroll
@@ -455,7 +531,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // ---- (C) mask: M[t][s] from the C B^T accumulator
             if (tid == 0) tc::bulk_wait_read0();     // the previous out tile has left shared memory
             bar_compute();
-            tc::mbar_wait(cb_done, c & 1, s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(cb_done, q & 1, s_abort, p.status, kStatusTimeout);
             tc::tc_fence_after();
             {
                 const int t = r16;
@@ -465,15 +541,15 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 float mv[16];
                 if (c16 > t) {
 #pragma unroll
-                    for (int j = 0; j < 16; j++) mv[j] = 0.f;
+                    for (int jj = 0; jj < 16; jj++) mv[jj] = 0.f;
                 } else {
                     const float at = cs->a2[t];
                     const int segt = cs->seg[t];
 #pragma unroll
-                    for (int j = 0; j < 16; j++) {
-                        const int sidx = c16 + j;
+                    for (int jj = 0; jj < 16; jj++) {
+                        const int sidx = c16 + jj;
                         const bool keep = sidx <= t && (quiet || cs->seg[sidx] == segt);
-                        mv[j] = keep ? __uint_as_float(r[j]) * ex2(at - cs->a2[sidx]) : 0.f;
+                        mv[jj] = keep ? __uint_as_float(r[jj]) * ex2(at - cs->a2[sidx]) : 0.f;
                     }
                 }
                 const uint4 lo = make_uint4(pack_bf16(mv[0], mv[1]), pack_bf16(mv[2], mv[3]),
@@ -488,7 +564,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             tc::mbar_arrive(ops_ready);
 
             // ---- (D) epilogue: out = (Ydiag + f Yoff + D u) SiLU(z)
-            tc::mbar_wait(mma_done, c & 1, s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(mma_done, q & 1, s_abort, p.status, kStatusTimeout);
             tc::tc_fence_after();
             {
                 const int t = r16;
@@ -508,12 +584,35 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     uint32_t ow[4];
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
-                        const int j = hh * 8 + e * 2;
-                        const float y0 = fmaf(f, __uint_as_float(ro[j]), __uint_as_float(ry[j])) + Dh * bf_lo(xw[e]);
-                        const float y1 = fmaf(f, __uint_as_float(ro[j + 1]), __uint_as_float(ry[j + 1])) + Dh * bf_hi(xw[e]);
+                        const int jj = hh * 8 + e * 2;
+                        const float y0 = fmaf(f, __uint_as_float(ro[jj]), __uint_as_float(ry[jj])) + Dh * bf_lo(xw[e]);
+                        const float y1 = fmaf(f, __uint_as_float(ro[jj + 1]), __uint_as_float(ry[jj + 1])) + Dh * bf_hi(xw[e]);
                         ow[e] = pack_bf16(y0 * silu_t(bf_lo(zw[e])), y1 * silu_t(bf_hi(zw[e])));
                     }
                     *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, col)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+            }
+            // ---- leaving the segment: h_out = k_c h_c + S_c -> the next segment or the caller
+            if (it.last()) {
+                uint32_t r[HR];
+                load_S(r);
+                const bool drop = carry_prev == kChunkReset;
+                const bool stream_end = it.c == nc - 1;
+                float* dst = stream_end ? (p.final_ssm ? p.final_ssm + str * 64 * NS : nullptr)
+                                        : p.hseg + (str * p.nseg + it.k) * 64 * NS;
+                if (dst != nullptr) {
+#pragma unroll
+                    for (int jj = 0; jj < HR; jj++)
+                        dst[(int64_t)(pcol + jj) * NS + nrow] =
+                            (drop ? 0.0f : carry_prev * hs[jj]) + __uint_as_float(r[jj]);
+                }
+                if (!stream_end) {
+                    bar_compute();
+                    if (tid == 0) {
+                        __threadfence();
+                        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + str * p.nseg + it.k),
+                                     "r"(p.epoch) : "memory");
+                    }
                 }
             }
             tc::fence_async_smem();
@@ -524,26 +623,6 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 tc::mbar_arrive(&empty[s]);
             }
             if (aborted) break;
-        }
-
-        // ---- final state: h_L = k_last h + S_last  ->  (b, h, p, n)
-        if (p.final_ssm != nullptr && !*s_abort && nc > 0) {
-            uint32_t r[HR];
-            if (NS == 128) {
-                tc::tmem_ld16(tmem + lane_base + kColS + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                tc::tmem_ld16(tmem + lane_base + kColS + half * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16 % HR]));
-            } else {
-                tc::tmem_ld16_x2_32(tmem + lane_base + kColS + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-            }
-            tc::tmem_wait_ld();
-            const bool drop = carry_prev == kChunkReset;
-            float* fs = p.final_ssm + bh * 64 * NS;
-            const int n = NS == 128 ? 32 * sub + lane : r16;
-#pragma unroll
-            for (int j = 0; j < HR; j++) {
-                const int pcol = NS == 128 ? half * 32 + j : c16 + j;
-                fs[(int64_t)pcol * NS + n] = (drop ? 0.0f : carry_prev * hs[j]) + __uint_as_float(r[j]);
-            }
         }
         if (tid == 0) tc::bulk_wait0();
     }
@@ -594,20 +673,63 @@ static bool encode_tile_map(CUtensorMap* m, const void* base, int width, int seq
 
 bool fused_path_available() { return tensor_map_encoder() != nullptr; }
 
+size_t fused_flag_count(int max_streams, int sm_count)
+{
+    return (size_t)kItemsPerSm * sm_count + max_streams;
+}
+size_t fused_handoff_floats(int max_streams, int dstate, int sm_count)
+{
+    return fused_flag_count(max_streams, sm_count) * 64 * dstate;
+}
+
+// Segments per stream: the count that minimises the makespan in chunk steps
+// within the hand-off buffers' capacity.  Items run in rounds of `grid`, but
+// the segments of one stream follow each other, so the makespan is at least
+// (segments) x (chunks per segment) as well; each step of a segment adds a
+// small hand-off cost.
+static void choose_segments(int streams, int nchunks, int grid, size_t cap_items, int& nseg, int& cps)
+{
+    double best = 1e300;
+    nseg = 1;
+    cps = nchunks;
+    for (int sg = 1; sg <= nchunks && sg <= 64; sg++) {
+        const int c = (nchunks + sg - 1) / sg;
+        const int se = (nchunks + c - 1) / c;
+        const size_t items = (size_t)streams * se;
+        if (items > cap_items && se > 1) break;
+        const double rounds = (double)((items + grid - 1) / grid);
+        const double cost = (rounds > se ? rounds : (double)se) * (c + 0.5);
+        if (cost < best - 1e-9) {
+            best = cost;
+            nseg = se;
+            cps = c;
+        }
+    }
+}
+
 template <int NS, bool CONV>
-static cudaError_t launch_t(const Shape& s, const FusedParams& fp, const CUtensorMap* maps,
+static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* maps, int sm_count,
                             cudaStream_t st)
 {
     auto kern = ssd_chunk_fused<NS, CONV>;
     const int smem = Layout<NS>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<s.batch * s.nheads, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], fp);
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int streams = s.batch * s.nheads, nc = s.nchunks();
+    int grid = sm_count * per_sm;                 // every CTA resident: hand-off waits end
+    choose_segments(streams, nc, grid, fused_flag_count(streams, sm_count), fp.nseg, fp.cps);
+    fp.nitems = streams * fp.nseg;
+    if (grid > fp.nitems) grid = fp.nitems;
+    kern<<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], fp);
     return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc, const float* dt,
-                               const float* acs, int* status, cudaStream_t st)
+                               const float* acs, int* status, const FusedWork& fw, cudaStream_t st)
 {
     if (!s.act_bf16 || s.headdim != 64 || (s.dstate != 64 && s.dstate != 128) || s.bc_norm)
         return cudaErrorNotSupported;
@@ -629,19 +751,25 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.seqlen = s.seqlen;
     fp.nheads = s.nheads;
     fp.ngroups = s.ngroups;
+    fp.epoch = fw.epoch;
     fp.dt = dt;
     fp.acs = acs;
     fp.seq = a.seq_idx;
     fp.D = a.D;
+    fp.x = (const bf16*)a.x;
     fp.conv_w = (const bf16*)a.conv_w;
     fp.conv_b = (const bf16*)a.conv_b;
     fp.init_conv = (const bf16*)a.init_conv;
     fp.init_ssm = a.init_ssm;
     fp.final_ssm = a.final_ssm;
+    fp.hseg = fw.hseg;
+    fp.flags = fw.flags;
     fp.status = status;
     if (s.dstate == 64)
-        return s.dconv == 4 ? launch_t<64, true>(s, fp, maps, st) : launch_t<64, false>(s, fp, maps, st);
-    return s.dconv == 4 ? launch_t<128, true>(s, fp, maps, st) : launch_t<128, false>(s, fp, maps, st);
+        return s.dconv == 4 ? launch_t<64, true>(s, fp, maps, fw.sm_count, st)
+                            : launch_t<64, false>(s, fp, maps, fw.sm_count, st);
+    return s.dconv == 4 ? launch_t<128, true>(s, fp, maps, fw.sm_count, st)
+                        : launch_t<128, false>(s, fp, maps, fw.sm_count, st);
 }
 
 }  // namespace ssd

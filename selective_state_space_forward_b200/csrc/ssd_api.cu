@@ -60,6 +60,7 @@ struct ssd_handle {
     const float *bn_w, *cn_w, *bn_bias, *cn_bias;
     cudaEvent_t ev_start, ev_stop;   // measurement hook (caller-owned), or null
     uint64_t launches;               // kernels launched since ssd_create
+    FusedWork fw;                    // fused path: segment hand-off buffers, epoch, SM count
 };
 
 namespace {
@@ -259,12 +260,25 @@ ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
         o_st = take((size_t)dd.max_batch * nc * H * P * N * sizeof(float));
     }
     if (path == SSD_PATH_FUSED && dd.dconv == 4) o_ubc = take(BL * 2 * G * N * 2);
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms < 1) sms = 1;
+    size_t o_hseg = 0, o_flags = 0, flag_bytes = 0;
+    if (path == SSD_PATH_FUSED) {
+        const int streams = dd.max_batch * dd.nheads;
+        o_hseg = take(fused_handoff_floats(streams, dd.dstate, sms) * sizeof(float));
+        flag_bytes = fused_flag_count(streams, sms) * sizeof(unsigned);
+        o_flags = take(flag_bytes);
+    }
     o_status = take(256);
 
     ssd_handle* h = new ssd_handle();
     h->d = dd;
     h->path = path;
-    cudaGetDevice(&h->device);
+    h->device = dev;
+    h->fw.sm_count = sms;
+    h->fw.epoch = 0;
     cudaError_t e = cudaMalloc(&h->ws, off);
     if (e != cudaSuccess) {
         delete h;
@@ -278,7 +292,10 @@ ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
     h->states = path == SSD_PATH_STAGED ? (float*)(h->ws + o_st) : nullptr;
     h->ubc = (path == SSD_PATH_FUSED && dd.dconv == 4) ? (void*)(h->ws + o_ubc) : nullptr;
     h->status = (int*)(h->ws + o_status);
+    h->fw.hseg = path == SSD_PATH_FUSED ? (float*)(h->ws + o_hseg) : nullptr;
+    h->fw.flags = path == SSD_PATH_FUSED ? (unsigned*)(h->ws + o_flags) : nullptr;
     e = cudaMemset(h->status, 0, 256);
+    if (e == cudaSuccess && flag_bytes) e = cudaMemset(h->fw.flags, 0, flag_bytes);
     if (e != cudaSuccess) {
         cudaFree(h->ws);
         delete h;
@@ -379,7 +396,8 @@ ssd_status ssd_forward(ssd_handle* h, int32_t batch, int32_t seqlen, const void*
     } else {
         if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_bc(s, a, h->ubc, st), "B|C conv kernel");
         SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, nullptr, st), "dt/cumsum kernel");
-        SSD_MAIN_LAUNCH(h, st, launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->status, st),
+        if (++h->fw.epoch == 0) h->fw.epoch = 1;      // flags hold the last call's epoch
+        SSD_MAIN_LAUNCH(h, st, launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->status, h->fw, st),
                         "fused chunk kernel");
     }
     if (a.final_conv) SSD_LAUNCH(h, launch_conv_state(s, a, st), "conv-state kernel");

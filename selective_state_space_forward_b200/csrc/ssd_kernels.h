@@ -62,10 +62,20 @@ cudaError_t launch_chunk_output(const Shape& s, const FwdArgs& a, const float* u
                                 cudaStream_t st);
 size_t chunk_output_smem_bytes(const Shape& s);
 size_t chunk_state_smem_bytes(const Shape& s);
-// KF: the fused chunk sweep (one CTA per row and head; state kept on chip).
+// KF: the fused chunk sweep (persistent; segments of a stream hand their
+// leaving state to the next segment through `hseg`, tagged in `flags` with
+// the call's epoch).
+struct FusedWork {
+    float* hseg;        // fused_handoff_floats(...) floats
+    unsigned* flags;    // fused_flag_count(...) words, zero at creation
+    unsigned epoch;     // distinct per call (never 0)
+    int sm_count;
+};
 bool fused_path_available();
+size_t fused_handoff_floats(int max_streams, int dstate, int sm_count);
+size_t fused_flag_count(int max_streams, int sm_count);
 cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc, const float* dt,
-                               const float* acs, int* status, cudaStream_t st);
+                               const float* acs, int* status, const FusedWork& fw, cudaStream_t st);
 // K6: one decode token per row, state updated in place.
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
                                cudaStream_t st);
