@@ -102,8 +102,8 @@ struct Layout {
     static constexpr int kHt = kXb + kTile;                   // h^T, NS rows x 128 B
     static constexpr int kScal = kHt + NS * 128;              // ChunkScalars[2]
     static constexpr int kHalo = kScal + 2 * (int)sizeof(ChunkScalars);   // u32 [2][3][32]
-    static constexpr int kBar = kHalo + 2 * 3 * 32 * 4;       // 8 mbarriers
-    static constexpr int kMisc = kBar + 8 * 8;                // tmem base, abort flag
+    static constexpr int kBar = kHalo + 2 * 3 * 32 * 4;       // 9 mbarriers (+1 spare)
+    static constexpr int kMisc = kBar + 10 * 8;               // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
 };
@@ -178,15 +178,18 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_out, FusedParams p)
 {
     using LY = Layout<NS>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base, derived from the shared array by pointer
+    // arithmetic so that every access through it compiles to ld/st.shared
+    uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     ChunkScalars* scal = (ChunkScalars*)(sm + LY::kScal);
     uint32_t* s_halo = (uint32_t*)(sm + LY::kHalo);
     uint64_t* bar = (uint64_t*)(sm + LY::kBar);
     uint64_t* full = bar;           // [2]
     uint64_t* empty = bar + 2;      // [2]
     uint64_t* cb_done = bar + 4;
-    uint64_t* ops_ready = bar + 5;
+    uint64_t* xready = bar + 5;     // conv tiles and h^T written
+    uint64_t* mready = bar + 8;     // mask operand written
     uint64_t* mma_done = bar + 6;
     uint64_t* drain = bar + 7;
     uint32_t* s_tmem = (uint32_t*)(sm + LY::kMisc);
@@ -202,7 +205,8 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             tc::mbar_init(&empty[i], 1);
         }
         tc::mbar_init(cb_done, 1);
-        tc::mbar_init(ops_ready, kComputeThreads);
+        tc::mbar_init(xready, kComputeThreads);
+        tc::mbar_init(mready, kComputeThreads);
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(drain, 1);
         *s_abort = 0;
@@ -321,13 +325,9 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                  tc::sdesc_sw128(a_b + off, 16, 1024), id_64, kk > 0);
                 }
                 tc::mma_commit(cb_done);
-                if (!tc::mbar_wait(ops_ready, q & 1, s_abort, p.status, kStatusTimeout)) break;
+                // the conv tiles and h^T are ready: Yoff and the chunk state need no mask
+                if (!tc::mbar_wait(xready, q & 1, s_abort, p.status, kStatusTimeout)) break;
                 tc::tc_fence_after();
-                // Ydiag = M Xd (K = s)
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++)
-                    tc::mma_bf16(tmem + kColY, tc::sdesc_sw128(a_mop + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(a_xd + kk * 32, 16, 1024), id_64, kk > 0);
                 // Yoff = C h^T (K = n; h^T is MN-major: rows n, 64 p per row)
 #pragma unroll
                 for (int kk = 0; kk < NS / 16; kk++) {
@@ -340,6 +340,13 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 for (int kk = 0; kk < 4; kk++)
                     tc::mma_bf16(tmem + kColS, tc::sdesc_sw128(a_b + kk * 2048, kTile, 1024),
                                  tc::sdesc_sw128(a_xs + kk * 32, 16, 1024), id_st, kk > 0);
+                if (!tc::mbar_wait(mready, q & 1, s_abort, p.status, kStatusTimeout)) break;
+                tc::tc_fence_after();
+                // Ydiag = M Xd (K = s)
+#pragma unroll
+                for (int kk = 0; kk < 4; kk++)
+                    tc::mma_bf16(tmem + kColY, tc::sdesc_sw128(a_mop + kk * 32, 16, 1024),
+                                 tc::sdesc_sw128(a_xd + kk * 32, 16, 1024), id_64, kk > 0);
                 tc::mma_commit(mma_done);
             }
         }
@@ -527,6 +534,11 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     *(uint4*)(sm + LY::kXs + tc::sw128_offset(2 * pp + e, r0)) = vs;
                 }
             }
+            // h^T and the conv tiles are written (and S of the last chunk read out of
+            // TMEM): Yoff and the chunk-state MMAs may start before the mask is done
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::mbar_arrive(xready);
 
             // ---- (C) mask: M[t][s] from the C B^T accumulator
             if (tid == 0) tc::bulk_wait_read0();     // the previous out tile has left shared memory
@@ -544,12 +556,27 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     for (int jj = 0; jj < 16; jj++) mv[jj] = 0.f;
                 } else {
                     const float at = cs->a2[t];
-                    const int segt = cs->seg[t];
+                    float as[16];
 #pragma unroll
-                    for (int jj = 0; jj < 16; jj++) {
-                        const int sidx = c16 + jj;
-                        const bool keep = sidx <= t && (quiet || cs->seg[sidx] == segt);
-                        mv[jj] = keep ? __uint_as_float(r[jj]) * ex2(at - cs->a2[sidx]) : 0.f;
+                    for (int j4 = 0; j4 < 4; j4++) {
+                        const float4 v = *reinterpret_cast<const float4*>(cs->a2 + c16 + 4 * j4);
+                        as[4 * j4] = v.x; as[4 * j4 + 1] = v.y; as[4 * j4 + 2] = v.z; as[4 * j4 + 3] = v.w;
+                    }
+                    // `quiet` is uniform over the block: two loop bodies, no per-element test
+                    if (quiet) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; jj++)
+                            mv[jj] = c16 + jj <= t ? __uint_as_float(r[jj]) * ex2(at - as[jj]) : 0.f;
+                    } else {
+                        const uint4 sv = *reinterpret_cast<const uint4*>(cs->seg + c16);
+                        const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+                        const uint32_t segt = cs->seg[t];
+#pragma unroll
+                        for (int jj = 0; jj < 16; jj++) {
+                            const uint32_t sj = (sw[jj >> 2] >> (8 * (jj & 3))) & 0xFFu;
+                            const bool keep = c16 + jj <= t && sj == segt;
+                            mv[jj] = keep ? __uint_as_float(r[jj]) * ex2(at - as[jj]) : 0.f;
+                        }
                     }
                 }
                 const uint4 lo = make_uint4(pack_bf16(mv[0], mv[1]), pack_bf16(mv[2], mv[3]),
@@ -561,7 +588,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
-            tc::mbar_arrive(ops_ready);
+            tc::mbar_arrive(mready);
 
             // ---- (D) epilogue: out = (Ydiag + f Yoff + D u) SiLU(z)
             tc::mbar_wait(mma_done, q & 1, s_abort, p.status, kStatusTimeout);
