@@ -190,6 +190,50 @@ uint64_t ssd_launch_count(const ssd_handle* h);
  * SSD_ERR_CUDA when the stream itself failed. */
 ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream);
 
+/*
+ * Allocation-free forward.  The method's pages have no counterpart to this
+ * entry point: it computes what ssd_forward computes on the FUSED path (same
+ * kernels, same arguments, same results), for callers that cannot allocate
+ * device memory and so cannot create a handle -- code that runs under a
+ * device-memory budget owned by someone else (a server that pre-sizes one
+ * pool for its whole life and refuses later cudaMalloc calls), and code on a
+ * latency-bound loop that cannot afford the device-wide synchronisation a
+ * cudaFree implies.
+ *
+ * Scratch: a static device array of 64 MiB per device that belongs to the
+ * loaded library (no cudaMalloc, cudaFree or allocating library call is
+ * made).  It holds 4 KiB of hand-off flags, then the segment hand-off states
+ * (64 * dstate fp32 per slot; at least one slot per (row, head) stream, at
+ * most 1024 slots), dt and the chunk cumsum ((batch, H, seqlen) fp32 each)
+ * and, when dconv = 4, the convolved B|C ((batch, seqlen, 2*G*N) bf16).
+ * A shape with more than 1024 streams (batch * H) or whose buffers exceed
+ * the 64 MiB returns SSD_ERR_SHAPE_EXCEEDS_MAX before any launch; for H = 32,
+ * G = 8, N = 64 that is about 28,000 tokens (batch * seqlen).
+ *
+ *   d           as for ssd_create; the shape must suit the FUSED path (bf16
+ *               activations, headdim 64, dstate 64 or 128, bc_norm 0; path
+ *               AUTO or FUSED, else SSD_ERR_UNSUPPORTED), and batch / seqlen
+ *               must respect max_batch / max_seqlen as with a handle.
+ *   x .. final_state, stream: as for ssd_forward.
+ *   status      device pointer to one int32 that the caller owns (required);
+ *               the kernels OR into it the bits ssd_check reports (1: a bounded
+ *               wait timed out and the outputs are invalid; 2: a kernel rejected
+ *               its launch shape).  This call neither reads nor clears it.
+ *
+ * The first call on each device does a one-time set-up with that device
+ * current: it looks up the array's device address (cudaGetSymbolAddress) and
+ * clears the flag words on `stream`.  Make that first call before any stream
+ * capture.  Every call on a device uses the same array, so calls that
+ * overlap on the GPU (on different streams without an ordering between
+ * them) race; calls on one stream, or ordered by events, do not.
+ */
+ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
+                               const void* x, const void* z, const float* dt_raw,
+                               const float* dt_bias, const float* A, const void* B, const void* C,
+                               const float* D, const void* conv_w, const void* conv_b,
+                               const int32_t* seq_idx, const void* init_state, void* out,
+                               void* final_state, int32_t* status, struct CUstream_st* stream);
+
 /* The calling thread's last error message ("" when none). */
 const char* ssd_last_error(void);
 

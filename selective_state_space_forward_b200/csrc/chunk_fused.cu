@@ -736,7 +736,7 @@ static void choose_segments(int streams, int nchunks, int grid, size_t cap_items
 
 template <int NS, bool CONV>
 static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* maps, int sm_count,
-                            cudaStream_t st)
+                            size_t max_items, cudaStream_t st)
 {
     auto kern = ssd_chunk_fused<NS, CONV>;
     const int smem = Layout<NS>::kAlloc;
@@ -748,7 +748,9 @@ static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* m
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int streams = s.batch * s.nheads, nc = s.nchunks();
     int grid = sm_count * per_sm;                 // every CTA resident: hand-off waits end
-    choose_segments(streams, nc, grid, fused_flag_count(streams, sm_count), fp.nseg, fp.cps);
+    const size_t cap = max_items ? max_items : fused_flag_count(streams, sm_count);
+    if (cap < (size_t)streams) return cudaErrorInvalidValue;
+    choose_segments(streams, nc, grid, cap, fp.nseg, fp.cps);
     fp.nitems = streams * fp.nseg;
     if (grid > fp.nitems) grid = fp.nitems;
     kern<<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], fp);
@@ -793,10 +795,10 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.flags = fw.flags;
     fp.status = status;
     if (s.dstate == 64)
-        return s.dconv == 4 ? launch_t<64, true>(s, fp, maps, fw.sm_count, st)
-                            : launch_t<64, false>(s, fp, maps, fw.sm_count, st);
-    return s.dconv == 4 ? launch_t<128, true>(s, fp, maps, fw.sm_count, st)
-                        : launch_t<128, false>(s, fp, maps, fw.sm_count, st);
+        return s.dconv == 4 ? launch_t<64, true>(s, fp, maps, fw.sm_count, fw.max_items, st)
+                            : launch_t<64, false>(s, fp, maps, fw.sm_count, fw.max_items, st);
+    return s.dconv == 4 ? launch_t<128, true>(s, fp, maps, fw.sm_count, fw.max_items, st)
+                        : launch_t<128, false>(s, fp, maps, fw.sm_count, fw.max_items, st);
 }
 
 }  // namespace ssd

@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "ssd.h"
@@ -200,6 +201,61 @@ ssd_status check_common(const ssd_handle* h, const void* x, const void* z, const
     }
     if (out == x || out == z || out == B || out == C)
         return fail(SSD_ERR_INVALID_ARG, "out may not alias an input");
+    return SSD_OK;
+}
+
+// ---- scratch of ssd_forward_noalloc --------------------------------------------
+// Callers that cannot allocate device memory (a fixed budget owned by someone
+// else, or a loop that cannot take cudaFree's device-wide synchronisation)
+// cannot create a handle; their forward keeps its workspace in a static device
+// array of this module instead.  Layout: the hand-off flags at the head (a
+// fixed place, so a flag word only ever holds an epoch), then per call the
+// hand-off states, dt, the cumsum and the convolved B|C.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;   // per device
+constexpr size_t kNoAllocMaxItems = 1024;                    // hand-off slots at most
+constexpr size_t kNoAllocFlagBytes = kNoAllocMaxItems * sizeof(unsigned);
+constexpr int kNoAllocMaxDevices = 64;
+static_assert(kNoAllocFlagBytes % 256 == 0, "the hand-off states start 256-byte aligned");
+
+struct NoAllocDevice {
+    unsigned char* base = nullptr;   // device address of the scratch array on this device
+    int sm_count = 0;
+    unsigned epoch = 0;              // the last epoch handed to a call on this device
+};
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+}  // namespace
+
+// Zero when the module loads; the flag words are cleared once more at set-up.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// The current device's scratch, with a fresh epoch for this call.  The first
+// call on a device (with that device current) looks the array's address up
+// and clears its flag words on `st`, ahead of the call's kernels.
+ssd_status noalloc_device(cudaStream_t st, NoAllocDevice& out)
+{
+    int dev = 0;
+    SSD_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return fail(SSD_ERR_UNSUPPORTED, "ssd_forward_noalloc serves devices 0 .. %d (current %d)",
+                    kNoAllocMaxDevices - 1, dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoAllocDevice& d = g_noalloc_dev[dev];
+    if (!d.base) {
+        void* p = nullptr;
+        SSD_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+        int sms = 0;
+        SSD_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev),
+                 "cudaDeviceGetAttribute(SM count)");
+        SSD_CUDA(cudaMemsetAsync(p, 0, kNoAllocFlagBytes, st), "scratch flag clear");
+        d.base = (unsigned char*)p;
+        d.sm_count = sms < 1 ? 1 : sms;
+    }
+    if (++d.epoch == 0) d.epoch = 1;   // flags hold earlier calls' epochs, never this one
+    out = d;
     return SSD_OK;
 }
 
@@ -501,6 +557,97 @@ ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream)
     return fail(SSD_ERR_DEVICE, "device status 0x%x:%s%s", word,
                 (word & kStatusTimeout) ? " a bounded wait timed out;" : "",
                 (word & kStatusBadLaunch) ? " a kernel rejected its launch shape;" : "");
+}
+
+ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen, const void* x,
+                               const void* z, const float* dt_raw, const float* dt_bias,
+                               const float* A, const void* B, const void* C, const float* D,
+                               const void* conv_w, const void* conv_b, const int32_t* seq_idx,
+                               const void* init_state, void* out, void* final_state,
+                               int32_t* status, struct CUstream_st* stream)
+{
+    g_err.clear();
+    SSD_TRY(validate_desc(d));
+    if (d->path == SSD_PATH_STAGED || !fused_supported(*d))
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "ssd_forward_noalloc runs the fused path only: bf16 activations, headdim 64, "
+                    "dstate 64 or 128, no B/C norm");
+    ssd_handle h{};   // holds the descriptor for the shared checks; owns no memory
+    h.d = *d;
+    h.d.chunk = 64;
+    h.d.path = SSD_PATH_FUSED;
+    h.path = SSD_PATH_FUSED;
+    SSD_TRY(check_handle_dims(&h, batch, seqlen));
+    SSD_TRY(check_ptr(status, "status", 4, true));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (batch == 0) return SSD_OK;
+    SSD_TRY(check_ptr(init_state, "init_state", 16, false));
+    SSD_TRY(check_ptr(final_state, "final_state", 16, false));
+    if (seqlen == 0) {   // no token: the state passes through unchanged
+        if (final_state && final_state != init_state) {
+            const size_t n = ssd_state_bytes(&h, batch);
+            SSD_CUDA(init_state ? cudaMemcpyAsync(final_state, init_state, n,
+                                                  cudaMemcpyDeviceToDevice, st)
+                                : cudaMemsetAsync(final_state, 0, n, st),
+                     "empty-sequence state copy");
+        }
+        return SSD_OK;
+    }
+    SSD_TRY(check_common(&h, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, out));
+    SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
+    if (out == init_state || out == final_state)
+        return fail(SSD_ERR_INVALID_ARG, "out may not alias a state buffer");
+
+    // Scratch plan: the token buffers first, then as many hand-off slots as
+    // the rest holds (at least one per stream, at most kNoAllocMaxItems).
+    const size_t H = h.d.nheads, N = h.d.dstate, G = h.d.ngroups;
+    const size_t streams = (size_t)batch * H;
+    const size_t slot = 64 * N * sizeof(float);
+    const size_t dt_bytes = align256((size_t)batch * H * seqlen * sizeof(float));
+    const size_t ubc_bytes = h.d.dconv == 4 ? align256((size_t)batch * seqlen * 2 * G * N * 2) : 0;
+    const size_t fixed = kNoAllocFlagBytes + 2 * dt_bytes + ubc_bytes;
+    if (streams > kNoAllocMaxItems || fixed + streams * slot > kNoAllocScratchBytes)
+        return fail(SSD_ERR_SHAPE_EXCEEDS_MAX,
+                    "batch %d x seqlen %d needs %zu bytes of scratch for %zu (row, head) streams; "
+                    "ssd_forward_noalloc's static scratch holds %zu bytes and %zu streams",
+                    batch, seqlen, fixed + streams * slot, streams, kNoAllocScratchBytes,
+                    kNoAllocMaxItems);
+    size_t items = (kNoAllocScratchBytes - fixed) / slot;
+    if (items > kNoAllocMaxItems) items = kNoAllocMaxItems;
+
+    NoAllocDevice dev;
+    SSD_TRY(noalloc_device(st, dev));
+    unsigned char* p = dev.base;
+    FusedWork fw;
+    fw.flags = (unsigned*)p;
+    fw.hseg = (float*)(p + kNoAllocFlagBytes);
+    fw.epoch = dev.epoch;
+    fw.sm_count = dev.sm_count;
+    fw.max_items = items;
+    size_t off = kNoAllocFlagBytes + items * slot;   // slot is a multiple of 256 bytes
+    float* dt = (float*)(p + off);
+    off += dt_bytes;
+    float* acs = (float*)(p + off);
+    off += dt_bytes;
+    void* ubc = h.d.dconv == 4 ? (void*)(p + off) : nullptr;
+
+    const Shape s = make_shape(&h, batch, seqlen);
+    FwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
+    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
+    a.init_ssm = (const float*)init_state;
+    a.init_conv = (init_state && s.dconv == 4) ? (const char*)init_state + conv_offset(h.d, batch)
+                                               : nullptr;
+    a.out = out;
+    a.final_ssm = (float*)final_state;
+    a.final_conv = (final_state && s.dconv == 4) ? (char*)final_state + conv_offset(h.d, batch)
+                                                 : nullptr;
+    if (s.dconv == 4) SSD_LAUNCH(&h, launch_conv_silu_bc(s, a, ubc, st), "B|C conv kernel");
+    SSD_LAUNCH(&h, launch_dt_cumsum(s, a, dt, acs, nullptr, st), "dt/cumsum kernel");
+    SSD_LAUNCH(&h, launch_chunk_fused(s, a, ubc, dt, acs, status, fw, st), "fused chunk kernel");
+    if (a.final_conv) SSD_LAUNCH(&h, launch_conv_state(s, a, st), "conv-state kernel");
+    return SSD_OK;
 }
 
 }  // extern "C"

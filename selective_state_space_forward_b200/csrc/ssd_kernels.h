@@ -70,6 +70,7 @@ struct FusedWork {
     unsigned* flags;    // fused_flag_count(...) words, zero at creation
     unsigned epoch;     // distinct per call (never 0)
     int sm_count;
+    size_t max_items;   // hand-off slots in hseg/flags; 0: fused_flag_count(streams, sm_count)
 };
 bool fused_path_available();
 size_t fused_handoff_floats(int max_streams, int dstate, int sm_count);

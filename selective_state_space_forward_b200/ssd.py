@@ -31,7 +31,7 @@ DTYPES = {"f32": (0, torch.float32), "bf16": (1, torch.bfloat16)}
 EXPORTS = ("ssd_create", "ssd_destroy", "ssd_get_path", "ssd_set_bc_norm", "ssd_state_bytes",
            "ssd_state_conv_offset", "ssd_forward", "ssd_step", "ssd_stage_conv", "ssd_stage_dt",
            "ssd_set_timing_events", "ssd_launch_count", "ssd_check", "ssd_last_error",
-           "ssd_status_string")
+           "ssd_status_string", "ssd_forward_noalloc")
 
 
 class SSDError(RuntimeError):
@@ -81,8 +81,9 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_last_error.restype = ctypes.c_char_p
     lib.ssd_status_string.argtypes = [ctypes.c_int]
     lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), i32, i32] + [vp] * 15 + [vp]
     for f in ("ssd_create", "ssd_set_bc_norm", "ssd_forward", "ssd_step", "ssd_stage_conv",
-              "ssd_stage_dt", "ssd_set_timing_events", "ssd_check"):
+              "ssd_stage_dt", "ssd_set_timing_events", "ssd_check", "ssd_forward_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -246,3 +247,31 @@ class Handle:
 
     def check(self, stream=None):
         _raise(self.lib, self.lib.ssd_check(self._h, _stream(stream)))
+
+
+def forward_noalloc(x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None, seq_idx=None,
+                    init_state=None, out=None, final_state=None, *, status, nheads, headdim,
+                    dstate, ngroups=1, dconv=4, max_batch=None, max_seqlen=None, path="auto",
+                    stream=None, lib=None):
+    """ssd_forward_noalloc: the fused forward with no handle and no device allocation by the
+    library (its scratch is a static device array).  `status` is a one-element int32 CUDA
+    tensor the kernels OR error bits into; `out` and the state buffers are laid out as for
+    Handle.forward.  Returns `out` (allocated like x when not given)."""
+    lib = lib or load_library()
+    at, f = torch.bfloat16, torch.float32
+    batch, seqlen = (x.shape[0], x.shape[1]) if x.dim() == 3 else (0, 0)
+    d = Desc(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv,
+             chunk=64, act_dtype=DTYPES["bf16"][0], a_mode=0, bc_norm=0,
+             max_batch=max_batch or max(batch, 1), max_seqlen=max_seqlen or max(seqlen, 1),
+             path=PATHS[path])
+    if out is None:
+        out = torch.empty_like(x)
+    _raise(lib, lib.ssd_forward_noalloc(
+        ctypes.byref(d), batch, seqlen, _ptr(x, at, "x"), _ptr(z, at, "z"),
+        _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"), _ptr(A, f, "A"),
+        _ptr(B, at, "B"), _ptr(C, at, "C"), _ptr(D, f, "D"), _ptr(conv_w, at, "conv_w"),
+        _ptr(conv_b, at, "conv_b"), _ptr(seq_idx, torch.int32, "seq_idx"),
+        _ptr(init_state, torch.uint8, "init_state"), _ptr(out, at, "out"),
+        _ptr(final_state, torch.uint8, "final_state"), _ptr(status, torch.int32, "status"),
+        _stream(stream)))
+    return out
