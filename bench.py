@@ -353,6 +353,8 @@ def bench_decode(args, torch, peaks):
     h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"],
               dev["D"], dev["conv_w"], dev["conv_b"], final_state=state)
     del dev["x"], dev["z"], dev["B"], dev["C"], dev["dt_raw"]
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()      # the prefill's inputs are not needed by the steps
     steps_in = []
     for i in range(8):
         si = make_step_inputs(w, i)

@@ -26,19 +26,24 @@
 // started earlier and the wait ends.  This keeps every SM busy to within one
 // item whatever the number of streams, and lets two CTAs share each SM.
 //
-// Roles (320 threads): warps 0-7 compute (state update, conv, masks,
-// epilogue; warp w reaches TMEM lanes 32*(w%4) .. +31 and takes the column
-// half w/4), warp 8 produces (TMA tile loads into a 2-stage ring plus the
-// chunk's per-token scalars: dt, decay weights, segment ids, carry), warp 9
-// issues the MMAs from one thread.  Every wait is bounded: after 1 s a waiter
-// raises the CTA's abort flag and the device status word, and all roles
-// drain and exit.
+// Roles (544 threads).  The work of a chunk splits in two: what does not
+// depend on the carried state (conv, operand tiles, C B^T, mask, Ydiag, the
+// chunk state S) and what does (the state update, Yoff, the epilogue).
+// Group A (warps 0-7) does the first part and its thread 0 issues those MMAs;
+// group B (warps 8-15) does the second, its thread 0 issuing Yoff and the TMA
+// store.  Operand tiles, Ydiag and S are double-buffered, so group A works on
+// chunk c+1 while group B finishes chunk c; warp 16 feeds both from a TMA
+// ring (tiles plus the chunk's per-token scalars).  A warp reaches TMEM lanes
+// 32*(w%4) .. +31.  Every wait is bounded: after 1 s a waiter raises the
+// CTA's abort flag and the device status word, and all roles drain and exit.
 //
 // Tile layouts (see tc05.cuh): x, z, B, C, out tiles are [64 tokens][64
 // channels] bf16 with the 128-byte swizzle, as TMA writes them; N = 128
 // operands are two such tiles side by side.  M=64 accumulators put row r in
 // TMEM lane 32*(r/16) + r%16; M=128 ones put row r in lane r.
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
@@ -47,14 +52,15 @@
 namespace ssd {
 namespace {
 
-constexpr int kComputeWarps = 8;
-constexpr int kComputeThreads = 32 * kComputeWarps;
-constexpr int kProducerWarp = kComputeWarps;
-constexpr int kMmaWarp = kComputeWarps + 1;
-constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kGroupWarps = 8;                       // warps per compute group
+constexpr int kGroupThreads = 32 * kGroupWarps;
+constexpr int kProducerWarp = 2 * kGroupWarps;       // after groups A (0-7) and B (8-15)
+constexpr int kThreads = 32 * (2 * kGroupWarps + 1);
+constexpr int kBarA = 1, kBarB = 2;                  // named barriers of the groups
 constexpr int kTile = 64 * 128;        // one [64][64] bf16 tile
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColCB = 0, kColY = 64, kColYO = 128, kColS = 192;
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns: C B^T; Ydiag [2]; Yoff; chunk state S [2]
+constexpr uint32_t kColCB = 0, kColY = 64, kColYO = 192, kColS = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kItemsPerSm = 16;        // bound on work items per SM (sizes the hand-off buffers)
 
@@ -92,37 +98,41 @@ struct ChunkScalars {
 
 template <int NS>
 struct Layout {
+    static constexpr int kStages = NS == 64 ? 3 : 2;          // TMA ring depth
     static constexpr int kBC = (NS / 64) * kTile;
     static constexpr int kStage = 2 * kTile + 2 * kBC;        // x, z, B, C
-    static constexpr int kRing = 2 * kStage;
-    static constexpr int kMop = kRing;                        // mask operand, then the out tile
-    static constexpr int kXd = kMop + kTile;
-    static constexpr int kXs = kXd + kTile;
-    static constexpr int kXb = kXs + kTile;                   // u in bf16, [t][p]
-    static constexpr int kHt = kXb + kTile;                   // h^T, NS rows x 128 B
-    static constexpr int kScal = kHt + NS * 128;              // ChunkScalars[2]
-    static constexpr int kHalo = kScal + 2 * (int)sizeof(ChunkScalars);   // u32 [2][3][32]
-    static constexpr int kBar = kHalo + 2 * 3 * 32 * 4;       // 9 mbarriers (+1 spare)
-    static constexpr int kMisc = kBar + 10 * 8;               // tmem base, abort flag
+    static constexpr int kRing = kStages * kStage;
+    static constexpr int kXb = kRing;                         // [2] u in bf16, [t][p]
+    static constexpr int kXd = kXb + 2 * kTile;               // [2] dt u, [p][t]
+    static constexpr int kXs = kXd + 2 * kTile;               // [2] decayed dt u, [p][t]
+    static constexpr int kMop = kXs + 2 * kTile;              // [2] mask operand, [t][s]
+    static constexpr int kOut = kMop + 2 * kTile;             // [2] out tiles
+    static constexpr int kHt = kOut + 2 * kTile;              // h^T, NS rows x 128 B
+    static constexpr int kScal = kHt + NS * 128;              // ChunkScalars[kStages]
+    static constexpr int kHalo = kScal + kStages * (int)sizeof(ChunkScalars);   // u32 [2][3][32]
+    static constexpr int kBar = kHalo + 2 * 3 * 32 * 4;
+    static constexpr int kNumBars = 2 * kStages + 12;
+    static constexpr int kMisc = kBar + kNumBars * 8;         // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
 };
 
-__device__ __forceinline__ void bar_compute()
+// Named barriers of the two compute groups (barrier 0 is __syncthreads).
+__device__ __forceinline__ void bar_group(int id)
 {
-    asm volatile("bar.sync 1, %0;" ::"n"(kComputeThreads) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kGroupThreads) : "memory");
 }
 
-// Compute-warp barrier that also returns the OR of v over the compute
-// threads, so every one of them takes the same branch afterwards.
-__device__ __forceinline__ int bar_compute_or(int v)
+// Group barrier that also returns the OR of v over the group, so every thread
+// of the group takes the same branch afterwards.
+__device__ __forceinline__ int bar_group_or(int id, int v)
 {
     uint32_t r;
     asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\t"
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(v), "n"(kComputeThreads)
+        : "r"(v), "r"(id), "n"(kGroupThreads)
         : "memory");
     return (int)r;
 }
@@ -171,13 +181,17 @@ struct StepIter {
     }
 };
 
+// Phase parity of the n-th completion (0-based) of a barrier.
+__device__ __forceinline__ uint32_t par(int n) { return (uint32_t)n & 1u; }
+
 template <int NS, bool CONV>
-__global__ void __launch_bounds__(kThreads, NS == 64 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, 1)
 ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
                 const __grid_constant__ CUtensorMap tm_out, FusedParams p)
 {
     using LY = Layout<NS>;
+    constexpr int NST = LY::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base, derived from the shared array by pointer
     // arithmetic so that every access through it compiles to ld/st.shared
@@ -185,13 +199,17 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     ChunkScalars* scal = (ChunkScalars*)(sm + LY::kScal);
     uint32_t* s_halo = (uint32_t*)(sm + LY::kHalo);
     uint64_t* bar = (uint64_t*)(sm + LY::kBar);
-    uint64_t* full = bar;           // [2]
-    uint64_t* empty = bar + 2;      // [2]
-    uint64_t* cb_done = bar + 4;
-    uint64_t* xready = bar + 5;     // conv tiles and h^T written
-    uint64_t* mready = bar + 8;     // mask operand written
-    uint64_t* mma_done = bar + 6;
-    uint64_t* drain = bar + 7;
+    uint64_t* full = bar;                  // [NST] tiles + scalars of a step landed
+    uint64_t* empty = bar + NST;           // [NST] group B released the stage
+    uint64_t* cb_done = bar + 2 * NST;     // C B^T of the next step in TMEM
+    uint64_t* s_done = cb_done + 1;        // [2] chunk state S(q) in TMEM
+    uint64_t* s_free = s_done + 2;         // [2] group B has read S(q)
+    uint64_t* y_done = s_free + 2;         // [2] Ydiag(q) done (with every earlier MMA of group A)
+                                           //     and the step's Xb written
+    uint64_t* yo_done = y_done + 2;        // Yoff(q)
+    uint64_t* epi_done = yo_done + 1;      // [2] group B is done with the step's operands
+    uint64_t* drain_a = epi_done + 2;
+    uint64_t* drain_b = drain_a + 1;
     uint32_t* s_tmem = (uint32_t*)(sm + LY::kMisc);
     volatile int* s_abort = (volatile int*)(sm + LY::kMisc + 4);
 
@@ -200,15 +218,20 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const int nc = (L + 63) / 64;
 
     if (tid == 0) {
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < NST; i++) {
             tc::mbar_init(&full[i], 33);     // producer: expect_tx arrive + 32 lane arrivals
             tc::mbar_init(&empty[i], 1);
         }
         tc::mbar_init(cb_done, 1);
-        tc::mbar_init(xready, kComputeThreads);
-        tc::mbar_init(mready, kComputeThreads);
-        tc::mbar_init(mma_done, 1);
-        tc::mbar_init(drain, 1);
+        tc::mbar_init(yo_done, 1);
+        tc::mbar_init(drain_a, 1);
+        tc::mbar_init(drain_b, 1);
+        for (int i = 0; i < 2; i++) {
+            tc::mbar_init(&s_done[i], 1);
+            tc::mbar_init(&s_free[i], 1);
+            tc::mbar_init(&y_done[i], 2);    // A's release arrive (Xb written) + the MMA commit
+            tc::mbar_init(&epi_done[i], 1);
+        }
         *s_abort = 0;
         tc::fence_mbar_init();
     }
@@ -227,35 +250,37 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    const int sub = warp & 3;                           // TMEM lane quarter of this warp
+    const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
         const uint32_t tx = (uint32_t)(2 * kTile + 2 * LY::kBC);
         int q = 0;
         for (StepIter it(p, nc); it.valid(); it.next(), q++) {
-            const int s = q & 1;
-            if (q >= 2 && !tc::mbar_wait(&empty[s], ((q >> 1) & 1) ^ 1, s_abort, p.status, kStatusTimeout))
+            const int st = q % NST;
+            if (q >= NST && !tc::mbar_wait(&empty[st], par(q / NST - 1), s_abort, p.status, kStatusTimeout))
                 break;
             const int b = it.b, h = it.h, g = h / (H / p.ngroups);
             const int t0 = it.c * 64;
             const int64_t bh = (int64_t)b * H + h;
-            uint8_t* st = sm + s * LY::kStage;
+            uint8_t* stg = sm + st * LY::kStage;
             if (lane == 0) {
-                tc::mbar_arrive_expect_tx(&full[s], tx);
-                tc::tma_load_3d(st, &tm_x, &full[s], h * 64, t0, b);
-                tc::tma_load_3d(st + kTile, &tm_z, &full[s], h * 64, t0, b);
+                tc::mbar_arrive_expect_tx(&full[st], tx);
+                tc::tma_load_3d(stg, &tm_x, &full[st], h * 64, t0, b);
+                tc::tma_load_3d(stg + kTile, &tm_z, &full[st], h * 64, t0, b);
 #pragma unroll
                 for (int jj = 0; jj < NS / 64; jj++) {
                     const int bx = g * NS + 64 * jj;
                     const int cx = (CONV ? p.ngroups * NS : 0) + g * NS + 64 * jj;
-                    tc::tma_load_3d(st + 2 * kTile + jj * kTile, &tm_b, &full[s], bx, t0, b);
-                    tc::tma_load_3d(st + 2 * kTile + LY::kBC + jj * kTile, &tm_c, &full[s], cx, t0, b);
+                    tc::tma_load_3d(stg + 2 * kTile + jj * kTile, &tm_b, &full[st], bx, t0, b);
+                    tc::tma_load_3d(stg + 2 * kTile + LY::kBC + jj * kTile, &tm_c, &full[st], cx, t0, b);
                 }
             }
             const int32_t* seq_row = p.seq ? p.seq + (int64_t)b * L : nullptr;
             const float* dt_row = p.dt + bh * L;
             const float* acs_row = p.acs + bh * L;
-            ChunkScalars* cs = &scal[s];
+            ChunkScalars* cs = &scal[st];
             const int Lc = min(64, L - t0);
             float dtv[2], acv[2];
             int bdv[2];
@@ -295,169 +320,75 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 cs->pre = pre;
             }
             __syncwarp();
-            tc::mbar_arrive(&full[s]);
+            tc::mbar_arrive(&full[st]);
         }
         // an aborting CTA lets its last loads land before the shared memory is released
-        for (int k2 = max(0, q - 2); k2 < q; k2++)
-            tc::mbar_drain(&full[k2 & 1], (k2 >> 1) & 1, p.status, kStatusTimeout);
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            const uint32_t id_64 = tc::idesc_bf16(64, 64, false, false);
-            const uint32_t id_yo = tc::idesc_bf16(64, 64, false, true);
-            const uint32_t id_st = tc::idesc_bf16(NS, 64, true, false);
-            const uint32_t a_mop = tc::smem_u32(sm + LY::kMop);
-            const uint32_t a_xd = tc::smem_u32(sm + LY::kXd);
-            const uint32_t a_xs = tc::smem_u32(sm + LY::kXs);
-            const uint32_t a_ht = tc::smem_u32(sm + LY::kHt);
-            int q = 0;
-            for (StepIter it(p, nc); it.valid(); it.next(), q++) {
-                const int s = q & 1;
-                if (!tc::mbar_wait(&full[s], (q >> 1) & 1, s_abort, p.status, kStatusTimeout)) break;
-                tc::tc_fence_after();
-                const uint32_t a_b = tc::smem_u32(sm + s * LY::kStage + 2 * kTile);
-                const uint32_t a_c = a_b + LY::kBC;
-                // C B^T: both K-major over n
-#pragma unroll
-                for (int kk = 0; kk < NS / 16; kk++) {
-                    const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
-                    tc::mma_bf16(tmem + kColCB, tc::sdesc_sw128(a_c + off, 16, 1024),
-                                 tc::sdesc_sw128(a_b + off, 16, 1024), id_64, kk > 0);
-                }
-                tc::mma_commit(cb_done);
-                // the conv tiles and h^T are ready: Yoff and the chunk state need no mask
-                if (!tc::mbar_wait(xready, q & 1, s_abort, p.status, kStatusTimeout)) break;
-                tc::tc_fence_after();
-                // Yoff = C h^T (K = n; h^T is MN-major: rows n, 64 p per row)
-#pragma unroll
-                for (int kk = 0; kk < NS / 16; kk++) {
-                    const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
-                    tc::mma_bf16(tmem + kColYO, tc::sdesc_sw128(a_c + off, 16, 1024),
-                                 tc::sdesc_sw128(a_ht + kk * 2048, 8192, 1024), id_yo, kk > 0);
-                }
-                // S_c^T[n][p] = B^T Xs (A = the B tile as MN-major over n, K = s)
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++)
-                    tc::mma_bf16(tmem + kColS, tc::sdesc_sw128(a_b + kk * 2048, kTile, 1024),
-                                 tc::sdesc_sw128(a_xs + kk * 32, 16, 1024), id_st, kk > 0);
-                if (!tc::mbar_wait(mready, q & 1, s_abort, p.status, kStatusTimeout)) break;
-                tc::tc_fence_after();
-                // Ydiag = M Xd (K = s)
-#pragma unroll
-                for (int kk = 0; kk < 4; kk++)
-                    tc::mma_bf16(tmem + kColY, tc::sdesc_sw128(a_mop + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(a_xd + kk * 32, 16, 1024), id_64, kk > 0);
-                tc::mma_commit(mma_done);
-            }
-        }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------------------ compute warps 0-7
-        const int cdim = H * 64 + 2 * p.ngroups * NS;
-        const int sub = warp & 3;                  // TMEM lane quarter
+        for (int k2 = max(0, q - NST); k2 < q; k2++)
+            tc::mbar_drain(&full[k2 % NST], par(k2 / NST), p.status, kStatusTimeout);
+    } else if (warp < kGroupWarps) {
+        // ------------------------------------------------------------ group A: conv, mask
+        // Warps 0-7.  Per step: conv -> Xb, Xd, Xs; [thread 0: S = B^T Xs]; mask from
+        // C B^T -> Mop; [thread 0: Ydiag = M Xd, then C B^T of the next step].
         const int half = warp >> 2;                // column half
-        const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
-        // M=64 accumulators: row r16, this thread's 16 columns start at c16
-        const int r16 = 16 * sub + (lane & 15);
+        const int r16 = 16 * sub + (lane & 15);    // M=64 accumulator row of this thread
         const int c16 = half * 16 + (lane < 16 ? 0 : 32);
-        // conv: channel pair pp, tokens 8*warp .. 8*warp+7
-        const int pp = lane;
-        const int r0 = 8 * warp;
-        // the carried state h: S^T[n][p] layout of the state MMA
-        constexpr int HR = NS == 128 ? 32 : 16;
-        const int nrow = NS == 128 ? 32 * sub + lane : r16;
-        const int pcol = NS == 128 ? half * 32 : c16;
-        float hs[HR];
+        const int pp = lane;                       // conv: channel pair 2pp, 2pp+1
+        const int r0 = 8 * warp;                   // conv: tokens r0 .. r0+7
+        const int cdim = H * 64 + 2 * p.ngroups * NS;
+        const bool issuer = tid == 0;
+        const uint32_t id_64 = tc::idesc_bf16(64, 64, false, false);
+        const uint32_t id_st = tc::idesc_bf16(NS, 64, true, false);
         float wk[2][4] = {{0.f, 0.f, 0.f, 1.f}, {0.f, 0.f, 0.f, 1.f}}, cbias[2] = {0.f, 0.f};
-        float Dh = 0.f, carry_prev = 0.f;
         int cur_h = -1;
-        auto load_S = [&](uint32_t (&r)[HR]) {
-            if (NS == 128) {
-                tc::tmem_ld16(tmem + lane_base + kColS + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                tc::tmem_ld16(tmem + lane_base + kColS + half * 32 + 16,
-                              *reinterpret_cast<uint32_t(*)[16]>(&r[16 % HR]));
-            } else {
-                tc::tmem_ld16_x2_32(tmem + lane_base + kColS + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+
+        // C B^T of one step into the CB columns (both operands K-major over n)
+        auto issue_cb = [&](int st) {
+            const uint32_t a_b = tc::smem_u32(sm + st * LY::kStage + 2 * kTile);
+            const uint32_t a_c = a_b + LY::kBC;
+#pragma unroll
+            for (int kk = 0; kk < NS / 16; kk++) {
+                const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
+                tc::mma_bf16(tmem + kColCB, tc::sdesc_sw128(a_c + off, 16, 1024),
+                             tc::sdesc_sw128(a_b + off, 16, 1024), id_64, kk > 0);
             }
-            tc::tmem_wait_ld();
+            tc::mma_commit(cb_done);
         };
+        if (issuer && tc::mbar_wait(&full[0], 0, s_abort, p.status, kStatusTimeout)) {
+            tc::tc_fence_after();
+            issue_cb(0);
+        }
 
         int q = 0;
-        for (StepIter it(p, nc); it.valid(); it.next(), q++) {
-            const int s = q & 1;
+        for (StepIter it(p, nc); it.valid(); q++) {
+            const int st = q % NST, i = q & 1;
             const int b = it.b, h = it.h, t0 = it.c * 64;
-            const int64_t str = (int64_t)b * H + h;
             const bool first = it.first();
-            // ---- per-head constants
-            if (h != cur_h) {
+            if (CONV && h != cur_h) {
                 cur_h = h;
-                Dh = p.D[h];
-                if (CONV) {
 #pragma unroll
-                    for (int e = 0; e < 2; e++) {
-                        const int ch = h * 64 + 2 * pp + e;
+                for (int e = 0; e < 2; e++) {
+                    const int ch = h * 64 + 2 * pp + e;
 #pragma unroll
-                        for (int kq = 0; kq < 4; kq++) wk[e][kq] = __bfloat162float(p.conv_w[(int64_t)ch * 4 + kq]);
-                        cbias[e] = __bfloat162float(p.conv_b[ch]);
-                    }
+                    for (int kq = 0; kq < 4; kq++) wk[e][kq] = __bfloat162float(p.conv_w[(int64_t)ch * 4 + kq]);
+                    cbias[e] = __bfloat162float(p.conv_b[ch]);
                 }
             }
             // On abort the waits return at once; every thread still runs the same
-            // sequence of compute barriers and leaves at the end of the iteration.
-            tc::mbar_wait(&full[s], (q >> 1) & 1, s_abort, p.status, kStatusTimeout);
-            const uint8_t* st = sm + s * LY::kStage;
-            const ChunkScalars* cs = &scal[s];
+            // sequence of group barriers and leaves at the end of the iteration.
+            tc::mbar_wait(&full[st], par(q / NST), s_abort, p.status, kStatusTimeout);
+            // the operand buffers [i] and Ydiag columns [i] are free once group B
+            // has finished step q-2
+            if (q >= 2) tc::mbar_wait(&epi_done[i], par((q >> 1) - 1), s_abort, p.status, kStatusTimeout);
+            const uint8_t* stg = sm + st * LY::kStage;
+            const ChunkScalars* cs = &scal[st];
             const uint32_t m0 = cs->m0, m1 = cs->m1, pre = cs->pre;
-            const float carry = cs->carry;
             const bool quiet = (m0 | m1 | pre) == 0;      // no boundary near this chunk
+            uint8_t* xb = sm + LY::kXb + i * kTile;
+            uint8_t* xd = sm + LY::kXd + i * kTile;
+            uint8_t* xs = sm + LY::kXs + i * kTile;
+            uint8_t* mop = sm + LY::kMop + i * kTile;
 
-            // ---- (A) state entering this chunk -> bf16 h^T (the Yoff operand)
-            if (first) {
-                const float* src = nullptr;
-                if (it.k == 0) {
-                    src = p.init_ssm ? p.init_ssm + str * 64 * NS : nullptr;
-                } else {
-                    // the previous segment's leaving state (an item started earlier)
-                    const unsigned* fl = p.flags + str * p.nseg + (it.k - 1);
-                    if (tid == 0) {
-                        const uint64_t tw = tc::global_ns();
-                        unsigned v;
-                        for (;;) {
-                            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(fl) : "memory");
-                            if (v == p.epoch || *s_abort) break;
-                            if (tc::global_ns() - tw > tc::kWaitLimitNs) {
-                                *s_abort = 1;
-                                atomicOr(p.status, kStatusTimeout);
-                                break;
-                            }
-                            __nanosleep(128);
-                        }
-                    }
-                    bar_compute();
-                    src = p.hseg + (str * p.nseg + (it.k - 1)) * 64 * NS;
-                }
-#pragma unroll
-                for (int jj = 0; jj < HR; jj++) hs[jj] = src ? __ldcg(src + (int64_t)(pcol + jj) * NS + nrow) : 0.f;
-            } else {
-                // h_c = k_{c-1} h_{c-1} + S_{c-1}  (S_{c-1} complete: mma_done of the last step)
-                uint32_t r[HR];
-                load_S(r);
-                const bool drop = carry_prev == kChunkReset;
-#pragma unroll
-                for (int jj = 0; jj < HR; jj++)
-                    hs[jj] = (drop ? 0.0f : carry_prev * hs[jj]) + __uint_as_float(r[jj]);
-            }
-#pragma unroll
-            for (int qq = 0; qq < HR / 8; qq++) {
-                const uint4 v = make_uint4(pack_bf16(hs[8 * qq], hs[8 * qq + 1]),
-                                           pack_bf16(hs[8 * qq + 2], hs[8 * qq + 3]),
-                                           pack_bf16(hs[8 * qq + 4], hs[8 * qq + 5]),
-                                           pack_bf16(hs[8 * qq + 6], hs[8 * qq + 7]));
-                *(uint4*)(sm + LY::kHt + tc::sw128_offset(nrow, pcol + 8 * qq)) = v;
-            }
-            carry_prev = carry;
-
-            // ---- (B) conv and the operand tiles: channels 2pp, 2pp+1; tokens r0 .. r0+7
+            // ---- conv and the operand tiles: channels 2pp, 2pp+1; tokens r0 .. r0+7
             {
                 const uint32_t* halo_in = s_halo + (q & 1) * 96;
                 uint32_t* halo_out = s_halo + ((q + 1) & 1) * 96;
@@ -466,7 +397,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 for (int qq = 0; qq < 11; qq++) {
                     const int row = r0 - 3 + qq;
                     if (row >= 0) {
-                        raw[qq] = *(const uint32_t*)(st + tc::sw128_offset(row, 2 * pp));
+                        raw[qq] = *(const uint32_t*)(stg + tc::sw128_offset(row, 2 * pp));
                     } else if (!CONV) {
                         raw[qq] = 0u;
                     } else if (!first) {
@@ -486,64 +417,84 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                     for (int jj = 0; jj < 3; jj++) halo_out[jj * 32 + pp] = raw[8 + jj];
                 }
-                float ud[2][8], us[2][8];
+                // `quiet` is uniform over the block: a tap-mask-free body for it
+                auto conv_tokens = [&](auto quiet_c) {
+                    constexpr bool QUIET = decltype(quiet_c)::value;
+                    float ud[2][8], us[2][8];
 #pragma unroll
-                for (int qq = 0; qq < 8; qq++) {
-                    const int t = r0 + qq;
-                    float u[2];
-                    if (CONV) {
-                        bool ok2 = true, ok1 = true, ok0 = true;
-                        if (!quiet) {
-                            auto bd = [&](int r) -> bool {
-                                if (r >= 32) return (m1 >> (r - 32)) & 1u;
-                                if (r >= 0) return (m0 >> r) & 1u;
-                                return (pre >> (r + 2)) & 1u;
-                            };
-                            ok2 = !bd(t);
-                            ok1 = ok2 && !bd(t - 1);
-                            ok0 = ok1 && !bd(t - 2);
+                    for (int qq = 0; qq < 8; qq++) {
+                        const int t = r0 + qq;
+                        float u[2];
+                        if (CONV) {
+                            bool ok2 = true, ok1 = true, ok0 = true;
+                            if (!QUIET) {
+                                auto bd = [&](int r) -> bool {
+                                    if (r >= 32) return (m1 >> (r - 32)) & 1u;
+                                    if (r >= 0) return (m0 >> r) & 1u;
+                                    return (pre >> (r + 2)) & 1u;
+                                };
+                                ok2 = !bd(t);
+                                ok1 = ok2 && !bd(t - 1);
+                                ok0 = ok1 && !bd(t - 2);
+                            }
+#pragma unroll
+                            for (int e = 0; e < 2; e++) {
+                                auto xv = [&](int k3) { return e ? bf_hi(raw[k3]) : bf_lo(raw[k3]); };
+                                float acc = fmaf(wk[e][3], xv(qq + 3), cbias[e]);
+                                if (QUIET) {
+                                    acc = fmaf(wk[e][2], xv(qq + 2), acc);
+                                    acc = fmaf(wk[e][1], xv(qq + 1), acc);
+                                    acc = fmaf(wk[e][0], xv(qq), acc);
+                                } else {
+                                    acc += ok2 ? wk[e][2] * xv(qq + 2) : 0.f;
+                                    acc += ok1 ? wk[e][1] * xv(qq + 1) : 0.f;
+                                    acc += ok0 ? wk[e][0] * xv(qq) : 0.f;
+                                }
+                                u[e] = silu_t(acc);
+                            }
+                        } else {
+                            u[0] = bf_lo(raw[qq + 3]);
+                            u[1] = bf_hi(raw[qq + 3]);
                         }
+                        *(uint32_t*)(xb + tc::sw128_offset(t, 2 * pp)) = pack_bf16(u[0], u[1]);
+                        const float dtt = cs->dt[t], wdt = cs->wd[t];
 #pragma unroll
                         for (int e = 0; e < 2; e++) {
-                            auto xv = [&](int k3) { return e ? bf_hi(raw[k3]) : bf_lo(raw[k3]); };
-                            float acc = fmaf(wk[e][3], xv(qq + 3), cbias[e]);
-                            acc += ok2 ? wk[e][2] * xv(qq + 2) : 0.f;
-                            acc += ok1 ? wk[e][1] * xv(qq + 1) : 0.f;
-                            acc += ok0 ? wk[e][0] * xv(qq) : 0.f;
-                            u[e] = silu_t(acc);
+                            ud[e][qq] = dtt * u[e];
+                            us[e][qq] = wdt * u[e];
                         }
-                    } else {
-                        u[0] = bf_lo(raw[qq + 3]);
-                        u[1] = bf_hi(raw[qq + 3]);
                     }
-                    *(uint32_t*)(sm + LY::kXb + tc::sw128_offset(t, 2 * pp)) = pack_bf16(u[0], u[1]);
-                    const float dtt = cs->dt[t], wdt = cs->wd[t];
 #pragma unroll
                     for (int e = 0; e < 2; e++) {
-                        ud[e][qq] = dtt * u[e];
-                        us[e][qq] = wdt * u[e];
+                        const uint4 vd = make_uint4(pack_bf16(ud[e][0], ud[e][1]), pack_bf16(ud[e][2], ud[e][3]),
+                                                    pack_bf16(ud[e][4], ud[e][5]), pack_bf16(ud[e][6], ud[e][7]));
+                        const uint4 vs = make_uint4(pack_bf16(us[e][0], us[e][1]), pack_bf16(us[e][2], us[e][3]),
+                                                    pack_bf16(us[e][4], us[e][5]), pack_bf16(us[e][6], us[e][7]));
+                        *(uint4*)(xd + tc::sw128_offset(2 * pp + e, r0)) = vd;
+                        *(uint4*)(xs + tc::sw128_offset(2 * pp + e, r0)) = vs;
                     }
-                }
-#pragma unroll
-                for (int e = 0; e < 2; e++) {
-                    const uint4 vd = make_uint4(pack_bf16(ud[e][0], ud[e][1]), pack_bf16(ud[e][2], ud[e][3]),
-                                                pack_bf16(ud[e][4], ud[e][5]), pack_bf16(ud[e][6], ud[e][7]));
-                    const uint4 vs = make_uint4(pack_bf16(us[e][0], us[e][1]), pack_bf16(us[e][2], us[e][3]),
-                                                pack_bf16(us[e][4], us[e][5]), pack_bf16(us[e][6], us[e][7]));
-                    *(uint4*)(sm + LY::kXd + tc::sw128_offset(2 * pp + e, r0)) = vd;
-                    *(uint4*)(sm + LY::kXs + tc::sw128_offset(2 * pp + e, r0)) = vs;
-                }
+                };
+                if (quiet) conv_tokens(std::true_type{});
+                else conv_tokens(std::false_type{});
             }
-            // h^T and the conv tiles are written (and S of the last chunk read out of
-            // TMEM): Yoff and the chunk-state MMAs may start before the mask is done
             tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::mbar_arrive(xready);
+            bar_group(kBarA);
+            // S_c^T[n][p] = B^T Xs into S[i] (A = the B tile as MN-major over n, K = s);
+            // S[i] last held S(q-2), which group B has read once it arrived on s_free[i]
+            if (issuer && (q < 2 || tc::mbar_wait(&s_free[i], par((q >> 1) - 1), s_abort, p.status,
+                                                   kStatusTimeout))) {
+                tc::tc_fence_after();
+                const uint32_t a_b = tc::smem_u32(stg + 2 * kTile);
+                const uint32_t a_xs = tc::smem_u32(xs);
+#pragma unroll
+                for (int kk = 0; kk < 4; kk++)
+                    tc::mma_bf16(tmem + kColS + i * 64, tc::sdesc_sw128(a_b + kk * 2048, kTile, 1024),
+                                 tc::sdesc_sw128(a_xs + kk * 32, 16, 1024), id_st, kk > 0);
+                tc::mma_commit(&s_done[i]);
+            }
 
-            // ---- (C) mask: M[t][s] from the C B^T accumulator
-            if (tid == 0) tc::bulk_wait_read0();     // the previous out tile has left shared memory
-            bar_compute();
-            tc::mbar_wait(cb_done, q & 1, s_abort, p.status, kStatusTimeout);
+            // ---- mask: M[t][s] from the C B^T accumulator
+            tc::mbar_wait(cb_done, par(q), s_abort, p.status, kStatusTimeout);
             tc::tc_fence_after();
             {
                 const int t = r16;
@@ -562,7 +513,6 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         const float4 v = *reinterpret_cast<const float4*>(cs->a2 + c16 + 4 * j4);
                         as[4 * j4] = v.x; as[4 * j4 + 1] = v.y; as[4 * j4 + 2] = v.z; as[4 * j4 + 3] = v.w;
                     }
-                    // `quiet` is uniform over the block: two loop bodies, no per-element test
                     if (quiet) {
 #pragma unroll
                         for (int jj = 0; jj < 16; jj++)
@@ -583,28 +533,170 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                                             pack_bf16(mv[4], mv[5]), pack_bf16(mv[6], mv[7]));
                 const uint4 hi = make_uint4(pack_bf16(mv[8], mv[9]), pack_bf16(mv[10], mv[11]),
                                             pack_bf16(mv[12], mv[13]), pack_bf16(mv[14], mv[15]));
-                *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, c16)) = lo;
-                *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, c16 + 8)) = hi;
+                *(uint4*)(mop + tc::sw128_offset(t, c16)) = lo;
+                *(uint4*)(mop + tc::sw128_offset(t, c16 + 8)) = hi;
             }
             tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::mbar_arrive(mready);
+            tc::tc_fence_before();                 // the CB columns have been read
+            it.next();
+            const int aborted = bar_group_or(kBarA, *s_abort);
+            if (issuer && !aborted) {
+                // release: group B reads this step's Xb after it acquires y_done[i]
+                tc::mbar_arrive(&y_done[i]);
+                tc::tc_fence_after();
+                // Ydiag = M Xd into Y[i] (K = s); its commit also covers C B^T and S of this step
+                const uint32_t a_mop = tc::smem_u32(mop), a_xd = tc::smem_u32(xd);
+#pragma unroll
+                for (int kk = 0; kk < 4; kk++)
+                    tc::mma_bf16(tmem + kColY + i * 64, tc::sdesc_sw128(a_mop + kk * 32, 16, 1024),
+                                 tc::sdesc_sw128(a_xd + kk * 32, 16, 1024), id_64, kk > 0);
+                tc::mma_commit(&y_done[i]);
+                // C B^T of the next step (the CB columns were read above)
+                if (it.valid()) {
+                    const int q1 = q + 1;
+                    if (tc::mbar_wait(&full[q1 % NST], par(q1 / NST), s_abort, p.status, kStatusTimeout)) {
+                        tc::tc_fence_after();
+                        issue_cb(q1 % NST);
+                    }
+                }
+            }
+            if (aborted) break;
+        }
+        if (issuer) {
+            tc::mma_commit(drain_a);
+            tc::mbar_drain(drain_a, 0, p.status, kStatusTimeout);
+        }
+    } else if (warp < 2 * kGroupWarps) {
+        // ------------------------------------------------------------ group B: state, epilogue
+        // Warps 8-15.  Per step: h_c = k h_{c-1} + S(q-1) (or the entering state) ->
+        // h^T; [thread 0: Yoff = C h^T]; out = (Ydiag + f Yoff + D u) SiLU(z) -> TMA store.
+        const int half = (warp - kGroupWarps) >> 2;
+        const int btid = tid - kGroupThreads;
+        const bool issuer = btid == 0;
+        const int r16 = 16 * sub + (lane & 15);
+        const int c16 = half * 16 + (lane < 16 ? 0 : 32);
+        // the carried state h: S^T[n][p] layout of the state MMA
+        constexpr int HR = NS == 128 ? 32 : 16;
+        const int nrow = NS == 128 ? 32 * sub + lane : r16;
+        const int pcol = NS == 128 ? half * 32 : c16;
+        const uint32_t id_yo = tc::idesc_bf16(64, 64, false, true);
+        const uint32_t a_ht = tc::smem_u32(sm + LY::kHt);
+        float hs[HR];
+        float Dh = 0.f, carry_prev = 0.f;
+        int cur_h = -1;
+        auto load_S = [&](int bi, uint32_t (&r)[HR]) {
+            const uint32_t col = kColS + bi * 64;
+            if (NS == 128) {
+                tc::tmem_ld16(tmem + lane_base + col + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                tc::tmem_ld16(tmem + lane_base + col + half * 32 + 16,
+                              *reinterpret_cast<uint32_t(*)[16]>(&r[16 % HR]));
+            } else {
+                tc::tmem_ld16_x2_32(tmem + lane_base + col + half * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+            }
+            tc::tmem_wait_ld();
+        };
 
-            // ---- (D) epilogue: out = (Ydiag + f Yoff + D u) SiLU(z)
-            tc::mbar_wait(mma_done, q & 1, s_abort, p.status, kStatusTimeout);
+        int q = 0;
+        for (StepIter it(p, nc); it.valid(); q++) {
+            const int st = q % NST, i = q & 1;
+            const int b = it.b, h = it.h, t0 = it.c * 64;
+            const int64_t str = (int64_t)b * H + h;
+            const bool first = it.first(), last = it.last();
+            const bool stream_end = it.c == nc - 1;
+            const int seg_k = it.k;
+            if (h != cur_h) {
+                cur_h = h;
+                Dh = p.D[h];
+            }
+            tc::mbar_wait(&full[st], par(q / NST), s_abort, p.status, kStatusTimeout);
+            const uint8_t* stg = sm + st * LY::kStage;
+            const ChunkScalars* cs = &scal[st];
+            const float carry = cs->carry;
+
+            // ---- state entering this chunk -> bf16 h^T (the Yoff operand)
+            if (first) {
+                const float* src = nullptr;
+                if (seg_k == 0) {
+                    src = p.init_ssm ? p.init_ssm + str * 64 * NS : nullptr;
+                } else {
+                    // the previous segment's leaving state (an item started earlier)
+                    const unsigned* fl = p.flags + str * p.nseg + (seg_k - 1);
+                    if (issuer) {
+                        const uint64_t tw = tc::global_ns();
+                        unsigned v;
+                        for (;;) {
+                            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(fl) : "memory");
+                            if (v == p.epoch || *s_abort) break;
+                            if (tc::global_ns() - tw > tc::kWaitLimitNs) {
+                                *s_abort = 1;
+                                atomicOr(p.status, kStatusTimeout);
+                                break;
+                            }
+                            __nanosleep(128);
+                        }
+                    }
+                    bar_group(kBarB);
+                    src = p.hseg + (str * p.nseg + (seg_k - 1)) * 64 * NS;
+                }
+#pragma unroll
+                for (int jj = 0; jj < HR; jj++) hs[jj] = src ? __ldcg(src + (int64_t)(pcol + jj) * NS + nrow) : 0.f;
+            } else {
+                // h_c = k_{c-1} h_{c-1} + S_{c-1}
+                tc::mbar_wait(&s_done[i ^ 1], par((q - 1) >> 1), s_abort, p.status, kStatusTimeout);
+                tc::tc_fence_after();
+                uint32_t r[HR];
+                load_S(i ^ 1, r);
+                const bool drop = carry_prev == kChunkReset;
+#pragma unroll
+                for (int jj = 0; jj < HR; jj++)
+                    hs[jj] = (drop ? 0.0f : carry_prev * hs[jj]) + __uint_as_float(r[jj]);
+            }
+#pragma unroll
+            for (int qq = 0; qq < HR / 8; qq++) {
+                const uint4 v = make_uint4(pack_bf16(hs[8 * qq], hs[8 * qq + 1]),
+                                           pack_bf16(hs[8 * qq + 2], hs[8 * qq + 3]),
+                                           pack_bf16(hs[8 * qq + 4], hs[8 * qq + 5]),
+                                           pack_bf16(hs[8 * qq + 6], hs[8 * qq + 7]));
+                *(uint4*)(sm + LY::kHt + tc::sw128_offset(nrow, pcol + 8 * qq)) = v;
+            }
+            carry_prev = carry;
+            tc::fence_async_smem();
+            tc::tc_fence_before();                 // S(q-1) has been read
+            if (issuer) tc::bulk_wait_read1();     // the out tile [i] of step q-2 has left
+            bar_group(kBarB);
+            if (issuer) {
+                tc::tc_fence_after();
+                // S[i^1] may be overwritten by S(q+1) now
+                if (q >= 1) tc::mbar_arrive(&s_free[i ^ 1]);
+                // Yoff = C h^T (K = n; h^T is MN-major: rows n, 64 p per row)
+                const uint32_t a_c = tc::smem_u32(stg + 2 * kTile + LY::kBC);
+#pragma unroll
+                for (int kk = 0; kk < NS / 16; kk++) {
+                    const uint32_t off = (kk >> 2) * kTile + (kk & 3) * 32;
+                    tc::mma_bf16(tmem + kColYO, tc::sdesc_sw128(a_c + off, 16, 1024),
+                                 tc::sdesc_sw128(a_ht + kk * 2048, 8192, 1024), id_yo, kk > 0);
+                }
+                tc::mma_commit(yo_done);
+            }
+
+            // ---- epilogue: out = (Ydiag + f Yoff + D u) SiLU(z)
+            tc::mbar_wait(&y_done[i], par(q >> 1), s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(yo_done, par(q), s_abort, p.status, kStatusTimeout);
             tc::tc_fence_after();
+            uint8_t* outt = sm + LY::kOut + i * kTile;
             {
                 const int t = r16;
                 const float f = cs->f[t];
-                const uint8_t* zt = st + kTile;
+                const uint8_t* zt = stg + kTile;
+                const uint8_t* xb = sm + LY::kXb + i * kTile;
                 uint32_t ry[16], ro[16];
-                tc::tmem_ld16_x2_32(tmem + lane_base + kColY + half * 16, ry);
+                tc::tmem_ld16_x2_32(tmem + lane_base + kColY + i * 64 + half * 16, ry);
                 tc::tmem_ld16_x2_32(tmem + lane_base + kColYO + half * 16, ro);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int hh = 0; hh < 2; hh++) {
                     const int col = c16 + hh * 8;
-                    const uint4 xv = *(const uint4*)(sm + LY::kXb + tc::sw128_offset(t, col));
+                    const uint4 xv = *(const uint4*)(xb + tc::sw128_offset(t, col));
                     const uint4 zv = *(const uint4*)(zt + tc::sw128_offset(t, col));
                     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                     const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
@@ -616,49 +708,54 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         const float y1 = fmaf(f, __uint_as_float(ro[jj + 1]), __uint_as_float(ry[jj + 1])) + Dh * bf_hi(xw[e]);
                         ow[e] = pack_bf16(y0 * silu_t(bf_lo(zw[e])), y1 * silu_t(bf_hi(zw[e])));
                     }
-                    *(uint4*)(sm + LY::kMop + tc::sw128_offset(t, col)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    *(uint4*)(outt + tc::sw128_offset(t, col)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
             // ---- leaving the segment: h_out = k_c h_c + S_c -> the next segment or the caller
-            if (it.last()) {
+            if (last) {
+                tc::mbar_wait(&s_done[i], par(q >> 1), s_abort, p.status, kStatusTimeout);
+                tc::tc_fence_after();
                 uint32_t r[HR];
-                load_S(r);
-                const bool drop = carry_prev == kChunkReset;
-                const bool stream_end = it.c == nc - 1;
+                load_S(i, r);
+                const bool drop = carry == kChunkReset;
                 float* dst = stream_end ? (p.final_ssm ? p.final_ssm + str * 64 * NS : nullptr)
-                                        : p.hseg + (str * p.nseg + it.k) * 64 * NS;
+                                        : p.hseg + (str * p.nseg + seg_k) * 64 * NS;
                 if (dst != nullptr) {
 #pragma unroll
                     for (int jj = 0; jj < HR; jj++)
                         dst[(int64_t)(pcol + jj) * NS + nrow] =
-                            (drop ? 0.0f : carry_prev * hs[jj]) + __uint_as_float(r[jj]);
+                            (drop ? 0.0f : carry * hs[jj]) + __uint_as_float(r[jj]);
                 }
                 if (!stream_end) {
-                    bar_compute();
-                    if (tid == 0) {
+                    bar_group(kBarB);
+                    if (issuer) {
                         __threadfence();
-                        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + str * p.nseg + it.k),
+                        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + str * p.nseg + seg_k),
                                      "r"(p.epoch) : "memory");
                     }
                 }
             }
             tc::fence_async_smem();
-            const int aborted = bar_compute_or(*s_abort);
-            if (tid == 0) {
-                tc::tma_store_3d(&tm_out, sm + LY::kMop, h * 64, t0, b);
+            tc::tc_fence_before();                 // Y[i], Yoff (and S[i]) have been read
+            it.next();
+            const int aborted = bar_group_or(kBarB, *s_abort);
+            if (issuer) {
+                tc::tc_fence_after();
+                tc::mbar_arrive(&epi_done[i]);
+                tc::tma_store_3d(&tm_out, outt, h * 64, t0, b);
                 tc::bulk_commit();
-                tc::mbar_arrive(&empty[s]);
+                tc::mbar_arrive(&empty[st]);
             }
             if (aborted) break;
         }
-        if (tid == 0) tc::bulk_wait0();
+        if (issuer) {
+            tc::mma_commit(drain_b);
+            tc::mbar_drain(drain_b, 0, p.status, kStatusTimeout);
+            tc::bulk_wait0();
+        }
     }
 
-    // ---- teardown: no MMA may still be running when the tensor memory is freed
-    if (warp == kMmaWarp && lane == 0) {
-        tc::mma_commit(drain);
-        tc::mbar_drain(drain, 0, p.status, kStatusTimeout);
-    }
+    // ---- teardown: every MMA has completed (drains above) before the tensor memory is freed
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -697,6 +794,9 @@ static bool encode_tile_map(CUtensorMap* m, const void* base, int width, int seq
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+static_assert(Layout<64>::kAlloc <= 227 * 1024 && Layout<128>::kAlloc <= 227 * 1024,
+              "the fused kernel's shared memory exceeds the per-CTA limit");
 
 bool fused_path_available() { return tensor_map_encoder() != nullptr; }
 
