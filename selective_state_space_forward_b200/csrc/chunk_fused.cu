@@ -7,11 +7,10 @@
 //
 //   conv      u_t = SiLU(conv(x)) for the head's 64 channels (K1's arithmetic;
 //             B and C of the group come pre-convolved from K1, or raw)
-//   operands  Xd[s] = dt_s u_s              (intra-chunk right operand)
 //             Xs[s] = exp(acs_last - acs_s) dt_s u_s  [seg_s = seg_last]
 //   CB        S = C B^T                      tcgen05, 64 x 64 x N
-//   mask      M[t,s] = S[t,s] exp(acs_t - acs_s)  [s <= t, seg_s = seg_t]
-//   Ydiag     M Xd                           tcgen05, 64 x 64 x 64
+//   mask      M[t,s] = S[t,s] exp(acs_t - acs_s) dt_s  [s <= t, seg_s = seg_t]
+//   Ydiag     M u                            tcgen05, 64 x 64 x 64
 //   Yoff      C h_c^T                        tcgen05, 64 x 64 x N (bf16 copy of h_c)
 //   chunk     S_c = B^T Xs                   tcgen05, N x 64 x 64
 //   state     h_{c+1} = k_c h_c + S_c        fp32, in registers
@@ -103,8 +102,7 @@ struct Layout {
     static constexpr int kStage = 2 * kTile + 2 * kBC;        // x, z, B, C
     static constexpr int kRing = kStages * kStage;
     static constexpr int kXb = kRing;                         // [2] u in bf16, [t][p]
-    static constexpr int kXd = kXb + 2 * kTile;               // [2] dt u, [p][t]
-    static constexpr int kXs = kXd + 2 * kTile;               // [2] decayed dt u, [p][t]
+    static constexpr int kXs = kXb + 2 * kTile;               // [2] decayed dt u, [p][t]
     static constexpr int kMop = kXs + 2 * kTile;              // [2] mask operand, [t][s]
     static constexpr int kOut = kMop + 2 * kTile;             // [2] out tiles
     static constexpr int kHt = kOut + 2 * kTile;              // h^T, NS rows x 128 B
@@ -327,8 +325,8 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             tc::mbar_drain(&full[k2 % NST], par(k2 / NST), p.status, kStatusTimeout);
     } else if (warp < kGroupWarps) {
         // ------------------------------------------------------------ group A: conv, mask
-        // Warps 0-7.  Per step: conv -> Xb, Xd, Xs; [thread 0: S = B^T Xs]; mask from
-        // C B^T -> Mop; [thread 0: Ydiag = M Xd, then C B^T of the next step].
+        // Warps 0-7.  Per step: conv -> Xb, Xs; [thread 0: S = B^T Xs]; mask from
+        // C B^T -> Mop; [thread 0: Ydiag = M u, then C B^T of the next step].
         const int half = warp >> 2;                // column half
         const int r16 = 16 * sub + (lane & 15);    // M=64 accumulator row of this thread
         const int c16 = half * 16 + (lane < 16 ? 0 : 32);
@@ -338,6 +336,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const bool issuer = tid == 0;
         const uint32_t id_64 = tc::idesc_bf16(64, 64, false, false);
         const uint32_t id_st = tc::idesc_bf16(NS, 64, true, false);
+        const uint32_t id_mn = tc::idesc_bf16(64, 64, false, true);
         float wk[2][4] = {{0.f, 0.f, 0.f, 1.f}, {0.f, 0.f, 0.f, 1.f}}, cbias[2] = {0.f, 0.f};
         int cur_h = -1;
 
@@ -384,7 +383,6 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const uint32_t m0 = cs->m0, m1 = cs->m1, pre = cs->pre;
             const bool quiet = (m0 | m1 | pre) == 0;      // no boundary near this chunk
             uint8_t* xb = sm + LY::kXb + i * kTile;
-            uint8_t* xd = sm + LY::kXd + i * kTile;
             uint8_t* xs = sm + LY::kXs + i * kTile;
             uint8_t* mop = sm + LY::kMop + i * kTile;
 
@@ -420,7 +418,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 // `quiet` is uniform over the block: a tap-mask-free body for it
                 auto conv_tokens = [&](auto quiet_c) {
                     constexpr bool QUIET = decltype(quiet_c)::value;
-                    float ud[2][8], us[2][8];
+                    float us[2][8];
 #pragma unroll
                     for (int qq = 0; qq < 8; qq++) {
                         const int t = r0 + qq;
@@ -457,20 +455,14 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                             u[1] = bf_hi(raw[qq + 3]);
                         }
                         *(uint32_t*)(xb + tc::sw128_offset(t, 2 * pp)) = pack_bf16(u[0], u[1]);
-                        const float dtt = cs->dt[t], wdt = cs->wd[t];
+                        const float wdt = cs->wd[t];
 #pragma unroll
-                        for (int e = 0; e < 2; e++) {
-                            ud[e][qq] = dtt * u[e];
-                            us[e][qq] = wdt * u[e];
-                        }
+                        for (int e = 0; e < 2; e++) us[e][qq] = wdt * u[e];
                     }
 #pragma unroll
                     for (int e = 0; e < 2; e++) {
-                        const uint4 vd = make_uint4(pack_bf16(ud[e][0], ud[e][1]), pack_bf16(ud[e][2], ud[e][3]),
-                                                    pack_bf16(ud[e][4], ud[e][5]), pack_bf16(ud[e][6], ud[e][7]));
                         const uint4 vs = make_uint4(pack_bf16(us[e][0], us[e][1]), pack_bf16(us[e][2], us[e][3]),
                                                     pack_bf16(us[e][4], us[e][5]), pack_bf16(us[e][6], us[e][7]));
-                        *(uint4*)(xd + tc::sw128_offset(2 * pp + e, r0)) = vd;
                         *(uint4*)(xs + tc::sw128_offset(2 * pp + e, r0)) = vs;
                     }
                 };
@@ -507,16 +499,20 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     for (int jj = 0; jj < 16; jj++) mv[jj] = 0.f;
                 } else {
                     const float at = cs->a2[t];
-                    float as[16];
+                    float as[16], ds[16];
 #pragma unroll
                     for (int j4 = 0; j4 < 4; j4++) {
                         const float4 v = *reinterpret_cast<const float4*>(cs->a2 + c16 + 4 * j4);
                         as[4 * j4] = v.x; as[4 * j4 + 1] = v.y; as[4 * j4 + 2] = v.z; as[4 * j4 + 3] = v.w;
+                        const float4 d = *reinterpret_cast<const float4*>(cs->dt + c16 + 4 * j4);
+                        ds[4 * j4] = d.x; ds[4 * j4 + 1] = d.y; ds[4 * j4 + 2] = d.z; ds[4 * j4 + 3] = d.w;
                     }
+#pragma unroll
+                    for (int jj = 0; jj < 16; jj++) ds[jj] *= __uint_as_float(r[jj]);   // C_t.B_s dt_s
                     if (quiet) {
 #pragma unroll
                         for (int jj = 0; jj < 16; jj++)
-                            mv[jj] = c16 + jj <= t ? __uint_as_float(r[jj]) * ex2(at - as[jj]) : 0.f;
+                            mv[jj] = c16 + jj <= t ? ds[jj] * ex2(at - as[jj]) : 0.f;
                     } else {
                         const uint4 sv = *reinterpret_cast<const uint4*>(cs->seg + c16);
                         const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
@@ -525,7 +521,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         for (int jj = 0; jj < 16; jj++) {
                             const uint32_t sj = (sw[jj >> 2] >> (8 * (jj & 3))) & 0xFFu;
                             const bool keep = c16 + jj <= t && sj == segt;
-                            mv[jj] = keep ? __uint_as_float(r[jj]) * ex2(at - as[jj]) : 0.f;
+                            mv[jj] = keep ? ds[jj] * ex2(at - as[jj]) : 0.f;
                         }
                     }
                 }
@@ -544,12 +540,13 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 // release: group B reads this step's Xb after it acquires y_done[i]
                 tc::mbar_arrive(&y_done[i]);
                 tc::tc_fence_after();
-                // Ydiag = M Xd into Y[i] (K = s); its commit also covers C B^T and S of this step
-                const uint32_t a_mop = tc::smem_u32(mop), a_xd = tc::smem_u32(xd);
+                // Ydiag = M u into Y[i] (K = s; u is [s][p], MN-major); its commit also
+                // covers C B^T and S of this step
+                const uint32_t a_mop = tc::smem_u32(mop), a_xb = tc::smem_u32(xb);
 #pragma unroll
                 for (int kk = 0; kk < 4; kk++)
                     tc::mma_bf16(tmem + kColY + i * 64, tc::sdesc_sw128(a_mop + kk * 32, 16, 1024),
-                                 tc::sdesc_sw128(a_xd + kk * 32, 16, 1024), id_64, kk > 0);
+                                 tc::sdesc_sw128(a_xb + kk * 2048, 8192, 1024), id_mn, kk > 0);
                 tc::mma_commit(&y_done[i]);
                 // C B^T of the next step (the CB columns were read above)
                 if (it.valid()) {

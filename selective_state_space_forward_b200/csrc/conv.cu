@@ -139,6 +139,80 @@ conv_silu_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
     }
 }
 
+// bf16 input: the same arithmetic with every input row of the thread (three
+// history rows + its eight tokens) requested before any is used, so each thread
+// keeps eleven 16-byte loads in flight -- enough bytes in flight per SM to run
+// near HBM bandwidth at two resident blocks.  Rows stay packed (4 registers
+// each) and are widened on use.
+template <typename OutT>
+__global__ void __launch_bounds__(256, 2)
+conv_silu_bf16_kernel(Shape s, const bf16* __restrict__ x, const bf16* __restrict__ Bm,
+                      const bf16* __restrict__ Cm, const bf16* __restrict__ w,
+                      const bf16* __restrict__ bias, const int32_t* __restrict__ seq,
+                      const bf16* __restrict__ hist0, OutT* __restrict__ u, int cbase)
+{
+    const int cd = s.conv_dim();
+    const int nvec = (cd - cbase) / 8;
+    const int ntg = (s.seqlen + kTokPerThread - 1) / kTokPerThread;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)s.batch * ntg * nvec) return;
+    const int v = (int)(gid % nvec);
+    const int64_t r = gid / nvec;
+    const int tg = (int)(r % ntg);
+    const int b = (int)(r / ntg);
+    const int c = cbase + v * 8;
+    const int L = s.seqlen;
+
+    int64_t stride;
+    int col;
+    const bf16* src = channel_src(s, x, Bm, Cm, c, stride, col);
+    src += (int64_t)b * L * stride + col;
+    const int t0 = tg * kTokPerThread;
+
+    Vec8<bf16> row[kTokPerThread + 3];      // rows t0-3 .. t0+7
+#pragma unroll
+    for (int j = 0; j < kTokPerThread + 3; j++) {
+        const int64_t tau = (int64_t)t0 - 3 + j;
+        if (tau >= 0 && tau < L) row[j].load(src + tau * stride);
+        else if (tau < 0 && hist0 != nullptr) row[j].load(hist0 + ((int64_t)b * 3 + (tau + 3)) * cd + c);
+        else row[j].zero();
+    }
+    Vec8<bf16> wv[4], bv;       // weight (channel i, tap k) = element 4*i + k
+#pragma unroll
+    for (int q = 0; q < 4; q++) wv[q].load(w + (int64_t)c * 4 + q * 8);
+    bv.load(bias + c);
+
+    const int32_t* seq_row = seq ? seq + (int64_t)b * L : nullptr;
+    uint32_t bdm = 0;           // bit j: boundary at position t0 - 2 + j
+#pragma unroll
+    for (int j = 0; j < kTokPerThread + 2; j++) {
+        const int64_t pos = (int64_t)t0 - 2 + j;
+        if (pos >= 1 && pos < L && is_boundary(seq_row, pos)) bdm |= 1u << j;
+    }
+
+    OutT* dst = u + (int64_t)b * L * (cd - cbase) + (c - cbase);
+#pragma unroll
+    for (int q = 0; q < kTokPerThread; q++) {
+        const int64_t t = t0 + q;
+        if (t >= L) break;
+        // tap k reads row t-3+k; valid when no boundary at positions t-2+k .. t
+        const bool ok2 = !((bdm >> (q + 2)) & 1u);
+        const bool ok1 = ok2 && !((bdm >> (q + 1)) & 1u);
+        const bool ok0 = ok1 && !((bdm >> q) & 1u);
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int e = 4 * i;
+            float acc = fmaf(wv[(e + 3) >> 3][(e + 3) & 7], row[q + 3][i], bv[i]);
+            acc += ok2 ? wv[(e + 2) >> 3][(e + 2) & 7] * row[q + 2][i] : 0.0f;
+            acc += ok1 ? wv[(e + 1) >> 3][(e + 1) & 7] * row[q + 1][i] : 0.0f;
+            acc += ok0 ? wv[e >> 3][e & 7] * row[q][i] : 0.0f;
+            o[i] = sizeof(OutT) == 2 ? silu_t(acc) : silu_f(acc);
+        }
+        store8(dst + t * (cd - cbase), o);
+    }
+}
+
 // Final conv history: slot i holds the raw input at L-3+i when it lies in the
 // last token's document, else 0.  Each thread reads its 3 slots before writing
 // them, so the initial and final history may be the same buffer.
@@ -188,9 +262,14 @@ static cudaError_t launch_conv(const Shape& s, const FwdArgs& a, OutT* u, int cb
     const int ntg = (s.seqlen + kTokPerThread - 1) / kTokPerThread;
     const int64_t total = (int64_t)s.batch * ntg * nvec;
     const int64_t blocks = (total + 255) / 256;
-    conv_silu_kernel<T, OutT><<<(unsigned)blocks, 256, 0, st>>>(
-        s, (const T*)a.x, (const T*)a.B, (const T*)a.C, (const T*)a.conv_w, (const T*)a.conv_b,
-        a.seq_idx, (const T*)a.init_conv, u, cbase);
+    if constexpr (sizeof(T) == 2)
+        conv_silu_bf16_kernel<OutT><<<(unsigned)blocks, 256, 0, st>>>(
+            s, (const bf16*)a.x, (const bf16*)a.B, (const bf16*)a.C, (const bf16*)a.conv_w,
+            (const bf16*)a.conv_b, a.seq_idx, (const bf16*)a.init_conv, u, cbase);
+    else
+        conv_silu_kernel<T, OutT><<<(unsigned)blocks, 256, 0, st>>>(
+            s, (const T*)a.x, (const T*)a.B, (const T*)a.C, (const T*)a.conv_w, (const T*)a.conv_b,
+            a.seq_idx, (const T*)a.init_conv, u, cbase);
     return cudaGetLastError();
 }
 
