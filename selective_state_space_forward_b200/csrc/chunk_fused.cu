@@ -88,12 +88,21 @@ struct ChunkScalars {
     float wd[64];      // [seg_t = seg_last] exp(acs_last - acs_t) dt_t
     float f[64];       // [seg_t = 0] exp(acs_t): weight of the carried-state term
     float a2[64];      // acs_t * log2(e)
+    float g[64];       // dt_s 2^(a2ref(block of s) - a2_s): column factor of the mask
     uint8_t seg[64];   // document boundaries at chunk positions 0 .. t
+    float a2ref[4];    // a2 at the last token of each 16-token block (within the chunk)
     float carry;       // exp(acs_last), or kChunkReset when the chunk holds a boundary
     uint32_t m0, m1;   // boundary at chunk position r (bit r of m0 | m1 << 32)
     uint32_t pre;      // bit 0: boundary at t0-2, bit 1: at t0-1
-    uint32_t pad[4];
+    uint32_t fast;     // bit b: the mask of column block b may use the factored decay
+    uint32_t pad[3];
 };
+static_assert(sizeof(ChunkScalars) % 16 == 0, "ChunkScalars keeps 16-byte alignment");
+
+// Largest decay (in log2 units) across a 16-token block for which the mask
+// factors exp2(a2_t - a2_s) into 2^(a2_t - a2ref) 2^(a2ref - a2_s): both factors
+// then stay within 2^-64 .. 2^64, far from fp32 under- and overflow.
+constexpr float kMaskBlockRange = 64.0f;
 
 template <int NS>
 struct Layout {
@@ -298,16 +307,35 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const int seg_last = __shfl_sync(0xffffffffu, last < 32 ? seg0 : seg1, last & 31);
             const float acs_last = __shfl_sync(0xffffffffu, last < 32 ? acv[0] : acv[1], last & 31);
             const int segv[2] = {seg0, seg1};
+            // the 16-token block of token r ends at min(r | 15, Lc - 1)
+            float a2ref[2];
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+                const int rref = min((hf * 32 + lane) | 15, last);
+                const float v0 = __shfl_sync(0xffffffffu, acv[0], rref & 31);
+                const float v1 = __shfl_sync(0xffffffffu, acv[1], rref & 31);
+                a2ref[hf] = (rref < 32 ? v0 : v1) * kLog2e;
+            }
 #pragma unroll
             for (int hf = 0; hf < 2; hf++) {
                 const int r = hf * 32 + lane;
                 const bool ok = r < Lc;
+                const float a2 = acv[hf] * kLog2e;
                 cs->dt[r] = dtv[hf];
                 cs->wd[r] = (ok && segv[hf] == seg_last) ? __expf(acs_last - acv[hf]) * dtv[hf] : 0.0f;
                 cs->f[r] = (ok && segv[hf] == 0) ? __expf(acv[hf]) : 0.0f;
-                cs->a2[r] = acv[hf] * kLog2e;
+                cs->a2[r] = a2;
+                cs->g[r] = ok ? dtv[hf] * ex2(fminf(a2ref[hf] - a2, 0.0f)) : 0.0f;
                 cs->seg[r] = (uint8_t)segv[hf];
             }
+            // block b may use the factored mask when the chunk holds no boundary and the
+            // decay across the block stays within kMaskBlockRange
+            const float a2first0 = __shfl_sync(0xffffffffu, acv[0], lane & 16) * kLog2e;
+            const float a2first1 = __shfl_sync(0xffffffffu, acv[1], lane & 16) * kLog2e;
+            const bool blk_ok0 = a2first0 - a2ref[0] <= kMaskBlockRange;
+            const bool blk_ok1 = a2first1 - a2ref[1] <= kMaskBlockRange;
+            const uint32_t okb0 = __ballot_sync(0xffffffffu, blk_ok0);
+            const uint32_t okb1 = __ballot_sync(0xffffffffu, blk_ok1);
             if (lane == 0) {
                 uint32_t pre = 0;
                 if (t0 - 2 >= 1 && is_boundary(seq_row, t0 - 2)) pre |= 1u;
@@ -316,6 +344,14 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 cs->m0 = m0;
                 cs->m1 = m1;
                 cs->pre = pre;
+                // lanes 0 and 16 hold blocks 0, 1 (first half) and 2, 3 (second half)
+                const uint32_t fb = ((okb0 & 1u) ? 1u : 0u) | ((okb0 >> 16) & 1u) << 1 |
+                                    ((okb1 & 1u) ? 1u : 0u) << 2 | ((okb1 >> 16) & 1u) << 3;
+                cs->fast = (m0 | m1) ? 0u : fb;
+            }
+            if (lane == 0 || lane == 16) {
+                cs->a2ref[lane >> 4] = a2ref[0];
+                cs->a2ref[2 + (lane >> 4)] = a2ref[1];
             }
             __syncwarp();
             tc::mbar_arrive(&full[st]);
@@ -497,6 +533,18 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 if (c16 > t) {
 #pragma unroll
                     for (int jj = 0; jj < 16; jj++) mv[jj] = 0.f;
+                } else if ((cs->fast >> (c16 >> 4)) & 1u) {
+                    // factored decay: 2^(a2_t - a2ref) per row times the column factor g_s
+                    const float fr = ex2(fminf(cs->a2[t] - cs->a2ref[c16 >> 4], kMaskBlockRange));
+                    float gs[16];
+#pragma unroll
+                    for (int j4 = 0; j4 < 4; j4++) {
+                        const float4 v = *reinterpret_cast<const float4*>(cs->g + c16 + 4 * j4);
+                        gs[4 * j4] = v.x; gs[4 * j4 + 1] = v.y; gs[4 * j4 + 2] = v.z; gs[4 * j4 + 3] = v.w;
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 16; jj++)
+                        mv[jj] = c16 + jj <= t ? (__uint_as_float(r[jj]) * fr) * gs[jj] : 0.f;
                 } else {
                     const float at = cs->a2[t];
                     float as[16], ds[16];

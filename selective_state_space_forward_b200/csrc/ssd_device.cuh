@@ -23,13 +23,15 @@ template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __flo
 // x * sigmoid(x), with an IEEE divide so fp32 stages stay near correctly rounded.
 __device__ __forceinline__ float silu_f(float v) { return v / (1.0f + expf(-v)); }
 
-// SiLU(v) = v (1 + tanh(v/2)) / 2 with one hardware tanh (PTX tanh.approx,
-// relative error ~2^-11): for results that are rounded to bf16 anyway.
+// SiLU(v) = v (1 + tanh(v/2)) / 2 = h + h tanh(h) with h = v/2, one hardware
+// tanh (PTX tanh.approx, relative error ~2^-11): for results that are rounded
+// to bf16 anyway.
 __device__ __forceinline__ float silu_t(float v)
 {
+    const float h = 0.5f * v;
     float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
-    return v * fmaf(0.5f, t, 0.5f);
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
 }
 
 // 2^x, hardware approximation (PTX ex2.approx).
