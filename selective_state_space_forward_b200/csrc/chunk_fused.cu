@@ -154,6 +154,49 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Packed fp32 pairs (the f32x2 arithmetic of sm_100): one instruction computes
+// both lanes, each rounded exactly as the scalar fma.rn / mul.rn would.
+__device__ __forceinline__ uint64_t p2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void p2split(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// both halves of a packed bf16 pair as an fp32 pair
+__device__ __forceinline__ uint64_t bf2(uint32_t w) { return p2(bf_lo(w), bf_hi(w)); }
+// SiLU of a pair, as silu_t: h + h tanh(h) with h = v/2
+__device__ __forceinline__ uint64_t silu2(uint64_t v)
+{
+    const uint64_t h = mul2(v, p2(0.5f, 0.5f));
+    float h0, h1, t0, t1;
+    p2split(h, h0, h1);
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(h0));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(h1));
+    return fma2(h, p2(t0, t1), h);
+}
+__device__ __forceinline__ uint32_t pack_bf16_2(uint64_t v)
+{
+    float lo, hi;
+    p2split(v, lo, hi);
+    return pack_bf16(lo, hi);
+}
+
 // The flattened step sequence a CTA walks: its work items in order, each item's
 // chunks in order.  Every role iterates it identically.
 struct StepIter {
@@ -374,6 +417,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const uint32_t id_st = tc::idesc_bf16(NS, 64, true, false);
         const uint32_t id_mn = tc::idesc_bf16(64, 64, false, true);
         float wk[2][4] = {{0.f, 0.f, 0.f, 1.f}, {0.f, 0.f, 0.f, 1.f}}, cbias[2] = {0.f, 0.f};
+        uint64_t wkp[4] = {0, 0, 0, 0}, cbp = 0;   // the same, channel pairs packed
         int cur_h = -1;
 
         // C B^T of one step into the CB columns (both operands K-major over n)
@@ -407,6 +451,9 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     for (int kq = 0; kq < 4; kq++) wk[e][kq] = __bfloat162float(p.conv_w[(int64_t)ch * 4 + kq]);
                     cbias[e] = __bfloat162float(p.conv_b[ch]);
                 }
+#pragma unroll
+                for (int kq = 0; kq < 4; kq++) wkp[kq] = p2(wk[0][kq], wk[1][kq]);
+                cbp = p2(cbias[0], cbias[1]);
             }
             // On abort the waits return at once; every thread still runs the same
             // sequence of group barriers and leaves at the end of the iteration.
@@ -459,7 +506,14 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                     for (int qq = 0; qq < 8; qq++) {
                         const int t = r0 + qq;
                         float u[2];
-                        if (CONV) {
+                        if (CONV && QUIET) {
+                            // both channels at once: four taps and the SiLU on fp32 pairs
+                            uint64_t acc = fma2(wkp[3], bf2(raw[qq + 3]), cbp);
+                            acc = fma2(wkp[2], bf2(raw[qq + 2]), acc);
+                            acc = fma2(wkp[1], bf2(raw[qq + 1]), acc);
+                            acc = fma2(wkp[0], bf2(raw[qq]), acc);
+                            p2split(silu2(acc), u[0], u[1]);
+                        } else if (CONV) {
                             bool ok2 = true, ok1 = true, ok0 = true;
                             if (!QUIET) {
                                 auto bd = [&](int r) -> bool {
@@ -492,8 +546,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         }
                         *(uint32_t*)(xb + tc::sw128_offset(t, 2 * pp)) = pack_bf16(u[0], u[1]);
                         const float wdt = cs->wd[t];
-#pragma unroll
-                        for (int e = 0; e < 2; e++) us[e][qq] = wdt * u[e];
+                        p2split(mul2(p2(u[0], u[1]), p2(wdt, wdt)), us[0][qq], us[1][qq]);
                     }
 #pragma unroll
                     for (int e = 0; e < 2; e++) {
@@ -542,9 +595,15 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         const float4 v = *reinterpret_cast<const float4*>(cs->g + c16 + 4 * j4);
                         gs[4 * j4] = v.x; gs[4 * j4 + 1] = v.y; gs[4 * j4 + 2] = v.z; gs[4 * j4 + 3] = v.w;
                     }
+                    const uint64_t frp = p2(fr, fr);
 #pragma unroll
-                    for (int jj = 0; jj < 16; jj++)
-                        mv[jj] = c16 + jj <= t ? (__uint_as_float(r[jj]) * fr) * gs[jj] : 0.f;
+                    for (int jj = 0; jj < 16; jj += 2) {
+                        float m0v, m1v;
+                        p2split(mul2(mul2(p2(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1])), frp),
+                                     p2(gs[jj], gs[jj + 1])), m0v, m1v);
+                        mv[jj] = c16 + jj <= t ? m0v : 0.f;
+                        mv[jj + 1] = c16 + jj + 1 <= t ? m1v : 0.f;
+                    }
                 } else {
                     const float at = cs->a2[t];
                     float as[16], ds[16];
@@ -691,10 +750,12 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 tc::tc_fence_after();
                 uint32_t r[HR];
                 load_S(i ^ 1, r);
-                const bool drop = carry_prev == kChunkReset;
+                const float cm = carry_prev == kChunkReset ? 0.0f : carry_prev;
+                const uint64_t cmp = p2(cm, cm);
 #pragma unroll
-                for (int jj = 0; jj < HR; jj++)
-                    hs[jj] = (drop ? 0.0f : carry_prev * hs[jj]) + __uint_as_float(r[jj]);
+                for (int jj = 0; jj < HR; jj += 2)
+                    p2split(fma2(cmp, p2(hs[jj], hs[jj + 1]), p2(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]))),
+                            hs[jj], hs[jj + 1]);
             }
 #pragma unroll
             for (int qq = 0; qq < HR / 8; qq++) {
@@ -732,6 +793,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             {
                 const int t = r16;
                 const float f = cs->f[t];
+                const uint64_t fp = p2(f, f), Dp = p2(Dh, Dh);
                 const uint8_t* zt = stg + kTile;
                 const uint8_t* xb = sm + LY::kXb + i * kTile;
                 uint32_t ry[16], ro[16];
@@ -749,9 +811,10 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
                         const int jj = hh * 8 + e * 2;
-                        const float y0 = fmaf(f, __uint_as_float(ro[jj]), __uint_as_float(ry[jj])) + Dh * bf_lo(xw[e]);
-                        const float y1 = fmaf(f, __uint_as_float(ro[jj + 1]), __uint_as_float(ry[jj + 1])) + Dh * bf_hi(xw[e]);
-                        ow[e] = pack_bf16(y0 * silu_t(bf_lo(zw[e])), y1 * silu_t(bf_hi(zw[e])));
+                        uint64_t y = fma2(fp, p2(__uint_as_float(ro[jj]), __uint_as_float(ro[jj + 1])),
+                                          p2(__uint_as_float(ry[jj]), __uint_as_float(ry[jj + 1])));
+                        y = fma2(Dp, bf2(xw[e]), y);
+                        ow[e] = pack_bf16_2(mul2(y, silu2(bf2(zw[e]))));
                     }
                     *(uint4*)(outt + tc::sw128_offset(t, col)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
