@@ -191,6 +191,26 @@ conv_silu_bf16_kernel(Shape s, const bf16* __restrict__ x, const bf16* __restric
     }
 
     OutT* dst = u + (int64_t)b * L * (cd - cbase) + (c - cbase);
+    if (bdm == 0) {
+        // no document boundary near these tokens: every tap is used
+#pragma unroll
+        for (int q = 0; q < kTokPerThread; q++) {
+            const int64_t t = t0 + q;
+            if (t >= L) break;
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const int e = 4 * i;
+                float acc = fmaf(wv[(e + 3) >> 3][(e + 3) & 7], row[q + 3][i], bv[i]);
+                acc = fmaf(wv[(e + 2) >> 3][(e + 2) & 7], row[q + 2][i], acc);
+                acc = fmaf(wv[(e + 1) >> 3][(e + 1) & 7], row[q + 1][i], acc);
+                acc = fmaf(wv[e >> 3][e & 7], row[q][i], acc);
+                o[i] = sizeof(OutT) == 2 ? silu_t(acc) : silu_f(acc);
+            }
+            store8(dst + t * (cd - cbase), o);
+        }
+        return;
+    }
 #pragma unroll
     for (int q = 0; q < kTokPerThread; q++) {
         const int64_t t = t0 + q;
