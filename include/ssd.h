@@ -72,7 +72,8 @@ typedef enum { SSD_A_PER_HEAD = 0, SSD_A_PER_TOKEN = 1 } ssd_a_mode;
  *  FUSED : one persistent chunk-sweep kernel per (row, head) that keeps the
  *          running state on chip (tcgen05 tensor-core contractions, bf16
  *          operands, fp32 accumulation); bf16 activations, headdim 64,
- *          d_state 64 or 128, no B/C norm.
+ *          d_state 64 or 128.  With bc_norm, each head's normalised B and C
+ *          tiles are built in shared memory and never written to memory.
  *  STAGED: the five-stage pipeline conv -> dt/cumsum -> chunk states ->
  *          state passing -> chunk outputs, fp32 arithmetic throughout; any
  *          supported shape and both dtypes.

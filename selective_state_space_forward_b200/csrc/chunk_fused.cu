@@ -80,6 +80,10 @@ struct FusedParams {
     float* hseg;              // (streams, nseg, 64, N) segment leaving states
     unsigned* flags;          // (streams, nseg)
     int* status;
+    // B/C RMSNorm + per-head bias (NORM kernels only)
+    const float* rinv;        // (B, L, 2G): 1/rms of B (g) and C (G + g) per token
+    const float *bn_w, *cn_w; // (N) or null (ones)
+    const float *bn_bias, *cn_bias;   // (H, N) or null (zeros)
 };
 
 // Per-token values of one chunk, written by the producer warp.
@@ -89,6 +93,7 @@ struct ChunkScalars {
     float f[64];       // [seg_t = 0] exp(acs_t): weight of the carried-state term
     float a2[64];      // acs_t * log2(e)
     float g[64];       // dt_s 2^(a2ref(block of s) - a2_s): column factor of the mask
+    float rb[64], rc[64];   // NORM: 1/rms of the token's B and C rows
     uint8_t seg[64];   // document boundaries at chunk positions 0 .. t
     float a2ref[4];    // a2 at the last token of each 16-token block (within the chunk)
     float carry;       // exp(acs_last), or kChunkReset when the chunk holds a boundary
@@ -118,7 +123,7 @@ struct Layout {
     static constexpr int kScal = kHt + NS * 128;              // ChunkScalars[kStages]
     static constexpr int kHalo = kScal + kStages * (int)sizeof(ChunkScalars);   // u32 [2][3][32]
     static constexpr int kBar = kHalo + 2 * 3 * 32 * 4;
-    static constexpr int kNumBars = 2 * kStages + 12;
+    static constexpr int kNumBars = 3 * kStages + 12;
     static constexpr int kMisc = kBar + kNumBars * 8;         // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack for 1024-byte alignment
@@ -234,7 +239,7 @@ struct StepIter {
 // Phase parity of the n-th completion (0-based) of a barrier.
 __device__ __forceinline__ uint32_t par(int n) { return (uint32_t)n & 1u; }
 
-template <int NS, bool CONV>
+template <int NS, bool CONV, bool NORM>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
@@ -260,6 +265,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     uint64_t* epi_done = yo_done + 1;      // [2] group B is done with the step's operands
     uint64_t* drain_a = epi_done + 2;
     uint64_t* drain_b = drain_a + 1;
+    uint64_t* norm_done = drain_b + 1;     // [NST] NORM: the stage's B and C tiles are normalised
     uint32_t* s_tmem = (uint32_t*)(sm + LY::kMisc);
     volatile int* s_abort = (volatile int*)(sm + LY::kMisc + 4);
 
@@ -271,6 +277,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int i = 0; i < NST; i++) {
             tc::mbar_init(&full[i], 33);     // producer: expect_tx arrive + 32 lane arrivals
             tc::mbar_init(&empty[i], 1);
+            tc::mbar_init(&norm_done[i], 1);
         }
         tc::mbar_init(cb_done, 1);
         tc::mbar_init(yo_done, 1);
@@ -370,6 +377,11 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 cs->a2[r] = a2;
                 cs->g[r] = ok ? dtv[hf] * ex2(fminf(a2ref[hf] - a2, 0.0f)) : 0.0f;
                 cs->seg[r] = (uint8_t)segv[hf];
+                if (NORM) {
+                    const int64_t tok = ((int64_t)b * L + (t0 + r)) * (2 * p.ngroups);
+                    cs->rb[r] = ok ? p.rinv[tok + g] : 0.0f;
+                    cs->rc[r] = ok ? p.rinv[tok + p.ngroups + g] : 0.0f;
+                }
             }
             // block b may use the factored mask when the chunk holds no boundary and the
             // decay across the block stays within kMaskBlockRange
@@ -432,6 +444,50 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
             tc::mma_commit(cb_done);
         };
+        // NORM: rewrite the B and C tiles of stage st (step with head hh) in place as
+        // B w / rms(B) + bias_h; thread tid takes 8 columns of rows tid / (NS/8) + k*(256/(NS/8))
+        auto normalise = [&](int st, int hh) {
+            uint8_t* stg = sm + st * LY::kStage;
+            const ChunkScalars* cs = &scal[st];
+            constexpr int kCh = NS / 8;                  // 8-column chunks per row
+            constexpr int kRowStep = kGroupThreads / kCh;
+            const int n8 = tid % kCh, n0 = n8 * 8;
+            const int tile = n0 >> 6, col = n0 & 63;
+#pragma unroll
+            for (int which = 0; which < 2; which++) {
+                const float* wv = which ? p.cn_w : p.bn_w;
+                const float* bv = which ? p.cn_bias : p.bn_bias;
+                float w8[8], b8[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    w8[j] = wv ? __ldg(wv + n0 + j) : 1.0f;
+                    b8[j] = bv ? __ldg(bv + (int64_t)hh * NS + n0 + j) : 0.0f;
+                }
+                uint8_t* tb = stg + 2 * kTile + which * LY::kBC + tile * kTile;
+#pragma unroll
+                for (int t = tid / kCh; t < 64; t += kRowStep) {
+                    const float ri = which ? cs->rc[t] : cs->rb[t];
+                    uint4* ptr = (uint4*)(tb + tc::sw128_offset(t, col));
+                    const uint4 v = *ptr;
+                    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const uint64_t sc = mul2(p2(w8[2 * j], w8[2 * j + 1]), p2(ri, ri));
+                        o[j] = pack_bf16_2(fma2(bf2(vw[j]), sc, p2(b8[2 * j], b8[2 * j + 1])));
+                    }
+                    *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        };
+        if (NORM) {
+            StepIter it0(p, nc);
+            tc::mbar_wait(&full[0], 0, s_abort, p.status, kStatusTimeout);
+            normalise(0, it0.h);
+            tc::fence_async_smem();
+            bar_group(kBarA);
+            if (issuer) tc::mbar_arrive(&norm_done[0]);
+        }
         if (issuer && tc::mbar_wait(&full[0], 0, s_abort, p.status, kStatusTimeout)) {
             tc::tc_fence_after();
             issue_cb(0);
@@ -639,9 +695,15 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 *(uint4*)(mop + tc::sw128_offset(t, c16)) = lo;
                 *(uint4*)(mop + tc::sw128_offset(t, c16 + 8)) = hi;
             }
+            it.next();
+            if (NORM && it.valid()) {
+                // the next step's B and C tiles, before its C B^T and Yoff read them
+                const int q1 = q + 1;
+                tc::mbar_wait(&full[q1 % NST], par(q1 / NST), s_abort, p.status, kStatusTimeout);
+                normalise(q1 % NST, it.h);
+            }
             tc::fence_async_smem();
             tc::tc_fence_before();                 // the CB columns have been read
-            it.next();
             const int aborted = bar_group_or(kBarA, *s_abort);
             if (issuer && !aborted) {
                 // release: group B reads this step's Xb after it acquires y_done[i]
@@ -658,6 +720,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 // C B^T of the next step (the CB columns were read above)
                 if (it.valid()) {
                     const int q1 = q + 1;
+                    if (NORM) tc::mbar_arrive(&norm_done[q1 % NST]);
                     if (tc::mbar_wait(&full[q1 % NST], par(q1 / NST), s_abort, p.status, kStatusTimeout)) {
                         tc::tc_fence_after();
                         issue_cb(q1 % NST);
@@ -774,6 +837,8 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 tc::tc_fence_after();
                 // S[i^1] may be overwritten by S(q+1) now
                 if (q >= 1) tc::mbar_arrive(&s_free[i ^ 1]);
+                // NORM: group A has normalised this step's C tile
+                if (NORM) tc::mbar_wait(&norm_done[st], par(q / NST), s_abort, p.status, kStatusTimeout);
                 // Yoff = C h^T (K = n; h^T is MN-major: rows n, 64 p per row)
                 const uint32_t a_c = tc::smem_u32(stg + 2 * kTile + LY::kBC);
 #pragma unroll
@@ -942,11 +1007,11 @@ static void choose_segments(int streams, int nchunks, int grid, size_t cap_items
     }
 }
 
-template <int NS, bool CONV>
+template <int NS, bool CONV, bool NORM>
 static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* maps, int sm_count,
                             size_t max_items, cudaStream_t st)
 {
-    auto kern = ssd_chunk_fused<NS, CONV>;
+    auto kern = ssd_chunk_fused<NS, CONV, NORM>;
     const int smem = Layout<NS>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -966,9 +1031,10 @@ static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* m
 }
 
 cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc, const float* dt,
-                               const float* acs, int* status, const FusedWork& fw, cudaStream_t st)
+                               const float* acs, const float* rinv, int* status, const FusedWork& fw,
+                               cudaStream_t st)
 {
-    if (!s.act_bf16 || s.headdim != 64 || (s.dstate != 64 && s.dstate != 128) || s.bc_norm)
+    if (!s.act_bf16 || s.headdim != 64 || (s.dstate != 64 && s.dstate != 128) || (s.bc_norm && !rinv))
         return cudaErrorNotSupported;
     const int HP = s.nheads * 64, GN = s.ngroups * s.dstate;
     CUtensorMap maps[5];
@@ -1002,11 +1068,19 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.hseg = fw.hseg;
     fp.flags = fw.flags;
     fp.status = status;
+    fp.rinv = rinv;
+    fp.bn_w = a.bn_w;
+    fp.cn_w = a.cn_w;
+    fp.bn_bias = a.bn_bias;
+    fp.cn_bias = a.cn_bias;
+#define SSD_FUSED_LAUNCH(NS_, CONV_, NORM_) launch_t<NS_, CONV_, NORM_>(s, fp, maps, fw.sm_count, fw.max_items, st)
+    const bool conv = s.dconv == 4, norm = s.bc_norm != 0;
     if (s.dstate == 64)
-        return s.dconv == 4 ? launch_t<64, true>(s, fp, maps, fw.sm_count, fw.max_items, st)
-                            : launch_t<64, false>(s, fp, maps, fw.sm_count, fw.max_items, st);
-    return s.dconv == 4 ? launch_t<128, true>(s, fp, maps, fw.sm_count, fw.max_items, st)
-                        : launch_t<128, false>(s, fp, maps, fw.sm_count, fw.max_items, st);
+        return conv ? (norm ? SSD_FUSED_LAUNCH(64, true, true) : SSD_FUSED_LAUNCH(64, true, false))
+                    : (norm ? SSD_FUSED_LAUNCH(64, false, true) : SSD_FUSED_LAUNCH(64, false, false));
+    return conv ? (norm ? SSD_FUSED_LAUNCH(128, true, true) : SSD_FUSED_LAUNCH(128, true, false))
+                : (norm ? SSD_FUSED_LAUNCH(128, false, true) : SSD_FUSED_LAUNCH(128, false, false));
+#undef SSD_FUSED_LAUNCH
 }
 
 }  // namespace ssd

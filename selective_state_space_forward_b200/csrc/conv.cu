@@ -233,6 +233,38 @@ conv_silu_bf16_kernel(Shape s, const bf16* __restrict__ x, const bf16* __restric
     }
 }
 
+// 1/rms of one N-long B or C row per thread: rinv[(b L + t) 2G + which G + g].
+__global__ void __launch_bounds__(256)
+bc_rms_kernel(Shape s, const bf16* __restrict__ Bm, const bf16* __restrict__ Cm,
+              const bf16* __restrict__ ubc, float* __restrict__ rinv)
+{
+    const int G = s.ngroups, N = s.dstate;
+    const int64_t rows = (int64_t)s.batch * s.seqlen * 2 * G;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= rows) return;
+    const int64_t tok = gid / (2 * G);
+    const int k = (int)(gid % (2 * G));          // which * G + g
+    const bf16* src = ubc ? ubc + tok * (2 * G * N) + (int64_t)k * N
+                          : (k < G ? Bm : Cm) + tok * (G * N) + (int64_t)(k % G) * N;
+    float ss = 0.0f;
+    for (int n = 0; n < N; n += 8) {
+        Vec8<bf16> v;
+        v.load(src + n);
+#pragma unroll
+        for (int j = 0; j < 8; j++) ss = fmaf(v[j], v[j], ss);
+    }
+    rinv[gid] = rsqrtf(ss / N + kNormEps);
+}
+
+cudaError_t launch_bc_rms(const Shape& s, const FwdArgs& a, const void* ubc, float* rinv, cudaStream_t st)
+{
+    if (!s.act_bf16 || s.dstate % 8) return cudaErrorInvalidValue;
+    const int64_t rows = (int64_t)s.batch * s.seqlen * 2 * s.ngroups;
+    bc_rms_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(
+        s, (const bf16*)a.B, (const bf16*)a.C, (const bf16*)ubc, rinv);
+    return cudaGetLastError();
+}
+
 // Final conv history: slot i holds the raw input at L-3+i when it lies in the
 // last token's document, else 0.  Each thread reads its 3 slots before writing
 // them, so the initial and final history may be the same buffer.

@@ -57,6 +57,7 @@ struct ssd_handle {
     float* cdecay;        // staged: (B, H, nc)
     float* states;        // staged: (B, nc, H, P, N)
     void* ubc;            // fused: conv'd B|C (B, L, 2GN) bf16
+    float* rinv;          // fused with bc_norm: 1/rms of every B and C row (B, L, 2G)
     int* status;          // device status word
     const float *bn_w, *cn_w, *bn_bias, *cn_bias;
     cudaEvent_t ev_start, ev_stop;   // measurement hook (caller-owned), or null
@@ -93,7 +94,7 @@ size_t conv_offset(const ssd_desc& d, int batch)
 bool fused_supported(const ssd_desc& d)
 {
     return fused_path_available() && d.act_dtype == SSD_DTYPE_BF16 && d.headdim == 64 &&
-           (d.dstate == 64 || d.dstate == 128) && !d.bc_norm;
+           (d.dstate == 64 || d.dstate == 128);
 }
 
 ssd_status validate_desc(const ssd_desc* d)
@@ -125,8 +126,7 @@ ssd_status validate_desc(const ssd_desc* d)
         return fail(SSD_ERR_INVALID_ARG, "path %d is not an ssd_path", d->path);
     if (d->path == SSD_PATH_FUSED && !fused_supported(*d))
         return fail(SSD_ERR_UNSUPPORTED,
-                    "the fused path needs bf16 activations, headdim 64, dstate 64 or 128 and "
-                    "no B/C norm");
+                    "the fused path needs bf16 activations, headdim 64 and dstate 64 or 128");
     return SSD_OK;
 }
 
@@ -316,6 +316,8 @@ ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
         o_st = take((size_t)dd.max_batch * nc * H * P * N * sizeof(float));
     }
     if (path == SSD_PATH_FUSED && dd.dconv == 4) o_ubc = take(BL * 2 * G * N * 2);
+    size_t o_rinv = 0;
+    if (path == SSD_PATH_FUSED && dd.bc_norm) o_rinv = take(BL * 2 * G * sizeof(float));
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -347,6 +349,7 @@ ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
     h->cdecay = path == SSD_PATH_STAGED ? (float*)(h->ws + o_cd) : nullptr;
     h->states = path == SSD_PATH_STAGED ? (float*)(h->ws + o_st) : nullptr;
     h->ubc = (path == SSD_PATH_FUSED && dd.dconv == 4) ? (void*)(h->ws + o_ubc) : nullptr;
+    h->rinv = (path == SSD_PATH_FUSED && dd.bc_norm) ? (float*)(h->ws + o_rinv) : nullptr;
     h->status = (int*)(h->ws + o_status);
     h->fw.hseg = path == SSD_PATH_FUSED ? (float*)(h->ws + o_hseg) : nullptr;
     h->fw.flags = path == SSD_PATH_FUSED ? (unsigned*)(h->ws + o_flags) : nullptr;
@@ -452,8 +455,10 @@ ssd_status ssd_forward(ssd_handle* h, int32_t batch, int32_t seqlen, const void*
     } else {
         if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_bc(s, a, h->ubc, st), "B|C conv kernel");
         SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, nullptr, st), "dt/cumsum kernel");
+        if (s.bc_norm) SSD_LAUNCH(h, launch_bc_rms(s, a, h->ubc, h->rinv, st), "B/C rms kernel");
         if (++h->fw.epoch == 0) h->fw.epoch = 1;      // flags hold the last call's epoch
-        SSD_MAIN_LAUNCH(h, st, launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->status, h->fw, st),
+        SSD_MAIN_LAUNCH(h, st,
+                        launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->rinv, h->status, h->fw, st),
                         "fused chunk kernel");
     }
     if (a.final_conv) SSD_LAUNCH(h, launch_conv_state(s, a, st), "conv-state kernel");
@@ -568,7 +573,7 @@ ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
 {
     g_err.clear();
     SSD_TRY(validate_desc(d));
-    if (d->path == SSD_PATH_STAGED || !fused_supported(*d))
+    if (d->path == SSD_PATH_STAGED || !fused_supported(*d) || d->bc_norm)
         return fail(SSD_ERR_UNSUPPORTED,
                     "ssd_forward_noalloc runs the fused path only: bf16 activations, headdim 64, "
                     "dstate 64 or 128, no B/C norm");
@@ -645,7 +650,7 @@ ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
                                                  : nullptr;
     if (s.dconv == 4) SSD_LAUNCH(&h, launch_conv_silu_bc(s, a, ubc, st), "B|C conv kernel");
     SSD_LAUNCH(&h, launch_dt_cumsum(s, a, dt, acs, nullptr, st), "dt/cumsum kernel");
-    SSD_LAUNCH(&h, launch_chunk_fused(s, a, ubc, dt, acs, status, fw, st), "fused chunk kernel");
+    SSD_LAUNCH(&h, launch_chunk_fused(s, a, ubc, dt, acs, nullptr, status, fw, st), "fused chunk kernel");
     if (a.final_conv) SSD_LAUNCH(&h, launch_conv_state(s, a, st), "conv-state kernel");
     return SSD_OK;
 }

@@ -75,8 +75,15 @@ struct FusedWork {
 bool fused_path_available();
 size_t fused_handoff_floats(int max_streams, int dstate, int sm_count);
 size_t fused_flag_count(int max_streams, int sm_count);
+// rinv: with bc_norm, (batch, seqlen, 2G) fp32 from launch_bc_rms, else null.
 cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc, const float* dt,
-                               const float* acs, int* status, const FusedWork& fw, cudaStream_t st);
+                               const float* acs, const float* rinv, int* status, const FusedWork& fw,
+                               cudaStream_t st);
+// Fused path with bc_norm: 1/sqrt(mean(row^2) + eps) of every B and C row,
+// rinv (batch, seqlen, 2G) fp32: B of group g at g, C at G + g.  Reads the
+// convolved B|C (ubc) when dconv = 4, else the raw B and C.
+cudaError_t launch_bc_rms(const Shape& s, const FwdArgs& a, const void* ubc, float* rinv,
+                          cudaStream_t st);
 // K6: one decode token per row, state updated in place.
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
                                cudaStream_t st);

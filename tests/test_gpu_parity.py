@@ -339,3 +339,25 @@ def test_empty_inputs():
     h.forward(e0, e0, ef[:0], dev["dt_bias"], dev["A"], eb[:0], eb[:0], dev["D"],
               dev["conv_w"], dev["conv_b"])
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("dstate,dconv,a_per_token", [(128, 1, True), (64, 4, False), (128, 4, True)])
+def test_bc_norm_on_the_fused_path(dstate, dconv, a_per_token):
+    """B/C RMSNorm + per-head bias on the fused kernel: groups shared by several
+    heads (so each head's bias must stay its own), norm weights other than one,
+    packed documents, with and without the conv."""
+    w = WORKLOADS["mamba3_siso"].with_(batch=2, seqlen=200, nheads=8, ngroups=2, dstate=dstate,
+                                       dconv=dconv, a_per_token=a_per_token,
+                                       documents="geometric", mean_doc_len=70, seed=21)
+    inp = make_inputs(w)
+    rng = np.random.Generator(np.random.PCG64(22))
+    inp["B_norm_w"] = (1.0 + 0.3 * rng.standard_normal(dstate)).astype(np.float32)
+    inp["C_norm_w"] = (1.0 + 0.3 * rng.standard_normal(dstate)).astype(np.float32)
+    inp["B_bias"] = (0.1 * rng.standard_normal((w.nheads, dstate))).astype(np.float32)
+    inp["C_bias"] = (0.1 * rng.standard_normal((w.nheads, dstate))).astype(np.float32)
+    res = oracle.forward(w.dims(), inp)
+    h = make_handle(w, "fused")
+    assert h.path == "fused"
+    dev = to_device(inp, w)
+    out, fs, fc, _ = run_forward(h, w, dev, init_state_of(h, w, inp))
+    _compare_all(w, inp, res, out, fs, fc, f"bc_norm N={dstate} conv={dconv}/fused")
