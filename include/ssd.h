@@ -146,6 +146,21 @@ ssd_status ssd_forward(ssd_handle* h, int32_t batch, int32_t seqlen,
                        struct CUstream_st* stream);
 
 /*
+ * Forward over a ragged batch: row b holds lengths[b] real tokens (a device
+ * int32 array of `batch` entries, each clamped to [0, seqlen]); the rest of
+ * the row is padding that is not part of the sequence.  Padding outputs are
+ * written as +0.0, and the final state and conv history are those after the
+ * row's last real token (a zero-length row hands init_state through).  Every
+ * other argument is as for ssd_forward; lengths may not be NULL.
+ */
+ssd_status ssd_forward_ragged(ssd_handle* h, int32_t batch, int32_t seqlen, const int32_t* lengths,
+                              const void* x, const void* z, const float* dt_raw,
+                              const float* dt_bias, const float* A, const void* B, const void* C,
+                              const float* D, const void* conv_w, const void* conv_b,
+                              const int32_t* seq_idx, const void* init_state, void* out,
+                              void* final_state, struct CUstream_st* stream);
+
+/*
  * One decode token per row (Mamba3Block.step: the same computation as forward
  * at L = 1 with the state carried).  Inputs are the forward's with seqlen 1:
  * x, z, out (batch, H*P); B, C (batch, G*N); dt_raw (batch, H); A (H) or

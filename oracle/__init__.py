@@ -54,7 +54,8 @@ class _Inputs(ctypes.Structure):
     _fields_ = [(n, _FP) for n in (
         "x", "z", "Bm", "Cm", "dt_raw", "dt_bias", "A", "D", "conv_w", "conv_b")] + [
         ("seq_idx", ctypes.POINTER(ctypes.c_int32))] + [
-        (n, _FP) for n in ("init_ssm", "init_conv", "bn_w", "cn_w", "bn_bias", "cn_bias")]
+        (n, _FP) for n in ("init_ssm", "init_conv", "bn_w", "cn_w", "bn_bias", "cn_bias")] + [
+        ("lengths", ctypes.POINTER(ctypes.c_int32))]
 
 
 def _bind(path: str):
@@ -112,6 +113,10 @@ def _marshal(dims: dict, inp: dict):
     if seq is not None:
         seq = np.ascontiguousarray(np.asarray(seq, dtype=np.int32))
         keep.append(seq)
+    lens = inp.get("lengths")
+    if lens is not None:
+        lens = np.ascontiguousarray(np.asarray(lens, dtype=np.int32))
+        keep.append(lens)
     i = _Inputs(
         x=_f32(inp["x"], keep), z=_f32(inp["z"], keep), Bm=_f32(inp["B"], keep),
         Cm=_f32(inp["C"], keep), dt_raw=_f32(inp["dt_raw"], keep),
@@ -120,7 +125,8 @@ def _marshal(dims: dict, inp: dict):
         seq_idx=seq.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if seq is not None else None,
         init_ssm=_f32(inp.get("init_ssm"), keep), init_conv=_f32(inp.get("init_conv"), keep),
         bn_w=_f32(inp.get("B_norm_w"), keep), cn_w=_f32(inp.get("C_norm_w"), keep),
-        bn_bias=_f32(inp.get("B_bias"), keep), cn_bias=_f32(inp.get("C_bias"), keep))
+        bn_bias=_f32(inp.get("B_bias"), keep), cn_bias=_f32(inp.get("C_bias"), keep),
+        lengths=lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if lens is not None else None)
     return d, i, keep
 
 

@@ -39,6 +39,11 @@
  *   8. after the last token: final SSM state h, and the last K-1 raw conv
  *      inputs, zeroed where they belong to another document than the last
  *      token's.
+ *   9. ragged batches: with per-row lengths, row b holds lengths[b] tokens and
+ *      the rest of the row is padding -- no token of the recurrence at all.
+ *      Padding outputs are +0.0, and the final state and conv history are
+ *      those after the row's last real token (a zero-length row hands its
+ *      initial state and history through unchanged).
  *
  * A decode step is this same computation at L = 1 with the state carried
  * (Mamba3Block.step: "the same computation as forward at L = 1").
@@ -68,6 +73,8 @@
  *             the oldest token
  *   bn_w, cn_w (dstate) or NULL (ones); bn_bias, cn_bias (nheads, dstate) or
  *             NULL (zeros) -- only read when bc_norm != 0
+ *   lengths   (batch) int32 real tokens per row, clamped to [0, seqlen], or
+ *             NULL (every row is seqlen long)
  * Outputs (double):
  *   out       (batch, seqlen, nheads*headdim)
  *   fin_ssm   (batch, nheads, headdim, dstate) or NULL
@@ -83,7 +90,16 @@ typedef struct {
     const int32_t *seq_idx;
     const float *init_ssm, *init_conv;
     const float *bn_w, *cn_w, *bn_bias, *cn_bias;
+    const int32_t *lengths;
 } oracle_inputs;
+
+/* Real tokens of row b. */
+static int row_len(const oracle_dims *d, const oracle_inputs *in, int b)
+{
+    if (!in->lengths) return d->seqlen;
+    const int v = in->lengths[b];
+    return v < 0 ? 0 : (v > d->seqlen ? d->seqlen : v);
+}
 
 static double softplus_exact(double v)
 {
@@ -167,7 +183,10 @@ static void run_pair(const oracle_dims *d, const oracle_inputs *in, int b, int h
         const float *s0 = in->init_ssm + ((size_t)b * H + h) * P * N;
         for (int i = 0; i < P * N; i++) hs[i] = s0[i];
     }
-    for (int t = 0; t < L; t++) {
+    const int Lb = row_len(d, in, b);
+    for (int t = Lb; t < L; t++)   /* padding */
+        for (int p = 0; p < P; p++) out[((size_t)b * L + t) * dx + h * P + p] = 0.0;
+    for (int t = 0; t < Lb; t++) {
         if (t > 0 && !same_doc(in, d, b, t - 1, t)) memset(hs, 0, sizeof(double) * P * N);
 
         for (int p = 0; p < P; p++) ux[p] = conv_silu(d, in, b, t, h * P + p);
@@ -271,9 +290,10 @@ int oracle_forward(const oracle_dims *d, const oracle_inputs *in,
     pthread_mutex_destroy(&j.lock);
 
     if (fin_conv && d->dconv > 1) {
-        const int K = d->dconv, cd = conv_dim_of(d), L = d->seqlen;
+        const int K = d->dconv, cd = conv_dim_of(d);
         for (int b = 0; b < d->batch; b++)
             for (int i = 0; i < K - 1; i++) {
+                const int L = row_len(d, in, b);   /* the row's last real token is L - 1 */
                 const int tau = L - (K - 1) + i;
                 for (int ch = 0; ch < cd; ch++) {
                     double v = 0.0;

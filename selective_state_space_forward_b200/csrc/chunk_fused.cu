@@ -70,6 +70,7 @@ struct FusedParams {
     const float* dt;          // (B, H, L) from K2
     const float* acs;         // (B, H, L) segmented cumsum from K2
     const int32_t* seq;       // (B, L) or null
+    const int32_t* lengths;   // (B) real tokens per row of a ragged batch, or null
     const float* D;
     const bf16* x;            // raw x, for the conv history at segment starts
     const bf16* conv_w;       // (conv_dim, 4) or null
@@ -100,7 +101,8 @@ struct ChunkScalars {
     uint32_t m0, m1;   // boundary at chunk position r (bit r of m0 | m1 << 32)
     uint32_t pre;      // bit 0: boundary at t0-2, bit 1: at t0-1
     uint32_t fast;     // bit b: the mask of column block b may use the factored decay
-    uint32_t pad[3];
+    uint32_t nvalid;   // real tokens of the chunk (rows from here on are ragged-batch padding)
+    uint32_t pad[2];
 };
 static_assert(sizeof(ChunkScalars) % 16 == 0, "ChunkScalars keeps 16-byte alignment");
 
@@ -335,6 +337,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
             }
             const int32_t* seq_row = p.seq ? p.seq + (int64_t)b * L : nullptr;
+            const int Lb = row_length(p.lengths, b, L);   // padding: dt = 0 (K2), no boundary
             const float* dt_row = p.dt + bh * L;
             const float* acs_row = p.acs + bh * L;
             ChunkScalars* cs = &scal[st];
@@ -347,7 +350,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const bool ok = t < L;
                 dtv[hf] = ok ? dt_row[t] : 0.0f;
                 acv[hf] = ok ? acs_row[t] : 0.0f;
-                bdv[hf] = ok ? is_boundary(seq_row, t) : 0;
+                bdv[hf] = t < Lb ? is_boundary(seq_row, t) : 0;
             }
             const uint32_t m0 = __ballot_sync(0xffffffffu, bdv[0]);
             const uint32_t m1 = __ballot_sync(0xffffffffu, bdv[1]);
@@ -393,8 +396,9 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const uint32_t okb1 = __ballot_sync(0xffffffffu, blk_ok1);
             if (lane == 0) {
                 uint32_t pre = 0;
-                if (t0 - 2 >= 1 && is_boundary(seq_row, t0 - 2)) pre |= 1u;
-                if (t0 - 1 >= 1 && is_boundary(seq_row, t0 - 1)) pre |= 2u;
+                if (t0 - 2 >= 1 && t0 - 2 < Lb && is_boundary(seq_row, t0 - 2)) pre |= 1u;
+                if (t0 - 1 >= 1 && t0 - 1 < Lb && is_boundary(seq_row, t0 - 1)) pre |= 2u;
+                cs->nvalid = (uint32_t)min(max(Lb - t0, 0), 64);
                 cs->carry = (m0 | m1) ? kChunkReset : __expf(acs_last);
                 cs->m0 = m0;
                 cs->m1 = m1;
@@ -881,6 +885,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         y = fma2(Dp, bf2(xw[e]), y);
                         ow[e] = pack_bf16_2(mul2(y, silu2(bf2(zw[e]))));
                     }
+                    if (t >= (int)cs->nvalid) ow[0] = ow[1] = ow[2] = ow[3] = 0u;   // ragged padding
                     *(uint4*)(outt + tc::sw128_offset(t, col)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
@@ -1058,6 +1063,7 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.dt = dt;
     fp.acs = acs;
     fp.seq = a.seq_idx;
+    fp.lengths = a.lengths;
     fp.D = a.D;
     fp.x = (const bf16*)a.x;
     fp.conv_w = (const bf16*)a.conv_w;

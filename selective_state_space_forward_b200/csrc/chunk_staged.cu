@@ -27,11 +27,12 @@
 
 namespace ssd {
 
-// Chunk-local segment ids: seg[t] = boundaries at positions t0 .. t0+t.
-__device__ void chunk_segments(const int32_t* seq_row, int t0, int Lc, int* seg, int* flag)
+// Chunk-local segment ids: seg[t] = boundaries at positions t0 .. t0+t (padding
+// positions, at or after the row length Lb, hold none).
+__device__ void chunk_segments(const int32_t* seq_row, int t0, int Lc, int Lb, int* seg, int* flag)
 {
     const int tid = threadIdx.x;
-    if (tid < kChunk) flag[tid] = (tid < Lc) ? is_boundary(seq_row, t0 + tid) : 0;
+    if (tid < kChunk) flag[tid] = (tid < Lc && t0 + tid < Lb) ? is_boundary(seq_row, t0 + tid) : 0;
     __syncthreads();
     if (tid < kChunk) {
         int acc = 0;
@@ -108,7 +109,8 @@ chunk_state_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float*
     int* seg = (int*)(wv + kChunk);    // [64]
     int* flag = seg + kChunk;          // [64]
 
-    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, seg, flag);
+    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc,
+                   row_length(a.lengths, b, L), seg, flag);
     const float* dtr = dt + ((int64_t)b * H + h) * L + t0;
     const float* acr = acs + ((int64_t)b * H + h) * L + t0;
     if (threadIdx.x < kChunk) {
@@ -175,7 +177,8 @@ chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float
     int* seg = (int*)(dv + kChunk);    // [64]
     int* flag = seg + kChunk;          // [64]
 
-    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, seg, flag);
+    const int Lb = row_length(a.lengths, b, L);
+    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, Lb, seg, flag);
     if (threadIdx.x < kChunk) {
         const int r = threadIdx.x;
         const int64_t o = ((int64_t)b * H + h) * L + t0 + r;
@@ -205,6 +208,10 @@ chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float
     for (int e = threadIdx.x; e < kChunk * P; e += blockDim.x) {
         const int t = e / P, p = e % P;
         if (t >= Lc) continue;
+        if (t0 + t >= Lb) {   // padding of a ragged row
+            ((T*)a.out)[((int64_t)b * L + t0 + t) * HP + h * P + p] = from_f<T>(0.0f);
+            continue;
+        }
         float y = 0.0f;
         for (int r = 0; r <= t; r++) y += cb[t * 65 + r] * xs[r * P + p];
         if (seg[t] == 0) {

@@ -271,8 +271,8 @@ cudaError_t launch_bc_rms(const Shape& s, const FwdArgs& a, const void* ubc, flo
 template <typename T>
 __global__ void __launch_bounds__(256)
 conv_state_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
-                  const T* __restrict__ Cm, const int32_t* __restrict__ seq, const T* hist0,
-                  T* hist1)
+                  const T* __restrict__ Cm, const int32_t* __restrict__ seq,
+                  const int32_t* __restrict__ lengths, const T* hist0, T* hist1)
 {
     const int cd = s.conv_dim();
     const int nvec = cd / 8;
@@ -287,12 +287,14 @@ conv_state_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
     const T* src = channel_src(s, x, Bm, Cm, c, stride, col);
     src += (int64_t)b * L * stride + col;
 
+    // the row's last real token is Lb - 1 (Lb = L unless the batch is ragged)
+    const int Lb = row_length(lengths, b, L);
     float vals[3][8];
 #pragma unroll
     for (int i = 0; i < 3; i++) {
-        const int64_t tau = (int64_t)L - 3 + i;
+        const int64_t tau = (int64_t)Lb - 3 + i;
         int ok = 1;
-        for (int64_t pos = (tau + 1 > 1 ? tau + 1 : 1); pos <= L - 1; pos++)
+        for (int64_t pos = (tau + 1 > 1 ? tau + 1 : 1); pos <= Lb - 1; pos++)
             ok &= !is_boundary(seq_row, pos);
         if (ok && tau >= 0) {
             load8(src + tau * stride, vals[i]);
@@ -343,11 +345,11 @@ cudaError_t launch_conv_state(const Shape& s, const FwdArgs& a, cudaStream_t st)
     const int64_t blocks = (total + 255) / 256;
     if (s.act_bf16)
         conv_state_kernel<bf16><<<(unsigned)blocks, 256, 0, st>>>(
-            s, (const bf16*)a.x, (const bf16*)a.B, (const bf16*)a.C, a.seq_idx,
+            s, (const bf16*)a.x, (const bf16*)a.B, (const bf16*)a.C, a.seq_idx, a.lengths,
             (const bf16*)a.init_conv, (bf16*)a.final_conv);
     else
         conv_state_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
-            s, (const float*)a.x, (const float*)a.B, (const float*)a.C, a.seq_idx,
+            s, (const float*)a.x, (const float*)a.B, (const float*)a.C, a.seq_idx, a.lengths,
             (const float*)a.init_conv, (float*)a.final_conv);
     return cudaGetLastError();
 }

@@ -45,7 +45,8 @@ __device__ __forceinline__ float warp_seg_scan(float v, int& start, int lane)
 __global__ void __launch_bounds__(256)
 dt_cumsum_kernel(Shape s, const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                  const float* __restrict__ A, const int32_t* __restrict__ seq,
-                 float* __restrict__ dt_out, float* __restrict__ acs_out, float* __restrict__ cdecay)
+                 const int32_t* __restrict__ lengths, float* __restrict__ dt_out,
+                 float* __restrict__ acs_out, float* __restrict__ cdecay)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -55,6 +56,7 @@ dt_cumsum_kernel(Shape s, const float* __restrict__ dt_raw, const float* __restr
     const int c = (int)((warp / H) % nc);
     const int b = (int)(warp / ((int64_t)H * nc));
     const int t0 = c * kChunk;
+    const int Lb = row_length(lengths, b, L);   // padding: dt = 0, no boundary
     const float bias = dt_bias[h];
     const float a_head = s.a_per_token ? 0.0f : A[h];
 
@@ -67,7 +69,7 @@ dt_cumsum_kernel(Shape s, const float* __restrict__ dt_raw, const float* __restr
         dtv[half] = 0.0f;
         dA[half] = 0.0f;
         bd[half] = 0;
-        if (t < L) {
+        if (t < Lb) {
             const int64_t i = ((int64_t)b * L + t) * H + h;
             dtv[half] = softplus_f(dt_raw[i] + bias);
             const float av = s.a_per_token ? fminf(A[i], -kAFloor) : a_head;
@@ -105,7 +107,7 @@ cudaError_t launch_dt_cumsum(const Shape& s, const FwdArgs& a, float* dt, float*
     const int64_t warps = (int64_t)s.batch * s.nchunks() * s.nheads;
     const int64_t blocks = (warps * 32 + 255) / 256;
     dt_cumsum_kernel<<<(unsigned)blocks, 256, 0, st>>>(s, a.dt_raw, a.dt_bias, a.A, a.seq_idx,
-                                                       dt, acs, cdecay);
+                                                       a.lengths, dt, acs, cdecay);
     return cudaGetLastError();
 }
 

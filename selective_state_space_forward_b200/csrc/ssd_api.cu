@@ -261,6 +261,72 @@ ssd_status noalloc_device(cudaStream_t st, NoAllocDevice& out)
 
 }  // namespace
 
+// ssd_forward and ssd_forward_ragged (lengths null: every row is seqlen long).
+static ssd_status forward_impl(ssd_handle* h, int32_t batch, int32_t seqlen, const int32_t* lengths,
+                               const void* x, const void* z, const float* dt_raw,
+                               const float* dt_bias, const float* A, const void* B, const void* C,
+                               const float* D, const void* conv_w, const void* conv_b,
+                               const int32_t* seq_idx, const void* init_state, void* out,
+                               void* final_state, struct CUstream_st* stream)
+{
+    g_err.clear();
+    SSD_TRY(check_handle_dims(h, batch, seqlen));
+    SSD_TRY(check_ptr(lengths, "lengths", 4, false));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (batch == 0) return SSD_OK;
+    SSD_TRY(check_ptr(init_state, "init_state", 16, false));
+    SSD_TRY(check_ptr(final_state, "final_state", 16, false));
+    if (seqlen == 0) {   // no token: the state passes through unchanged
+        if (final_state && final_state != init_state) {
+            const size_t n = ssd_state_bytes(h, batch);
+            SSD_CUDA(init_state ? cudaMemcpyAsync(final_state, init_state, n,
+                                                  cudaMemcpyDeviceToDevice, st)
+                                : cudaMemsetAsync(final_state, 0, n, st),
+                     "empty-sequence state copy");
+        }
+        return SSD_OK;
+    }
+    SSD_TRY(check_common(h, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, out));
+    SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
+    if (out == init_state || out == final_state)
+        return fail(SSD_ERR_INVALID_ARG, "out may not alias a state buffer");
+
+    const Shape s = make_shape(h, batch, seqlen);
+    FwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.lengths = lengths;
+    a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
+    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
+    a.init_ssm = (const float*)init_state;
+    a.init_conv = (init_state && s.dconv == 4) ? (const char*)init_state + conv_offset(h->d, batch)
+                                               : nullptr;
+    a.out = out;
+    a.final_ssm = (float*)final_state;
+    a.final_conv = (final_state && s.dconv == 4) ? (char*)final_state + conv_offset(h->d, batch)
+                                                 : nullptr;
+    a.bn_w = h->bn_w; a.cn_w = h->cn_w; a.bn_bias = h->bn_bias; a.cn_bias = h->cn_bias;
+
+    if (h->path == SSD_PATH_STAGED) {
+        if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_all(s, a, h->u, st), "conv kernel");
+        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, h->cdecay, st), "dt/cumsum kernel");
+        SSD_LAUNCH(h, launch_chunk_state(s, a, h->u, h->dt, h->acs, h->states, st),
+                   "chunk-state kernel");
+        SSD_LAUNCH(h, launch_state_passing(s, a, h->cdecay, h->states, st), "state-passing kernel");
+        SSD_MAIN_LAUNCH(h, st, launch_chunk_output(s, a, h->u, h->dt, h->acs, h->states, st),
+                        "chunk-output kernel");
+    } else {
+        if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_bc(s, a, h->ubc, st), "B|C conv kernel");
+        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, nullptr, st), "dt/cumsum kernel");
+        if (s.bc_norm) SSD_LAUNCH(h, launch_bc_rms(s, a, h->ubc, h->rinv, st), "B/C rms kernel");
+        if (++h->fw.epoch == 0) h->fw.epoch = 1;      // flags hold the last call's epoch
+        SSD_MAIN_LAUNCH(h, st,
+                        launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->rinv, h->status, h->fw, st),
+                        "fused chunk kernel");
+    }
+    if (a.final_conv) SSD_LAUNCH(h, launch_conv_state(s, a, st), "conv-state kernel");
+    return SSD_OK;
+}
+
 extern "C" {
 
 const char* ssd_last_error(void) { return g_err.c_str(); }
@@ -410,59 +476,23 @@ ssd_status ssd_forward(ssd_handle* h, int32_t batch, int32_t seqlen, const void*
                        const int32_t* seq_idx, const void* init_state, void* out,
                        void* final_state, struct CUstream_st* stream)
 {
-    g_err.clear();
-    SSD_TRY(check_handle_dims(h, batch, seqlen));
-    cudaStream_t st = (cudaStream_t)stream;
-    if (batch == 0) return SSD_OK;
-    SSD_TRY(check_ptr(init_state, "init_state", 16, false));
-    SSD_TRY(check_ptr(final_state, "final_state", 16, false));
-    if (seqlen == 0) {   // no token: the state passes through unchanged
-        if (final_state && final_state != init_state) {
-            const size_t n = ssd_state_bytes(h, batch);
-            SSD_CUDA(init_state ? cudaMemcpyAsync(final_state, init_state, n,
-                                                  cudaMemcpyDeviceToDevice, st)
-                                : cudaMemsetAsync(final_state, 0, n, st),
-                     "empty-sequence state copy");
-        }
-        return SSD_OK;
-    }
-    SSD_TRY(check_common(h, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, out));
-    SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
-    if (out == init_state || out == final_state)
-        return fail(SSD_ERR_INVALID_ARG, "out may not alias a state buffer");
+    return forward_impl(h, batch, seqlen, nullptr, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b,
+                        seq_idx, init_state, out, final_state, stream);
+}
 
-    const Shape s = make_shape(h, batch, seqlen);
-    FwdArgs a;
-    a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
-    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
-    a.init_ssm = (const float*)init_state;
-    a.init_conv = (init_state && s.dconv == 4) ? (const char*)init_state + conv_offset(h->d, batch)
-                                               : nullptr;
-    a.out = out;
-    a.final_ssm = (float*)final_state;
-    a.final_conv = (final_state && s.dconv == 4) ? (char*)final_state + conv_offset(h->d, batch)
-                                                 : nullptr;
-    a.bn_w = h->bn_w; a.cn_w = h->cn_w; a.bn_bias = h->bn_bias; a.cn_bias = h->cn_bias;
-
-    if (h->path == SSD_PATH_STAGED) {
-        if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_all(s, a, h->u, st), "conv kernel");
-        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, h->cdecay, st), "dt/cumsum kernel");
-        SSD_LAUNCH(h, launch_chunk_state(s, a, h->u, h->dt, h->acs, h->states, st),
-                   "chunk-state kernel");
-        SSD_LAUNCH(h, launch_state_passing(s, a, h->cdecay, h->states, st), "state-passing kernel");
-        SSD_MAIN_LAUNCH(h, st, launch_chunk_output(s, a, h->u, h->dt, h->acs, h->states, st),
-                        "chunk-output kernel");
-    } else {
-        if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_bc(s, a, h->ubc, st), "B|C conv kernel");
-        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, nullptr, st), "dt/cumsum kernel");
-        if (s.bc_norm) SSD_LAUNCH(h, launch_bc_rms(s, a, h->ubc, h->rinv, st), "B/C rms kernel");
-        if (++h->fw.epoch == 0) h->fw.epoch = 1;      // flags hold the last call's epoch
-        SSD_MAIN_LAUNCH(h, st,
-                        launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->rinv, h->status, h->fw, st),
-                        "fused chunk kernel");
+ssd_status ssd_forward_ragged(ssd_handle* h, int32_t batch, int32_t seqlen, const int32_t* lengths,
+                              const void* x, const void* z, const float* dt_raw,
+                              const float* dt_bias, const float* A, const void* B, const void* C,
+                              const float* D, const void* conv_w, const void* conv_b,
+                              const int32_t* seq_idx, const void* init_state, void* out,
+                              void* final_state, struct CUstream_st* stream)
+{
+    if (!lengths) {
+        g_err.clear();
+        return fail(SSD_ERR_INVALID_ARG, "lengths is NULL");
     }
-    if (a.final_conv) SSD_LAUNCH(h, launch_conv_state(s, a, st), "conv-state kernel");
-    return SSD_OK;
+    return forward_impl(h, batch, seqlen, lengths, x, z, dt_raw, dt_bias, A, B, C, D, conv_w,
+                        conv_b, seq_idx, init_state, out, final_state, stream);
 }
 
 ssd_status ssd_step(ssd_handle* h, int32_t batch, const void* x, const void* z,

@@ -90,4 +90,15 @@ __device__ __forceinline__ int is_boundary(const int32_t* seq_row, int64_t r)
     return (seq_row != nullptr && r > 0) ? (seq_row[r] != seq_row[r - 1]) : 0;
 }
 
+// Real tokens of row b of a ragged batch (lengths null: every row is L long);
+// lengths are clamped to [0, L].  Padding tokens after them carry dt = 0 and
+// no document boundary, so the state passes them unchanged, and their outputs
+// are written as +0.0.
+__device__ __forceinline__ int row_length(const int32_t* lengths, int b, int L)
+{
+    if (lengths == nullptr) return L;
+    const int v = lengths[b];
+    return v < 0 ? 0 : (v > L ? L : v);
+}
+
 }  // namespace ssd

@@ -37,6 +37,7 @@ struct FwdArgs {
     float* final_ssm;        // or null
     void* final_conv;        // or null
     const float *bn_w, *cn_w, *bn_bias, *cn_bias;  // B/C norm parameters (nullable)
+    const int32_t* lengths;  // (batch) real tokens per row of a ragged batch, or null
 };
 
 // K1: conv + SiLU of every x|B|C channel into u (batch, seqlen, conv_dim) fp32.

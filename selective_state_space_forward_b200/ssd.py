@@ -31,7 +31,7 @@ DTYPES = {"f32": (0, torch.float32), "bf16": (1, torch.bfloat16)}
 EXPORTS = ("ssd_create", "ssd_destroy", "ssd_get_path", "ssd_set_bc_norm", "ssd_state_bytes",
            "ssd_state_conv_offset", "ssd_forward", "ssd_step", "ssd_stage_conv", "ssd_stage_dt",
            "ssd_set_timing_events", "ssd_launch_count", "ssd_check", "ssd_last_error",
-           "ssd_status_string", "ssd_forward_noalloc")
+           "ssd_status_string", "ssd_forward_noalloc", "ssd_forward_ragged")
 
 
 class SSDError(RuntimeError):
@@ -70,6 +70,7 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_state_conv_offset.argtypes = [vp, i32]
     lib.ssd_state_conv_offset.restype = sz
     lib.ssd_forward.argtypes = [vp, i32, i32] + [vp] * 14 + [vp]
+    lib.ssd_forward_ragged.argtypes = [vp, i32, i32] + [vp] * 15 + [vp]
     lib.ssd_step.argtypes = [vp, i32] + [vp] * 13
     lib.ssd_stage_conv.argtypes = [vp, i32, i32] + [vp] * 9
     lib.ssd_stage_dt.argtypes = [vp, i32, i32] + [vp] * 7
@@ -83,7 +84,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), i32, i32] + [vp] * 15 + [vp]
     for f in ("ssd_create", "ssd_set_bc_norm", "ssd_forward", "ssd_step", "ssd_stage_conv",
-              "ssd_stage_dt", "ssd_set_timing_events", "ssd_check", "ssd_forward_noalloc"):
+              "ssd_stage_dt", "ssd_set_timing_events", "ssd_check", "ssd_forward_noalloc",
+              "ssd_forward_ragged"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -184,12 +186,23 @@ class Handle:
             _ptr(B_bias, f, "B_bias"), _ptr(C_bias, f, "C_bias")))
 
     def forward(self, x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None, seq_idx=None,
-                init_state=None, out=None, final_state=None, stream=None):
-        """ssd_forward; returns `out` (allocated like x when not given)."""
+                init_state=None, out=None, final_state=None, stream=None, lengths=None):
+        """ssd_forward, or ssd_forward_ragged when `lengths` (an int32 CUDA tensor of
+        per-row real-token counts) is given; returns `out` (allocated like x when not given)."""
         at, f = self.torch_dtype, torch.float32
         batch, seqlen = (x.shape[0], x.shape[1]) if x.dim() == 3 else (0, 0)
         if out is None:
             out = torch.empty_like(x)
+        if lengths is not None:
+            _raise(self.lib, self.lib.ssd_forward_ragged(
+                self._h, batch, seqlen, _ptr(lengths, torch.int32, "lengths"), _ptr(x, at, "x"),
+                _ptr(z, at, "z"), _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"),
+                _ptr(A, f, "A"), _ptr(B, at, "B"), _ptr(C, at, "C"), _ptr(D, f, "D"),
+                _ptr(conv_w, at, "conv_w"), _ptr(conv_b, at, "conv_b"),
+                _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(init_state, torch.uint8, "init_state"),
+                _ptr(out, at, "out"), _ptr(final_state, torch.uint8, "final_state"),
+                _stream(stream)))
+            return out
         _raise(self.lib, self.lib.ssd_forward(
             self._h, batch, seqlen, _ptr(x, at, "x"), _ptr(z, at, "z"),
             _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"), _ptr(A, f, "A"),

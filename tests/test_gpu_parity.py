@@ -361,3 +361,63 @@ def test_bc_norm_on_the_fused_path(dstate, dconv, a_per_token):
     dev = to_device(inp, w)
     out, fs, fc, _ = run_forward(h, w, dev, init_state_of(h, w, inp))
     _compare_all(w, inp, res, out, fs, fc, f"bc_norm N={dstate} conv={dconv}/fused")
+
+
+def _ragged_case():
+    w = _small("mini_k3_mixer", batch=4, seqlen=300, mean_doc_len=90).with_(init_state=True)
+    inp = make_inputs(w)
+    lengths = np.array([300, 128, 0, 65], dtype=np.int32)
+    return w, inp, lengths
+
+
+def _run_ragged(h, w, dev, init, lengths):
+    fin = h.new_state(w.batch)
+    lens = torch.from_numpy(lengths).cuda()
+    out = h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"],
+                    dev["C"], dev["D"], dev["conv_w"], dev["conv_b"], seq_idx=dev["seq_idx"],
+                    init_state=init, final_state=fin, lengths=lens)
+    torch.cuda.synchronize()
+    h.check()
+    return out, fin
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_ragged_batch_matches_oracle_with_zero_padding(path):
+    """Ragged lengths (the full row, exactly two chunks, nothing, one chunk + 1):
+    every element against the oracle, padding exactly +0.0, final state and conv
+    history after each row's last real token."""
+    w, inp, lengths = _ragged_case()
+    res = oracle.forward(w.dims(), dict(inp, lengths=lengths))
+    h = make_handle(w, path)
+    dev = to_device(inp, w)
+    out, fin = _run_ragged(h, w, dev, init_state_of(h, w, inp), lengths)
+    bits = out.view(torch.int16)
+    for b, L in enumerate(lengths):
+        assert bool(torch.all(bits[b, L:] == 0)), f"row {b}: padding is not +0.0"
+    s, c = state_to_numpy(h, fin, w.batch)
+    _compare_all(w, inp, res, out.double().cpu().numpy(), s, c, f"ragged/{h.path}")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_ragged_rows_equal_rows_run_alone(path):
+    w, inp, lengths = _ragged_case()
+    h = make_handle(w, path)
+    dev = to_device(inp, w)
+    out, fin = _run_ragged(h, w, dev, init_state_of(h, w, inp), lengths)
+    s_all, c_all = state_to_numpy(h, fin, w.batch)
+    o_all = out.double().cpu().numpy()
+    for b, L in enumerate(lengths):
+        if L == 0:
+            continue
+        wb = w.with_(batch=1, seqlen=int(L))
+        one = {k: (None if v is None else
+                   (np.ascontiguousarray(v[b:b + 1, :L]) if k in ("x", "z", "B", "C", "dt_raw", "seq_idx")
+                    else (np.ascontiguousarray(v[b:b + 1]) if k in ("init_ssm", "init_conv") else v)))
+               for k, v in inp.items()}
+        h1 = make_handle(wb, path)
+        o1, s1, c1, _ = run_forward(h1, wb, to_device(one, wb), init_state_of(h1, wb, one))
+        rel = np.linalg.norm(o_all[b, :L] - o1[0]) / max(np.linalg.norm(o1[0]), 1e-30)
+        assert rel <= 1e-6, f"row {b}: rel-L2 {rel:.2e} against the row run alone"
+        assert np.allclose(s_all[b], s1[0], rtol=1e-6, atol=1e-6 * np.abs(s1[0]).max())
+        if c1 is not None:
+            assert np.array_equal(c_all[b], c1[0])

@@ -36,6 +36,9 @@ MUTANTS = {
     "norm_uses_C_bias_for_B": ("ub[n] = ub[n] * rb * wb + bb;", "ub[n] = ub[n] * rb * wb + bc;"),
     "output_before_update": ("hp[n] = decay * hp[n] + dxp * ub[n];\n                y += uc[n] * hp[n];",
                              "y += uc[n] * hp[n];\n                hp[n] = decay * hp[n] + dxp * ub[n];"),
+    "padding_runs_the_recurrence": ("    for (int t = 0; t < Lb; t++) {", "    for (int t = 0; t < L; t++) {"),
+    "final_history_ignores_length": ("const int L = row_len(d, in, b);   /* the row's last real token is L - 1 */",
+                                     "const int L = d->seqlen;"),
 }
 
 
@@ -106,6 +109,40 @@ def _battery(lib) -> list:
     r2 = oracle.forward(dict(w.dims(), ngroups=2, bc_norm=0), flat)
     if not np.max(np.abs(r["out"] - r2["out"])) <= 1e-5 * np.max(np.abs(r2["out"])):
         failed.append("bcnorm_wiring")
+    # 5. ragged lengths: a row equals the matrix form over its real tokens, padding is +0.0,
+    #    and the final conv history holds the last real raw inputs
+    w = Workload("r", 3, 70, 2, 4, 5, 1, 4, "f32", init_state=True, seed=25)
+    inp = make_inputs(w)
+    rng = np.random.default_rng(2)
+    inp["init_conv"] = rng.standard_normal((3, 3, w.conv_dim)).astype(np.float32)
+    lens = np.array([70, 33, 2], np.int32)
+    res = oracle.forward(w.dims(), dict(inp, lengths=lens), lib=lib)
+    ok = True
+    for b in range(3):
+        L = int(lens[b])
+        pad = res["out"][b, L:]
+        ok &= bool(np.all(pad == 0.0) and not np.any(np.signbit(pad)))
+        # the conv'd x|B|C of the row's real tokens, then the matrix form on them
+        row = {k: (None if v is None else (v[b:b + 1, :L] if k in ("x", "z", "B", "C", "dt_raw")
+                                           else (v[b:b + 1] if k in ("init_ssm", "init_conv") else v)))
+               for k, v in inp.items()}
+        wr = w.with_(batch=1, seqlen=L)
+        u = oracle.conv_stage(wr.dims(), row)[0]   # the unmodified oracle's conv stage
+        HP, GN = 8, 5
+        flat = dict(row, x=u[None, :, :HP].astype(np.float32), B=u[None, :, HP:HP + GN].astype(np.float32),
+                    C=u[None, :, HP + GN:].astype(np.float32), conv_w=None, conv_b=None)
+        dims1 = dict(wr.dims(), dconv=1)
+        for h in range(2):
+            x, z, Bm, Cm, dt, a, D, seq, h0 = head_inputs(flat, dims1, 0, h)
+            y, hf = quadratic_form(x, z, Bm, Cm, dt, a, D, seq, h0)
+            got = res["out"][b, :L, h * 4:(h + 1) * 4]
+            ok &= bool(np.max(np.abs(got - y)) <= 1e-6 * np.max(np.abs(y)))
+            ok &= bool(np.max(np.abs(res["final_ssm"][b, h] - hf)) <= 1e-6 * np.max(np.abs(hf)))
+        raw = np.concatenate([inp["init_conv"][b].astype(np.float64),
+                              np.concatenate([inp["x"][b, :L], inp["B"][b, :L], inp["C"][b, :L]], axis=1)])
+        ok &= bool(np.array_equal(res["final_conv"][b], raw[-3:]))
+    if not ok:
+        failed.append("ragged")
     return failed
 
 

@@ -406,3 +406,53 @@ def test_document_ids_are_compared_between_neighbours(oracle_mod):
     assert np.array_equal(r1["out"], r2["out"])
     assert np.array_equal(r1["final_ssm"], r2["final_ssm"])
     assert np.array_equal(r1["final_conv"], r2["final_conv"])
+
+
+def _row_slice(inp, b, L):
+    """Row b of a batch, truncated to its first L tokens, as a batch of one."""
+    per_tok = ("x", "z", "B", "C", "dt_raw", "seq_idx")
+    out = {}
+    for k, v in inp.items():
+        if v is None:
+            out[k] = None
+        elif k in per_tok or (k == "A" and v.ndim == 3):
+            out[k] = np.ascontiguousarray(v[b:b + 1, :L])
+        elif k in ("init_ssm", "init_conv"):
+            out[k] = np.ascontiguousarray(v[b:b + 1])
+        else:
+            out[k] = v
+    return out
+
+
+@pytest.mark.parametrize("a_per_token", [False, True])
+def test_ragged_rows_equal_truncated_rows(oracle_mod, a_per_token):
+    """Ragged lengths: each row equals the same row run alone over its real
+    tokens, padding outputs are exactly +0.0, and a zero-length row hands its
+    initial state and conv history through unchanged."""
+    w = _small(batch=4, seqlen=150, dconv=4, init_state=True, a_per_token=a_per_token,
+               documents="geometric", mean_doc_len=40)
+    inp = make_inputs(w)
+    rng = np.random.Generator(np.random.PCG64(5))
+    inp["init_conv"] = (0.5 * rng.standard_normal((w.batch, 3, w.conv_dim))).astype(np.float32)
+    lengths = np.array([150, 77, 0, 1], dtype=np.int32)
+    res = oracle_mod.forward(w.dims(), dict(inp, lengths=lengths))
+    for b, L in enumerate(lengths):
+        pad = res["out"][b, L:]
+        assert np.all(pad == 0.0) and not np.any(np.signbit(pad)), "padding must be +0.0"
+        if L == 0:
+            assert np.array_equal(res["final_ssm"][b], inp["init_ssm"][b].astype(np.float64))
+            assert np.array_equal(res["final_conv"][b], inp["init_conv"][b].astype(np.float64))
+            continue
+        one = oracle_mod.forward(w.with_(batch=1, seqlen=int(L)).dims(), _row_slice(inp, b, int(L)))
+        assert np.array_equal(res["out"][b, :L], one["out"][0])
+        assert np.array_equal(res["final_ssm"][b], one["final_ssm"][0])
+        assert np.array_equal(res["final_conv"][b], one["final_conv"][0])
+
+
+def test_full_lengths_equal_no_lengths(oracle_mod):
+    w = _small(batch=2, seqlen=90, dconv=4, documents="geometric", mean_doc_len=30)
+    inp = make_inputs(w)
+    a = oracle_mod.forward(w.dims(), inp)
+    b = oracle_mod.forward(w.dims(), dict(inp, lengths=np.full(w.batch, w.seqlen, np.int32)))
+    for k in ("out", "final_ssm", "final_conv"):
+        assert np.array_equal(a[k], b[k])
