@@ -241,7 +241,7 @@ struct StepIter {
 // Phase parity of the n-th completion (0-based) of a barrier.
 __device__ __forceinline__ uint32_t par(int n) { return (uint32_t)n & 1u; }
 
-template <int NS, bool CONV, bool NORM>
+template <int NS, bool CONV, bool NORM, bool RAG>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
@@ -337,7 +337,8 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
             }
             const int32_t* seq_row = p.seq ? p.seq + (int64_t)b * L : nullptr;
-            const int Lb = row_length(p.lengths, b, L);   // padding: dt = 0 (K2), no boundary
+            // ragged batch: padding after the row's real tokens has dt = 0 (K2) and no boundary
+            const int Lb = RAG ? row_length(p.lengths, b, L) : L;
             const float* dt_row = p.dt + bh * L;
             const float* acs_row = p.acs + bh * L;
             ChunkScalars* cs = &scal[st];
@@ -398,7 +399,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 uint32_t pre = 0;
                 if (t0 - 2 >= 1 && t0 - 2 < Lb && is_boundary(seq_row, t0 - 2)) pre |= 1u;
                 if (t0 - 1 >= 1 && t0 - 1 < Lb && is_boundary(seq_row, t0 - 1)) pre |= 2u;
-                cs->nvalid = (uint32_t)min(max(Lb - t0, 0), 64);
+                if (RAG) cs->nvalid = (uint32_t)min(max(Lb - t0, 0), 64);
                 cs->carry = (m0 | m1) ? kChunkReset : __expf(acs_last);
                 cs->m0 = m0;
                 cs->m1 = m1;
@@ -885,7 +886,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         y = fma2(Dp, bf2(xw[e]), y);
                         ow[e] = pack_bf16_2(mul2(y, silu2(bf2(zw[e]))));
                     }
-                    if (t >= (int)cs->nvalid) ow[0] = ow[1] = ow[2] = ow[3] = 0u;   // ragged padding
+                    if (RAG && t >= (int)cs->nvalid) ow[0] = ow[1] = ow[2] = ow[3] = 0u;   // padding
                     *(uint4*)(outt + tc::sw128_offset(t, col)) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
             }
@@ -1012,11 +1013,11 @@ static void choose_segments(int streams, int nchunks, int grid, size_t cap_items
     }
 }
 
-template <int NS, bool CONV, bool NORM>
+template <int NS, bool CONV, bool NORM, bool RAG>
 static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* maps, int sm_count,
                             size_t max_items, cudaStream_t st)
 {
-    auto kern = ssd_chunk_fused<NS, CONV, NORM>;
+    auto kern = ssd_chunk_fused<NS, CONV, NORM, RAG>;
     const int smem = Layout<NS>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -1079,8 +1080,10 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.cn_w = a.cn_w;
     fp.bn_bias = a.bn_bias;
     fp.cn_bias = a.cn_bias;
-#define SSD_FUSED_LAUNCH(NS_, CONV_, NORM_) launch_t<NS_, CONV_, NORM_>(s, fp, maps, fw.sm_count, fw.max_items, st)
-    const bool conv = s.dconv == 4, norm = s.bc_norm != 0;
+    const bool conv = s.dconv == 4, norm = s.bc_norm != 0, rag = a.lengths != nullptr;
+#define SSD_FUSED_LAUNCH(NS_, CONV_, NORM_)                                                     \
+    (rag ? launch_t<NS_, CONV_, NORM_, true>(s, fp, maps, fw.sm_count, fw.max_items, st)        \
+         : launch_t<NS_, CONV_, NORM_, false>(s, fp, maps, fw.sm_count, fw.max_items, st))
     if (s.dstate == 64)
         return conv ? (norm ? SSD_FUSED_LAUNCH(64, true, true) : SSD_FUSED_LAUNCH(64, true, false))
                     : (norm ? SSD_FUSED_LAUNCH(64, false, true) : SSD_FUSED_LAUNCH(64, false, false));
