@@ -93,6 +93,10 @@ typedef struct {
     int32_t max_batch;   /* >= 1 */
     int32_t max_seqlen;  /* >= 1 */
     int32_t path;        /* ssd_path */
+    int32_t validate_finite;  /* 1: after every forward / step, scan out and the
+                                 fp32 state for NaN or infinity; ssd_check then
+                                 reports SSD_ERR_DEVICE.  Costs one extra read of
+                                 the results.  0: no check. */
 } ssd_desc;
 
 /* Create a handle for one layer shape.  Validates d, picks the path, and
@@ -202,8 +206,10 @@ ssd_status ssd_set_timing_events(ssd_handle* h, void* start, void* stop);
 uint64_t ssd_launch_count(const ssd_handle* h);
 
 /* Wait for `stream`, then read and clear the handle's device status word.
- * SSD_ERR_DEVICE when a kernel reported an error (ssd_last_error says which),
- * SSD_ERR_CUDA when the stream itself failed. */
+ * SSD_ERR_DEVICE when a kernel reported an error -- a bounded wait that timed
+ * out, a rejected launch shape, or (validate_finite) a NaN or infinity in the
+ * results; ssd_last_error says which -- and SSD_ERR_CUDA when the stream
+ * itself failed. */
 ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream);
 
 /*
@@ -234,7 +240,8 @@ ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream);
  *   status      device pointer to one int32 that the caller owns (required);
  *               the kernels OR into it the bits ssd_check reports (1: a bounded
  *               wait timed out and the outputs are invalid; 2: a kernel rejected
- *               its launch shape).  This call neither reads nor clears it.
+ *               its launch shape; 4: with validate_finite, a NaN or infinity in
+ *               out or the final state).  This call neither reads nor clears it.
  *
  * The first call on each device does a one-time set-up with that device
  * current: it looks up the array's device address (cudaGetSymbolAddress) and

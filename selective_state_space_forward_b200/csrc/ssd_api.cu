@@ -124,6 +124,8 @@ ssd_status validate_desc(const ssd_desc* d)
         return fail(SSD_ERR_INVALID_ARG, "max_batch and max_seqlen must be >= 1");
     if (d->path < SSD_PATH_AUTO || d->path > SSD_PATH_STAGED)
         return fail(SSD_ERR_INVALID_ARG, "path %d is not an ssd_path", d->path);
+    if (d->validate_finite != 0 && d->validate_finite != 1)
+        return fail(SSD_ERR_INVALID_ARG, "validate_finite must be 0 or 1 (got %d)", d->validate_finite);
     if (d->path == SSD_PATH_FUSED && !fused_supported(*d))
         return fail(SSD_ERR_UNSUPPORTED,
                     "the fused path needs bf16 activations, headdim 64 and dstate 64 or 128");
@@ -324,6 +326,15 @@ static ssd_status forward_impl(ssd_handle* h, int32_t batch, int32_t seqlen, con
                         "fused chunk kernel");
     }
     if (a.final_conv) SSD_LAUNCH(h, launch_conv_state(s, a, st), "conv-state kernel");
+    if (h->d.validate_finite) {
+        const size_t ob = (size_t)batch * seqlen * h->d.nheads * h->d.headdim * act_size(h->d);
+        SSD_LAUNCH(h, launch_finite_check(out, ob, s.act_bf16, h->status, st), "finite check");
+        if (final_state)
+            SSD_LAUNCH(h, launch_finite_check(final_state, (size_t)batch * h->d.nheads * h->d.headdim *
+                                                               h->d.dstate * sizeof(float),
+                                              false, h->status, st),
+                       "finite check");
+    }
     return SSD_OK;
 }
 
@@ -516,6 +527,15 @@ ssd_status ssd_step(ssd_handle* h, int32_t batch, const void* x, const void* z,
     SSD_MAIN_LAUNCH(h, (cudaStream_t)stream,
                     launch_decode_step(s, a, (float*)state, hist, (cudaStream_t)stream),
                     "decode kernel");
+    if (h->d.validate_finite) {
+        const size_t ob = (size_t)batch * h->d.nheads * h->d.headdim * act_size(h->d);
+        SSD_LAUNCH(h, launch_finite_check(out, ob, s.act_bf16, h->status, (cudaStream_t)stream),
+                   "finite check");
+        SSD_LAUNCH(h, launch_finite_check(state, (size_t)batch * h->d.nheads * h->d.headdim *
+                                                     h->d.dstate * sizeof(float),
+                                          false, h->status, (cudaStream_t)stream),
+                   "finite check");
+    }
     return SSD_OK;
 }
 
@@ -589,9 +609,10 @@ ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream)
     SSD_CUDA(cudaMemcpy(&word, h->status, sizeof word, cudaMemcpyDeviceToHost), "status read");
     if (word == 0) return SSD_OK;
     SSD_CUDA(cudaMemset(h->status, 0, sizeof word), "status clear");
-    return fail(SSD_ERR_DEVICE, "device status 0x%x:%s%s", word,
+    return fail(SSD_ERR_DEVICE, "device status 0x%x:%s%s%s", word,
                 (word & kStatusTimeout) ? " a bounded wait timed out;" : "",
-                (word & kStatusBadLaunch) ? " a kernel rejected its launch shape;" : "");
+                (word & kStatusBadLaunch) ? " a kernel rejected its launch shape;" : "",
+                (word & kStatusNonFinite) ? " a non-finite value in the results;" : "");
 }
 
 ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen, const void* x,
@@ -682,6 +703,14 @@ ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
     SSD_LAUNCH(&h, launch_dt_cumsum(s, a, dt, acs, nullptr, st), "dt/cumsum kernel");
     SSD_LAUNCH(&h, launch_chunk_fused(s, a, ubc, dt, acs, nullptr, status, fw, st), "fused chunk kernel");
     if (a.final_conv) SSD_LAUNCH(&h, launch_conv_state(s, a, st), "conv-state kernel");
+    if (h.d.validate_finite) {
+        SSD_LAUNCH(&h, launch_finite_check(out, (size_t)batch * seqlen * H * 64 * 2, true, status, st),
+                   "finite check");
+        if (final_state)
+            SSD_LAUNCH(&h, launch_finite_check(final_state, streams * 64 * N * sizeof(float), false,
+                                               status, st),
+                       "finite check");
+    }
     return SSD_OK;
 }
 

@@ -15,6 +15,7 @@ namespace ssd {
 // Device status word bits (read and cleared by ssd_check).
 constexpr int kStatusTimeout = 1;   // a bounded wait gave up
 constexpr int kStatusBadLaunch = 2; // a kernel saw a launch shape it cannot serve
+constexpr int kStatusNonFinite = 4; // validate_finite: a result holds a NaN or an infinity
 
 // Shapes of one call, resolved by the host layer.
 struct Shape {
@@ -85,6 +86,10 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
 // convolved B|C (ubc) when dconv = 4, else the raw B and C.
 cudaError_t launch_bc_rms(const Shape& s, const FwdArgs& a, const void* ubc, float* rinv,
                           cudaStream_t st);
+// validate_finite: OR kStatusNonFinite into *status when the `bytes` bytes at
+// data (bf16 or fp32 values; 16-byte aligned, a multiple of 16 bytes) hold a
+// NaN or an infinity.
+cudaError_t launch_finite_check(const void* data, size_t bytes, bool bf16, int* status, cudaStream_t st);
 // K6: one decode token per row, state updated in place.
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
                                cudaStream_t st);

@@ -43,7 +43,7 @@ class SSDError(RuntimeError):
 class Desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "nheads", "headdim", "dstate", "ngroups", "dconv", "chunk", "act_dtype", "a_mode",
-        "bc_norm", "max_batch", "max_seqlen", "path")]
+        "bc_norm", "max_batch", "max_seqlen", "path", "validate_finite")]
 
 
 _lib = None
@@ -123,7 +123,7 @@ class Handle:
 
     def __init__(self, nheads, headdim, dstate, ngroups=1, dconv=4, act_dtype="bf16",
                  a_per_token=False, bc_norm=False, max_batch=1, max_seqlen=1, path="auto",
-                 lib=None):
+                 validate_finite=False, lib=None):
         self.lib = lib or load_library()
         self.nheads, self.headdim, self.dstate, self.ngroups = nheads, headdim, dstate, ngroups
         self.dconv, self.act_dtype = dconv, act_dtype
@@ -132,7 +132,7 @@ class Handle:
         d = Desc(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv,
                  chunk=64, act_dtype=DTYPES[act_dtype][0], a_mode=int(bool(a_per_token)),
                  bc_norm=int(bool(bc_norm)), max_batch=max_batch, max_seqlen=max_seqlen,
-                 path=PATHS[path])
+                 path=PATHS[path], validate_finite=int(bool(validate_finite)))
         h = ctypes.c_void_p()
         _raise(self.lib, self.lib.ssd_create(ctypes.byref(d), ctypes.byref(h)))
         self._h = h

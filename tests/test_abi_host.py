@@ -79,6 +79,7 @@ def _desc(**kw):
     (dict(bc_norm=2), 1, "bc_norm"),
     (dict(max_batch=0), 1, "max_batch"),
     (dict(path=9), 1, "path"),
+    (dict(validate_finite=2), 1, "validate_finite"),
     (dict(path=1, act_dtype=0), 2, "fused"),
     (dict(path=1, headdim=32), 2, "fused"),
 ])

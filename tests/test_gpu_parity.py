@@ -421,3 +421,22 @@ def test_ragged_rows_equal_rows_run_alone(path):
         assert np.allclose(s_all[b], s1[0], rtol=1e-6, atol=1e-6 * np.abs(s1[0]).max())
         if c1 is not None:
             assert np.array_equal(c_all[b], c1[0])
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_ragged_batch_without_conv_with_bc_norm(path):
+    """The ragged variant of the no-conv, B/C-norm, d_state-128 kernels (per-token A)."""
+    w = _small("mamba3_siso", batch=3, seqlen=200, nheads=8, ngroups=2)
+    inp = make_inputs(w)
+    lengths = np.array([200, 70, 0], dtype=np.int32)
+    res = oracle.forward(w.dims(), dict(inp, lengths=lengths))
+    h = make_handle(w, path)
+    dev = to_device(inp, w)
+    if w.bc_norm:
+        h.set_bc_norm(dev["B_norm_w"], dev["C_norm_w"], dev["B_bias"], dev["C_bias"])
+    out, fin = _run_ragged(h, w, dev, init_state_of(h, w, inp), lengths)
+    bits = out.view(torch.int16)
+    for b, L in enumerate(lengths):
+        assert bool(torch.all(bits[b, L:] == 0)), f"row {b}: padding is not +0.0"
+    s, c = state_to_numpy(h, fin, w.batch)
+    _compare_all(w, inp, res, out.double().cpu().numpy(), s, c, f"ragged norm/{h.path}")

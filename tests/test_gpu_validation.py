@@ -100,3 +100,38 @@ def test_check_reports_clean_status(case):
     h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"],
               dev["D"], dev["conv_w"], dev["conv_b"], seq_idx=dev["seq_idx"])
     h.check()
+
+
+@pytest.mark.parametrize("path", ["staged", "auto"])
+def test_validate_finite_reports_a_nan_in_the_results(path):
+    """validate_finite: clean forward and step calls check clean; a NaN planted in
+    z reaches out and ssd_check reports it; the check clears the word."""
+    w = WORKLOADS["mini_k3_mixer"].with_(batch=1, seqlen=128, mean_doc_len=50)
+    inp = make_inputs(w)
+    dev = to_device(inp, w)
+    h = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, w.act_dtype,
+                   max_batch=1, max_seqlen=128, path=path, validate_finite=True)
+    fin = h.new_state(1)
+
+    def fwd():
+        return h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"],
+                         dev["C"], dev["D"], dev["conv_w"], dev["conv_b"], seq_idx=dev["seq_idx"],
+                         final_state=fin)
+
+    fwd()
+    h.check()
+    dev["z"][0, 5, 3] = float("nan")
+    fwd()
+    with pytest.raises(ssd.SSDError, match="non-finite"):
+        h.check()
+    dev["z"][0, 5, 3] = 0.0
+    fwd()
+    h.check()
+    # the decode step: a NaN in z reaches out
+    x1, z1 = dev["x"][:, 0].contiguous(), dev["z"][:, 0].contiguous()
+    z1[0, 7] = float("nan")
+    h.step(x1, z1, dev["dt_raw"][:, 0].contiguous(), dev["dt_bias"], dev["A"],
+           dev["B"][:, 0].contiguous(), dev["C"][:, 0].contiguous(), dev["D"], dev["conv_w"],
+           dev["conv_b"], state=fin)
+    with pytest.raises(ssd.SSDError, match="non-finite"):
+        h.check()
