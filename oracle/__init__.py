@@ -58,6 +58,15 @@ class _Inputs(ctypes.Structure):
         ("lengths", ctypes.POINTER(ctypes.c_int32))]
 
 
+class _S6Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seqlen", "d_inner", "dstate")]
+
+
+class _S6Inputs(ctypes.Structure):
+    _fields_ = [(n, _FP) for n in ("u", "delta", "delta_bias", "A_log", "Bm", "Cm", "D", "z",
+                                   "init")]
+
+
 def _bind(path: str):
     lib = ctypes.CDLL(path)
     dp = ctypes.POINTER(ctypes.c_double)
@@ -72,6 +81,9 @@ def _bind(path: str):
     lib.oracle_bcnorm.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Inputs), dp, dp]
     lib.oracle_bcnorm.restype = ctypes.c_int
     lib.oracle_default_threads.restype = ctypes.c_int
+    lib.oracle_s6_forward.argtypes = [ctypes.POINTER(_S6Dims), ctypes.POINTER(_S6Inputs),
+                                      ctypes.c_int, dp, dp]
+    lib.oracle_s6_forward.restype = ctypes.c_int
     return lib
 
 
@@ -212,3 +224,27 @@ def step(dims: dict, inp: dict, state_ssm, state_conv, threads: int = 0, lib=Non
     i["init_ssm"] = state_ssm
     i["init_conv"] = state_conv
     return forward(d, i, threads=threads, lib=lib)
+
+
+def s6_forward(inp: dict, threads: int = 0, lib=None) -> dict:
+    """The Mamba-1 selective scan (S6), sequential fp64.
+
+    inp: numpy arrays u, delta, z (batch, seqlen, d_inner; z may be None), B, C
+    (batch, seqlen, dstate), A_log (d_inner, dstate), delta_bias, D (d_inner),
+    init (batch, d_inner, dstate) or None.  Returns {"out": (batch, seqlen,
+    d_inner) f64, "final": (batch, d_inner, dstate) f64}.
+    """
+    lib = _load(lib)
+    Bb, L, DI = inp["u"].shape
+    N = inp["B"].shape[2]
+    keep = []
+    d = _S6Dims(batch=Bb, seqlen=L, d_inner=DI, dstate=N)
+    i = _S6Inputs(u=_f32(inp["u"], keep), delta=_f32(inp["delta"], keep),
+                  delta_bias=_f32(inp["delta_bias"], keep), A_log=_f32(inp["A_log"], keep),
+                  Bm=_f32(inp["B"], keep), Cm=_f32(inp["C"], keep), D=_f32(inp["D"], keep),
+                  z=_f32(inp.get("z"), keep), init=_f32(inp.get("init"), keep))
+    out = np.full((Bb, L, DI), np.nan)
+    fin = np.full((Bb, DI, N), np.nan)
+    if lib.oracle_s6_forward(ctypes.byref(d), ctypes.byref(i), int(threads), _dptr(out), _dptr(fin)) < 0:
+        raise ValueError("oracle_s6_forward rejected its arguments")
+    return {"out": out, "final": fin}

@@ -367,3 +367,111 @@ int oracle_bcnorm(const oracle_dims *d, const oracle_inputs *in, double *bh, dou
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------
+ * Mamba-1 selective scan (S6) -- the second scan the pages describe, for the
+ * Falcon-Mamba port (falcon_mamba.ts header, "Mamba-1 / S6"):
+ *
+ *   per batch row b and channel d (d_inner of them), state size N:
+ *     A[d,n] = -exp(clamp(A_log[d,n], -10, 5))       (selective_scan.ts, quoted
+ *                                                      by the falcon_mamba.ts header)
+ *     dt_t   = softplus(delta_t[d] + delta_bias[d])   ("softplus(dt + bias)", no clamp)
+ *     h[n]  <- exp(dt_t A[d,n]) h[n] + dt_t u_t[d] B_t[n]
+ *     y_t    = sum_n C_t[n] h[n] + D[d] u_t[d];   out = y_t * silu(z_t[d]) (no z: y_t)
+ *
+ * A is diagonal (one decay per channel and state), B and C are shared by all
+ * channels of a token, u is the already convolved input (the conv sits before
+ * the x_proj projection that produces delta, B and C).  Same fp64, one-token-
+ * at-a-time evaluation as oracle_forward; rows run in parallel threads.
+ *
+ * Layouts (row-major, float32 in):
+ *   u, delta, z   (batch, seqlen, d_inner)   (z may be NULL)
+ *   Bm, Cm        (batch, seqlen, dstate)
+ *   A_log         (d_inner, dstate);  delta_bias, D (d_inner)
+ *   init          (batch, d_inner, dstate) or NULL (zeros)
+ * Out (double): out (batch, seqlen, d_inner); fin (batch, d_inner, dstate) or NULL.
+ */
+typedef struct {
+    int batch, seqlen, d_inner, dstate;
+} oracle_s6_dims;
+
+typedef struct {
+    const float *u, *delta, *delta_bias, *A_log, *Bm, *Cm, *D, *z, *init;
+} oracle_s6_inputs;
+
+typedef struct {
+    const oracle_s6_dims *d;
+    const oracle_s6_inputs *in;
+    double *out, *fin;
+    int next;
+    pthread_mutex_t lock;
+} s6_job;
+
+static void s6_row(const oracle_s6_dims *d, const oracle_s6_inputs *in, int b, double *out, double *fin)
+{
+    const int L = d->seqlen, DI = d->d_inner, N = d->dstate;
+    double *h = malloc(sizeof(double) * (size_t)DI * N);
+    double *a = malloc(sizeof(double) * (size_t)DI * N);
+    if (!h || !a) abort();
+    for (int c = 0; c < DI; c++)
+        for (int n = 0; n < N; n++) {
+            double al = in->A_log[(size_t)c * N + n];
+            if (al < -10.0) al = -10.0;
+            if (al > 5.0) al = 5.0;
+            a[(size_t)c * N + n] = -exp(al);
+            h[(size_t)c * N + n] = in->init ? in->init[((size_t)b * DI + c) * N + n] : 0.0;
+        }
+    for (int t = 0; t < L; t++) {
+        const size_t tok = (size_t)b * L + t;
+        const float *Bt = in->Bm + tok * N, *Ct = in->Cm + tok * N;
+        for (int c = 0; c < DI; c++) {
+            const double dt = softplus_exact((double)in->delta[tok * DI + c] + in->delta_bias[c]);
+            const double uv = in->u[tok * DI + c];
+            double *hc = h + (size_t)c * N;
+            double y = 0.0;
+            for (int n = 0; n < N; n++) {
+                hc[n] = exp(dt * a[(size_t)c * N + n]) * hc[n] + dt * uv * Bt[n];
+                y += Ct[n] * hc[n];
+            }
+            y += in->D[c] * uv;
+            out[tok * DI + c] = in->z ? y * silu(in->z[tok * DI + c]) : y;
+        }
+    }
+    if (fin) memcpy(fin + (size_t)b * DI * N, h, sizeof(double) * (size_t)DI * N);
+    free(h); free(a);
+}
+
+static void *s6_worker(void *arg)
+{
+    s6_job *j = arg;
+    for (;;) {
+        pthread_mutex_lock(&j->lock);
+        const int b = j->next++;
+        pthread_mutex_unlock(&j->lock);
+        if (b >= j->d->batch) break;
+        s6_row(j->d, j->in, b, j->out, j->fin);
+    }
+    return NULL;
+}
+
+/* Returns the number of threads used, or -1 on a bad argument. */
+int oracle_s6_forward(const oracle_s6_dims *d, const oracle_s6_inputs *in, int nthreads,
+                      double *out, double *fin)
+{
+    if (!d || !in || !out || d->batch < 0 || d->seqlen < 1 || d->d_inner < 1 || d->dstate < 1)
+        return -1;
+    if (!in->u || !in->delta || !in->delta_bias || !in->A_log || !in->Bm || !in->Cm || !in->D)
+        return -1;
+    s6_job j;
+    j.d = d; j.in = in; j.out = out; j.fin = fin; j.next = 0;
+    pthread_mutex_init(&j.lock, NULL);
+    if (nthreads <= 0) nthreads = oracle_default_threads();
+    if (nthreads > d->batch) nthreads = d->batch > 0 ? d->batch : 1;
+    pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int i = 1; i < nthreads; i++) pthread_create(&th[i], NULL, s6_worker, &j);
+    s6_worker(&j);
+    for (int i = 1; i < nthreads; i++) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&j.lock);
+    return nthreads;
+}

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 
 from brute_force import head_inputs, quadratic_form, silu
+from test_oracle_s6 import _inputs as _s6_inputs, _matrix_form as _s6_matrix_form
 from selective_state_space_forward_b200.synthetic import Workload, make_inputs
 
 import oracle
@@ -39,6 +40,13 @@ MUTANTS = {
     "padding_runs_the_recurrence": ("    for (int t = 0; t < Lb; t++) {", "    for (int t = 0; t < L; t++) {"),
     "final_history_ignores_length": ("const int L = row_len(d, in, b);   /* the row's last real token is L - 1 */",
                                      "const int L = d->seqlen;"),
+    "s6_no_clamp": ("            if (al < -10.0) al = -10.0;\n            if (al > 5.0) al = 5.0;\n", ""),
+    "s6_decay_sign": ("hc[n] = exp(dt * a[(size_t)c * N + n]) * hc[n] + dt * uv * Bt[n];",
+                      "hc[n] = exp(-dt * a[(size_t)c * N + n]) * hc[n] + dt * uv * Bt[n];"),
+    "s6_output_with_B": ("                y += Ct[n] * hc[n];", "                y += Bt[n] * hc[n];"),
+    "s6_drop_D": ("            y += in->D[c] * uv;", "            y += 0.0 * uv;"),
+    "s6_no_gate": ("out[tok * DI + c] = in->z ? y * silu(in->z[tok * DI + c]) : y;",
+                   "out[tok * DI + c] = y;"),
 }
 
 
@@ -143,6 +151,15 @@ def _battery(lib) -> list:
         ok &= bool(np.array_equal(res["final_conv"][b], raw[-3:]))
     if not ok:
         failed.append("ragged")
+    # 6. S6: the matrix form, with A_log values beyond both clamp bounds
+    inp = _s6_inputs(B=1, L=30, DI=3, N=4, seed=26)
+    inp["A_log"][0, 0] = 7.0
+    inp["A_log"][1, 2] = -12.0
+    r = oracle.s6_forward(inp, lib=lib)
+    y, hf = _s6_matrix_form(inp)
+    if not (np.max(np.abs(r["out"] - y)) <= 1e-10 * np.max(np.abs(y)) and
+            np.max(np.abs(r["final"] - hf)) <= 1e-10 * np.max(np.abs(hf))):
+        failed.append("s6_matrix_form")
     return failed
 
 
