@@ -257,6 +257,29 @@ ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
                                const int32_t* seq_idx, const void* init_state, void* out,
                                void* final_state, int32_t* status, struct CUstream_st* stream);
 
+/*
+ * Mamba-1 selective scan (S6), the scan of the Falcon-Mamba port (falcon_mamba.ts
+ * header: a Mamba-1 / S6 model; A = -exp(clamp(A_log, -10, 5)) as
+ * selective_scan.ts computes it; dt = softplus(dt + bias)).  Per row b and
+ * channel d (d_inner channels, state size dstate):
+ *   h[n] <- exp(dt A[d,n]) h[n] + dt u B[n];  y = C.h + D[d] u;  out = y SiLU(z)
+ * No handle: the call allocates nothing and keeps no state between calls.
+ *   u, z, out   (batch, seqlen, d_inner) act_dtype; u is the convolved input,
+ *               z NULL = no gate; out may not alias an input
+ *   delta       (batch, seqlen, d_inner) fp32, before softplus
+ *   delta_bias, D (d_inner) fp32;  A_log (d_inner, dstate) fp32
+ *   B, C        (batch, seqlen, dstate) act_dtype, shared by every channel
+ *   init_state, final_state  (batch, d_inner, dstate) fp32, or NULL (zeros / not
+ *               written); they may be the same buffer
+ *   dstate      8, 16 or 32 (else SSD_ERR_UNSUPPORTED); act_dtype an ssd_dtype
+ * Arguments are validated before any launch, as for ssd_forward.
+ */
+ssd_status ssd_s6_forward(int32_t batch, int32_t seqlen, int32_t d_inner, int32_t dstate,
+                          int32_t act_dtype, const void* u, const float* delta,
+                          const float* delta_bias, const float* A_log, const void* B,
+                          const void* C, const float* D, const void* z, const float* init_state,
+                          void* out, float* final_state, struct CUstream_st* stream);
+
 /* The calling thread's last error message ("" when none). */
 const char* ssd_last_error(void);
 

@@ -615,6 +615,55 @@ ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream)
                 (word & kStatusNonFinite) ? " a non-finite value in the results;" : "");
 }
 
+ssd_status ssd_s6_forward(int32_t batch, int32_t seqlen, int32_t d_inner, int32_t dstate,
+                          int32_t act_dtype, const void* u, const float* delta,
+                          const float* delta_bias, const float* A_log, const void* B,
+                          const void* C, const float* D, const void* z, const float* init_state,
+                          void* out, float* final_state, struct CUstream_st* stream)
+{
+    g_err.clear();
+    if (batch < 0 || seqlen < 0)
+        return fail(SSD_ERR_INVALID_ARG, "batch (%d) and seqlen (%d) must be >= 0", batch, seqlen);
+    if (d_inner < 1) return fail(SSD_ERR_INVALID_ARG, "d_inner must be >= 1 (got %d)", d_inner);
+    if (dstate != 8 && dstate != 16 && dstate != 32)
+        return fail(SSD_ERR_UNSUPPORTED, "dstate must be 8, 16 or 32 (got %d)", dstate);
+    if (act_dtype != SSD_DTYPE_F32 && act_dtype != SSD_DTYPE_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "act_dtype %d is not an ssd_dtype", act_dtype);
+    const size_t ea = act_dtype == SSD_DTYPE_BF16 ? 2 : 4;
+    SSD_TRY(check_ptr(init_state, "init_state", 4, false));
+    SSD_TRY(check_ptr(final_state, "final_state", 4, false));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (batch == 0) return SSD_OK;
+    if (seqlen == 0) {   // no token: the state passes through unchanged
+        if (final_state && final_state != init_state) {
+            const size_t n = (size_t)batch * d_inner * dstate * sizeof(float);
+            SSD_CUDA(init_state ? cudaMemcpyAsync(final_state, init_state, n, cudaMemcpyDeviceToDevice, st)
+                                : cudaMemsetAsync(final_state, 0, n, st),
+                     "empty-sequence state copy");
+        }
+        return SSD_OK;
+    }
+    SSD_TRY(check_ptr(u, "u", ea, true));
+    SSD_TRY(check_ptr(delta, "delta", 4, true));
+    SSD_TRY(check_ptr(delta_bias, "delta_bias", 4, true));
+    SSD_TRY(check_ptr(A_log, "A_log", 4, true));
+    SSD_TRY(check_ptr(B, "B", ea, true));
+    SSD_TRY(check_ptr(C, "C", ea, true));
+    SSD_TRY(check_ptr(D, "D", 4, true));
+    SSD_TRY(check_ptr(z, "z", ea, false));
+    SSD_TRY(check_ptr(out, "out", ea, true));
+    if (out == u || out == z || out == B || out == C)
+        return fail(SSD_ERR_INVALID_ARG, "out may not alias an input");
+    S6Args s;
+    s.batch = batch; s.seqlen = seqlen; s.d_inner = d_inner; s.dstate = dstate;
+    s.bf16 = act_dtype == SSD_DTYPE_BF16;
+    s.u = u; s.B = B; s.C = C; s.z = z;
+    s.delta = delta; s.delta_bias = delta_bias; s.A_log = A_log; s.D = D;
+    s.init = init_state; s.out = out; s.fin = final_state;
+    SSD_CUDA(launch_s6_scan(s, st), "S6 scan kernel");
+    return SSD_OK;
+}
+
 ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen, const void* x,
                                const void* z, const float* dt_raw, const float* dt_bias,
                                const float* A, const void* B, const void* C, const float* D,

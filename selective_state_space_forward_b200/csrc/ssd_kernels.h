@@ -90,6 +90,16 @@ cudaError_t launch_bc_rms(const Shape& s, const FwdArgs& a, const void* ubc, flo
 // data (bf16 or fp32 values; 16-byte aligned, a multiple of 16 bytes) hold a
 // NaN or an infinity.
 cudaError_t launch_finite_check(const void* data, size_t bytes, bool bf16, int* status, cudaStream_t st);
+// Mamba-1 selective scan (S6): device pointers of one call.
+struct S6Args {
+    int batch, seqlen, d_inner, dstate, bf16;
+    const void *u, *B, *C, *z;          // act dtype; z may be null
+    const float *delta, *delta_bias, *A_log, *D;
+    const float* init;                  // (batch, d_inner, dstate) or null
+    void* out;
+    float* fin;                         // or null
+};
+cudaError_t launch_s6_scan(const S6Args& s, cudaStream_t st);
 // K6: one decode token per row, state updated in place.
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
                                cudaStream_t st);

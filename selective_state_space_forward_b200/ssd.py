@@ -31,7 +31,7 @@ DTYPES = {"f32": (0, torch.float32), "bf16": (1, torch.bfloat16)}
 EXPORTS = ("ssd_create", "ssd_destroy", "ssd_get_path", "ssd_set_bc_norm", "ssd_state_bytes",
            "ssd_state_conv_offset", "ssd_forward", "ssd_step", "ssd_stage_conv", "ssd_stage_dt",
            "ssd_set_timing_events", "ssd_launch_count", "ssd_check", "ssd_last_error",
-           "ssd_status_string", "ssd_forward_noalloc", "ssd_forward_ragged")
+           "ssd_status_string", "ssd_forward_noalloc", "ssd_forward_ragged", "ssd_s6_forward")
 
 
 class SSDError(RuntimeError):
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_state_conv_offset.restype = sz
     lib.ssd_forward.argtypes = [vp, i32, i32] + [vp] * 14 + [vp]
     lib.ssd_forward_ragged.argtypes = [vp, i32, i32] + [vp] * 15 + [vp]
+    lib.ssd_s6_forward.argtypes = [i32, i32, i32, i32, i32] + [vp] * 11 + [vp]
     lib.ssd_step.argtypes = [vp, i32] + [vp] * 13
     lib.ssd_stage_conv.argtypes = [vp, i32, i32] + [vp] * 9
     lib.ssd_stage_dt.argtypes = [vp, i32, i32] + [vp] * 7
@@ -85,7 +86,7 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), i32, i32] + [vp] * 15 + [vp]
     for f in ("ssd_create", "ssd_set_bc_norm", "ssd_forward", "ssd_step", "ssd_stage_conv",
               "ssd_stage_dt", "ssd_set_timing_events", "ssd_check", "ssd_forward_noalloc",
-              "ssd_forward_ragged"):
+              "ssd_forward_ragged", "ssd_s6_forward"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -286,5 +287,27 @@ def forward_noalloc(x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None,
         _ptr(conv_b, at, "conv_b"), _ptr(seq_idx, torch.int32, "seq_idx"),
         _ptr(init_state, torch.uint8, "init_state"), _ptr(out, at, "out"),
         _ptr(final_state, torch.uint8, "final_state"), _ptr(status, torch.int32, "status"),
+        _stream(stream)))
+    return out
+
+
+def s6_forward(u, delta, delta_bias, A_log, B, C, D, z=None, init_state=None, out=None,
+               final_state=None, stream=None, lib=None):
+    """ssd_s6_forward (the Mamba-1 selective scan); returns `out` (allocated like u when
+    not given).  u, z, B, C: bf16 or fp32 CUDA tensors; the rest fp32."""
+    lib = lib or load_library()
+    f = torch.float32
+    if u.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("u must be bf16 or fp32")
+    at = u.dtype
+    batch, seqlen, d_inner = u.shape
+    dstate = A_log.shape[1]
+    if out is None:
+        out = torch.empty_like(u)
+    _raise(lib, lib.ssd_s6_forward(
+        batch, seqlen, d_inner, dstate, 1 if at == torch.bfloat16 else 0, _ptr(u, at, "u"),
+        _ptr(delta, f, "delta"), _ptr(delta_bias, f, "delta_bias"), _ptr(A_log, f, "A_log"),
+        _ptr(B, at, "B"), _ptr(C, at, "C"), _ptr(D, f, "D"), _ptr(z, at, "z"),
+        _ptr(init_state, f, "init_state"), _ptr(out, at, "out"), _ptr(final_state, f, "final_state"),
         _stream(stream)))
     return out

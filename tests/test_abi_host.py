@@ -23,7 +23,7 @@ def lib():
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ssd_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_what_the_binding_lists():
@@ -39,7 +39,7 @@ def _declared_param_counts():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     out = {}
-    for m in re.finditer(r"\b(ssd_[a-z_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+    for m in re.finditer(r"\b(ssd_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
         params = m.group(2).strip()
         out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
     return out
