@@ -48,6 +48,7 @@ def parse_args(argv=None):
     p.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--no-s6", action="store_true", help="skip the Mamba-1 (S6) scan measurement")
     return p.parse_args(argv)
 
 
@@ -404,6 +405,65 @@ def bench_decode(args, torch, peaks):
             "traffic": measured_traffic(f"decode:{DECODE_WORKLOAD}", "decode")}
 
 
+# Mamba-1 selective scan (S6) at the Falcon-Mamba-7B mixer shape.
+S6_SHAPE = dict(batch=2, seqlen=4096, d_inner=8192, dstate=16)
+# MUFU (transcendental) issue rate assumed for the roofline: 16 results per clock per SM.
+MUFU_PER_SM_CLK = 16
+
+
+def bench_s6(args, torch, peaks, sm_mhz):
+    """ssd_s6_forward over synthetic Falcon-Mamba-7B mixer inputs (bf16 u, z, B, C; fp32
+    dt, A_log, D, states), each call timed alone with CUDA events; the inputs (674 MB) are
+    larger than L2.  Rooflines: HBM bytes, and the MUFU pipe, which takes the dstate
+    exponentials of every (token, channel) plus the softplus and the gate's tanh."""
+    from selective_state_space_forward_b200 import ssd
+    Bb, L, DI, N = (S6_SHAPE[k] for k in ("batch", "seqlen", "d_inner", "dstate"))
+    g = torch.Generator(device="cuda").manual_seed(9)
+    bf = torch.bfloat16
+
+    def rnd(*shape, dtype=torch.float32):
+        return torch.randn(*shape, generator=g, device="cuda").to(dtype)
+
+    u, z = rnd(Bb, L, DI, dtype=bf), rnd(Bb, L, DI, dtype=bf)
+    delta = rnd(Bb, L, DI) - 2.0
+    Bm, Cm = rnd(Bb, L, N, dtype=bf), rnd(Bb, L, N, dtype=bf)
+    A_log = torch.log(torch.rand(DI, N, generator=g, device="cuda") * (N - 1) + 1.0)
+    dbias = torch.rand(DI, generator=g, device="cuda") * -2.0
+    D = torch.rand(DI, generator=g, device="cuda")
+    state = torch.zeros(Bb, DI, N, device="cuda")
+    out = torch.empty_like(u)
+
+    def call():
+        ssd.s6_forward(u, delta, dbias, A_log, Bm, Cm, D, z=z, init_state=state, out=out,
+                       final_state=state)
+
+    for _ in range(3):
+        call()
+    ts = []
+    for _ in range(max(5, min(args.steps, 20))):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = sorted(ts)[len(ts) // 2]
+    tc = Bb * L * DI
+    nbytes = tc * (2 + 4 + 2 + 2) + 2 * Bb * L * N * 2 + 2 * Bb * DI * N * 4
+    mufu = tc * (N + 3)
+    mhz = sm_mhz or 1965
+    mufu_peak = 148 * MUFU_PER_SM_CLK * mhz * 1e6
+    return {"workload": "falcon_mamba_7b_mixer: Mamba-1 selective scan, batch 2 x 4096 tokens, "
+                        "d_inner 8192, d_state 16, bf16 u/z/B/C, fp32 dt/A/D/state",
+            "ms_per_call": round(ms, 4), "tokens_per_s": Bb * L / (ms * 1e-3),
+            "roofline": {"bound": "alu", "unit": "Gop/s (MUFU)", "achieved": round(mufu / (ms * 1e-3) / 1e9, 1),
+                         "peak": round(mufu_peak / 1e9, 1), "frac": round(mufu / (ms * 1e-3) / mufu_peak, 4),
+                         "peak_source": f"148 SMs x {MUFU_PER_SM_CLK} MUFU results/clk x {mhz} MHz"},
+            "hbm": {"algorithmic_bytes": nbytes, "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                    "frac_of_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "l2": "inputs larger than L2 (674 MB), no flush"}
+
+
 # ---------------------------------------------------------------------------------------
 _INPUT_CACHE = {}
 
@@ -498,6 +558,10 @@ def main(argv=None):
     if not args.no_decode and rank == 0:
         torch.cuda.empty_cache()
         decode = bench_decode(args, torch, peaks)
+    s6 = None
+    if not args.no_s6 and rank == 0:
+        torch.cuda.empty_cache()
+        s6 = bench_s6(args, torch, peaks, fwd["clocks"].get("sm_mhz"))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         v, desc, threads, _ = cpu_oracle_run(None)
@@ -508,7 +572,7 @@ def main(argv=None):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic", "config": config_block(world),
                 "path": fwd["path"], "roofline": fwd["roofline"],
-                "forward_roofline": fwd["forward_roofline"], "decode": decode,
+                "forward_roofline": fwd["forward_roofline"], "decode": decode, "s6": s6,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": fwd["launches"],
                 "clocks": fwd["clocks"]}
         print(json.dumps(line), flush=True)
