@@ -67,6 +67,12 @@ class _S6Inputs(ctypes.Structure):
                                    "init")]
 
 
+class _Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.POINTER(ctypes.c_double)) for n in (
+        "x", "z", "Bm", "Cm", "dt_raw", "dt_bias", "A", "D", "conv_w", "conv_b",
+        "bn_w", "cn_w", "bn_bias", "cn_bias")]
+
+
 def _bind(path: str):
     lib = ctypes.CDLL(path)
     dp = ctypes.POINTER(ctypes.c_double)
@@ -84,6 +90,9 @@ def _bind(path: str):
     lib.oracle_s6_forward.argtypes = [ctypes.POINTER(_S6Dims), ctypes.POINTER(_S6Inputs),
                                       ctypes.c_int, dp, dp]
     lib.oracle_s6_forward.restype = ctypes.c_int
+    lib.oracle_backward.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Inputs), _FP,
+                                    ctypes.c_int, ctypes.POINTER(_Grads)]
+    lib.oracle_backward.restype = ctypes.c_int
     return lib
 
 
@@ -248,3 +257,40 @@ def s6_forward(inp: dict, threads: int = 0, lib=None) -> dict:
     if lib.oracle_s6_forward(ctypes.byref(d), ctypes.byref(i), int(threads), _dptr(out), _dptr(fin)) < 0:
         raise ValueError("oracle_s6_forward rejected its arguments")
     return {"out": out, "final": fin}
+
+
+def backward(dims: dict, inp: dict, gout, threads: int = 0, lib=None) -> dict:
+    """Gradients of a zero-state prefill (the vector-Jacobian product of forward).
+
+    dims / inp as for ``forward`` (init_ssm and init_conv must be None); gout is
+    the gradient of the loss with respect to ``out``, (batch, seqlen, H*P).
+    Returns float64 gradients under the input names: x, z, B, C, dt_raw,
+    dt_bias, A, D, and conv_w, conv_b (with a conv) and B_norm_w, C_norm_w,
+    B_bias, C_bias (with the B/C norm); the others are None.
+    """
+    lib = _load(lib)
+    if inp.get("init_ssm") is not None or inp.get("init_conv") is not None:
+        raise ValueError("backward is defined for a zero-state prefill only")
+    d, i, keep = _marshal(dims, inp)
+    Bb, L, H, P, N, G, K = (dims["batch"], dims["seqlen"], dims["nheads"], dims["headdim"],
+                            dims["dstate"], dims["ngroups"], dims.get("dconv", 1))
+    cd = H * P + 2 * G * N
+    norm = bool(dims.get("bc_norm"))
+    g = {
+        "x": np.zeros((Bb, L, H * P)), "z": np.zeros((Bb, L, H * P)),
+        "B": np.zeros((Bb, L, G * N)), "C": np.zeros((Bb, L, G * N)),
+        "dt_raw": np.zeros((Bb, L, H)), "dt_bias": np.zeros(H),
+        "A": np.zeros((Bb, L, H) if dims.get("a_per_token") else H), "D": np.zeros(H),
+        "conv_w": np.zeros((cd, K)) if K > 1 else None, "conv_b": np.zeros(cd) if K > 1 else None,
+        "B_norm_w": np.zeros(N) if norm else None, "C_norm_w": np.zeros(N) if norm else None,
+        "B_bias": np.zeros((H, N)) if norm else None, "C_bias": np.zeros((H, N)) if norm else None,
+    }
+    gr = _Grads(x=_dptr(g["x"]), z=_dptr(g["z"]), Bm=_dptr(g["B"]), Cm=_dptr(g["C"]),
+                dt_raw=_dptr(g["dt_raw"]), dt_bias=_dptr(g["dt_bias"]), A=_dptr(g["A"]),
+                D=_dptr(g["D"]), conv_w=_dptr(g["conv_w"]), conv_b=_dptr(g["conv_b"]),
+                bn_w=_dptr(g["B_norm_w"]), cn_w=_dptr(g["C_norm_w"]),
+                bn_bias=_dptr(g["B_bias"]), cn_bias=_dptr(g["C_bias"]))
+    go = _f32(gout, keep)
+    if lib.oracle_backward(ctypes.byref(d), ctypes.byref(i), go, int(threads), ctypes.byref(gr)) < 0:
+        raise ValueError("oracle_backward rejected its arguments")
+    return g

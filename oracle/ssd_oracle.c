@@ -475,3 +475,372 @@ int oracle_s6_forward(const oracle_s6_dims *d, const oracle_s6_inputs *in, int n
     pthread_mutex_destroy(&j.lock);
     return nthreads;
 }
+
+/* ------------------------------------------------------------------------------------
+ * Backward of a zero-state prefill: the vector-Jacobian product of
+ * oracle_forward (mojolearn Mamba3Block, method "backward": the gradients of
+ * the loss with respect to the forward input and every weight, given the
+ * gradient of the output; nothing with respect to a carried state, and no
+ * final-state cotangent -- so init_ssm and init_conv must be NULL).
+ *
+ * Plain reverse-mode differentiation of the same per-token steps 1-9, in
+ * double precision, done per batch row:
+ *
+ *   forward sweep   per head, token by token, keeping every state h_t;
+ *   reverse sweep   per head, from the row's last real token to the first:
+ *     out = y silu(z)          gy = gout silu(z),  gz = gout y silu'(z)
+ *     y = C.h_t + D u_x        gC += gy h_t, gh_t += gy C, gD += gy u_x, gu_x += gy D
+ *     h_t = e h_{t-1} + dt u_x B
+ *                              ge = <gh_t, h_{t-1}>, gdt += <gh_t, u_x B>,
+ *                              gu_x += dt gh_t B, gB += dt gh_t^T u_x,
+ *                              gh_{t-1} = e gh_t, or 0 when t starts a document
+ *     e = exp(dt a)            gdt += ge e a,  ga = ge e dt
+ *     dt = softplus(v)         gv = gdt sigmoid(v) -> dt_raw[t], dt_bias
+ *     a = min(A, -1e-4)        ga passes where A <= -1e-4, else 0 (per-token A)
+ *     B^ = B r w + bias, r = (mean(B^2) + 1e-5)^(-1/2)
+ *                              gw += gB^ B r, gbias += gB^,
+ *                              gB = r w gB^ - (r^3 / N) B <gB^, w B>
+ *   then the conv of the row:  u = silu(pre), pre = b + sum_k w_k x[t-3+k] (same document)
+ *                              gpre = gu silu'(pre), gb += gpre, gw_k += gpre x[.],
+ *                              gx[.] += gpre w_k
+ *
+ * B and C (and their conv channels) are shared by the heads of a group, so
+ * their gradients are sums over those heads.  Weight gradients are summed
+ * per row, and then over rows in row order.  Padding tokens of a ragged row
+ * (t >= lengths[b]) take no part: every gradient there is 0 and the output
+ * gradient there is ignored.
+ *
+ * gout has the layout of out (float32).  Gradients (double) have the layout
+ * of the input they belong to; the conv ones (conv_w, conv_b) are only
+ * written when dconv > 1 and the norm ones (bn_w .. cn_bias) only when
+ * bc_norm != 0.
+ */
+typedef struct {
+    double *x, *z, *Bm, *Cm, *dt_raw, *dt_bias, *A, *D, *conv_w, *conv_b;
+    double *bn_w, *cn_w, *bn_bias, *cn_bias;
+} oracle_grads;
+
+/* Weight gradients of one batch row (summed over rows afterwards). */
+typedef struct {
+    double *dt_bias, *A, *D, *conv_w, *conv_b, *bn_w, *cn_w, *bn_bias, *cn_bias;
+} row_wgrads;
+
+/* What token t of head h sees: u_x (P), the raw group B/C after the conv (N),
+ * the per-head B^/C^ (N), the norms' 1/rms, dt, its softplus argument, the
+ * decay rate and whether the per-token floor replaced it. */
+typedef struct {
+    double *ux, *ub, *uc, *bh, *ch;
+    double rb, rc, dt, v, a, decay;
+    int floored;
+} tok_terms;
+
+static void token_terms(const oracle_dims *d, const oracle_inputs *in, int b, int h, int t,
+                        tok_terms *k)
+{
+    const int P = d->headdim, N = d->dstate, H = d->nheads;
+    const int g = h / (H / d->ngroups);
+    const int dx = H * P, gn = d->ngroups * N;
+    for (int p = 0; p < P; p++) k->ux[p] = conv_silu(d, in, b, t, h * P + p);
+    for (int n = 0; n < N; n++) {
+        k->ub[n] = conv_silu(d, in, b, t, dx + g * N + n);
+        k->uc[n] = conv_silu(d, in, b, t, dx + gn + g * N + n);
+    }
+    k->rb = k->rc = 1.0;
+    if (d->bc_norm) {
+        double sb = 0.0, sc = 0.0;
+        for (int n = 0; n < N; n++) { sb += k->ub[n] * k->ub[n]; sc += k->uc[n] * k->uc[n]; }
+        k->rb = 1.0 / sqrt(sb / N + 1e-5);
+        k->rc = 1.0 / sqrt(sc / N + 1e-5);
+    }
+    for (int n = 0; n < N; n++) {
+        if (d->bc_norm) {
+            const double wb = in->bn_w ? in->bn_w[n] : 1.0, wc = in->cn_w ? in->cn_w[n] : 1.0;
+            const double bb = in->bn_bias ? in->bn_bias[(size_t)h * N + n] : 0.0;
+            const double bc = in->cn_bias ? in->cn_bias[(size_t)h * N + n] : 0.0;
+            k->bh[n] = k->ub[n] * k->rb * wb + bb;
+            k->ch[n] = k->uc[n] * k->rc * wc + bc;
+        } else {
+            k->bh[n] = k->ub[n];
+            k->ch[n] = k->uc[n];
+        }
+    }
+    const size_t tok = (size_t)b * d->seqlen + t;
+    k->v = (double)in->dt_raw[tok * H + h] + in->dt_bias[h];
+    k->dt = softplus_exact(k->v);
+    k->floored = 0;
+    if (d->a_per_token) {
+        k->a = in->A[tok * H + h];
+        if (k->a > -1e-4) { k->a = -1e-4; k->floored = 1; }
+    } else {
+        k->a = in->A[h];
+    }
+    k->decay = exp(k->dt * k->a);
+}
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* d silu(v) / dv */
+static double silu_grad(double v)
+{
+    const double s = sigmoid(v);
+    return s * (1.0 + v * (1.0 - s));
+}
+
+/* Pre-activation of conv channel ch at (b, t) (no initial history: zero-state prefill). */
+static double conv_pre(const oracle_dims *d, const oracle_inputs *in, int b, int t, int ch)
+{
+    const int K = d->dconv;
+    double acc = in->conv_b[ch];
+    for (int k = 0; k < K; k++) {
+        const int tau = t - (K - 1) + k;
+        if (tau >= 0 && same_doc(in, d, b, tau, t))
+            acc += (double)in->conv_w[(size_t)ch * K + k] * xbc_raw(d, in, b, tau, ch);
+    }
+    return acc;
+}
+
+static void backward_row(const oracle_dims *d, const oracle_inputs *in, const float *gout, int b,
+                         const oracle_grads *gr, row_wgrads *wg)
+{
+    const int L = d->seqlen, P = d->headdim, N = d->dstate, H = d->nheads, G = d->ngroups;
+    const int dx = H * P, gn = G * N, cd = conv_dim_of(d), K = d->dconv;
+    const int Lb = row_len(d, in, b);
+    double *gu = calloc((size_t)L * cd, sizeof(double));     /* gradient of the conv output */
+    double *hist = malloc(sizeof(double) * ((size_t)(Lb > 0 ? Lb : 1) * P * N));
+    double *gh = malloc(sizeof(double) * (size_t)P * N);
+    double *buf = malloc(sizeof(double) * (size_t)(P + 4 * N));
+    double *gux = malloc(sizeof(double) * (size_t)P);
+    double *gbh = malloc(sizeof(double) * (size_t)N), *gch = malloc(sizeof(double) * (size_t)N);
+    if (!gu || !hist || !gh || !buf || !gux || !gbh || !gch) abort();
+    tok_terms k;
+    k.ux = buf; k.ub = buf + P; k.uc = k.ub + N; k.bh = k.uc + N; k.ch = k.bh + N;
+
+    for (int h = 0; h < H; h++) {
+        const int g = h / (H / G);
+        /* forward sweep: every state h_t after its update */
+        for (int t = 0; t < Lb; t++) {
+            token_terms(d, in, b, h, t, &k);
+            const int carry = t > 0 && same_doc(in, d, b, t - 1, t);
+            double *ht = hist + (size_t)t * P * N;
+            for (int p = 0; p < P; p++)
+                for (int n = 0; n < N; n++) {
+                    const double prev = carry ? hist[((size_t)(t - 1) * P + p) * N + n] : 0.0;
+                    ht[p * N + n] = k.decay * prev + k.dt * k.ux[p] * k.bh[n];
+                }
+        }
+        /* reverse sweep */
+        memset(gh, 0, sizeof(double) * (size_t)P * N);
+        for (int t = Lb - 1; t >= 0; t--) {
+            token_terms(d, in, b, h, t, &k);
+            const size_t tok = (size_t)b * L + t;
+            const int carry = t > 0 && same_doc(in, d, b, t - 1, t);
+            const double *ht = hist + (size_t)t * P * N;
+            const double *hprev = carry ? hist + (size_t)(t - 1) * P * N : NULL;
+            for (int n = 0; n < N; n++) { gbh[n] = 0.0; gch[n] = 0.0; }
+            for (int p = 0; p < P; p++) {
+                double y = 0.0;
+                for (int n = 0; n < N; n++) y += k.ch[n] * ht[p * N + n];
+                y += in->D[h] * k.ux[p];
+                const double zv = in->z[tok * dx + h * P + p];
+                const double go = gout[tok * dx + h * P + p];
+                const double gy = go * silu(zv);
+                gr->z[tok * dx + h * P + p] = go * y * silu_grad(zv);
+                wg->D[h] += gy * k.ux[p];
+                gux[p] = gy * in->D[h];
+                for (int n = 0; n < N; n++) {
+                    gch[n] += gy * ht[p * N + n];
+                    gh[p * N + n] += gy * k.ch[n];
+                }
+            }
+            double gdecay = 0.0, gdt = 0.0;
+            for (int p = 0; p < P; p++)
+                for (int n = 0; n < N; n++) {
+                    const double ghv = gh[p * N + n];
+                    if (hprev) gdecay += ghv * hprev[p * N + n];
+                    gdt += ghv * k.ux[p] * k.bh[n];
+                    gux[p] += k.dt * ghv * k.bh[n];
+                    gbh[n] += k.dt * ghv * k.ux[p];
+                }
+            gdt += gdecay * k.decay * k.a;
+            const double ga = gdecay * k.decay * k.dt;
+            const double gv = gdt * sigmoid(k.v);
+            gr->dt_raw[tok * H + h] = gv;
+            wg->dt_bias[h] += gv;
+            if (d->a_per_token) gr->A[tok * H + h] = k.floored ? 0.0 : ga;
+            else wg->A[h] += ga;
+
+            /* B^ / C^ back to the group's conv outputs */
+            double *gub = gu + (size_t)t * cd + dx + g * N;
+            double *guc = gu + (size_t)t * cd + dx + gn + g * N;
+            if (d->bc_norm) {
+                double sb = 0.0, sc = 0.0;
+                for (int n = 0; n < N; n++) {
+                    const double wb = in->bn_w ? in->bn_w[n] : 1.0, wc = in->cn_w ? in->cn_w[n] : 1.0;
+                    wg->bn_w[n] += gbh[n] * k.ub[n] * k.rb;
+                    wg->cn_w[n] += gch[n] * k.uc[n] * k.rc;
+                    wg->bn_bias[(size_t)h * N + n] += gbh[n];
+                    wg->cn_bias[(size_t)h * N + n] += gch[n];
+                    sb += gbh[n] * wb * k.ub[n];
+                    sc += gch[n] * wc * k.uc[n];
+                }
+                for (int n = 0; n < N; n++) {
+                    const double wb = in->bn_w ? in->bn_w[n] : 1.0, wc = in->cn_w ? in->cn_w[n] : 1.0;
+                    gub[n] += k.rb * wb * gbh[n] - k.rb * k.rb * k.rb / N * k.ub[n] * sb;
+                    guc[n] += k.rc * wc * gch[n] - k.rc * k.rc * k.rc / N * k.uc[n] * sc;
+                }
+            } else {
+                for (int n = 0; n < N; n++) { gub[n] += gbh[n]; guc[n] += gch[n]; }
+            }
+            for (int p = 0; p < P; p++) gu[(size_t)t * cd + h * P + p] += gux[p];
+
+            /* the adjoint state handed to token t-1 */
+            if (carry)
+                for (int i = 0; i < P * N; i++) gh[i] *= k.decay;
+            else
+                memset(gh, 0, sizeof(double) * (size_t)P * N);
+        }
+    }
+
+    /* conv (+ SiLU) of the row, back to the raw x|B|C inputs */
+    double *graw = calloc((size_t)L * cd, sizeof(double));
+    if (!graw) abort();
+    for (int t = 0; t < Lb; t++)
+        for (int ch = 0; ch < cd; ch++) {
+            const double gv = gu[(size_t)t * cd + ch];
+            if (K == 1) { graw[(size_t)t * cd + ch] += gv; continue; }
+            const double gpre = gv * silu_grad(conv_pre(d, in, b, t, ch));
+            wg->conv_b[ch] += gpre;
+            for (int kk = 0; kk < K; kk++) {
+                const int tau = t - (K - 1) + kk;
+                if (tau < 0 || !same_doc(in, d, b, tau, t)) continue;
+                wg->conv_w[(size_t)ch * K + kk] += gpre * xbc_raw(d, in, b, tau, ch);
+                graw[(size_t)tau * cd + ch] += gpre * in->conv_w[(size_t)ch * K + kk];
+            }
+        }
+    for (int t = 0; t < L; t++) {
+        const size_t row = (size_t)b * L + t;
+        for (int c = 0; c < dx; c++) gr->x[row * dx + c] = graw[(size_t)t * cd + c];
+        for (int c = 0; c < gn; c++) {
+            gr->Bm[row * gn + c] = graw[(size_t)t * cd + dx + c];
+            gr->Cm[row * gn + c] = graw[(size_t)t * cd + dx + gn + c];
+        }
+    }
+    /* padding tokens: nothing reaches them */
+    for (int t = Lb; t < L; t++) {
+        const size_t tok = (size_t)b * L + t;
+        for (int c = 0; c < dx; c++) gr->z[tok * dx + c] = 0.0;
+        for (int hh = 0; hh < H; hh++) {
+            gr->dt_raw[tok * H + hh] = 0.0;
+            if (d->a_per_token) gr->A[tok * H + hh] = 0.0;
+        }
+    }
+    free(gu); free(hist); free(gh); free(buf); free(gux); free(gbh); free(gch); free(graw);
+}
+
+typedef struct {
+    const oracle_dims *d;
+    const oracle_inputs *in;
+    const float *gout;
+    const oracle_grads *gr;
+    row_wgrads *rows;
+    int next;
+    pthread_mutex_t lock;
+} bwd_job;
+
+static void *bwd_worker(void *arg)
+{
+    bwd_job *j = arg;
+    for (;;) {
+        pthread_mutex_lock(&j->lock);
+        const int b = j->next++;
+        pthread_mutex_unlock(&j->lock);
+        if (b >= j->d->batch) break;
+        backward_row(j->d, j->in, j->gout, b, j->gr, &j->rows[b]);
+    }
+    return NULL;
+}
+
+/* Returns the number of threads used, or -1 on a bad argument. */
+int oracle_backward(const oracle_dims *d, const oracle_inputs *in, const float *gout,
+                    int nthreads, const oracle_grads *gr)
+{
+    if (!d || !in || !gout || !gr) return -1;
+    if (d->batch < 0 || d->seqlen < 1 || d->nheads < 1 || d->headdim < 1 || d->dstate < 1 ||
+        d->ngroups < 1 || d->nheads % d->ngroups || d->dconv < 1)
+        return -1;
+    if (in->init_ssm || in->init_conv) return -1;          /* zero-state prefill only */
+    if (d->dconv > 1 && (!in->conv_w || !in->conv_b || !gr->conv_w || !gr->conv_b)) return -1;
+    if (d->bc_norm && (!gr->bn_w || !gr->cn_w || !gr->bn_bias || !gr->cn_bias)) return -1;
+    if (!gr->x || !gr->z || !gr->Bm || !gr->Cm || !gr->dt_raw || !gr->dt_bias || !gr->A || !gr->D)
+        return -1;
+
+    const int H = d->nheads, N = d->dstate, K = d->dconv, cd = conv_dim_of(d);
+    /* one block of weight gradients per row: dt_bias, A (per head), D, conv_w, conv_b,
+     * bn_w, cn_w, bn_bias, cn_bias */
+    const size_t per_row = (size_t)3 * H + (size_t)cd * K + cd + 2 * (size_t)N + 2 * (size_t)H * N;
+    const int rows = d->batch > 0 ? d->batch : 1;
+    double *pool = calloc(per_row * rows, sizeof(double));
+    row_wgrads *rw = malloc(sizeof(row_wgrads) * (size_t)rows);
+    if (!pool || !rw) abort();
+    for (int b = 0; b < rows; b++) {
+        double *q = pool + per_row * b;
+        rw[b].dt_bias = q; q += H;
+        rw[b].A = q; q += H;
+        rw[b].D = q; q += H;
+        rw[b].conv_w = q; q += (size_t)cd * K;
+        rw[b].conv_b = q; q += cd;
+        rw[b].bn_w = q; q += N;
+        rw[b].cn_w = q; q += N;
+        rw[b].bn_bias = q; q += (size_t)H * N;
+        rw[b].cn_bias = q;
+    }
+
+    bwd_job j;
+    j.d = d; j.in = in; j.gout = gout; j.gr = gr; j.rows = rw; j.next = 0;
+    pthread_mutex_init(&j.lock, NULL);
+    if (nthreads <= 0) nthreads = oracle_default_threads();
+    if (nthreads > d->batch) nthreads = d->batch > 0 ? d->batch : 1;
+    pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int i = 1; i < nthreads; i++) pthread_create(&th[i], NULL, bwd_worker, &j);
+    bwd_worker(&j);
+    for (int i = 1; i < nthreads; i++) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&j.lock);
+
+    /* sum the rows' weight gradients in row order */
+    for (int i = 0; i < H; i++) {
+        double sbias = 0.0, sa = 0.0, sd = 0.0;
+        for (int b = 0; b < d->batch; b++) { sbias += rw[b].dt_bias[i]; sa += rw[b].A[i]; sd += rw[b].D[i]; }
+        gr->dt_bias[i] = sbias;
+        gr->D[i] = sd;
+        if (!d->a_per_token) gr->A[i] = sa;
+    }
+    if (K > 1) {
+        for (size_t i = 0; i < (size_t)cd * K; i++) {
+            double s = 0.0;
+            for (int b = 0; b < d->batch; b++) s += rw[b].conv_w[i];
+            gr->conv_w[i] = s;
+        }
+        for (int i = 0; i < cd; i++) {
+            double s = 0.0;
+            for (int b = 0; b < d->batch; b++) s += rw[b].conv_b[i];
+            gr->conv_b[i] = s;
+        }
+    }
+    if (d->bc_norm) {
+        for (int i = 0; i < N; i++) {
+            double sb = 0.0, sc = 0.0;
+            for (int b = 0; b < d->batch; b++) { sb += rw[b].bn_w[i]; sc += rw[b].cn_w[i]; }
+            gr->bn_w[i] = sb;
+            gr->cn_w[i] = sc;
+        }
+        for (size_t i = 0; i < (size_t)H * N; i++) {
+            double sb = 0.0, sc = 0.0;
+            for (int b = 0; b < d->batch; b++) { sb += rw[b].bn_bias[i]; sc += rw[b].cn_bias[i]; }
+            gr->bn_bias[i] = sb;
+            gr->cn_bias[i] = sc;
+        }
+    }
+    free(pool); free(rw);
+    return nthreads;
+}

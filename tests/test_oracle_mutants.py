@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 
 from brute_force import head_inputs, quadratic_form, silu
+from test_oracle_backward import case as _bwd_case, check_directional as _bwd_directional
 from test_oracle_s6 import _inputs as _s6_inputs, _matrix_form as _s6_matrix_form
 from selective_state_space_forward_b200.synthetic import Workload, make_inputs
 
@@ -24,11 +25,11 @@ MUTANTS = {
     "drop_D_skip": ("y += in->D[h] * ux[p];", "y += 0.0 * ux[p];"),
     "decay_sign": ("const double decay = exp(dt * a);", "const double decay = exp(-dt * a);"),
     "no_document_reset": ("memset(hs, 0, sizeof(double) * P * N);", "(void)0;"),
-    "conv_taps_reversed": ("in->conv_w[(size_t)ch * K + k]", "in->conv_w[(size_t)ch * K + (K - 1 - k)]"),
+    "conv_taps_reversed": ("in->conv_w[(size_t)ch * K + k] * v;", "in->conv_w[(size_t)ch * K + (K - 1 - k)] * v;"),
     "update_with_C": ("hp[n] = decay * hp[n] + dxp * ub[n];", "hp[n] = decay * hp[n] + dxp * uc[n];"),
     "no_gate_silu": ("out[tok * dx + h * P + p] = y * silu(zv);", "out[tok * dx + h * P + p] = y * zv;"),
-    "groups_interleaved": ("const int g = h / (H / d->ngroups);\n    const int dx",
-                           "const int g = h % d->ngroups;\n    const int dx"),
+    "groups_interleaved": ("const int g = h / (H / d->ngroups);\n    const int dx = H * P, gn = d->ngroups * N;\n    double *hs",
+                           "const int g = h % d->ngroups;\n    const int dx = H * P, gn = d->ngroups * N;\n    double *hs"),
     "dt_bias_dropped": ("softplus_exact((double)in->dt_raw[tok * H + h] + in->dt_bias[h])",
                         "softplus_exact((double)in->dt_raw[tok * H + h])"),
     "a_floor_inverted": ("if (a > -1e-4) a = -1e-4;", "if (a < -1e-4) a = -1e-4;"),
@@ -37,7 +38,7 @@ MUTANTS = {
     "norm_uses_C_bias_for_B": ("ub[n] = ub[n] * rb * wb + bb;", "ub[n] = ub[n] * rb * wb + bc;"),
     "output_before_update": ("hp[n] = decay * hp[n] + dxp * ub[n];\n                y += uc[n] * hp[n];",
                              "y += uc[n] * hp[n];\n                hp[n] = decay * hp[n] + dxp * ub[n];"),
-    "padding_runs_the_recurrence": ("    for (int t = 0; t < Lb; t++) {", "    for (int t = 0; t < L; t++) {"),
+    "padding_runs_the_recurrence": ("= 0.0;\n    for (int t = 0; t < Lb; t++) {", "= 0.0;\n    for (int t = 0; t < L; t++) {"),
     "final_history_ignores_length": ("const int L = row_len(d, in, b);   /* the row's last real token is L - 1 */",
                                      "const int L = d->seqlen;"),
     "s6_no_clamp": ("            if (al < -10.0) al = -10.0;\n            if (al > 5.0) al = 5.0;\n", ""),
@@ -47,6 +48,22 @@ MUTANTS = {
     "s6_drop_D": ("            y += in->D[c] * uv;", "            y += 0.0 * uv;"),
     "s6_no_gate": ("out[tok * DI + c] = in->z ? y * silu(in->z[tok * DI + c]) : y;",
                    "out[tok * DI + c] = y;"),
+    "bwd_drop_decay_term_of_dt": ("gdt += gdecay * k.decay * k.a;", "(void)gdecay;"),
+    "bwd_no_adjoint_reset": ("            else\n                memset(gh, 0, sizeof(double) * (size_t)P * N);",
+                             "            else\n                (void)0;"),
+    "bwd_norm_cross_term_sign": ("gub[n] += k.rb * wb * gbh[n] - k.rb * k.rb * k.rb / N * k.ub[n] * sb;",
+                                 "gub[n] += k.rb * wb * gbh[n] + k.rb * k.rb * k.rb / N * k.ub[n] * sb;"),
+    "bwd_conv_taps_reversed": ("graw[(size_t)tau * cd + ch] += gpre * in->conv_w[(size_t)ch * K + kk];",
+                               "graw[(size_t)tau * cd + ch] += gpre * in->conv_w[(size_t)ch * K + (K - 1 - kk)];"),
+    "bwd_conv_without_silu_grad": ("const double gpre = gv * silu_grad(conv_pre(d, in, b, t, ch));",
+                                   "const double gpre = gv;"),
+    "bwd_floored_A_passes": ("gr->A[tok * H + h] = k.floored ? 0.0 : ga;", "gr->A[tok * H + h] = ga;"),
+    "bwd_gate_uses_silu": ("go * y * silu_grad(zv);", "go * y * silu(zv);"),
+    "bwd_softplus_grad_at_dt": ("const double gv = gdt * sigmoid(k.v);", "const double gv = gdt * sigmoid(k.dt);"),
+    "bwd_group_gradient_overwritten": ("for (int n = 0; n < N; n++) { gub[n] += gbh[n]; guc[n] += gch[n]; }",
+                                       "for (int n = 0; n < N; n++) { gub[n] = gbh[n]; guc[n] = gch[n]; }"),
+    "bwd_decay_grad_with_new_state": ("if (hprev) gdecay += ghv * hprev[p * N + n];",
+                                      "if (hprev) gdecay += ghv * ht[p * N + n];"),
 }
 
 
@@ -160,6 +177,12 @@ def _battery(lib) -> list:
     if not (np.max(np.abs(r["out"] - y)) <= 1e-10 * np.max(np.abs(y)) and
             np.max(np.abs(r["final"] - hf)) <= 1e-10 * np.max(np.abs(hf))):
         failed.append("s6_matrix_form")
+    # 7. backward: directional derivatives of the unmodified forward, with and without
+    #    conv / documents / the B/C norm / per-token A
+    for conv, seed in ((True, 27), (False, 28)):
+        dims, inp, gout = _bwd_case(conv, seed=seed)
+        if _bwd_directional(dims, inp, gout, seed=seed, lib=lib):
+            failed.append("backward_%s" % ("conv" if conv else "norm"))
     return failed
 
 
