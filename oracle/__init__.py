@@ -93,6 +93,9 @@ def _bind(path: str):
     lib.oracle_backward.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Inputs), _FP,
                                     ctypes.c_int, ctypes.POINTER(_Grads)]
     lib.oracle_backward.restype = ctypes.c_int
+    lib.oracle_gated_norm.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                      dp, _FP, dp]
+    lib.oracle_gated_norm.restype = ctypes.c_int
     return lib
 
 
@@ -294,3 +297,23 @@ def backward(dims: dict, inp: dict, gout, threads: int = 0, lib=None) -> dict:
     if lib.oracle_backward(ctypes.byref(d), ctypes.byref(i), go, int(threads), ctypes.byref(gr)) < 0:
         raise ValueError("oracle_backward rejected its arguments")
     return g
+
+
+def gated_norm(gated, weight=None, group: int | None = None, eps: float = 1e-5, lib=None):
+    """RMSNorm of the gated scan output (``forward``'s out = y * silu(z)) times
+    the per-channel weight: upstream Mamba-2's norm(y * silu(z)).
+
+    gated: (..., d_inner) float64; weight: (d_inner) or None (ones); group:
+    channels per norm group (default d_inner, one norm per token).
+    """
+    lib = _load(lib)
+    g = np.ascontiguousarray(np.asarray(gated, dtype=np.float64))
+    d_inner = g.shape[-1]
+    rows = g.size // d_inner if d_inner else 0
+    keep = []
+    out = np.empty_like(g)
+    rc = lib.oracle_gated_norm(int(rows), int(d_inner), int(group or d_inner), float(eps),
+                               _dptr(g), _f32(weight, keep), _dptr(out))
+    if rc != 0:
+        raise ValueError("oracle_gated_norm rejected its arguments")
+    return out

@@ -844,3 +844,34 @@ int oracle_backward(const oracle_dims *d, const oracle_inputs *in, const float *
     free(pool); free(rw);
     return nthreads;
 }
+
+/* ------------------------------------------------------------------------------------
+ * Gated RMSNorm after the scan: upstream Mamba-2's norm(y * silu(z)) with the
+ * weight mixer.norm.weight of shape (d_inner) -- codestral_mamba.ts weight-port
+ * header (tensor list, and reconciliation 3: upstream computes
+ * "norm(y * silu(z))").  The gated product y * silu(z) is exactly what
+ * oracle_forward returns as out, so this step takes that output:
+ *
+ *   for each token row and each group of `group` consecutive channels
+ *   (group == d_inner: one norm over the whole row):
+ *     r = 1 / sqrt(mean over the group of g^2 + eps);   out[c] = g[c] * r * w[c]
+ *
+ * g, out: (rows, d_inner) double (may alias); w: (d_inner) float32 or NULL
+ * (ones).  Returns 0, or -1 on a bad argument.
+ */
+int oracle_gated_norm(int rows, int d_inner, int group, double eps, const double *g,
+                      const float *w, double *out)
+{
+    if (rows < 0 || d_inner < 1 || group < 1 || d_inner % group || !(eps >= 0.0) || !g || !out)
+        return -1;
+    for (int r = 0; r < rows; r++)
+        for (int c0 = 0; c0 < d_inner; c0 += group) {
+            const double *gv = g + (size_t)r * d_inner + c0;
+            double ss = 0.0;
+            for (int c = 0; c < group; c++) ss += gv[c] * gv[c];
+            const double rs = 1.0 / sqrt(ss / group + eps);
+            for (int c = 0; c < group; c++)
+                out[(size_t)r * d_inner + c0 + c] = gv[c] * rs * (w ? w[c0 + c] : 1.0);
+        }
+    return 0;
+}

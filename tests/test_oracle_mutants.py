@@ -13,6 +13,7 @@ import pytest
 
 from brute_force import head_inputs, quadratic_form, silu
 from test_oracle_backward import case as _bwd_case, check_directional as _bwd_directional
+from test_oracle_gated_norm import check_gated_norm as _gated_norm_checks
 from test_oracle_s6 import _inputs as _s6_inputs, _matrix_form as _s6_matrix_form
 from selective_state_space_forward_b200.synthetic import Workload, make_inputs
 
@@ -62,6 +63,11 @@ MUTANTS = {
     "bwd_softplus_grad_at_dt": ("const double gv = gdt * sigmoid(k.v);", "const double gv = gdt * sigmoid(k.dt);"),
     "bwd_group_gradient_overwritten": ("for (int n = 0; n < N; n++) { gub[n] += gbh[n]; guc[n] += gch[n]; }",
                                        "for (int n = 0; n < N; n++) { gub[n] = gbh[n]; guc[n] = gch[n]; }"),
+    "norm_mean_over_the_row": ("const double rs = 1.0 / sqrt(ss / group + eps);",
+                               "const double rs = 1.0 / sqrt(ss / d_inner + eps);"),
+    "norm_eps_outside_the_root": ("const double rs = 1.0 / sqrt(ss / group + eps);",
+                                  "const double rs = 1.0 / (sqrt(ss / group) + eps);"),
+    "norm_weight_by_group_position": ("gv[c] * rs * (w ? w[c0 + c] : 1.0);", "gv[c] * rs * (w ? w[c] : 1.0);"),
     "bwd_decay_grad_with_new_state": ("if (hprev) gdecay += ghv * hprev[p * N + n];",
                                       "if (hprev) gdecay += ghv * ht[p * N + n];"),
 }
@@ -183,6 +189,8 @@ def _battery(lib) -> list:
         dims, inp, gout = _bwd_case(conv, seed=seed)
         if _bwd_directional(dims, inp, gout, seed=seed, lib=lib):
             failed.append("backward_%s" % ("conv" if conv else "norm"))
+    # 8. the gated RMSNorm after the scan
+    failed += ["gated_norm_" + n for n in _gated_norm_checks(lib)]
     return failed
 
 
