@@ -113,6 +113,64 @@ def _ptr(t, dtype=None, name="tensor"):
     return t.data_ptr() or None
 
 
+def _need(t, count: int, name: str):
+    """Refuse a tensor that holds fewer elements than the call reads or writes
+    through its pointer (the C ABI sees only the pointer)."""
+    if isinstance(t, torch.Tensor) and t.numel() < count:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call touches {count}")
+
+
+def _align256(v: int) -> int:
+    return (v + 255) & ~255
+
+
+def state_bytes_for(nheads, headdim, dstate, ngroups, dconv, act_dtype, batch) -> int:
+    """ssd_state_bytes without a handle: the fp32 SSM state (batch, H, P, N), then
+    at the next 256-byte boundary the conv history (batch, 3, conv_dim) in the
+    activation dtype (none when dconv is 1), the whole rounded up to 256 bytes."""
+    n = _align256(batch * nheads * headdim * dstate * 4)
+    if dconv == 4:
+        es = 2 if act_dtype == "bf16" else 4
+        n += batch * 3 * (nheads * headdim + 2 * ngroups * dstate) * es
+    return _align256(n)
+
+
+def check_forward_sizes(dims: dict, batch: int, seqlen: int, state_bytes: int, *, x, z, dt_raw,
+                        dt_bias, A, B, C, D, conv_w=None, conv_b=None, seq_idx=None,
+                        init_state=None, out=None, final_state=None, lengths=None):
+    """Element counts of a forward's (or, at seqlen 1, a step's) tensors against
+    the shape the call reads: every pointer the library dereferences must
+    cover what it touches.  dims: nheads, headdim, dstate, ngroups, dconv,
+    a_per_token."""
+    H, P, N, G = dims["nheads"], dims["headdim"], dims["dstate"], dims["ngroups"]
+    tok = batch * seqlen
+    for t, n in (("x", x), ("z", z), ("out", out)):
+        _need(n, tok * H * P, t)
+    _need(B, tok * G * N, "B")
+    _need(C, tok * G * N, "C")
+    _need(dt_raw, tok * H, "dt_raw")
+    _need(dt_bias, H, "dt_bias")
+    _need(D, H, "D")
+    _need(A, tok * H if dims.get("a_per_token") else H, "A")
+    if dims.get("dconv", 1) == 4:
+        cd = H * P + 2 * G * N
+        _need(conv_w, cd * 4, "conv_w")
+        _need(conv_b, cd, "conv_b")
+    _need(seq_idx, tok, "seq_idx")
+    _need(lengths, batch, "lengths")
+    _need(init_state, state_bytes, "init_state")
+    _need(final_state, state_bytes, "final_state")
+
+
+def _rows(x, per_token: int, name: str, rank: int = 3):
+    """(batch, seqlen) of a (batch, seqlen, per_token) activation tensor."""
+    if not isinstance(x, torch.Tensor) or x.dim() != rank or x.shape[-1] != per_token:
+        want = "(batch, seqlen, %d)" % per_token if rank == 3 else "(batch, %d)" % per_token
+        got = tuple(x.shape) if isinstance(x, torch.Tensor) else type(x).__name__
+        raise ValueError(f"{name} must be {want}, got {got}")
+    return (x.shape[0], x.shape[1]) if rank == 3 else (x.shape[0], 1)
+
+
 def _stream(stream):
     if stream is None:
         return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
@@ -139,6 +197,11 @@ class Handle:
         self._h = h
         self._keep = ()
         self.path = PATH_NAMES.get(self.lib.ssd_get_path(h), "?")
+
+    @property
+    def dims(self) -> dict:
+        return dict(nheads=self.nheads, headdim=self.headdim, dstate=self.dstate,
+                    ngroups=self.ngroups, dconv=self.dconv, a_per_token=self.a_per_token)
 
     @property
     def conv_dim(self):
@@ -191,9 +254,13 @@ class Handle:
         """ssd_forward, or ssd_forward_ragged when `lengths` (an int32 CUDA tensor of
         per-row real-token counts) is given; returns `out` (allocated like x when not given)."""
         at, f = self.torch_dtype, torch.float32
-        batch, seqlen = (x.shape[0], x.shape[1]) if x.dim() == 3 else (0, 0)
+        batch, seqlen = _rows(x, self.nheads * self.headdim, "x")
         if out is None:
             out = torch.empty_like(x)
+        check_forward_sizes(self.dims, batch, seqlen, self.state_bytes(batch), x=x, z=z,
+                            dt_raw=dt_raw, dt_bias=dt_bias, A=A, B=B, C=C, D=D, conv_w=conv_w,
+                            conv_b=conv_b, seq_idx=seq_idx, init_state=init_state, out=out,
+                            final_state=final_state, lengths=lengths)
         if lengths is not None:
             _raise(self.lib, self.lib.ssd_forward_ragged(
                 self._h, batch, seqlen, _ptr(lengths, torch.int32, "lengths"), _ptr(x, at, "x"),
@@ -217,10 +284,16 @@ class Handle:
              out=None, stream=None):
         """ssd_step: one token per row, `state` updated in place; returns `out`."""
         at, f = self.torch_dtype, torch.float32
+        batch = x.shape[0] if isinstance(x, torch.Tensor) and x.dim() >= 1 else 0
+        if not isinstance(x, torch.Tensor) or x.numel() != batch * self.nheads * self.headdim:
+            raise ValueError(f"x must hold one token of {self.nheads * self.headdim} channels per row")
         if out is None:
             out = torch.empty_like(x)
+        check_forward_sizes(self.dims, batch, 1, self.state_bytes(batch), x=x, z=z, dt_raw=dt_raw,
+                            dt_bias=dt_bias, A=A, B=B, C=C, D=D, conv_w=conv_w, conv_b=conv_b,
+                            init_state=state, out=out)
         _raise(self.lib, self.lib.ssd_step(
-            self._h, x.shape[0], _ptr(x, at, "x"), _ptr(z, at, "z"), _ptr(dt_raw, f, "dt_raw"),
+            self._h, batch, _ptr(x, at, "x"), _ptr(z, at, "z"), _ptr(dt_raw, f, "dt_raw"),
             _ptr(dt_bias, f, "dt_bias"), _ptr(A, f, "A"), _ptr(B, at, "B"), _ptr(C, at, "C"),
             _ptr(D, f, "D"), _ptr(conv_w, at, "conv_w"), _ptr(conv_b, at, "conv_b"),
             _ptr(state, torch.uint8, "state"), _ptr(out, at, "out"), _stream(stream)))
@@ -229,9 +302,17 @@ class Handle:
     def stage_conv(self, x, B, C, conv_w, conv_b, seq_idx=None, init_state=None, u=None,
                    stream=None):
         at = self.torch_dtype
-        batch, seqlen = x.shape[0], x.shape[1]
+        batch, seqlen = _rows(x, self.nheads * self.headdim, "x")
         if u is None:
             u = torch.empty(batch, seqlen, self.conv_dim, dtype=torch.float32, device=x.device)
+        gn = self.ngroups * self.dstate
+        _need(B, batch * seqlen * gn, "B")
+        _need(C, batch * seqlen * gn, "C")
+        _need(conv_w, self.conv_dim * 4, "conv_w")
+        _need(conv_b, self.conv_dim, "conv_b")
+        _need(seq_idx, batch * seqlen, "seq_idx")
+        _need(init_state, self.state_bytes(batch), "init_state")
+        _need(u, batch * seqlen * self.conv_dim, "u")
         _raise(self.lib, self.lib.ssd_stage_conv(
             self._h, batch, seqlen, _ptr(x, at, "x"), _ptr(B, at, "B"), _ptr(C, at, "C"),
             _ptr(conv_w, at, "conv_w"), _ptr(conv_b, at, "conv_b"),
@@ -241,7 +322,10 @@ class Handle:
 
     def stage_dt(self, dt_raw, dt_bias, A, seq_idx=None, stream=None):
         f = torch.float32
-        batch, seqlen = dt_raw.shape[0], dt_raw.shape[1]
+        batch, seqlen = _rows(dt_raw, self.nheads, "dt_raw")
+        _need(dt_bias, self.nheads, "dt_bias")
+        _need(A, batch * seqlen * self.nheads if self.a_per_token else self.nheads, "A")
+        _need(seq_idx, batch * seqlen, "seq_idx")
         dt = torch.empty(batch, self.nheads, seqlen, dtype=f, device=dt_raw.device)
         acs = torch.empty_like(dt)
         _raise(self.lib, self.lib.ssd_stage_dt(
@@ -273,13 +357,20 @@ def forward_noalloc(x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None,
     Handle.forward.  Returns `out` (allocated like x when not given)."""
     lib = lib or load_library()
     at, f = torch.bfloat16, torch.float32
-    batch, seqlen = (x.shape[0], x.shape[1]) if x.dim() == 3 else (0, 0)
+    batch, seqlen = _rows(x, nheads * headdim, "x")
     d = Desc(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv,
              chunk=64, act_dtype=DTYPES["bf16"][0], a_mode=0, bc_norm=0,
              max_batch=max_batch or max(batch, 1), max_seqlen=max_seqlen or max(seqlen, 1),
              path=PATHS[path])
     if out is None:
         out = torch.empty_like(x)
+    dims = dict(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv)
+    check_forward_sizes(dims, batch, seqlen,
+                        state_bytes_for(nheads, headdim, dstate, ngroups, dconv, "bf16", batch),
+                        x=x, z=z, dt_raw=dt_raw, dt_bias=dt_bias, A=A, B=B, C=C, D=D,
+                        conv_w=conv_w, conv_b=conv_b, seq_idx=seq_idx, init_state=init_state,
+                        out=out, final_state=final_state)
+    _need(status, 1, "status")
     _raise(lib, lib.ssd_forward_noalloc(
         ctypes.byref(d), batch, seqlen, _ptr(x, at, "x"), _ptr(z, at, "z"),
         _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"), _ptr(A, f, "A"),
@@ -300,10 +391,16 @@ def s6_forward(u, delta, delta_bias, A_log, B, C, D, z=None, init_state=None, ou
     if u.dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("u must be bf16 or fp32")
     at = u.dtype
+    if u.dim() != 3:
+        raise ValueError(f"u must be (batch, seqlen, d_inner), got {tuple(u.shape)}")
     batch, seqlen, d_inner = u.shape
+    if not isinstance(A_log, torch.Tensor) or A_log.dim() != 2 or A_log.shape[0] != d_inner:
+        raise ValueError(f"A_log must be (d_inner, dstate) = ({d_inner}, dstate)")
     dstate = A_log.shape[1]
     if out is None:
         out = torch.empty_like(u)
+    check_s6_sizes(batch, seqlen, d_inner, dstate, delta=delta, delta_bias=delta_bias, B=B, C=C,
+                   D=D, z=z, init_state=init_state, out=out, final_state=final_state)
     _raise(lib, lib.ssd_s6_forward(
         batch, seqlen, d_inner, dstate, 1 if at == torch.bfloat16 else 0, _ptr(u, at, "u"),
         _ptr(delta, f, "delta"), _ptr(delta_bias, f, "delta_bias"), _ptr(A_log, f, "A_log"),
@@ -311,3 +408,18 @@ def s6_forward(u, delta, delta_bias, A_log, B, C, D, z=None, init_state=None, ou
         _ptr(init_state, f, "init_state"), _ptr(out, at, "out"), _ptr(final_state, f, "final_state"),
         _stream(stream)))
     return out
+
+
+def check_s6_sizes(batch, seqlen, d_inner, dstate, *, delta, delta_bias, B, C, D, z=None,
+                   init_state=None, out=None, final_state=None):
+    """Element counts of ssd_s6_forward's tensors against the shape it reads."""
+    tok = batch * seqlen
+    _need(delta, tok * d_inner, "delta")
+    _need(z, tok * d_inner, "z")
+    _need(out, tok * d_inner, "out")
+    _need(B, tok * dstate, "B")
+    _need(C, tok * dstate, "C")
+    _need(delta_bias, d_inner, "delta_bias")
+    _need(D, d_inner, "D")
+    _need(init_state, batch * d_inner * dstate, "init_state")
+    _need(final_state, batch * d_inner * dstate, "final_state")

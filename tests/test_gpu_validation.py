@@ -135,3 +135,14 @@ def test_validate_finite_reports_a_nan_in_the_results(path):
            dev["conv_b"], state=fin)
     with pytest.raises(ssd.SSDError, match="non-finite"):
         h.check()
+
+
+@pytest.mark.parametrize("name", ["mini_k3_mixer", "mamba3_siso", "tiny_fp32"])
+def test_state_bytes_without_a_handle_match_the_library(name):
+    """The binding sizes ssd_forward_noalloc's state buffers itself; its count
+    must be ssd_state_bytes'."""
+    w = WORKLOADS[name]
+    h = make_handle(w, max_batch=3, max_seqlen=64)
+    for b in (0, 1, 3):
+        assert ssd.state_bytes_for(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv,
+                                   w.act_dtype, b) == h.state_bytes(b)
