@@ -88,3 +88,38 @@ def test_s6_refuses_bad_arguments_by_name():
     b16 = torch.zeros(1, 8, 16, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ssd.SSDError, match="out may not alias"):
         ssd.s6_forward(u, f, v, a16, b16, b16, v, out=u)
+
+
+def test_s6_split_sequence_continues_through_the_state():
+    """Scanning tokens [0, 100) and then [100, 300) from the carried state gives
+    the outputs and final state of one scan over [0, 300)."""
+    inp = _inputs(2, 300, 200, 16, seed=11)
+    out, fin = _gpu(inp)
+    first = dict(inp, u=inp["u"][:, :100], delta=inp["delta"][:, :100], z=inp["z"][:, :100],
+                 B=inp["B"][:, :100], C=inp["C"][:, :100])
+    o1, f1 = _gpu(first)
+    second = dict(inp, u=inp["u"][:, 100:], delta=inp["delta"][:, 100:], z=inp["z"][:, 100:],
+                  B=inp["B"][:, 100:], C=inp["C"][:, 100:], init=f1.astype(np.float32))
+    o2, f2 = _gpu(second)
+    assert_close(np.concatenate([o1, o2], axis=1), out, "bf16", "S6 split outputs")
+    assert_close(f2, fin, "bf16", "S6 split final state")
+
+
+def test_s6_empty_inputs():
+    """No token: the state passes through (zeros without an initial state); no row: nothing."""
+    DI, N = 40, 8
+    u = torch.empty(2, 0, DI, dtype=torch.bfloat16, device="cuda")
+    f = torch.empty(2, 0, DI, dtype=torch.float32, device="cuda")
+    bc = torch.empty(2, 0, N, dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros(DI, dtype=torch.float32, device="cuda")
+    a = torch.zeros(DI, N, dtype=torch.float32, device="cuda")
+    init = torch.randn(2, DI, N, device="cuda")
+    fin = torch.full((2, DI, N), 7.0, device="cuda")
+    ssd.s6_forward(u, f, v, a, bc, bc, v, init_state=init, final_state=fin)
+    torch.cuda.synchronize()
+    assert torch.equal(fin, init)
+    ssd.s6_forward(u, f, v, a, bc, bc, v, final_state=fin)
+    torch.cuda.synchronize()
+    assert bool(torch.all(fin == 0.0))
+    ssd.s6_forward(u[:0], f[:0], v, a, bc[:0], bc[:0], v)
+    torch.cuda.synchronize()
