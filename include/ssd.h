@@ -272,7 +272,11 @@ ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
  *   init_state, final_state  (batch, d_inner, dstate) fp32, or NULL (zeros / not
  *               written); they may be the same buffer
  *   dstate      8, 16 or 32 (else SSD_ERR_UNSUPPORTED); act_dtype an ssd_dtype
- * Arguments are validated before any launch, as for ssd_forward.
+ * All pointers are contiguous row-major device memory that the caller owns,
+ * aligned to their element size; the call is asynchronous on `stream`.
+ * batch = 0 is a no-op; seqlen = 0 copies init_state to final_state (zeros
+ * without an initial state).  Arguments are validated before any launch, as
+ * for ssd_forward, and a refusal names the argument (ssd_last_error).
  */
 ssd_status ssd_s6_forward(int32_t batch, int32_t seqlen, int32_t d_inner, int32_t dstate,
                           int32_t act_dtype, const void* u, const float* delta,
