@@ -440,3 +440,31 @@ def test_ragged_batch_without_conv_with_bc_norm(path):
         assert bool(torch.all(bits[b, L:] == 0)), f"row {b}: padding is not +0.0"
     s, c = state_to_numpy(h, fin, w.batch)
     _compare_all(w, inp, res, out.double().cpu().numpy(), s, c, f"ragged norm/{h.path}")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_packed_documents_match_separate_calls(path):
+    """Each document of a packed row against the same document run as its own
+    call (model card, Checkpoint and training: packed and separately launched
+    documents differ only by the reduction order of the fused prefix sums).
+    Both runs see the same bf16 operands; the chunk grid falls differently on
+    the document, so the results agree to the bf16 tolerance, not bit for bit.
+    Documents of 1 token and boundaries on and beside the 64-token chunk edges
+    are included."""
+    w = _small("mini_k3_mixer", batch=1, seqlen=260, documents="none", init_state=False, seed=41)
+    inp = make_inputs(w)
+    seq = _docs_row(w.seqlen, [37, 64, 65, 150, 151, 230])[None]
+    inp["seq_idx"] = seq
+    h = make_handle(w, path)
+    packed, _, _, _ = run_forward(h, w, to_device(inp, w), None, final=False)
+    for k in range(int(seq.max()) + 1):
+        idx = np.flatnonzero(seq[0] == k)
+        lo, hi = int(idx[0]), int(idx[-1]) + 1
+        wk = w.with_(seqlen=hi - lo)
+        one = {key: (None if v is None else
+                     (np.ascontiguousarray(v[:, lo:hi]) if key in ("x", "z", "B", "C", "dt_raw")
+                      else v)) for key, v in inp.items()}
+        one["seq_idx"] = None
+        hk = make_handle(wk, path)
+        alone, _, _, _ = run_forward(hk, wk, to_device(one, wk), None, final=False)
+        assert_close(packed[:, lo:hi], alone, "bf16", f"document {k} packed vs alone ({h.path})")

@@ -207,6 +207,35 @@ def test_documents_are_isolated_bitwise(oracle_mod):
             assert np.array_equal(res["final_conv"], base["final_conv"]), k
 
 
+def test_packed_documents_equal_separate_calls(oracle_mod):
+    """A document packed in a row gives the outputs of the same document run as
+    its own call, bit for bit (model card, Checkpoint and training: packed and
+    separately launched documents differ only by the GPU's reduction order;
+    the sequential oracle has none).  The first document also carries the
+    row's initial state, and the last one hands its state out."""
+    w = _small(dconv=4, seqlen=160, batch=1, init_state=True, a_per_token=True)
+    inp = make_inputs(w)
+    rng = np.random.default_rng(4)
+    inp["init_conv"] = rng.standard_normal((1, 3, w.conv_dim)).astype(np.float32)
+    seq = _docs_with_boundaries(w.seqlen, [1, 40, 64, 65, 100])[None]
+    inp["seq_idx"] = seq
+    packed = oracle_mod.forward(w.dims(), inp)
+    ndoc = int(seq.max()) + 1
+    for k in range(ndoc):
+        idx = np.flatnonzero(seq[0] == k)
+        lo, hi = int(idx[0]), int(idx[-1]) + 1
+        alone = dict(inp, seq_idx=None)
+        for key in ("x", "z", "B", "C", "dt_raw", "A"):
+            alone[key] = np.ascontiguousarray(inp[key][:, lo:hi])
+        if k > 0:
+            alone["init_ssm"] = alone["init_conv"] = None
+        r = oracle_mod.forward(dict(w.dims(), seqlen=hi - lo), alone)
+        assert np.array_equal(r["out"][0], packed["out"][0, lo:hi]), k
+        if k == ndoc - 1:
+            assert np.array_equal(r["final_ssm"], packed["final_ssm"])
+            assert np.array_equal(r["final_conv"], packed["final_conv"])
+
+
 def test_prefill_then_steps_continues_the_sequence(oracle_mod):
     """forward(L1) -> state -> steps == forward(L1 + M) (Mamba3Block.step: decoding
     continues a prefill).  The state crosses the call boundary as fp32."""
