@@ -468,3 +468,31 @@ def test_packed_documents_match_separate_calls(path):
         hk = make_handle(wk, path)
         alone, _, _, _ = run_forward(hk, wk, to_device(one, wk), None, final=False)
         assert_close(packed[:, lo:hi], alone, "bf16", f"document {k} packed vs alone ({h.path})")
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("name", ["mini_k3_mixer", "mamba3_siso"])
+def test_forward_of_one_token_equals_the_step(name, path):
+    """Mamba3Block.step is the forward at L = 1 with the state carried: the
+    decode kernel and a one-token forward from the same state give the same
+    output and the same new state (to the bf16 tolerance: different kernels)."""
+    w = _small(name, batch=3, seqlen=70, documents="none")
+    inp = make_inputs(w)
+    h = make_handle(w, path)
+    dev = to_device(inp, w)
+    _, _, _, state = run_forward(h, w, dev, None)
+    carried = state.clone()
+    si = make_step_inputs(w, 0)
+    o_step = _step_run(h, w, dev, si, state)
+    torch.cuda.synchronize()
+
+    w1 = w.with_(seqlen=1)
+    one = dict(inp)
+    one.update({k: v[:, None] for k, v in si.items()})
+    one["seq_idx"] = None
+    o_fwd, s_fwd, c_fwd, _ = run_forward(h, w1, to_device(one, w1), carried)
+    assert_close(o_step.double().cpu().numpy()[:, None], o_fwd, w.act_dtype, "step vs forward out")
+    s_step, c_step = state_to_numpy(h, state, w.batch)
+    assert_close(s_step, s_fwd, w.act_dtype, "step vs forward state")
+    if c_step is not None:
+        assert np.array_equal(c_step, c_fwd)
