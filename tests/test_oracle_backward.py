@@ -14,7 +14,9 @@ differentiation, which shares nothing with the hand-written reverse sweep:
     documents' inputs), and packed-versus-alone equality of a document's
     gradients;
   * ragged rows: padding takes no gradient, and a row's gradients equal the
-    same row run alone over its real tokens.
+    same row run alone over its real tokens;
+  * autograd (torch, float64, CPU) of an independent implementation: the SSD
+    matrix form of the whole forward, conv and B/C norm included.
 
 Inputs are put on a coarse binary grid (multiples of 2^-8) so that every
 perturbed value x +- e v (e = 2^-12, 2^-13, |v| <= 4) is exactly a float32: the
@@ -203,3 +205,70 @@ def test_backward_refuses_a_carried_state(oracle_mod):
         oracle.backward(dims, dict(inp, init_ssm=np.zeros((1, 4, 3, 5), np.float32)), gout)
     with pytest.raises(ValueError):
         oracle.backward(dims, dict(inp, init_conv=np.zeros((1, 3, 22), np.float32)), gout)
+
+
+def _torch_matrix_form(dims, inp):
+    """The whole forward in the SSD matrix form, in float64 torch ops on the CPU:
+    conv (document-masked taps) + SiLU, the B/C norm, softplus dt, the floored
+    per-token A, y = (L o C B^T o dt) x + D x, out = y SiLU(z).  It shares no
+    loop with the oracle's token-by-token recurrence; autograd gives its
+    gradients.  Returns (out, leaves) with leaves the inputs requiring grad."""
+    import torch
+    Bb, L, H, P, N, G, K = (dims["batch"], dims["seqlen"], dims["nheads"], dims["headdim"],
+                            dims["dstate"], dims["ngroups"], dims["dconv"])
+    leaves = {k: torch.tensor(np.asarray(v, np.float64), requires_grad=True)
+              for k, v in inp.items() if isinstance(v, np.ndarray) and v.dtype == np.float32}
+    seq = np.zeros((Bb, L), np.int64) if inp.get("seq_idx") is None else np.asarray(inp["seq_idx"])
+    # doc[b, t]: the document ordinal (boundaries where neighbours differ)
+    doc = np.concatenate([np.zeros((Bb, 1), np.int64),
+                          np.cumsum(seq[:, 1:] != seq[:, :-1], axis=1)], axis=1)
+    raw = torch.cat([leaves["x"], leaves["B"], leaves["C"]], dim=-1)
+    if K == 4:
+        pre = leaves["conv_b"].expand_as(raw)
+        for k in range(4):
+            sh = 3 - k
+            shifted = torch.zeros_like(raw)
+            shifted[:, sh:] = raw[:, :L - sh]
+            ok = np.zeros((Bb, L), bool)
+            ok[:, sh:] = doc[:, sh:] == doc[:, :L - sh]
+            pre = pre + leaves["conv_w"][:, k] * shifted * torch.tensor(ok, dtype=torch.float64)[..., None]
+        u = pre * torch.sigmoid(pre)
+    else:
+        u = raw
+    HP, GN = H * P, G * N
+    ux = u[..., :HP].reshape(Bb, L, H, P)
+    gmap = torch.tensor([h // (H // G) for h in range(H)])
+    ub = u[..., HP:HP + GN].reshape(Bb, L, G, N)[:, :, gmap]
+    uc = u[..., HP + GN:].reshape(Bb, L, G, N)[:, :, gmap]
+    if dims.get("bc_norm"):
+        ub = ub * torch.rsqrt((ub ** 2).mean(-1, keepdim=True) + 1e-5) * leaves["B_norm_w"] + leaves["B_bias"]
+        uc = uc * torch.rsqrt((uc ** 2).mean(-1, keepdim=True) + 1e-5) * leaves["C_norm_w"] + leaves["C_bias"]
+    dt = torch.nn.functional.softplus(leaves["dt_raw"] + leaves["dt_bias"])          # (Bb, L, H)
+    a = torch.clamp(leaves["A"], max=-1e-4) if dims.get("a_per_token") else leaves["A"].expand(Bb, L, H)
+    cs = torch.cumsum(dt * a, dim=1)
+    t = np.arange(L)
+    keep = torch.tensor((t[:, None] >= t[None, :])[None] & (doc[:, :, None] == doc[:, None, :]))
+    diff = cs[:, :, None, :] - cs[:, None, :, :]                                   # (Bb, t, s, H)
+    decay = torch.exp(torch.where(keep[..., None], diff, torch.full_like(diff, -torch.inf)))
+    cb = torch.einsum("btgn,bsgn->btsg", uc, ub)                                   # per head
+    M = cb * decay * dt[:, None, :, :]
+    y = torch.einsum("btsh,bshp->bthp", M, ux) + leaves["D"][:, None] * ux
+    z = leaves["z"].reshape(Bb, L, H, P)
+    out = (y * z * torch.sigmoid(z)).reshape(Bb, L, HP)
+    return out, leaves
+
+
+@pytest.mark.parametrize("conv", [True, False], ids=["conv_docs_groups", "bcnorm_per_token_A"])
+def test_gradients_equal_autograd_of_the_matrix_form(oracle_mod, conv):
+    import torch
+    dims, inp, gout = case(conv, seed=51 if conv else 52)
+    out, leaves = _torch_matrix_form(dims, inp)
+    ref = oracle.forward(dims, inp, final=False)["out"]
+    assert np.max(np.abs(out.detach().numpy() - ref)) <= 1e-11 * np.max(np.abs(ref))
+    names = sorted(k for k, v in oracle.backward(dims, inp, gout).items() if v is not None)
+    want = torch.autograd.grad((out * torch.tensor(gout, dtype=torch.float64)).sum(),
+                               [leaves[k] for k in names])
+    got = oracle.backward(dims, inp, gout)
+    for k, wv in zip(names, want):
+        wv = wv.numpy()
+        assert np.max(np.abs(got[k] - wv)) <= 1e-10 * max(np.max(np.abs(wv)), 1e-300), k
