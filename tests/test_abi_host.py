@@ -96,11 +96,45 @@ def test_null_handle_is_refused(lib):
     assert st == 1 and "handle" in lib.ssd_last_error().decode()
     st = lib.ssd_step(None, 1, *([None] * 13))
     assert st == 1
-    assert st == 1
     assert lib.ssd_check(None, None) == 1
     assert lib.ssd_get_path(None) == -1
     assert lib.ssd_state_bytes(None, 1) == 0
     lib.ssd_destroy(None)   # no-op
+
+
+def _s6(lib, batch=1, seqlen=8, d_inner=16, dstate=16, act_dtype=1, **ptrs):
+    names = ("u", "delta", "delta_bias", "A_log", "B", "C", "D", "z", "init", "out", "fin")
+    # distinct, aligned, never dereferenced: every case is refused before a launch
+    p = {n: 0x10000 * (i + 1) for i, n in enumerate(names)}
+    p.update(ptrs)
+    return lib.ssd_s6_forward(batch, seqlen, d_inner, dstate, act_dtype,
+                              *[p[n] for n in names], None)
+
+
+@pytest.mark.parametrize("kw,status,word", [
+    (dict(dstate=12), 2, "dstate"),
+    (dict(act_dtype=5), 1, "act_dtype"),
+    (dict(batch=-1), 1, "batch"),
+    (dict(d_inner=0), 1, "d_inner"),
+    (dict(init=0x10002), 3, "init_state"),
+    (dict(u=None), 1, "u"),
+    (dict(A_log=None), 1, "A_log"),
+    (dict(out=0x10000), 1, "alias"),
+])
+def test_s6_bad_arguments_are_refused_by_name(lib, kw, status, word):
+    assert _s6(lib, **kw) == status
+    assert word in lib.ssd_last_error().decode()
+
+
+def test_s6_empty_batch_is_a_no_op(lib):
+    assert _s6(lib, batch=0) == 0
+
+
+def test_noalloc_refuses_bad_descriptors(lib):
+    st = lib.ssd_forward_noalloc(ctypes.byref(_desc(nheads=0)), 1, 1, *([None] * 16))
+    assert st == 1 and "nheads" in lib.ssd_last_error().decode()
+    st = lib.ssd_forward_noalloc(ctypes.byref(_desc(path=2)), 1, 1, *([None] * 16))
+    assert st == 2 and "fused path only" in lib.ssd_last_error().decode()
 
 
 def test_missing_library_fails_loudly(tmp_path):
