@@ -17,6 +17,8 @@ Extra keys: `roofline` (dominant kernel against measured HBM bandwidth),
 (decode_b256 single-token step, GB/s), `e2e` (host buffers, copies inside the
 timed region), `cpu_baseline` (the fp64 oracle on this host's cores),
 `clocks` (SM clock and throttle reasons sampled during the timed region).
+`cpu_baseline.single_thread` gives the oracle's one-thread rate on the tiny
+fp32 case and on one (row, head) pair of the bench workload.
 """
 from __future__ import annotations
 
@@ -500,6 +502,27 @@ def cpu_oracle_run(max_seconds: float | None = None):
     return tokens_equiv / dt, desc, r["threads"], dt
 
 
+def cpu_oracle_single_thread() -> dict:
+    """One host thread of the oracle: the whole tiny_fp32 case, and one (row,
+    head) pair of the bench workload over its full 8192 tokens; tokens/s in
+    full-width tokens (all heads)."""
+    import oracle
+    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
+    res = {}
+    for name, pairs in (("tiny_fp32", None), (WORKLOAD, [(0, 0)])):
+        w = WORKLOADS[name]
+        if name not in _INPUT_CACHE:
+            _INPUT_CACHE[name] = make_inputs(w)
+        t0 = time.time()
+        oracle.forward(w.dims(), _INPUT_CACHE[name], pairs=pairs, threads=1, final=True)
+        dt = time.time() - t0
+        npairs = w.batch * w.nheads if pairs is None else len(pairs)
+        tokens = npairs * w.seqlen / w.nheads
+        res[name] = {"tokens_per_s": tokens / dt, "seconds": round(dt, 4),
+                     "sample": f"{npairs} (row, head) pair(s) x {w.seqlen} tokens, 1 thread"}
+    return res
+
+
 def _cut(inp, L):
     keys = ("x", "z", "B", "C", "dt_raw", "seq_idx")
     return {k: (v[:, :L] if (v is not None and k in keys) else v) for k, v in inp.items()}
@@ -565,7 +588,8 @@ def main(argv=None):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         v, desc, threads, _ = cpu_oracle_run(None)
-        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "single_thread": cpu_oracle_single_thread()}
     if rank == 0:
         line = {"metric": METRIC, "value": fwd["value"], "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": fwd["ms_per_step"],
