@@ -4,21 +4,28 @@ decode-step GB/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one ssd_forward over the mini_k3_mixer workload (batch 5 x 8192
-tokens, 32 heads x 64, d_state 64, 8 B/C groups, conv 4, packed documents)
-with its inputs resident in HBM; the whole hot path runs in the library's
-kernels (conv, dt/cumsum, chunk scan with state passing, gated output, final
-state).  Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs
-its own batch -- the scan has no cross-row exchange -- so the scaling is weak
-and `value` counts every rank's tokens over the slowest rank's device time.
+One step = one ssd_forward over the headline workload, long_7b (a 7B-class
+Mamba-2 layer: batch 2 x 16384 tokens, 128 heads x 64, d_state 128, 8 B/C
+groups, conv 4, nonzero initial state) -- the largest configuration that fits
+one GPU -- with its inputs resident in HBM; the whole hot path runs in the
+library's kernels (conv, dt/cumsum, chunk scan with state passing, gated
+output, final state).  Rank 0 prints one JSON line.  With N > 1 (torchrun)
+every rank runs its own batch -- the scan has no cross-row exchange -- so the
+scaling is weak and `value` counts every rank's tokens over the slowest rank's
+device time.
+
+The timed region is the K-step loop, run R times back to back (R chosen so the
+region lasts at least half a second and the clock sampler sees it); every
+repetition times exactly K steps and `ms_per_step` is their mean.
 
 Extra keys: `roofline` (dominant kernel against measured HBM bandwidth),
-`forward_roofline` (whole forward against its compulsory bytes), `decode`
-(decode_b256 single-token step, GB/s), `e2e` (host buffers, copies inside the
-timed region), `cpu_baseline` (the fp64 oracle on this host's cores),
-`clocks` (SM clock and throttle reasons sampled during the timed region).
-`cpu_baseline.single_thread` gives the oracle's one-thread rate on the tiny
-fp32 case and on one (row, head) pair of the bench workload.
+`forward_roofline` (whole forward against its compulsory bytes), `configs`
+(the same measurement, rooflines and CPU baseline for mini_k3_mixer and
+mamba3_siso), `decode` (decode_b256 single-token step, GB/s), `e2e` (host
+buffers, copies inside the timed region), `cpu_baseline` (the fp64 oracle on
+this host's cores), `clocks` (SM clock and throttle reasons sampled during the
+timed region).  `cpu_baseline.single_thread` gives the oracle's one-thread
+rate on one (row, head) pair of the workload.
 """
 from __future__ import annotations
 
@@ -34,7 +41,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "SSD mixer tokens/s (B·L/s) at 1 B200 and % of roofline; decode-step GB/s"
-WORKLOAD = "mini_k3_mixer"
+WORKLOAD = "long_7b"                        # the headline configuration
+EXTRA_WORKLOADS = ("mini_k3_mixer", "mamba3_siso")
+MIN_TIMED_S = 0.5                            # shortest timed region (clock samples)
 DECODE_WORKLOAD = "decode_b256"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "kernel_traffic.json")
@@ -51,6 +60,13 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-s6", action="store_true", help="skip the Mamba-1 (S6) scan measurement")
+    p.add_argument("--workload", default=WORKLOAD,
+                   choices=["long_7b", "mini_k3_mixer", "mamba3_siso"],
+                   help="the workload of the headline measurement (default long_7b)")
+    p.add_argument("--min-timed-s", type=float, default=MIN_TIMED_S,
+                   help="shortest timed region in seconds (the K-step loop is repeated)")
+    p.add_argument("--no-extra", action="store_true",
+                   help="time the headline workload only (skip mini_k3_mixer and mamba3_siso)")
     return p.parse_args(argv)
 
 
@@ -232,15 +248,71 @@ def main_kernel_bytes(w, path: str) -> int:
     return u + BL * (2 * HP * a + 2 * H * 4) + seq + w.batch * nc * H * w.headdim * w.dstate * 4
 
 
-def bench_forward(args, torch, rank, world, local_rank, peaks):
+def _timed_loop(torch, stream, step, K: int, world: int, h=None, clk_index: int = 0,
+                min_s: float = MIN_TIMED_S):
+    """Run the K-step loop R times back to back inside one sampled region (R so
+    that the region lasts at least min_s seconds); every repetition times exactly
+    K steps with CUDA events on `stream`.  When a handle is given, its main
+    kernel is bracketed by per-step events too.  Returns (mean ms per step,
+    mean main-kernel ms or None, R, clocks summary, the handle's kernel launches
+    in the whole timed region)."""
+    probe0, probe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    probe0.record(stream)
+    for _ in range(K):
+        step()
+    probe1.record(stream)
+    torch.cuda.synchronize()
+    est = max(probe0.elapsed_time(probe1) / 1e3, 1e-6)
+    R = max(1, int(-(-min_s // est)))
+    if world > 1:       # every rank runs the same number of repetitions
+        import torch.distributed as dist
+        t = torch.tensor([R], dtype=torch.int64, device=torch.device("cuda", clk_index))
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        R = int(t.item())
+    reps = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(R)]
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(K)] for _ in range(R)] if h is not None else None
+    for ev in [e for pair in reps for e in pair] + (
+            [e for rep in kev for pair in rep for e in pair] if kev else []):
+        ev.record(stream)          # materialise the events so their handles exist
+    torch.cuda.synchronize()
+    barrier(world)
+    launches0 = h.launch_count() if h is not None else 0
+    with ClockSampler(clk_index) as clk:
+        for r in range(R):
+            reps[r][0].record(stream)
+            for i in range(K):
+                if kev is not None:
+                    h.set_timing_events(*kev[r][i])
+                step()
+            reps[r][1].record(stream)
+        torch.cuda.synchronize()
+    launches = (h.launch_count() - launches0) if h is not None else None
+    if h is not None:
+        h.set_timing_events(None, None)
+    barrier(world)
+    ms = sum(a.elapsed_time(b) for a, b in reps) / (R * K)
+    kern = (sum(a.elapsed_time(b) for rep in kev for a, b in rep) / (R * K)) if kev else None
+    return ms, kern, R, clk.summary(), launches
+
+
+def bench_forward(args, torch, rank, world, local_rank, peaks, wname=WORKLOAD):
     from selective_state_space_forward_b200 import ssd
     from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[wname]
     inp = make_inputs(w)
     dev = _device_inputs(w, inp, torch)
     h = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, w.act_dtype,
                    a_per_token=w.a_per_token, bc_norm=w.bc_norm, max_batch=w.batch,
                    max_seqlen=w.seqlen, path=args.path)
+    if w.bc_norm:
+        h.set_bc_norm(dev["B_norm_w"], dev["C_norm_w"], dev["B_bias"], dev["C_bias"])
+    init = None
+    if inp.get("init_ssm") is not None:
+        init = h.new_state(w.batch)
+        ssm, _ = h.state_views(init, w.batch)
+        ssm.copy_(torch.from_numpy(inp["init_ssm"]))
     fin = h.new_state(w.batch)
     out = torch.empty_like(dev["x"])
     stream = torch.cuda.current_stream()
@@ -248,49 +320,32 @@ def bench_forward(args, torch, rank, world, local_rank, peaks):
     def step():
         h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"],
                   dev["C"], dev["D"], dev["conv_w"], dev["conv_b"], seq_idx=dev["seq_idx"],
-                  out=out, final_state=fin, stream=stream)
+                  init_state=init, out=out, final_state=fin, stream=stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
-    for a_, b_ in ev:   # materialise the events so their handles exist
-        a_.record(stream)
-        b_.record(stream)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    barrier(world)
-    launches0 = h.launch_count()
-    with ClockSampler(local_rank) as clk:
-        t0.record(stream)
-        for i in range(K):
-            h.set_timing_events(*ev[i])
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize()
-    launches = h.launch_count() - launches0
-    h.set_timing_events(None, None)
-    barrier(world)
-    local_ms = t0.elapsed_time(t1) / K
-    kern_ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / K
+    local_ms, kern_ms, R, clocks, launches = _timed_loop(torch, stream, step, K, world, h,
+                                                         local_rank, args.min_timed_s)
     h.check()
     max_ms, total_tokens = aggregate(local_ms, w.tokens, world,
                                      device=torch.device("cuda", local_rank))
 
     kb = main_kernel_bytes(w, h.path)
     achieved = kb / (kern_ms * 1e-3) / 1e9
-    traffic = measured_traffic(f"{h.path}:{WORKLOAD}", h.path)
+    traffic = measured_traffic(f"{h.path}:{wname}", h.path)
     fb = forward_bytes(w)["bytes"]
     roof_ms = fb / (peaks["hbm_gbs"] * 1e9) * 1e3
     res = {
         "value": total_tokens / (max_ms * 1e-3),
         "ms_per_step": max_ms,
+        "repeats": R,
         "tokens_per_rank": w.tokens,
         "path": h.path,
         "launches": launches,
-        "clocks": clk.summary(),
+        "launches_per_step": launches / (R * K) if launches is not None else None,
+        "clocks": clocks,
         "roofline": {"bound": "hbm", "kernel": "ssd_chunk_fused" if h.path == "fused"
                      else "chunk_output_kernel", "achieved": round(achieved, 1),
                      "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
@@ -300,15 +355,16 @@ def bench_forward(args, torch, rank, world, local_rank, peaks):
                              "roofline_tokens_per_s": w.tokens / (roof_ms * 1e-3),
                              "frac": round(roof_ms / local_ms, 4)},
     }
-    return res, (w, inp, h, dev, out, fin)
+    return res, (w, inp, h, dev, out, fin, init)
 
 
 def bench_e2e(args, torch, ctx, world, local_rank):
     """Same forward through the public call with the step's inputs in pinned host
     memory: H2D copies, the call, and the D2H read of the output are timed."""
-    w, inp, h, dev, out, fin = ctx
+    w, inp, h, dev, out, fin, init = ctx
     stream = torch.cuda.current_stream()
-    keys = ["x", "z", "B", "C", "dt_raw"] + (["seq_idx"] if dev["seq_idx"] is not None else [])
+    keys = ["x", "z", "B", "C", "dt_raw"] + (["seq_idx"] if dev["seq_idx"] is not None else []) + (
+        ["A"] if w.a_per_token else [])
     host = {k: dev[k].cpu().pin_memory() for k in keys}
     dbuf = {k: torch.empty_like(dev[k]) for k in keys}
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -318,9 +374,10 @@ def bench_e2e(args, torch, ctx, world, local_rank):
     def step():
         for k in keys:
             dbuf[k].copy_(host[k], non_blocking=True)
-        h.forward(dbuf["x"], dbuf["z"], dbuf["dt_raw"], dev["dt_bias"], dev["A"], dbuf["B"],
-                  dbuf["C"], dev["D"], dev["conv_w"], dev["conv_b"],
-                  seq_idx=dbuf.get("seq_idx"), out=out, final_state=fin, stream=stream)
+        h.forward(dbuf["x"], dbuf["z"], dbuf["dt_raw"], dev["dt_bias"],
+                  dbuf["A"] if w.a_per_token else dev["A"], dbuf["B"], dbuf["C"], dev["D"],
+                  dev["conv_w"], dev["conv_b"], seq_idx=dbuf.get("seq_idx"), init_state=init,
+                  out=out, final_state=fin, stream=stream)
         hout.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -470,15 +527,20 @@ def bench_s6(args, torch, peaks, sm_mhz):
 _INPUT_CACHE = {}
 
 
-def cpu_oracle_run(max_seconds: float | None = None):
-    """The fp64 oracle on this host's cores over (part of) the bench workload.
+def _inputs(wname):
+    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
+    if wname not in _INPUT_CACHE:
+        _INPUT_CACHE[wname] = make_inputs(WORKLOADS[wname])
+    return _INPUT_CACHE[wname]
+
+
+def cpu_oracle_run(wname: str = WORKLOAD, max_seconds: float | None = None):
+    """The fp64 oracle on this host's cores over (part of) workload `wname`.
     Returns (tokens-equivalent per second, description, threads, seconds)."""
     import oracle
-    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
-    w = WORKLOADS[WORKLOAD]
-    if WORKLOAD not in _INPUT_CACHE:
-        _INPUT_CACHE[WORKLOAD] = make_inputs(w)
-    inp = _INPUT_CACHE[WORKLOAD]
+    from selective_state_space_forward_b200.synthetic import WORKLOADS
+    w = WORKLOADS[wname]
+    inp = _inputs(wname)
     cores = oracle.default_threads()
     pairs = [(b, hh) for b in range(w.batch) for hh in range(w.nheads)]
     L = w.seqlen
@@ -497,49 +559,51 @@ def cpu_oracle_run(max_seconds: float | None = None):
     r = oracle.forward(dims, inp, pairs=pairs, threads=0, final=True)
     dt = time.time() - t0
     tokens_equiv = len(pairs) * L / w.nheads
-    desc = (f"{len(pairs)} (row, head) pairs of {WORKLOAD} over {L} tokens each "
-            f"(= {tokens_equiv:.0f} full-width tokens of 32 heads), fp64")
+    desc = (f"{len(pairs)} (row, head) pairs of {wname} over {L} tokens each "
+            f"(= {tokens_equiv:.0f} full-width tokens of {w.nheads} heads), fp64")
     return tokens_equiv / dt, desc, r["threads"], dt
 
 
-def cpu_oracle_single_thread() -> dict:
-    """One host thread of the oracle: the whole tiny_fp32 case, and one (row,
-    head) pair of the bench workload over its full 8192 tokens; tokens/s in
-    full-width tokens (all heads)."""
+def cpu_oracle_single_thread(wname: str = WORKLOAD) -> dict:
+    """One host thread of the oracle on one (row, head) pair of workload `wname`
+    over its full length; tokens/s in full-width tokens (all heads)."""
     import oracle
-    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
-    res = {}
-    for name, pairs in (("tiny_fp32", None), (WORKLOAD, [(0, 0)])):
-        w = WORKLOADS[name]
-        if name not in _INPUT_CACHE:
-            _INPUT_CACHE[name] = make_inputs(w)
-        t0 = time.time()
-        oracle.forward(w.dims(), _INPUT_CACHE[name], pairs=pairs, threads=1, final=True)
-        dt = time.time() - t0
-        npairs = w.batch * w.nheads if pairs is None else len(pairs)
-        tokens = npairs * w.seqlen / w.nheads
-        res[name] = {"tokens_per_s": tokens / dt, "seconds": round(dt, 4),
-                     "sample": f"{npairs} (row, head) pair(s) x {w.seqlen} tokens, 1 thread"}
-    return res
+    from selective_state_space_forward_b200.synthetic import WORKLOADS
+    w = WORKLOADS[wname]
+    t0 = time.time()
+    oracle.forward(w.dims(), _inputs(wname), pairs=[(0, 0)], threads=1, final=True)
+    dt = time.time() - t0
+    tokens = w.seqlen / w.nheads
+    return {"tokens_per_s": tokens / dt, "seconds": round(dt, 4),
+            "sample": f"1 (row, head) pair x {w.seqlen} tokens of {wname}, 1 thread"}
 
 
 def _cut(inp, L):
     keys = ("x", "z", "B", "C", "dt_raw", "seq_idx")
-    return {k: (v[:, :L] if (v is not None and k in keys) else v) for k, v in inp.items()}
+    out = {k: (v[:, :L] if (v is not None and k in keys) else v) for k, v in inp.items()}
+    if inp.get("A") is not None and inp["A"].ndim == 3:      # per-token A
+        out["A"] = inp["A"][:, :L]
+    return out
+
+
+def cpu_baseline_block(wname: str, seconds: float) -> dict:
+    v, desc, threads, _ = cpu_oracle_run(wname, seconds)
+    return {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
+            "single_thread": cpu_oracle_single_thread(wname)}
 
 
 def reference_arm(args):
     """The oracle, as it stands, timed on the host cores: each step is a
-    bounded sample of the bench workload."""
+    bounded sample of the headline workload."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     budget = 150.0 / max(1, args.steps + args.warmup)
     for _ in range(args.warmup):
-        cpu_oracle_run(budget)
+        cpu_oracle_run(args.workload, budget)
     vals, descs, threads, wall = [], None, None, 0.0
     for _ in range(args.steps):
-        v, descs, threads, dt = cpu_oracle_run(budget)
+        v, descs, threads, dt = cpu_oracle_run(args.workload, budget)
         vals.append(v)
         wall += dt
     value = sum(vals) / len(vals)
@@ -547,7 +611,7 @@ def reference_arm(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": wall / max(1, args.steps) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(args.gpus),
+            "config": config_block(args.gpus, args.workload),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": descs},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -557,12 +621,26 @@ def reference_arm(args):
     return 0
 
 
-def config_block(n):
-    return {"workload": f"{WORKLOAD}: Mamba-2 SSD mixer, batch 5 x 8192 tokens per GPU, "
-                        "32 heads x 64, d_state 64, 8 B/C groups, conv kernel 4, packed documents "
-                        "(geometric lengths, mean 1500), bf16 activations, fp32 dt/A/D/state",
-            "global_batch": 5 * n, "seq_len": 8192, "parallelism": f"dp{n} (independent rows)",
-            "l2": "inputs larger than L2 (595 MB per step), no flush"}
+WORKLOAD_TEXT = {
+    "long_7b": "long_7b: 7B-class Mamba-2 layer, batch 2 x 16384 tokens per GPU, 128 heads x 64, "
+               "d_state 128, 8 B/C groups, conv kernel 4, initial state N(0, 0.1), one document "
+               "per row, bf16 activations, fp32 dt/A/D/state",
+    "mini_k3_mixer": "mini_k3_mixer: Mamba-2 SSD mixer, batch 5 x 8192 tokens per GPU, 32 heads "
+                     "x 64, d_state 64, 8 B/C groups, conv kernel 4, packed documents (geometric "
+                     "lengths, mean 1500), bf16 activations, fp32 dt/A/D/state",
+    "mamba3_siso": "mamba3_siso: Mamba-3-sized SISO scan, batch 4 x 4096 tokens per GPU, 80 heads "
+                   "x 64, d_state 128, 1 group, no conv, per-token A floored at 1e-4, B/C RMSNorm "
+                   "+ per-head bias, bf16 activations, fp32 dt/A/D/state",
+}
+
+
+def config_block(n, wname=WORKLOAD):
+    from selective_state_space_forward_b200.synthetic import WORKLOADS
+    w = WORKLOADS[wname]
+    fb = forward_bytes(w)["bytes"]
+    return {"workload": WORKLOAD_TEXT[wname], "global_batch": w.batch * n, "seq_len": w.seqlen,
+            "parallelism": f"dp{n} (independent rows)",
+            "l2": f"inputs larger than L2 ({fb / 1e6:.0f} MB per step), no flush"}
 
 
 def main(argv=None):
@@ -574,9 +652,17 @@ def main(argv=None):
     torch.cuda.set_device(local_rank)
     rank, world = dist_init("nccl")
     peaks = load_peaks()
-    fwd, ctx = bench_forward(args, torch, rank, world, local_rank, peaks)
+    fwd, ctx = bench_forward(args, torch, rank, world, local_rank, peaks, args.workload)
     e2e = None if args.no_e2e else bench_e2e(args, torch, ctx, world, local_rank)
     del ctx
+    torch.cuda.empty_cache()
+    configs = {}
+    if not args.no_extra:
+        for wname in [n for n in (WORKLOAD,) + EXTRA_WORKLOADS if n != args.workload]:
+            r, c = bench_forward(args, torch, rank, world, local_rank, peaks, wname)
+            del c
+            torch.cuda.empty_cache()
+            configs[wname] = dict(r, config=config_block(world, wname))
     decode = None
     if not args.no_decode and rank == 0:
         torch.cuda.empty_cache()
@@ -587,18 +673,20 @@ def main(argv=None):
         s6 = bench_s6(args, torch, peaks, fwd["clocks"].get("sm_mhz"))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, desc, threads, _ = cpu_oracle_run(None)
-        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "single_thread": cpu_oracle_single_thread()}
+        cpu = cpu_baseline_block(args.workload, 20.0)
+        for wname in configs:
+            configs[wname]["cpu_baseline"] = cpu_baseline_block(wname, 6.0)
     if rank == 0:
         line = {"metric": METRIC, "value": fwd["value"], "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": fwd["ms_per_step"],
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic", "config": config_block(world),
-                "path": fwd["path"], "roofline": fwd["roofline"],
-                "forward_roofline": fwd["forward_roofline"], "decode": decode, "s6": s6,
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": fwd["launches"],
-                "clocks": fwd["clocks"]}
+                "repeats": fwd["repeats"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_block(world, args.workload), "path": fwd["path"],
+                "roofline": fwd["roofline"],
+                "forward_roofline": fwd["forward_roofline"], "configs": configs,
+                "decode": decode, "s6": s6, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": fwd["launches"],
+                "gpu_launches_per_step": fwd["launches_per_step"], "clocks": fwd["clocks"]}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

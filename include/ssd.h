@@ -224,7 +224,11 @@ ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream);
  *
  * Scratch: a static device array of 64 MiB per device that belongs to the
  * loaded library (no cudaMalloc, cudaFree or allocating library call is
- * made).  It holds 4 KiB of hand-off flags, then the segment hand-off states
+ * made).  Because the array is part of the library's device code, every
+ * device on which that code is loaded holds the 64 MiB until the process
+ * exits, whether or not this entry point is ever called: from the library's
+ * first kernel launch on the device under lazy module loading (the CUDA
+ * default), from its load under eager loading.  It holds 4 KiB of hand-off flags, then the segment hand-off states
  * (64 * dstate fp32 per slot; at least one slot per (row, head) stream, at
  * most 1024 slots), dt and the chunk cumsum ((batch, H, seqlen) fp32 each)
  * and, when dconv = 4, the convolved B|C ((batch, seqlen, 2*G*N) bf16).

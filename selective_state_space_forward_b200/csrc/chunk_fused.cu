@@ -1032,7 +1032,22 @@ static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* m
     choose_segments(streams, nc, grid, cap, fp.nseg, fp.cps);
     fp.nitems = streams * fp.nseg;
     if (grid > fp.nitems) grid = fp.nitems;
-    kern<<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], fp);
+    // A cooperative launch makes co-residency of the whole grid a condition of
+    // the launch: on a GPU shared with other work (another stream's kernels, a
+    // reduced SM partition) it is refused with an error instead of starting CTAs
+    // whose hand-off waits could only time out.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], fp);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -349,22 +349,25 @@ class Handle:
 
 def forward_noalloc(x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None, seq_idx=None,
                     init_state=None, out=None, final_state=None, *, status, nheads, headdim,
-                    dstate, ngroups=1, dconv=4, max_batch=None, max_seqlen=None, path="auto",
-                    stream=None, lib=None):
+                    dstate, ngroups=1, dconv=4, a_per_token=False, validate_finite=False,
+                    max_batch=None, max_seqlen=None, path="auto", stream=None, lib=None):
     """ssd_forward_noalloc: the fused forward with no handle and no device allocation by the
     library (its scratch is a static device array).  `status` is a one-element int32 CUDA
     tensor the kernels OR error bits into; `out` and the state buffers are laid out as for
-    Handle.forward.  Returns `out` (allocated like x when not given)."""
+    Handle.forward.  a_per_token: A is (batch, seqlen, H), floored at magnitude 1e-4;
+    validate_finite: the call also scans out and the final state for NaN or infinity and
+    ORs bit 4 into `status`.  Returns `out` (allocated like x when not given)."""
     lib = lib or load_library()
     at, f = torch.bfloat16, torch.float32
     batch, seqlen = _rows(x, nheads * headdim, "x")
     d = Desc(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv,
-             chunk=64, act_dtype=DTYPES["bf16"][0], a_mode=0, bc_norm=0,
+             chunk=64, act_dtype=DTYPES["bf16"][0], a_mode=int(bool(a_per_token)), bc_norm=0,
              max_batch=max_batch or max(batch, 1), max_seqlen=max_seqlen or max(seqlen, 1),
-             path=PATHS[path])
+             path=PATHS[path], validate_finite=int(bool(validate_finite)))
     if out is None:
         out = torch.empty_like(x)
-    dims = dict(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv)
+    dims = dict(nheads=nheads, headdim=headdim, dstate=dstate, ngroups=ngroups, dconv=dconv,
+                a_per_token=bool(a_per_token))
     check_forward_sizes(dims, batch, seqlen,
                         state_bytes_for(nheads, headdim, dstate, ngroups, dconv, "bf16", batch),
                         x=x, z=z, dt_raw=dt_raw, dt_bias=dt_bias, A=A, B=B, C=C, D=D,

@@ -34,12 +34,13 @@ CASES = [
 ]
 
 
-def _noalloc(w, dev, init, fin, status, out=None):
+def _noalloc(w, dev, init, fin, status, out=None, validate_finite=False):
     return ssd.forward_noalloc(
         dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"],
         dev["D"], dev["conv_w"], dev["conv_b"], seq_idx=dev["seq_idx"], init_state=init,
         out=out, final_state=fin, status=status, nheads=w.nheads, headdim=w.headdim,
-        dstate=w.dstate, ngroups=w.ngroups, dconv=w.dconv)
+        dstate=w.dstate, ngroups=w.ngroups, dconv=w.dconv, a_per_token=w.a_per_token,
+        validate_finite=validate_finite)
 
 
 def _handle_forward(h, w, dev, init):
@@ -157,3 +158,50 @@ def test_noalloc_refuses_what_the_fused_path_does_not_serve():
                             status=None, nheads=w.nheads, headdim=w.headdim, dstate=w.dstate,
                             ngroups=w.ngroups, dconv=w.dconv)
     assert e.value.status == 1
+
+
+def test_noalloc_per_token_a_matches_forward():
+    """Per-token A (floored at magnitude 1e-4), d_state 128, no conv: the no-alloc
+    call against ssd_forward on a handle made with the same a_mode."""
+    w = WORKLOADS["mamba3_siso"].with_(batch=2, seqlen=300, nheads=8, bc_norm=False, seed=13)
+    inp = make_inputs(w)
+    inp["A"][0, 5:9, 2] = np.array([0.0, -1e-6, -1e-4, -3.0], dtype=np.float32)
+    dev = to_device(inp, w)
+    h = make_handle(w)
+    assert h.path == "fused"
+    want_out, want_fin = _handle_forward(h, w, dev, None)
+    status = _status_word()
+    fin = h.new_state(w.batch)
+    out = _noalloc(w, dev, None, fin, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    _close(out, want_out, "per-token A out")
+    _close(h.state_views(fin, w.batch)[0], h.state_views(want_fin, w.batch)[0],
+           "per-token A final ssm")
+
+
+def test_noalloc_validate_finite_reports_like_forward():
+    """validate_finite: a clean call leaves the status word at 0; a NaN planted in
+    one token of x reaches out and the final state, and the call ORs the
+    non-finite bit (4) into the status word, as ssd_forward's check reports it."""
+    w = CASES[0].with_(seqlen=200)
+    inp = make_inputs(w, seed=5)
+    dev = to_device(inp, w)
+    status = _status_word()
+    fin = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, "bf16",
+                     max_batch=w.batch, max_seqlen=w.seqlen).new_state(w.batch)
+    _noalloc(w, dev, None, fin, status, validate_finite=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    dev["x"][0, 150, 3] = float("nan")
+    _noalloc(w, dev, None, fin, status, validate_finite=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) & 4, f"status {int(status.item()):#x}"
+    h = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, "bf16",
+                   max_batch=w.batch, max_seqlen=w.seqlen, validate_finite=True)
+    h.forward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"], dev["B"], dev["C"],
+              dev["D"], dev["conv_w"], dev["conv_b"], seq_idx=dev["seq_idx"],
+              final_state=h.new_state(w.batch))
+    with pytest.raises(ssd.SSDError) as e:
+        h.check()
+    assert e.value.status == 6 and "non-finite" in str(e.value)
