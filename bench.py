@@ -21,7 +21,9 @@ repetition times exactly K steps and `ms_per_step` is their mean.
 Extra keys: `roofline` (dominant kernel against measured HBM bandwidth),
 `forward_roofline` (whole forward against its compulsory bytes), `configs`
 (the same measurement, rooflines and CPU baseline for mini_k3_mixer and
-mamba3_siso), `decode` (decode_b256 single-token step, GB/s), `e2e` (host
+mamba3_siso), `decode` (decode_b256 single-token step, GB/s), `backward`
+(ssd_backward on mini_k3_mixer), `packed_gated_norm` (the forward on a packed
+in_proj input followed by the gated RMSNorm), `e2e` (host
 buffers, copies inside the timed region), `cpu_baseline` (the fp64 oracle on
 this host's cores), `clocks` (SM clock and throttle reasons sampled during the
 timed region).  `cpu_baseline.single_thread` gives the oracle's one-thread
@@ -60,6 +62,8 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-s6", action="store_true", help="skip the Mamba-1 (S6) scan measurement")
+    p.add_argument("--no-backward", action="store_true",
+                   help="skip the backward and the packed-input gated-norm measurements")
     p.add_argument("--workload", default=WORKLOAD,
                    choices=["long_7b", "mini_k3_mixer", "mamba3_siso"],
                    help="the workload of the headline measurement (default long_7b)")
@@ -464,6 +468,110 @@ def bench_decode(args, torch, peaks):
             "traffic": measured_traffic(f"decode:{DECODE_WORKLOAD}", "decode")}
 
 
+def _event_ms(torch, fn, reps: int) -> float:
+    """Median CUDA-event time of fn() on the current stream over `reps` calls."""
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return sorted(ts)[len(ts) // 2]
+
+
+def bench_backward(args, torch, peaks, wname="mini_k3_mixer"):
+    """ssd_backward (zero-state prefill) over a full workload: the forward
+    recompute on the staged kernels plus the backward kernels, timed as one
+    call with CUDA events; the timing hook brackets the backward kernels alone.
+    Compulsory bytes: x, z, B, C, dt_raw and gout read once, the fp32 gradients
+    of x, z, B, C, dt_raw written once (weights and the small per-head vectors
+    are negligible)."""
+    from selective_state_space_forward_b200 import ssd
+    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs, make_output_grad
+    w = WORKLOADS[wname]
+    inp = make_inputs(w)
+    dev = _device_inputs(w, inp, torch)
+    h = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, w.act_dtype,
+                   a_per_token=w.a_per_token, bc_norm=w.bc_norm, max_batch=w.batch,
+                   max_seqlen=w.seqlen)
+    gout = torch.from_numpy(make_output_grad(w, 11)).to(dev["x"].dtype).cuda()
+    ws = torch.empty(h.backward_workspace_bytes(w.batch, w.seqlen), dtype=torch.uint8,
+                     device="cuda")
+    grads = {}
+
+    def call():
+        grads.update(h.backward(dev["x"], dev["z"], dev["dt_raw"], dev["dt_bias"], dev["A"],
+                                dev["B"], dev["C"], dev["D"], dev["conv_w"], dev["conv_b"],
+                                gout=gout, seq_idx=dev["seq_idx"], workspace=ws, grads=grads))
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = _event_ms(torch, call, max(5, min(args.steps, 20)))
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h.set_timing_events(k0, k1)
+    call()
+    torch.cuda.synchronize()
+    kern_ms = k0.elapsed_time(k1)
+    h.set_timing_events(None, None)
+    h.check()
+    a = 2 if w.act_dtype == "bf16" else 4
+    BL, HP, GN, H = w.tokens, w.nheads * w.headdim, w.ngroups * w.dstate, w.nheads
+    nbytes = BL * ((3 * HP + 2 * GN) * a + H * 4) + BL * (2 * HP + 2 * GN + H) * 4
+    return {"workload": WORKLOAD_TEXT[wname], "ms_per_call": round(ms, 4),
+            "backward_kernels_ms": round(kern_ms, 4), "tokens_per_s": BL / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "unit": "GB/s", "compulsory_bytes": nbytes,
+                         "achieved": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                         "frac": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "arithmetic": "fp32 SIMT (forward recompute on the staged kernels, then the "
+                          "backward kernels)",
+            "workspace_bytes": ws.numel()}
+
+
+def bench_packed_norm(args, torch, peaks, wname="mini_k3_mixer"):
+    """The forward reading a packed in_proj row [z | x | B | C | dt_raw] in place,
+    followed by the gated RMSNorm (group d_inner / ngroups), against the plain
+    contiguous forward on the same workload."""
+    from selective_state_space_forward_b200 import ssd
+    from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
+    w = WORKLOADS[wname]
+    inp = make_inputs(w)
+    dev = _device_inputs(w, inp, torch)
+    h = ssd.Handle(w.nheads, w.headdim, w.dstate, w.ngroups, w.dconv, w.act_dtype,
+                   a_per_token=w.a_per_token, bc_norm=w.bc_norm, max_batch=w.batch,
+                   max_seqlen=w.seqlen)
+    bf = dev["x"].dtype
+    packed = torch.cat([dev["z"], dev["x"], dev["B"], dev["C"], dev["dt_raw"].to(bf)], dim=2)
+    del dev["x"], dev["z"], dev["B"], dev["C"]
+    torch.cuda.empty_cache()
+    HP = w.nheads * w.headdim
+    weight = torch.ones(HP, device="cuda")
+    out = torch.empty(w.batch, w.seqlen, HP, dtype=bf, device="cuda")
+    fin = h.new_state(w.batch)
+    h.set_gated_norm(weight, group_size=HP // w.ngroups)
+
+    def call():
+        h.forward_packed(packed, dev["dt_bias"], dev["A"], dev["D"], dev["conv_w"], dev["conv_b"],
+                         seq_idx=dev["seq_idx"], out=out, final_state=fin)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = _event_ms(torch, call, max(5, min(args.steps, 20)))
+    h.check()
+    fb = forward_bytes(w)["bytes"] + HP * 4
+    return {"workload": WORKLOADS[wname].name + ": packed in_proj input (row stride "
+                        f"{packed.shape[2]} bf16), gated RMSNorm over groups of {HP // w.ngroups}",
+            "ms_per_step": round(ms, 4), "tokens_per_s": w.tokens / (ms * 1e-3),
+            "forward_roofline": {"compulsory_bytes": fb,
+                                 "frac": round(fb / (peaks["hbm_gbs"] * 1e9) / (ms * 1e-3), 4)},
+            "note": "the norm re-reads and re-writes out once: the kernels move "
+                    f"{fb + 2 * w.tokens * HP * 2} bytes against {fb} compulsory"}
+
+
 # Mamba-1 selective scan (S6) at the Falcon-Mamba-7B mixer shape.
 S6_SHAPE = dict(batch=2, seqlen=4096, d_inner=8192, dstate=16)
 # MUFU (transcendental) issue rate assumed for the roofline: 16 results per clock per SM.
@@ -667,6 +775,12 @@ def main(argv=None):
     if not args.no_decode and rank == 0:
         torch.cuda.empty_cache()
         decode = bench_decode(args, torch, peaks)
+    backward = packed = None
+    if not args.no_backward and rank == 0:
+        torch.cuda.empty_cache()
+        backward = bench_backward(args, torch, peaks)
+        torch.cuda.empty_cache()
+        packed = bench_packed_norm(args, torch, peaks)
     s6 = None
     if not args.no_s6 and rank == 0:
         torch.cuda.empty_cache()
@@ -684,7 +798,8 @@ def main(argv=None):
                 "config": config_block(world, args.workload), "path": fwd["path"],
                 "roofline": fwd["roofline"],
                 "forward_roofline": fwd["forward_roofline"], "configs": configs,
-                "decode": decode, "s6": s6, "cpu_baseline": cpu, "e2e": e2e,
+                "decode": decode, "backward": backward, "packed_gated_norm": packed, "s6": s6,
+                "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": fwd["launches"],
                 "gpu_launches_per_step": fwd["launches_per_step"], "clocks": fwd["clocks"]}
         print(json.dumps(line), flush=True)

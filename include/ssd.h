@@ -118,6 +118,20 @@ int32_t ssd_get_path(const ssd_handle* h);
 ssd_status ssd_set_bc_norm(ssd_handle* h, const float* B_norm_w, const float* C_norm_w,
                            const float* B_bias, const float* C_bias);
 
+/* Gated RMSNorm after the scan (the upstream Mamba-2 block's norm(y * silu(z));
+ * codestral_mamba.ts header: `mixer.norm.weight [d_inner]`, reconciliation 3).
+ * With enable = 1, every later ssd_forward / ssd_forward_ragged / ssd_step
+ * rewrites out in place as out * weight / sqrt(mean(out^2) + eps), the mean
+ * taken over each group of group_size consecutive channels of a token
+ * (group_size 0 = H*P, one norm per token; otherwise it must divide H*P, be a
+ * multiple of 8 and be at most 16384).  weight: (H*P) fp32 device pointer that
+ * stays valid while calls run, or NULL (ones).  eps in [0, 1]; the Mamba3Block
+ * norms use 1e-5.  Padding tokens of a ragged batch stay +0.0.  enable = 0
+ * turns the norm off (the other arguments are then ignored).  The norm adds one
+ * read and one write of out; validate_finite checks the normed out. */
+ssd_status ssd_set_gated_norm(ssd_handle* h, int32_t enable, const float* weight,
+                              int32_t group_size, float eps);
+
 /* Bytes of one state buffer for `batch` rows: the fp32 SSM state
  * (batch, H, P, N), then, at ssd_state_conv_offset, the conv history
  * (batch, dconv-1, conv_dim) in act_dtype, oldest token first (absent when
@@ -163,6 +177,22 @@ ssd_status ssd_forward_ragged(ssd_handle* h, int32_t batch, int32_t seqlen, cons
                               const float* D, const void* conv_w, const void* conv_b,
                               const int32_t* seq_idx, const void* init_state, void* out,
                               void* final_state, struct CUstream_st* stream);
+
+/*
+ * Forward over a packed in_proj output, read in place through row strides
+ * (codestral_mamba.ts header: the Mamba-2 in_proj row splits as
+ * [gate z | x|B|C | dt]).  zxbcdt is (batch, seqlen, ld) in act_dtype, and each
+ * token's row holds, from column 0: z (H*P), x (H*P), B (G*N), C (G*N) and
+ * dt_raw (H, in act_dtype rather than fp32); columns from 2*H*P + 2*G*N + H up
+ * to ld are ignored.  ld * element size must be a multiple of 16 bytes and
+ * zxbcdt 16-byte aligned.  Everything else is as for ssd_forward: the results
+ * equal ssd_forward over the same values split into contiguous tensors.
+ */
+ssd_status ssd_forward_packed(ssd_handle* h, int32_t batch, int32_t seqlen, const void* zxbcdt,
+                              int64_t ld, const float* dt_bias, const float* A, const float* D,
+                              const void* conv_w, const void* conv_b, const int32_t* seq_idx,
+                              const void* init_state, void* out, void* final_state,
+                              struct CUstream_st* stream);
 
 /*
  * One decode token per row (Mamba3Block.step: the same computation as forward
@@ -211,6 +241,61 @@ uint64_t ssd_launch_count(const ssd_handle* h);
  * results; ssd_last_error says which -- and SSD_ERR_CUDA when the stream
  * itself failed. */
 ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream);
+
+/*
+ * Gradients of the backward, all fp32 device buffers owned by the caller, each
+ * with the layout of the input it belongs to.  x, z, B, C and dt_raw are
+ * required; a NULL weight gradient is not computed.
+ */
+typedef struct {
+    float* x;         /* (batch, seqlen, H*P) */
+    float* z;         /* (batch, seqlen, H*P) */
+    float* B;         /* (batch, seqlen, G*N) */
+    float* C;         /* (batch, seqlen, G*N) */
+    float* dt_raw;    /* (batch, seqlen, H) */
+    float* dt_bias;   /* (H) */
+    float* A;         /* (H), or (batch, seqlen, H) when a_mode = PER_TOKEN */
+    float* D;         /* (H) */
+    float* conv_w;    /* (conv_dim, 4); NULL when dconv = 1 */
+    float* conv_b;    /* (conv_dim); NULL when dconv = 1 */
+    float* B_norm_w;  /* (N); only with bc_norm */
+    float* C_norm_w;  /* (N); only with bc_norm */
+    float* B_bias;    /* (H, N); only with bc_norm */
+    float* C_bias;    /* (H, N); only with bc_norm */
+} ssd_grads;
+
+/* Bytes of the device workspace ssd_backward needs for `batch` rows of
+ * `seqlen` tokens (0 for a NULL handle or negative sizes). */
+size_t ssd_backward_workspace_bytes(const ssd_handle* h, int32_t batch, int32_t seqlen);
+
+/*
+ * Backward of a zero-state prefill (mojolearn Mamba3Block, method "backward":
+ * the gradients of the loss with respect to the input and every weight, given
+ * the gradient of the output): the vector-Jacobian product of ssd_forward with
+ * no initial state, without a final-state cotangent.  The model card's gate
+ * ("Checkpoint and training") holds: a loss on one packed document gives
+ * exactly zero gradient on every other document's inputs.
+ *   x .. seq_idx  as for ssd_forward (lengths: as for ssd_forward_ragged, or
+ *                 NULL; padding tokens take no gradient and their gout is ignored)
+ *   gout          (batch, seqlen, H*P) act_dtype: gradient of the loss w.r.t. out
+ *   grads         the outputs (see ssd_grads); written, not accumulated
+ *   workspace     device memory of at least ssd_backward_workspace_bytes(h, batch,
+ *                 seqlen) bytes, 256-byte aligned, owned by the caller; its
+ *                 contents on entry do not matter
+ * With bc_norm, the handle's ssd_set_bc_norm parameters are used and their
+ * gradients can be asked for.  The arithmetic is fp32 throughout: the forward
+ * quantities are recomputed by the staged kernels, and weight gradients are
+ * summed in a fixed order, so a call repeats bit for bit.  headdim <= 64 and
+ * dstate <= 128 (else SSD_ERR_UNSUPPORTED).  Asynchronous on `stream`; the
+ * timing hook (ssd_set_timing_events) brackets the backward kernels that follow
+ * the forward recompute.
+ */
+ssd_status ssd_backward(ssd_handle* h, int32_t batch, int32_t seqlen, const int32_t* lengths,
+                        const void* x, const void* z, const float* dt_raw, const float* dt_bias,
+                        const float* A, const void* B, const void* C, const float* D,
+                        const void* conv_w, const void* conv_b, const int32_t* seq_idx,
+                        const void* gout, const ssd_grads* grads, void* workspace,
+                        size_t workspace_bytes, struct CUstream_st* stream);
 
 /*
  * Allocation-free forward.  The method's pages have no counterpart to this

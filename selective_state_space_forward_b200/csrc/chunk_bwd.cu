@@ -1,0 +1,717 @@
+// chunk_bwd.cu -- the backward (vector-Jacobian product) of the chunked scan, fp32.
+//
+// mojolearn Mamba3Block, method "backward": given the gradient of the loss
+// with respect to the output, the gradients with respect to the input and
+// every weight of a zero-state prefill (no carried state, no final-state
+// cotangent).  The model card ("Checkpoint and training") fixes what the
+// gradients must respect: a loss on one packed document gives exactly zero
+// gradient on every other document.
+//
+// The forward is the chunked form of the staged path (chunk_staged.cu): with
+// E[t,s] = exp(acs_t - acs_s), M[t,s] = (C^_t . B^_s) E[t,s] dt_s on the
+// causal same-segment mask of a chunk, f_t = [seg_t = 0] exp(acs_t),
+// w_s = [seg_s = seg_last] exp(acs_last - acs_s) dt_s and k_c the chunk's carry,
+//
+//   y_t      = sum_s M[t,s] x_s + f_t C^_t . Hin_c + D x_t ,  out_t = y_t SiLU(z_t)
+//   Hin_{c+1} = k_c Hin_c + S_c ,  S_c = sum_s w_s x_s (outer) B^_s .
+//
+// Its reverse, with gy = gout SiLU(z):
+//
+//   gHout_c  = sum_t f_t gy_t (outer) C^_t                 (bwd_state_out_kernel)
+//   gHin_c   = gHout_c + k_c gHin_{c+1},  gS_c = gHin_{c+1}  (bwd_state_scan_kernel)
+//   per chunk and head (bwd_chunk_kernel):
+//     gz       = gout y SiLU'(z),           gD += gy . x
+//     gM[t,s]  = gy_t . x_s                 gx_s += sum_t M[t,s] gy_t + D gy_s + w_s gS_c B^_s
+//     gC^_t    = sum_s gM E dt_s B^_s + f_t gy_t Hin_c
+//     gB^_s    = sum_t gM E dt_s C^_t + w_s x_s gS_c
+//     gacs     from E (row sums minus column sums of gM M), f_t, w_s and k_c,
+//     gdt      from M and w_s;  gdA = reverse segmented cumsum of gacs;
+//     gdt += gdA a, ga = gdA dt;  gdt_raw = gdt sigmoid(dt_raw + dt_bias)
+//   per group and token (bwd_bc_group_kernel): the heads' gB^, gC^ summed and
+//     taken back through the B/C RMSNorm (weight and per-head bias gradients);
+//   per channel (bwd_conv_kernel): back through SiLU and the 4-tap causal conv,
+//     with the same document rule as the forward.
+//
+// Weight gradients are written as per-block partial sums and added up by
+// bwd_reduce_kernel in a fixed order, so results repeat bit for bit.
+#include "ssd_device.cuh"
+#include "ssd_kernels.h"
+#include "staged_rows.cuh"
+
+namespace ssd {
+
+constexpr int kBwdThreads = 256;
+constexpr int kConvSeg = 128;          // tokens per thread of the conv backward
+
+__device__ __forceinline__ float sigmoid_f(float v) { return 1.0f / (1.0f + expf(-v)); }
+// d SiLU(v) / dv
+__device__ __forceinline__ float silu_grad_f(float v)
+{
+    const float s = sigmoid_f(v);
+    return s * (1.0f + v * (1.0f - s));
+}
+
+// Sum of v over the block (every thread gets the total); red holds >= 32 floats.
+__device__ float block_sum(float v, float* red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncthreads();
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float t = 0.0f;
+    for (int i = 0; i < nw; i++) t += red[i];
+    return t;
+}
+
+// ---------------------------------------------------------------------------------
+// gHout_c[p,n] = sum_t f_t gy_t[p] C^_t[n]: the gradient of the state entering
+// chunk c through the chunk's own outputs.  Written into gs.
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_state_out_kernel(Shape s, FwdArgs a, BwdBufs w)
+{
+    extern __shared__ float sm[];
+    const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
+    const int HP = H * P;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
+    float* cs = sm;                    // [64][N]
+    float* gf = cs + kChunk * N;       // [64][P]  f_t gy_t
+    float* ft = gf + kChunk * P;       // [64]
+    int* seg = (int*)(ft + kChunk);    // [64]
+    int* flag = seg + kChunk;          // [64]
+
+    const int Lb = row_length(a.lengths, b, L);
+    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, Lb, seg, flag);
+    if (threadIdx.x < kChunk) {
+        const int r = threadIdx.x;
+        const int64_t o = ((int64_t)b * H + h) * L + t0 + r;
+        ft[r] = (r < Lc && t0 + r < Lb && seg[r] == 0) ? expf(w.acs[o]) : 0.0f;
+    }
+    load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 1, cs, N);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kChunk * P; e += blockDim.x) {
+        const int t = e / P, p = e % P;
+        float v = 0.0f;
+        if (ft[t] != 0.0f) {
+            const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
+            v = ft[t] * to_f(((const T*)w.gout)[o]) * silu_f(to_f(((const T*)a.z)[o]));
+        }
+        gf[t * P + p] = v;
+    }
+    __syncthreads();
+    float* dst = w.gs + (((int64_t)b * nc + c) * H + h) * P * N;
+    for (int e = threadIdx.x; e < P * N; e += blockDim.x) {
+        const int p = e / N, n = e % N;
+        float acc = 0.0f;
+        for (int t = 0; t < Lc; t++) acc += gf[t * P + p] * cs[t * N + n];
+        dst[e] = acc;
+    }
+}
+
+// Reverse state scan, one thread per state element: on entry gs holds gHout_c,
+// on exit gS_c = gHin_{c+1} (zero for the last chunk: no final-state cotangent).
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_state_scan_kernel(Shape s, const float* __restrict__ cdecay, float* __restrict__ gs)
+{
+    const int PN = s.headdim * s.dstate, H = s.nheads, nc = s.nchunks();
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)s.batch * H * PN) return;
+    const int e = (int)(gid % PN);
+    const int h = (int)((gid / PN) % H);
+    const int b = (int)(gid / ((int64_t)PN * H));
+    const float* kd = cdecay + ((int64_t)b * H + h) * nc;
+    float g = 0.0f;                       // gHin_{c+1}
+    for (int c = nc - 1; c >= 0; c--) {
+        float* sp = gs + (((int64_t)b * nc + c) * H + h) * PN + e;
+        const float gout_c = *sp;
+        *sp = g;
+        const float k = kd[c];
+        g = (k == kChunkReset) ? gout_c : gout_c + k * g;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// The per-(chunk, head) gradients.  256 threads; P <= 64 and N <= 128.
+constexpr int kMaxXe = kChunk * 64 / kBwdThreads;     // x elements per thread
+constexpr int kMaxBe = kChunk * 128 / kBwdThreads;    // B elements per thread
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads)
+bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
+{
+    extern __shared__ float sm[];
+    const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
+    const int HP = H * P, NB = N + 1, cd = s.conv_dim();
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = c * kChunk, Lc = min(kChunk, L - t0), last = Lc - 1;
+    const int tid = threadIdx.x;
+    float* cs = sm;                    // [64][N]   C^
+    float* bs = cs + kChunk * N;       // [64][NB]  B^
+    float* xs = bs + kChunk * NB;      // [64][P]   x (conv output)
+    float* gy = xs + kChunk * P;       // [64][P]   gradient of y
+    float* hb = gy + kChunk * P;       // [P][NB]   Hin_c, then gS_c
+    float* cbe = hb + P * NB;          // [64][65]  (C^_t . B^_s) E[t,s] on the mask
+    float* gm = cbe + kChunk * 65;     // [64][65]  scratch; gM; then gM E dt_s
+    float* ac = gm + kChunk * 65;      // [64] acs
+    float* dv = ac + kChunk;           // [64] dt
+    float* ft = dv + kChunk;           // [64] weight of the carried-state term
+    float* ws = ft + kChunk;           // [64] chunk-state weight
+    float* gac = ws + kChunk;          // [64] gradient of acs
+    float* gdv = gac + kChunk;         // [64] gradient of dt
+    float* red = gdv + kChunk;         // [64] per-token scratch
+    float* red2 = red + kChunk;        // [32] block reduction scratch
+    int* seg = (int*)(red2 + 32);      // [64]
+    int* flag = seg + kChunk;          // [64]
+
+    const int Lb = row_length(a.lengths, b, L);
+    chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, Lb, seg, flag);
+    const int64_t bh = (int64_t)b * H + h;
+    if (tid < kChunk) {
+        const int64_t o = bh * L + t0 + tid;
+        ac[tid] = tid < Lc ? w.acs[o] : 0.0f;
+        dv[tid] = tid < Lc ? w.dt[o] : 0.0f;
+        gac[tid] = 0.0f;
+        gdv[tid] = 0.0f;
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        ft[tid] = (tid < Lc && seg[tid] == 0) ? expf(ac[tid]) : 0.0f;
+        ws[tid] = (tid < Lc && seg[tid] == seg[last]) ? expf(ac[last] - ac[tid]) * dv[tid] : 0.0f;
+    }
+    load_x_rows<T>(s, a, w.u, b, h, t0, Lc, xs, P);
+    load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 1, cs, N);
+    load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 0, bs, NB);
+    const float* hp = w.hin + (((int64_t)b * nc + c) * H + h) * P * N;
+    for (int e = tid; e < P * N; e += blockDim.x) hb[(e / N) * NB + e % N] = hp[e];
+    __syncthreads();
+
+    // (C^_t . B^_s) E[t,s]
+    for (int e = tid; e < kChunk * kChunk; e += blockDim.x) {
+        const int t = e / kChunk, r = e % kChunk;
+        float v = 0.0f;
+        if (r <= t && t < Lc && seg[r] == seg[t]) {
+            float dot = 0.0f;
+            for (int n = 0; n < N; n++) dot += cs[t * N + n] * bs[r * NB + n];
+            v = dot * expf(ac[t] - ac[r]);
+        }
+        cbe[t * 65 + r] = v;
+    }
+    __syncthreads();
+
+    // y recomputed; gy, gz; the carried-state term's share of gacs; gD
+    const float Dh = a.D[h];
+    float dpart = 0.0f;
+    for (int e = tid; e < kChunk * P; e += blockDim.x) {
+        const int t = e / P, p = e % P;
+        float gyv = 0.0f, prod = 0.0f;
+        if (t < Lc) {
+            const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
+            if (t0 + t < Lb) {
+                float y = 0.0f;
+                for (int r = 0; r <= t; r++) y += cbe[t * 65 + r] * dv[r] * xs[r * P + p];
+                float off = 0.0f;
+                if (ft[t] != 0.0f)
+                    for (int n = 0; n < N; n++) off += cs[t * N + n] * hb[p * NB + n];
+                y += ft[t] * off + Dh * xs[t * P + p];
+                const float zv = to_f(((const T*)a.z)[o]);
+                const float go = to_f(((const T*)w.gout)[o]);
+                gyv = go * silu_f(zv);
+                w.gz[o] = go * y * silu_grad_f(zv);
+                prod = ft[t] * gyv * off;
+                dpart += gyv * xs[t * P + p];
+            } else {
+                w.gz[o] = 0.0f;
+            }
+        }
+        gy[t * P + p] = gyv;
+        gm[t * 65 + p] = prod;
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        float acc = 0.0f;
+        for (int p = 0; p < P; p++) acc += gm[tid * 65 + p];
+        gac[tid] += acc;
+    }
+    dpart = block_sum(dpart, red2);
+    __syncthreads();
+
+    // gM[t,s] = gy_t . x_s on the mask
+    for (int e = tid; e < kChunk * kChunk; e += blockDim.x) {
+        const int t = e / kChunk, r = e % kChunk;
+        float v = 0.0f;
+        if (r <= t && t < Lc && seg[r] == seg[t])
+            for (int p = 0; p < P; p++) v += gy[t * P + p] * xs[r * P + p];
+        gm[t * 65 + r] = v;
+    }
+    __syncthreads();
+    // acs through E: + row sums, - column sums of gM M; dt through M
+    if (tid < kChunk) {
+        const int t = tid;
+        float acc = 0.0f;
+        for (int r = 0; r <= t; r++) acc += gm[t * 65 + r] * cbe[t * 65 + r] * dv[r];
+        gac[t] += acc;
+    } else if (tid < 2 * kChunk) {
+        const int r = tid - kChunk;
+        float acc = 0.0f, gd = 0.0f;
+        for (int t = r; t < kChunk; t++) {
+            const float g = gm[t * 65 + r] * cbe[t * 65 + r];
+            acc += g * dv[r];
+            gd += g;
+        }
+        red[r] = acc;
+        gdv[r] += gd;
+    }
+    __syncthreads();
+    if (tid < kChunk) gac[tid] -= red[tid];
+    // gM -> gradient of (C^_t . B^_s): gM E dt_s
+    for (int e = tid; e < kChunk * kChunk; e += blockDim.x) {
+        const int t = e / kChunk, r = e % kChunk;
+        const float g = gm[t * 65 + r];
+        gm[t * 65 + r] = g != 0.0f ? g * expf(ac[t] - ac[r]) * dv[r] : 0.0f;
+    }
+    __syncthreads();
+
+    // gx (intra-chunk and D), kept in registers until the chunk-state part is added
+    float gx_r[kMaxXe];
+#pragma unroll
+    for (int k = 0; k < kMaxXe; k++) {
+        const int e = tid + k * kBwdThreads;
+        float v = 0.0f;
+        if (e < kChunk * P) {
+            const int r = e / P, p = e % P;
+            if (r < Lc) {
+                for (int t = r; t < Lc; t++) v += cbe[t * 65 + r] * gy[t * P + p];
+                v = v * dv[r] + Dh * gy[r * P + p];
+            }
+        }
+        gx_r[k] = v;
+    }
+    // gC^ (complete), written per head
+    for (int e = tid; e < kChunk * N; e += blockDim.x) {
+        const int t = e / N, n = e % N;
+        if (t >= Lc) continue;
+        float v = 0.0f;
+        for (int r = 0; r <= t; r++) v += gm[t * 65 + r] * bs[r * NB + n];
+        if (ft[t] != 0.0f) {
+            float o = 0.0f;
+            for (int p = 0; p < P; p++) o += gy[t * P + p] * hb[p * NB + n];
+            v += ft[t] * o;
+        }
+        w.gch[(((int64_t)b * L + t0 + t) * H + h) * N + n] = v;
+    }
+    // gB^ (intra-chunk part)
+    float gb_r[kMaxBe];
+#pragma unroll
+    for (int k = 0; k < kMaxBe; k++) {
+        const int e = tid + k * kBwdThreads;
+        float v = 0.0f;
+        if (e < kChunk * N) {
+            const int r = e / N, n = e % N;
+            for (int t = r; t < Lc; t++) v += gm[t * 65 + r] * cs[t * N + n];
+        }
+        gb_r[k] = v;
+    }
+    __syncthreads();
+
+    // gS_c replaces Hin_c; gk = <gS_c, Hin_c> is the carry's gradient
+    const float* gsp = w.gs + (((int64_t)b * nc + c) * H + h) * P * N;
+    float gk = 0.0f;
+    for (int e = tid; e < P * N; e += blockDim.x) {
+        const int i = (e / N) * NB + e % N;
+        const float g = gsp[e];
+        gk += g * hb[i];
+        hb[i] = g;
+    }
+    gk = block_sum(gk, red2);
+    __syncthreads();
+
+    // chunk state: gXs = gS B^_s -> gx += w_s gXs; gw_s = gXs . x_s; gB^_s += w_s x_s gS
+#pragma unroll
+    for (int k = 0; k < kMaxXe; k++) {
+        const int e = tid + k * kBwdThreads;
+        if (e < kChunk * P) {
+            const int r = e / P, p = e % P;
+            float g = 0.0f;
+            for (int n = 0; n < N; n++) g += hb[p * NB + n] * bs[r * NB + n];
+            gx_r[k] += ws[r] * g;
+            gm[r * 65 + p] = g * xs[r * P + p];
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxBe; k++) {
+        const int e = tid + k * kBwdThreads;
+        if (e < kChunk * N) {
+            const int r = e / N, n = e % N;
+            if (r < Lc) {
+                float g = 0.0f;
+                for (int p = 0; p < P; p++) g += xs[r * P + p] * hb[p * NB + n];
+                w.gbh[(((int64_t)b * L + t0 + r) * H + h) * N + n] = gb_r[k] + ws[r] * g;
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxXe; k++) {
+        const int e = tid + k * kBwdThreads;
+        if (e < kChunk * P) {
+            const int r = e / P, p = e % P;
+            if (r < Lc) w.gu[((int64_t)b * L + t0 + r) * cd + h * P + p] = gx_r[k];
+        }
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        float acc = 0.0f;
+        for (int p = 0; p < P; p++) acc += gm[tid * 65 + p];
+        red[tid] = acc;                               // gradient of w_s
+    }
+    __syncthreads();
+    if (tid < Lc && seg[tid] == seg[last]) {
+        gac[tid] -= red[tid] * ws[tid];
+        gdv[tid] += red[tid] * expf(ac[last] - ac[tid]);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float gl = 0.0f;
+        for (int r = 0; r < Lc; r++) gl += red[r] * ws[r];
+        const float kc = w.cdecay[bh * nc + c];
+        if (kc != kChunkReset) gl += gk * kc;         // k_c = exp(acs_last)
+        gac[last] += gl;
+    }
+    __syncthreads();
+
+    // dA = dt a feeds acs through the segmented in-chunk cumsum: gdA is its reverse
+    if (tid < kChunk) {
+        float gv = 0.0f, ga = 0.0f;
+        if (tid < Lc) {
+            const int j = tid;
+            float gda = 0.0f;
+            for (int t = j; t < Lc && seg[t] == seg[j]; t++) gda += gac[t];
+            const int64_t tok = (int64_t)b * L + t0 + j;
+            const bool real = t0 + j < Lb;
+            float av;
+            bool floored = false;
+            if (s.a_per_token) {
+                const float Av = a.A[tok * H + h];
+                av = fminf(Av, -kAFloor);
+                floored = Av > -kAFloor;
+            } else {
+                av = a.A[h];
+            }
+            if (real) {
+                gv = (gdv[j] + gda * av) * sigmoid_f(a.dt_raw[tok * H + h] + a.dt_bias[h]);
+                ga = floored ? 0.0f : gda * dv[j];
+            }
+            w.gdt_raw[tok * H + h] = gv;
+            if (s.a_per_token && w.gA) w.gA[tok * H + h] = ga;
+        }
+        red[tid] = gv;
+        gm[tid] = ga;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float sdt = 0.0f, sa = 0.0f;
+        for (int j = 0; j < Lc; j++) {
+            sdt += red[j];
+            sa += gm[j];
+        }
+        const int64_t pi = ((int64_t)b * nc + c) * H + h;
+        w.p_dtb[pi] = sdt;
+        w.p_A[pi] = sa;
+        w.p_D[pi] = dpart;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Per (row, 64-token block, group): sum the group's heads' gB^ and gC^, then (with
+// the B/C norm) go back through B^ = B r w + bias_h.  128 threads, n = tid (+128).
+template <typename T>
+__global__ void __launch_bounds__(128)
+bwd_bc_group_kernel(Shape s, FwdArgs a, BwdBufs w)
+{
+    extern __shared__ float sm[];
+    const int N = s.dstate, H = s.nheads, G = s.ngroups, L = s.seqlen, hg = H / G;
+    const int HP = H * s.headdim, GN = G * N, cd = s.conv_dim();
+    const int tb = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int ntb = gridDim.x;
+    const int tid = threadIdx.x;
+    float* acc = sm;                   // [2][hg][N] per-head bias gradient of this block
+    float* red = acc + 2 * hg * N;     // [32]
+    const bool norm = s.bc_norm != 0;
+    if (norm)
+        for (int i = tid; i < 2 * hg * N; i += blockDim.x) acc[i] = 0.0f;
+    float wacc[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};   // [which][n slot] norm-weight gradient
+    __syncthreads();
+    for (int t = tb * kChunk; t < min(L, (tb + 1) * kChunk); t++) {
+        const int64_t tok = (int64_t)b * L + t;
+        for (int which = 0; which < 2; which++) {
+            const float* gh = which ? w.gch : w.gbh;
+            const float* wn = which ? a.cn_w : a.bn_w;
+            float gsum[2] = {0.0f, 0.0f}, uv[2] = {0.0f, 0.0f};
+            float ss = 0.0f, dot = 0.0f;
+            for (int k = 0; k < 2; k++) {
+                const int n = tid + 128 * k;
+                if (n >= N) continue;
+                for (int j = 0; j < hg; j++) {
+                    const float v = gh[(tok * H + g * hg + j) * N + n];
+                    gsum[k] += v;
+                    if (norm) acc[(which * hg + j) * N + n] += v;
+                }
+                if (norm) {
+                    const int64_t ch = HP + which * GN + g * N + n;
+                    uv[k] = w.u ? w.u[tok * cd + ch]
+                                : to_f(((const T*)(which ? a.C : a.B))[tok * GN + g * N + n]);
+                    ss += uv[k] * uv[k];
+                    dot += gsum[k] * (wn ? wn[n] : 1.0f) * uv[k];
+                }
+            }
+            float r = 1.0f, r3n = 0.0f;
+            if (norm) {
+                ss = block_sum(ss, red);
+                dot = block_sum(dot, red);
+                r = rsqrtf(ss / N + kNormEps);
+                r3n = r * r * r / N;
+            }
+            for (int k = 0; k < 2; k++) {
+                const int n = tid + 128 * k;
+                if (n >= N) continue;
+                float gval = gsum[k];
+                if (norm) {
+                    const float wv = wn ? wn[n] : 1.0f;
+                    gval = r * wv * gsum[k] - r3n * uv[k] * dot;
+                    wacc[which][k] += gsum[k] * uv[k] * r;
+                }
+                w.gu[tok * cd + HP + which * GN + g * N + n] = gval;
+            }
+        }
+    }
+    if (!norm) return;
+    __syncthreads();
+    // partials: p_nw (B, ntb, G, 2, N), p_nb (B, ntb, 2, H, N)
+    for (int which = 0; which < 2; which++)
+        for (int k = 0; k < 2; k++) {
+            const int n = tid + 128 * k;
+            if (n < N) w.p_nw[((((int64_t)b * ntb + tb) * G + g) * 2 + which) * N + n] = wacc[which][k];
+        }
+    for (int i = tid; i < 2 * hg * N; i += blockDim.x) {
+        const int which = i / (hg * N), j = (i / N) % hg, n = i % N;
+        w.p_nb[((((int64_t)b * ntb + tb) * 2 + which) * H + g * hg + j) * N + n] = acc[i];
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Back through SiLU and the causal conv: one thread per (row, channel, segment of
+// kConvSeg tokens); channels fastest, so a warp reads consecutive channels of a
+// token row.  gconv partials (B, nseg, cd, 5): four taps, then the bias.
+template <typename T>
+__global__ void __launch_bounds__(256)
+bwd_conv_kernel(Shape s, FwdArgs a, BwdBufs w)
+{
+    const int cd = s.conv_dim(), L = s.seqlen;
+    const int nseg = (L + kConvSeg - 1) / kConvSeg;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)s.batch * nseg * cd) return;
+    const int ch = (int)(gid % cd);
+    const int sg = (int)((gid / cd) % nseg);
+    const int b = (int)(gid / ((int64_t)cd * nseg));
+    const int HP = s.nheads * s.headdim, GN = s.ngroups * s.dstate;
+    const T* src;
+    float* dst;
+    int64_t stride;
+    int col;
+    if (ch < HP) { src = (const T*)a.x; dst = w.gx; stride = HP; col = ch; }
+    else if (ch < HP + GN) { src = (const T*)a.B; dst = w.gB; stride = GN; col = ch - HP; }
+    else { src = (const T*)a.C; dst = w.gC; stride = GN; col = ch - HP - GN; }
+    src += (int64_t)b * L * stride + col;
+    dst += (int64_t)b * L * stride + col;
+    const float* gu = w.gu + (int64_t)b * L * cd + ch;
+    const int Lb = row_length(a.lengths, b, L);
+    const int ts = sg * kConvSeg, te = min(L, ts + kConvSeg);
+
+    if (s.dconv == 1) {       // no conv: the gradient of the raw input is gu itself
+        for (int t = ts; t < te; t++) dst[(int64_t)t * stride] = t < Lb ? gu[(int64_t)t * cd] : 0.0f;
+        return;
+    }
+    const int32_t* seq_row = a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr;
+    float wk[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) wk[k] = to_f(((const T*)a.conv_w)[(int64_t)ch * 4 + k]);
+    const float cb = to_f(((const T*)a.conv_b)[ch]);
+    float gw[4] = {0.0f, 0.0f, 0.0f, 0.0f}, gbias = 0.0f;
+    // window of raw inputs x[t-3 .. t] and boundary flags at t-2 .. t
+    float xw[4];
+#pragma unroll
+    for (int k = 0; k < 3; k++) {
+        const int tau = ts - 3 + k;
+        xw[k] = (tau >= 0 && tau < Lb) ? to_f(src[(int64_t)tau * stride]) : 0.0f;
+    }
+    int bd1 = (ts - 2 >= 1 && ts - 2 < Lb) ? is_boundary(seq_row, ts - 2) : 0;   // at t-2
+    int bd2 = (ts - 1 >= 1 && ts - 1 < Lb) ? is_boundary(seq_row, ts - 1) : 0;   // at t-1
+    float gxw[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // pending gx at t-3 .. t
+    const int tend = min(te + 3, Lb);
+    for (int t = ts; t < tend; t++) {
+        xw[3] = to_f(src[(int64_t)t * stride]);
+        const int bd3 = is_boundary(seq_row, t);
+        // tap k reads x[t-3+k]; valid while no boundary lies in (t-3+k, t]
+        const bool ok3 = true;
+        const bool ok2 = !bd3;
+        const bool ok1 = ok2 && !bd2;
+        const bool ok0 = ok1 && !bd1 && t - 3 >= 0;
+        const bool okk[4] = {ok0, ok1 && t - 2 >= 0, ok2 && t - 1 >= 0, ok3};
+        float pre = cb;
+#pragma unroll
+        for (int k = 0; k < 4; k++) pre += okk[k] ? wk[k] * xw[k] : 0.0f;
+        const float gpre = gu[(int64_t)t * cd] * silu_grad_f(pre);
+        if (t < te) {
+            gbias += gpre;
+#pragma unroll
+            for (int k = 0; k < 4; k++) gw[k] += okk[k] ? gpre * xw[k] : 0.0f;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; k++) gxw[k] += okk[k] ? gpre * wk[k] : 0.0f;
+        // x[t-3] has all its contributions (tokens t-3 .. t): emit it
+        if (t - 3 >= ts && t - 3 < te) dst[(int64_t)(t - 3) * stride] = gxw[0];
+        gxw[0] = gxw[1]; gxw[1] = gxw[2]; gxw[2] = gxw[3]; gxw[3] = 0.0f;
+        xw[0] = xw[1]; xw[1] = xw[2]; xw[2] = xw[3];
+        bd1 = bd2; bd2 = bd3;
+    }
+    // tokens whose later taps lie past the row's real end, and padding
+    for (int tau = max(ts, tend - 3); tau < te; tau++) {
+        const int k = tau - (tend - 3);      // gxw[k] holds x[tend-3+k]
+        dst[(int64_t)tau * stride] = (tau < Lb && k >= 0 && k < 3) ? gxw[k] : 0.0f;
+    }
+    float* pc = w.p_conv + (((int64_t)b * nseg + sg) * cd + ch) * 5;
+#pragma unroll
+    for (int k = 0; k < 4; k++) pc[k] = gw[k];
+    pc[4] = gbias;
+}
+
+// out[m] = sum over r of in[r * ld + m], r in order (weight-gradient partials).
+__global__ void __launch_bounds__(256)
+bwd_reduce_kernel(const float* __restrict__ in, int64_t R, int64_t M, int64_t ld,
+                  float* __restrict__ out)
+{
+    const int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= M) return;
+    float acc = 0.0f;
+    for (int64_t r = 0; r < R; r++) acc += in[r * ld + m];
+    out[m] = acc;
+}
+
+// The conv partials (R, cd, 5) summed over r in order: taps to gconv_w (cd, 4),
+// the fifth column to gconv_b (cd).
+__global__ void __launch_bounds__(256)
+bwd_conv_reduce_kernel(const float* __restrict__ in, int64_t R, int cd, float* __restrict__ gw,
+                       float* __restrict__ gb)
+{
+    const int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= (int64_t)cd * 5) return;
+    float acc = 0.0f;
+    for (int64_t r = 0; r < R; r++) acc += in[r * cd * 5 + m];
+    const int ch = (int)(m / 5), k = (int)(m % 5);
+    if (k < 4) gw[(int64_t)ch * 4 + k] = acc;
+    else gb[ch] = acc;
+}
+
+// ---------------------------------------------------------------------------------
+// host side
+
+size_t bwd_chunk_smem_bytes(const Shape& s)
+{
+    const size_t P = s.headdim, N = s.dstate, NB = N + 1;
+    return sizeof(float) * (kChunk * N + kChunk * NB + 2 * kChunk * P + P * NB + 2 * kChunk * 65 +
+                            8 * kChunk + 32) + sizeof(int) * 2 * kChunk;
+}
+
+static size_t state_out_smem_bytes(const Shape& s)
+{
+    return sizeof(float) * (kChunk * (size_t)s.dstate + kChunk * (size_t)s.headdim + kChunk) +
+           sizeof(int) * 2 * kChunk;
+}
+
+bool bwd_supported(const Shape& s)
+{
+    return s.headdim <= 64 && s.dstate <= 128 && bwd_chunk_smem_bytes(s) <= 227 * 1024;
+}
+
+template <typename K>
+static cudaError_t set_smem(K kern, size_t bytes)
+{
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename T>
+static cudaError_t launch_bwd_t(const Shape& s, const FwdArgs& a, const BwdBufs& w, int* launches,
+                                cudaStream_t st)
+{
+    cudaError_t e;
+    const dim3 cgrid(s.nchunks(), s.nheads, s.batch);
+    const size_t so = state_out_smem_bytes(s);
+    if ((e = set_smem(bwd_state_out_kernel<T>, so)) != cudaSuccess) return e;
+    bwd_state_out_kernel<T><<<cgrid, kBwdThreads, so, st>>>(s, a, w);
+    ++*launches;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const int64_t nel = (int64_t)s.batch * s.nheads * s.headdim * s.dstate;
+    bwd_state_scan_kernel<<<(unsigned)((nel + 255) / 256), 256, 0, st>>>(s, w.cdecay, w.gs);
+    ++*launches;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const size_t sc = bwd_chunk_smem_bytes(s);
+    if ((e = set_smem(bwd_chunk_kernel<T>, sc)) != cudaSuccess) return e;
+    bwd_chunk_kernel<T><<<cgrid, kBwdThreads, sc, st>>>(s, a, w);
+    ++*launches;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const int ntb = s.nchunks();
+    const int hg = s.nheads / s.ngroups;
+    const size_t sg = sizeof(float) * (2 * (size_t)hg * s.dstate + 32);
+    if ((e = set_smem(bwd_bc_group_kernel<T>, sg)) != cudaSuccess) return e;
+    bwd_bc_group_kernel<T><<<dim3(ntb, s.ngroups, s.batch), 128, sg, st>>>(s, a, w);
+    ++*launches;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const int nseg = (s.seqlen + kConvSeg - 1) / kConvSeg;
+    const int64_t nth = (int64_t)s.batch * nseg * s.conv_dim();
+    bwd_conv_kernel<T><<<(unsigned)((nth + 255) / 256), 256, 0, st>>>(s, a, w);
+    ++*launches;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    // weight gradients: fixed-order sums of the partials
+    auto reduce = [&](const float* in, int64_t R, int64_t M, int64_t ld, float* out) -> cudaError_t {
+        if (!out || M == 0) return cudaSuccess;
+        bwd_reduce_kernel<<<(unsigned)((M + 255) / 256), 256, 0, st>>>(in, R, M, ld, out);
+        ++*launches;
+        return cudaGetLastError();
+    };
+    const int64_t rc = (int64_t)s.batch * s.nchunks(), Hh = s.nheads;
+    if ((e = reduce(w.p_dtb, rc, Hh, Hh, w.g_dt_bias)) != cudaSuccess) return e;
+    if ((e = reduce(w.p_D, rc, Hh, Hh, w.g_D)) != cudaSuccess) return e;
+    if (!s.a_per_token && (e = reduce(w.p_A, rc, Hh, Hh, w.gA)) != cudaSuccess) return e;
+    if (s.dconv == 4) {
+        const int cd = s.conv_dim();
+        bwd_conv_reduce_kernel<<<(unsigned)(((int64_t)cd * 5 + 255) / 256), 256, 0, st>>>(
+            w.p_conv, (int64_t)s.batch * nseg, cd, w.gconv_w, w.gconv_b);
+        ++*launches;
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (s.bc_norm) {
+        const int64_t N = s.dstate, HN = Hh * N;
+        const int64_t rn = (int64_t)s.batch * ntb * s.ngroups, rb = (int64_t)s.batch * ntb;
+        if ((e = reduce(w.p_nw, rn, N, 2 * N, w.g_bnw)) != cudaSuccess) return e;
+        if ((e = reduce(w.p_nw + N, rn, N, 2 * N, w.g_cnw)) != cudaSuccess) return e;
+        if ((e = reduce(w.p_nb, rb, HN, 2 * HN, w.g_bnb)) != cudaSuccess) return e;
+        if ((e = reduce(w.p_nb + HN, rb, HN, 2 * HN, w.g_cnb)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_backward(const Shape& s, const FwdArgs& a, const BwdBufs& w, int* launches,
+                            cudaStream_t st)
+{
+    return s.act_bf16 ? launch_bwd_t<bf16>(s, a, w, launches, st)
+                      : launch_bwd_t<float>(s, a, w, launches, st);
+}
+
+}  // namespace ssd

@@ -73,6 +73,7 @@ struct FusedParams {
     const int32_t* lengths;   // (B) real tokens per row of a ragged batch, or null
     const float* D;
     const bf16* x;            // raw x, for the conv history at segment starts
+    int64_t ld_x;             // its row stride (elements)
     const bf16* conv_w;       // (conv_dim, 4) or null
     const bf16* conv_b;
     const bf16* init_conv;    // (B, 3, conv_dim) or null
@@ -549,7 +550,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         // or the caller's conv history before token 0
                         const int tok = t0 + row;
                         raw[qq] = tok >= 0
-                            ? *(const uint32_t*)(p.x + ((int64_t)b * L + tok) * (H * 64) + h * 64 + 2 * pp)
+                            ? *(const uint32_t*)(p.x + ((int64_t)b * L + tok) * p.ld_x + h * 64 + 2 * pp)
                             : (p.init_conv ? *(const uint32_t*)(p.init_conv + ((int64_t)b * 3 + (tok + 3)) * cdim +
                                                                h * 64 + 2 * pp)
                                            : 0u);
@@ -960,13 +961,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 // [64 channels x 64 tokens] bf16 boxes with the 128-byte swizzle over a
-// (batch, seqlen, width) row-major tensor.
-static bool encode_tile_map(CUtensorMap* m, const void* base, int width, int seqlen, int batch)
+// (batch, seqlen, width) tensor whose rows lie ld elements apart (ld = width
+// when contiguous; a column block of a packed in_proj row otherwise).
+static bool encode_tile_map(CUtensorMap* m, const void* base, int width, int64_t ld, int seqlen,
+                            int batch)
 {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)width, (cuuint64_t)seqlen, (cuuint64_t)batch};
-    const cuuint64_t strides[2] = {(cuuint64_t)width * 2, (cuuint64_t)width * 2 * seqlen};
+    const cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * seqlen};
     const cuuint32_t box[3] = {64, 64, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
@@ -1059,15 +1062,15 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
         return cudaErrorNotSupported;
     const int HP = s.nheads * 64, GN = s.ngroups * s.dstate;
     CUtensorMap maps[5];
-    bool ok = encode_tile_map(&maps[0], a.x, HP, s.seqlen, s.batch) &&
-              encode_tile_map(&maps[1], a.z, HP, s.seqlen, s.batch) &&
-              encode_tile_map(&maps[4], a.out, HP, s.seqlen, s.batch);
+    bool ok = encode_tile_map(&maps[0], a.x, HP, a.ld_x, s.seqlen, s.batch) &&
+              encode_tile_map(&maps[1], a.z, HP, a.ld_z, s.seqlen, s.batch) &&
+              encode_tile_map(&maps[4], a.out, HP, HP, s.seqlen, s.batch);
     if (s.dconv == 4) {
-        ok = ok && encode_tile_map(&maps[2], ubc, 2 * GN, s.seqlen, s.batch);
+        ok = ok && encode_tile_map(&maps[2], ubc, 2 * GN, 2 * GN, s.seqlen, s.batch);
         maps[3] = maps[2];
     } else {
-        ok = ok && encode_tile_map(&maps[2], a.B, GN, s.seqlen, s.batch) &&
-             encode_tile_map(&maps[3], a.C, GN, s.seqlen, s.batch);
+        ok = ok && encode_tile_map(&maps[2], a.B, GN, a.ld_bc, s.seqlen, s.batch) &&
+             encode_tile_map(&maps[3], a.C, GN, a.ld_bc, s.seqlen, s.batch);
     }
     if (!ok) return cudaErrorInvalidValue;
     FusedParams fp;
@@ -1082,6 +1085,7 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.lengths = a.lengths;
     fp.D = a.D;
     fp.x = (const bf16*)a.x;
+    fp.ld_x = a.ld_x;
     fp.conv_w = (const bf16*)a.conv_w;
     fp.conv_b = (const bf16*)a.conv_b;
     fp.init_conv = (const bf16*)a.init_conv;

@@ -22,14 +22,19 @@ namespace ssd {
 
 constexpr int kTokPerThread = 8;
 
+// Row strides (elements) of the raw x and B|C inputs.
+struct RawStrides {
+    int64_t x, bc;
+};
+
 template <typename T>
-__device__ __forceinline__ const T* channel_src(const Shape& s, const T* x, const T* B, const T* C,
-                                               int c, int64_t& stride, int& col)
+__device__ __forceinline__ const T* channel_src(const Shape& s, RawStrides ld, const T* x, const T* B,
+                                               const T* C, int c, int64_t& stride, int& col)
 {
     const int HP = s.nheads * s.headdim, GN = s.ngroups * s.dstate;
-    if (c < HP) { stride = HP; col = c; return x; }
-    if (c < HP + GN) { stride = GN; col = c - HP; return B; }
-    stride = GN; col = c - HP - GN; return C;
+    if (c < HP) { stride = ld.x; col = c; return x; }
+    if (c < HP + GN) { stride = ld.bc; col = c - HP; return B; }
+    stride = ld.bc; col = c - HP - GN; return C;
 }
 
 // Eight consecutive elements kept in their storage form (fewer registers than
@@ -70,7 +75,7 @@ __global__ void __launch_bounds__(256, 3)
 conv_silu_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
                  const T* __restrict__ Cm, const T* __restrict__ w, const T* __restrict__ bias,
                  const int32_t* __restrict__ seq, const T* __restrict__ hist0,
-                 OutT* __restrict__ u, int cbase)
+                 OutT* __restrict__ u, int cbase, RawStrides ld)
 {
     const int cd = s.conv_dim();
     const int nvec = (cd - cbase) / 8;
@@ -86,7 +91,7 @@ conv_silu_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
 
     int64_t stride;
     int col;
-    const T* src = channel_src(s, x, Bm, Cm, c, stride, col);
+    const T* src = channel_src(s, ld, x, Bm, Cm, c, stride, col);
     src += (int64_t)b * L * stride + col;
 
     Vec8<T> wv[4], bv;          // weight (channel i, tap k) = element 4*i + k
@@ -149,7 +154,8 @@ __global__ void __launch_bounds__(256, 2)
 conv_silu_bf16_kernel(Shape s, const bf16* __restrict__ x, const bf16* __restrict__ Bm,
                       const bf16* __restrict__ Cm, const bf16* __restrict__ w,
                       const bf16* __restrict__ bias, const int32_t* __restrict__ seq,
-                      const bf16* __restrict__ hist0, OutT* __restrict__ u, int cbase)
+                      const bf16* __restrict__ hist0, OutT* __restrict__ u, int cbase,
+                      RawStrides ld)
 {
     const int cd = s.conv_dim();
     const int nvec = (cd - cbase) / 8;
@@ -165,7 +171,7 @@ conv_silu_bf16_kernel(Shape s, const bf16* __restrict__ x, const bf16* __restric
 
     int64_t stride;
     int col;
-    const bf16* src = channel_src(s, x, Bm, Cm, c, stride, col);
+    const bf16* src = channel_src(s, ld, x, Bm, Cm, c, stride, col);
     src += (int64_t)b * L * stride + col;
     const int t0 = tg * kTokPerThread;
 
@@ -236,7 +242,7 @@ conv_silu_bf16_kernel(Shape s, const bf16* __restrict__ x, const bf16* __restric
 // 1/rms of one N-long B or C row per thread: rinv[(b L + t) 2G + which G + g].
 __global__ void __launch_bounds__(256)
 bc_rms_kernel(Shape s, const bf16* __restrict__ Bm, const bf16* __restrict__ Cm,
-              const bf16* __restrict__ ubc, float* __restrict__ rinv)
+              const bf16* __restrict__ ubc, float* __restrict__ rinv, int64_t ld_bc)
 {
     const int G = s.ngroups, N = s.dstate;
     const int64_t rows = (int64_t)s.batch * s.seqlen * 2 * G;
@@ -245,7 +251,7 @@ bc_rms_kernel(Shape s, const bf16* __restrict__ Bm, const bf16* __restrict__ Cm,
     const int64_t tok = gid / (2 * G);
     const int k = (int)(gid % (2 * G));          // which * G + g
     const bf16* src = ubc ? ubc + tok * (2 * G * N) + (int64_t)k * N
-                          : (k < G ? Bm : Cm) + tok * (G * N) + (int64_t)(k % G) * N;
+                          : (k < G ? Bm : Cm) + tok * ld_bc + (int64_t)(k % G) * N;
     float ss = 0.0f;
     for (int n = 0; n < N; n += 8) {
         Vec8<bf16> v;
@@ -261,7 +267,7 @@ cudaError_t launch_bc_rms(const Shape& s, const FwdArgs& a, const void* ubc, flo
     if (!s.act_bf16 || s.dstate % 8) return cudaErrorInvalidValue;
     const int64_t rows = (int64_t)s.batch * s.seqlen * 2 * s.ngroups;
     bc_rms_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(
-        s, (const bf16*)a.B, (const bf16*)a.C, (const bf16*)ubc, rinv);
+        s, (const bf16*)a.B, (const bf16*)a.C, (const bf16*)ubc, rinv, a.ld_bc);
     return cudaGetLastError();
 }
 
@@ -272,7 +278,7 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 conv_state_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
                   const T* __restrict__ Cm, const int32_t* __restrict__ seq,
-                  const int32_t* __restrict__ lengths, const T* hist0, T* hist1)
+                  const int32_t* __restrict__ lengths, const T* hist0, T* hist1, RawStrides ld)
 {
     const int cd = s.conv_dim();
     const int nvec = cd / 8;
@@ -284,7 +290,7 @@ conv_state_kernel(Shape s, const T* __restrict__ x, const T* __restrict__ Bm,
     const int32_t* seq_row = seq ? seq + (int64_t)b * L : nullptr;
     int64_t stride;
     int col;
-    const T* src = channel_src(s, x, Bm, Cm, c, stride, col);
+    const T* src = channel_src(s, ld, x, Bm, Cm, c, stride, col);
     src += (int64_t)b * L * stride + col;
 
     // the row's last real token is Lb - 1 (Lb = L unless the batch is ragged)
@@ -319,11 +325,12 @@ static cudaError_t launch_conv(const Shape& s, const FwdArgs& a, OutT* u, int cb
     if constexpr (sizeof(T) == 2)
         conv_silu_bf16_kernel<OutT><<<(unsigned)blocks, 256, 0, st>>>(
             s, (const bf16*)a.x, (const bf16*)a.B, (const bf16*)a.C, (const bf16*)a.conv_w,
-            (const bf16*)a.conv_b, a.seq_idx, (const bf16*)a.init_conv, u, cbase);
+            (const bf16*)a.conv_b, a.seq_idx, (const bf16*)a.init_conv, u, cbase,
+            RawStrides{a.ld_x, a.ld_bc});
     else
         conv_silu_kernel<T, OutT><<<(unsigned)blocks, 256, 0, st>>>(
             s, (const T*)a.x, (const T*)a.B, (const T*)a.C, (const T*)a.conv_w, (const T*)a.conv_b,
-            a.seq_idx, (const T*)a.init_conv, u, cbase);
+            a.seq_idx, (const T*)a.init_conv, u, cbase, RawStrides{a.ld_x, a.ld_bc});
     return cudaGetLastError();
 }
 
@@ -346,11 +353,11 @@ cudaError_t launch_conv_state(const Shape& s, const FwdArgs& a, cudaStream_t st)
     if (s.act_bf16)
         conv_state_kernel<bf16><<<(unsigned)blocks, 256, 0, st>>>(
             s, (const bf16*)a.x, (const bf16*)a.B, (const bf16*)a.C, a.seq_idx, a.lengths,
-            (const bf16*)a.init_conv, (bf16*)a.final_conv);
+            (const bf16*)a.init_conv, (bf16*)a.final_conv, RawStrides{a.ld_x, a.ld_bc});
     else
         conv_state_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
             s, (const float*)a.x, (const float*)a.B, (const float*)a.C, a.seq_idx, a.lengths,
-            (const float*)a.init_conv, (float*)a.final_conv);
+            (const float*)a.init_conv, (float*)a.final_conv, RawStrides{a.ld_x, a.ld_bc});
     return cudaGetLastError();
 }
 

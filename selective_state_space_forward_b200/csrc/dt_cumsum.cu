@@ -43,7 +43,8 @@ __device__ __forceinline__ float warp_seg_scan(float v, int& start, int lane)
 }
 
 __global__ void __launch_bounds__(256)
-dt_cumsum_kernel(Shape s, const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
+dt_cumsum_kernel(Shape s, const void* __restrict__ dt_raw, int64_t ld_dt, int dt_bf16,
+                 const float* __restrict__ dt_bias,
                  const float* __restrict__ A, const int32_t* __restrict__ seq,
                  const int32_t* __restrict__ lengths, float* __restrict__ dt_out,
                  float* __restrict__ acs_out, float* __restrict__ cdecay)
@@ -71,7 +72,9 @@ dt_cumsum_kernel(Shape s, const float* __restrict__ dt_raw, const float* __restr
         bd[half] = 0;
         if (t < Lb) {
             const int64_t i = ((int64_t)b * L + t) * H + h;
-            dtv[half] = softplus_f(dt_raw[i] + bias);
+            const int64_t id = ((int64_t)b * L + t) * ld_dt + h;
+            const float raw = dt_bf16 ? to_f(((const bf16*)dt_raw)[id]) : ((const float*)dt_raw)[id];
+            dtv[half] = softplus_f(raw + bias);
             const float av = s.a_per_token ? fminf(A[i], -kAFloor) : a_head;
             dA[half] = dtv[half] * av;
             bd[half] = is_boundary(seq_row, t);
@@ -106,7 +109,7 @@ cudaError_t launch_dt_cumsum(const Shape& s, const FwdArgs& a, float* dt, float*
 {
     const int64_t warps = (int64_t)s.batch * s.nchunks() * s.nheads;
     const int64_t blocks = (warps * 32 + 255) / 256;
-    dt_cumsum_kernel<<<(unsigned)blocks, 256, 0, st>>>(s, a.dt_raw, a.dt_bias, a.A, a.seq_idx,
+    dt_cumsum_kernel<<<(unsigned)blocks, 256, 0, st>>>(s, a.dt_raw, a.ld_dt, a.dt_act, a.dt_bias, a.A, a.seq_idx,
                                                        a.lengths, dt, acs, cdecay);
     return cudaGetLastError();
 }

@@ -60,6 +60,9 @@ struct ssd_handle {
     float* rinv;          // fused with bc_norm: 1/rms of every B and C row (B, L, 2G)
     int* status;          // device status word
     const float *bn_w, *cn_w, *bn_bias, *cn_bias;
+    int gn_on, gn_group;             // gated RMSNorm after the scan (ssd_set_gated_norm)
+    const float* gn_w;
+    float gn_eps;
     cudaEvent_t ev_start, ev_stop;   // measurement hook (caller-owned), or null
     uint64_t launches;               // kernels launched since ssd_create
     FusedWork fw;                    // fused path: segment hand-off buffers, epoch, SM count
@@ -261,15 +264,51 @@ ssd_status noalloc_device(cudaStream_t st, NoAllocDevice& out)
     return SSD_OK;
 }
 
+// Workspace of ssd_backward: byte offsets of its buffers (256-byte aligned).
+struct BwdPlan {
+    size_t u, dt, acs, cdecay, hin, gs, gu, gbh, gch, pdtb, pA, pD, pconv, pnw, pnb, total;
+};
+
+BwdPlan bwd_plan(const ssd_desc& d, int batch, int seqlen)
+{
+    BwdPlan p;
+    memset(&p, 0, sizeof p);
+    const size_t B = batch, L = seqlen, H = d.nheads, P = d.headdim, N = d.dstate, G = d.ngroups;
+    const size_t nc = (L + 63) / 64, cd = conv_dim(d), nseg = (L + 127) / 128;
+    size_t off = 0;
+    auto take = [&](size_t floats) { size_t o = off; off = align256(off + floats * sizeof(float)); return o; };
+    if (d.dconv == 4) p.u = take(B * L * cd);
+    p.dt = take(B * H * L);
+    p.acs = take(B * H * L);
+    p.cdecay = take(B * H * nc);
+    p.hin = take(B * nc * H * P * N);
+    p.gs = take(B * nc * H * P * N);
+    p.gu = take(B * L * cd);
+    p.gbh = take(B * L * H * N);
+    p.gch = take(B * L * H * N);
+    p.pdtb = take(B * nc * H);
+    p.pA = take(B * nc * H);
+    p.pD = take(B * nc * H);
+    if (d.dconv == 4) p.pconv = take(B * nseg * cd * 5);
+    if (d.bc_norm) {
+        p.pnw = take(B * nc * G * 2 * N);
+        p.pnb = take(B * nc * 2 * H * N);
+    }
+    p.total = off;
+    return p;
+}
+
 }  // namespace
 
 // ssd_forward and ssd_forward_ragged (lengths null: every row is seqlen long).
+// ld_in > 0: x, z, B, C and dt_raw are column blocks of rows ld_in elements apart,
+// dt_raw in the activation dtype (a packed in_proj output).
 static ssd_status forward_impl(ssd_handle* h, int32_t batch, int32_t seqlen, const int32_t* lengths,
-                               const void* x, const void* z, const float* dt_raw,
+                               const void* x, const void* z, const void* dt_raw,
                                const float* dt_bias, const float* A, const void* B, const void* C,
                                const float* D, const void* conv_w, const void* conv_b,
                                const int32_t* seq_idx, const void* init_state, void* out,
-                               void* final_state, struct CUstream_st* stream)
+                               void* final_state, struct CUstream_st* stream, int64_t ld_in = 0)
 {
     g_err.clear();
     SSD_TRY(check_handle_dims(h, batch, seqlen));
@@ -288,7 +327,7 @@ static ssd_status forward_impl(ssd_handle* h, int32_t batch, int32_t seqlen, con
         }
         return SSD_OK;
     }
-    SSD_TRY(check_common(h, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, out));
+    SSD_TRY(check_common(h, x, z, (const float*)dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, out));
     SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
     if (out == init_state || out == final_state)
         return fail(SSD_ERR_INVALID_ARG, "out may not alias a state buffer");
@@ -296,9 +335,14 @@ static ssd_status forward_impl(ssd_handle* h, int32_t batch, int32_t seqlen, con
     const Shape s = make_shape(h, batch, seqlen);
     FwdArgs a;
     memset(&a, 0, sizeof a);
+    default_strides(a, s);
+    if (ld_in > 0) {
+        a.ld_x = a.ld_z = a.ld_bc = a.ld_dt = ld_in;
+        a.dt_act = 1;
+    }
     a.lengths = lengths;
     a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
-    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
+    a.dt_raw = (const float*)dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
     a.init_ssm = (const float*)init_state;
     a.init_conv = (init_state && s.dconv == 4) ? (const char*)init_state + conv_offset(h->d, batch)
                                                : nullptr;
@@ -326,6 +370,9 @@ static ssd_status forward_impl(ssd_handle* h, int32_t batch, int32_t seqlen, con
                         "fused chunk kernel");
     }
     if (a.final_conv) SSD_LAUNCH(h, launch_conv_state(s, a, st), "conv-state kernel");
+    if (h->gn_on)
+        SSD_LAUNCH(h, launch_gated_norm(s, out, h->gn_w, h->gn_group, h->gn_eps, lengths, st),
+                   "gated norm kernel");
     if (h->d.validate_finite) {
         const size_t ob = (size_t)batch * seqlen * h->d.nheads * h->d.headdim * act_size(h->d);
         SSD_LAUNCH(h, launch_finite_check(out, ob, s.act_bf16, h->status, st), "finite check");
@@ -467,6 +514,31 @@ ssd_status ssd_set_bc_norm(ssd_handle* h, const float* B_norm_w, const float* C_
     return SSD_OK;
 }
 
+ssd_status ssd_set_gated_norm(ssd_handle* h, int32_t enable, const float* weight,
+                              int32_t group_size, float eps)
+{
+    g_err.clear();
+    if (!h) return fail(SSD_ERR_INVALID_ARG, "handle is NULL");
+    if (enable != 0 && enable != 1) return fail(SSD_ERR_INVALID_ARG, "enable must be 0 or 1 (got %d)", enable);
+    if (!enable) {
+        h->gn_on = 0;
+        return SSD_OK;
+    }
+    const int HP = h->d.nheads * h->d.headdim;
+    const int gs = group_size == 0 ? HP : group_size;
+    if (!ssd::gated_norm_group_ok(HP, gs))
+        return fail(SSD_ERR_INVALID_ARG,
+                    "group_size %d must divide H*P = %d, be a multiple of 8 and at most 16384",
+                    group_size, HP);
+    if (!(eps >= 0.0f) || eps > 1.0f) return fail(SSD_ERR_INVALID_ARG, "eps must lie in [0, 1] (got %g)", (double)eps);
+    SSD_TRY(check_ptr(weight, "weight", 4, false));
+    h->gn_on = 1;
+    h->gn_w = weight;
+    h->gn_group = gs;
+    h->gn_eps = eps;
+    return SSD_OK;
+}
+
 size_t ssd_state_conv_offset(const ssd_handle* h, int32_t batch)
 {
     if (!h || batch < 0) return 0;
@@ -506,6 +578,34 @@ ssd_status ssd_forward_ragged(ssd_handle* h, int32_t batch, int32_t seqlen, cons
                         conv_b, seq_idx, init_state, out, final_state, stream);
 }
 
+ssd_status ssd_forward_packed(ssd_handle* h, int32_t batch, int32_t seqlen, const void* zxbcdt,
+                              int64_t ld, const float* dt_bias, const float* A, const float* D,
+                              const void* conv_w, const void* conv_b, const int32_t* seq_idx,
+                              const void* init_state, void* out, void* final_state,
+                              struct CUstream_st* stream)
+{
+    g_err.clear();
+    if (!h) return fail(SSD_ERR_INVALID_ARG, "handle is NULL");
+    const int64_t HP = (int64_t)h->d.nheads * h->d.headdim, GN = (int64_t)h->d.ngroups * h->d.dstate;
+    const int64_t need = 2 * HP + 2 * GN + h->d.nheads;
+    const size_t es = act_size(h->d);
+    if (ld < need)
+        return fail(SSD_ERR_INVALID_ARG, "ld %lld is below the packed row width 2*H*P + 2*G*N + H = %lld",
+                    (long long)ld, (long long)need);
+    if ((ld * (int64_t)es) % 16)
+        return fail(SSD_ERR_ALIGNMENT, "ld * element size (%lld bytes) must be a multiple of 16",
+                    (long long)(ld * (int64_t)es));
+    if (batch > 0 && seqlen > 0) SSD_TRY(check_ptr(zxbcdt, "zxbcdt", 16, true));
+    const char* base = (const char*)zxbcdt;
+    const void* z = base;
+    const void* x = base ? base + HP * es : nullptr;
+    const void* B = base ? base + 2 * HP * es : nullptr;
+    const void* C = base ? base + (2 * HP + GN) * es : nullptr;
+    const void* dt = base ? base + (2 * HP + 2 * GN) * es : nullptr;
+    return forward_impl(h, batch, seqlen, nullptr, x, z, dt, dt_bias, A, B, C, D, conv_w, conv_b,
+                        seq_idx, init_state, out, final_state, stream, ld);
+}
+
 ssd_status ssd_step(ssd_handle* h, int32_t batch, const void* x, const void* z,
                     const float* dt_raw, const float* dt_bias, const float* A, const void* B,
                     const void* C, const float* D, const void* conv_w, const void* conv_b,
@@ -520,6 +620,7 @@ ssd_status ssd_step(ssd_handle* h, int32_t batch, const void* x, const void* z,
     const Shape s = make_shape(h, batch, 1);
     FwdArgs a;
     memset(&a, 0, sizeof a);
+    default_strides(a, s);
     a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
     a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.out = out;
     a.bn_w = h->bn_w; a.cn_w = h->cn_w; a.bn_bias = h->bn_bias; a.cn_bias = h->cn_bias;
@@ -527,6 +628,10 @@ ssd_status ssd_step(ssd_handle* h, int32_t batch, const void* x, const void* z,
     SSD_MAIN_LAUNCH(h, (cudaStream_t)stream,
                     launch_decode_step(s, a, (float*)state, hist, (cudaStream_t)stream),
                     "decode kernel");
+    if (h->gn_on)
+        SSD_LAUNCH(h, launch_gated_norm(s, out, h->gn_w, h->gn_group, h->gn_eps, nullptr,
+                                        (cudaStream_t)stream),
+                   "gated norm kernel");
     if (h->d.validate_finite) {
         const size_t ob = (size_t)batch * h->d.nheads * h->d.headdim * act_size(h->d);
         SSD_LAUNCH(h, launch_finite_check(out, ob, s.act_bf16, h->status, (cudaStream_t)stream),
@@ -559,6 +664,7 @@ ssd_status ssd_stage_conv(ssd_handle* h, int32_t batch, int32_t seqlen, const vo
     const Shape s = make_shape(h, batch, seqlen);
     FwdArgs a;
     memset(&a, 0, sizeof a);
+    default_strides(a, s);
     a.x = x; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b; a.seq_idx = seq_idx;
     a.init_conv = init_state ? (const char*)init_state + conv_offset(h->d, batch) : nullptr;
     SSD_LAUNCH(h, launch_conv_silu_all(s, a, u, (cudaStream_t)stream), "conv kernel");
@@ -581,6 +687,7 @@ ssd_status ssd_stage_dt(ssd_handle* h, int32_t batch, int32_t seqlen, const floa
     const Shape s = make_shape(h, batch, seqlen);
     FwdArgs a;
     memset(&a, 0, sizeof a);
+    default_strides(a, s);
     a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.seq_idx = seq_idx;
     SSD_LAUNCH(h, launch_dt_cumsum(s, a, dt, acs, nullptr, (cudaStream_t)stream),
                "dt/cumsum kernel");
@@ -664,6 +771,107 @@ ssd_status ssd_s6_forward(int32_t batch, int32_t seqlen, int32_t d_inner, int32_
     return SSD_OK;
 }
 
+size_t ssd_backward_workspace_bytes(const ssd_handle* h, int32_t batch, int32_t seqlen)
+{
+    if (!h || batch < 0 || seqlen < 0) return 0;
+    return bwd_plan(h->d, batch, seqlen).total;
+}
+
+ssd_status ssd_backward(ssd_handle* h, int32_t batch, int32_t seqlen, const int32_t* lengths,
+                        const void* x, const void* z, const float* dt_raw, const float* dt_bias,
+                        const float* A, const void* B, const void* C, const float* D,
+                        const void* conv_w, const void* conv_b, const int32_t* seq_idx,
+                        const void* gout, const ssd_grads* grads, void* workspace,
+                        size_t workspace_bytes, struct CUstream_st* stream)
+{
+    g_err.clear();
+    SSD_TRY(check_handle_dims(h, batch, seqlen));
+    if (!grads) return fail(SSD_ERR_INVALID_ARG, "grads is NULL");
+    SSD_TRY(check_ptr(lengths, "lengths", 4, false));
+    const Shape s = make_shape(h, batch, seqlen);
+    if (!bwd_supported(s))
+        return fail(SSD_ERR_UNSUPPORTED, "the backward serves headdim <= 64 and dstate <= 128 "
+                                         "(got headdim %d, dstate %d)", s.headdim, s.dstate);
+    if (batch == 0 || seqlen == 0) return SSD_OK;
+    SSD_TRY(check_ptr(gout, "gout", 16, true));
+    SSD_TRY(check_common(h, x, z, dt_raw, dt_bias, A, B, C, D, conv_w, conv_b, gout));
+    SSD_TRY(check_ptr(seq_idx, "seq_idx", 4, false));
+    SSD_TRY(check_ptr(grads->x, "grads->x", 16, true));
+    SSD_TRY(check_ptr(grads->z, "grads->z", 16, true));
+    SSD_TRY(check_ptr(grads->B, "grads->B", 16, true));
+    SSD_TRY(check_ptr(grads->C, "grads->C", 16, true));
+    SSD_TRY(check_ptr(grads->dt_raw, "grads->dt_raw", 4, true));
+    SSD_TRY(check_ptr(grads->dt_bias, "grads->dt_bias", 4, false));
+    SSD_TRY(check_ptr(grads->A, "grads->A", 4, false));
+    SSD_TRY(check_ptr(grads->D, "grads->D", 4, false));
+    SSD_TRY(check_ptr(grads->conv_w, "grads->conv_w", 4, false));
+    SSD_TRY(check_ptr(grads->conv_b, "grads->conv_b", 4, false));
+    SSD_TRY(check_ptr(grads->B_norm_w, "grads->B_norm_w", 4, false));
+    SSD_TRY(check_ptr(grads->C_norm_w, "grads->C_norm_w", 4, false));
+    SSD_TRY(check_ptr(grads->B_bias, "grads->B_bias", 4, false));
+    SSD_TRY(check_ptr(grads->C_bias, "grads->C_bias", 4, false));
+    if (h->d.dconv == 1 && (grads->conv_w || grads->conv_b))
+        return fail(SSD_ERR_INVALID_ARG, "grads->conv_w/conv_b must be NULL when dconv is 1");
+    if (!h->d.bc_norm && (grads->B_norm_w || grads->C_norm_w || grads->B_bias || grads->C_bias))
+        return fail(SSD_ERR_INVALID_ARG, "norm gradients need a handle created with bc_norm = 1");
+    SSD_TRY(check_ptr(workspace, "workspace", 256, true));
+    const BwdPlan pl = bwd_plan(h->d, batch, seqlen);
+    if (workspace_bytes < pl.total)
+        return fail(SSD_ERR_INVALID_ARG, "workspace_bytes %zu is below the %zu bytes the call needs "
+                    "(ssd_backward_workspace_bytes)", workspace_bytes, pl.total);
+    cudaStream_t st = (cudaStream_t)stream;
+
+    FwdArgs a;
+    memset(&a, 0, sizeof a);
+    default_strides(a, s);
+    a.lengths = lengths;
+    a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
+    a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
+    a.bn_w = h->bn_w; a.cn_w = h->cn_w; a.bn_bias = h->bn_bias; a.cn_bias = h->cn_bias;
+    char* ws = (char*)workspace;
+    BwdBufs w;
+    memset(&w, 0, sizeof w);
+    float* u = s.dconv == 4 ? (float*)(ws + pl.u) : nullptr;
+    float* dt = (float*)(ws + pl.dt);
+    float* acs = (float*)(ws + pl.acs);
+    float* cdecay = (float*)(ws + pl.cdecay);
+    float* hin = (float*)(ws + pl.hin);
+    w.u = u; w.dt = dt; w.acs = acs; w.cdecay = cdecay; w.hin = hin;
+    w.gs = (float*)(ws + pl.gs);
+    w.gout = gout;
+    w.gu = (float*)(ws + pl.gu);
+    w.gbh = (float*)(ws + pl.gbh);
+    w.gch = (float*)(ws + pl.gch);
+    w.p_dtb = (float*)(ws + pl.pdtb);
+    w.p_A = (float*)(ws + pl.pA);
+    w.p_D = (float*)(ws + pl.pD);
+    w.p_conv = s.dconv == 4 ? (float*)(ws + pl.pconv) : nullptr;
+    w.p_nw = s.bc_norm ? (float*)(ws + pl.pnw) : nullptr;
+    w.p_nb = s.bc_norm ? (float*)(ws + pl.pnb) : nullptr;
+    w.gx = grads->x; w.gz = grads->z; w.gB = grads->B; w.gC = grads->C;
+    w.gdt_raw = grads->dt_raw; w.gA = grads->A;
+    w.g_dt_bias = grads->dt_bias; w.g_D = grads->D;
+    w.gconv_w = grads->conv_w; w.gconv_b = grads->conv_b;
+    w.g_bnw = grads->B_norm_w; w.g_cnw = grads->C_norm_w;
+    w.g_bnb = grads->B_bias; w.g_cnb = grads->C_bias;
+    if (s.dconv == 4 && (!w.gconv_w) != (!w.gconv_b))
+        return fail(SSD_ERR_INVALID_ARG, "grads->conv_w and grads->conv_b must both be set or both be NULL");
+
+    // forward recompute on the staged kernels: conv output, dt and the cumsum, the
+    // states entering every chunk (zero initial state)
+    if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_all(s, a, u, st), "conv kernel");
+    SSD_LAUNCH(h, launch_dt_cumsum(s, a, dt, acs, cdecay, st), "dt/cumsum kernel");
+    SSD_LAUNCH(h, launch_chunk_state(s, a, u, dt, acs, hin, st), "chunk-state kernel");
+    SSD_LAUNCH(h, launch_state_passing(s, a, cdecay, hin, st), "state-passing kernel");
+    int nl = 0;
+    if (h->ev_start) SSD_CUDA(cudaEventRecord(h->ev_start, st), "timing event");
+    const cudaError_t e = launch_backward(s, a, w, &nl, st);
+    h->launches += nl;
+    if (e != cudaSuccess) return cuda_fail(e, "backward kernels");
+    if (h->ev_stop) SSD_CUDA(cudaEventRecord(h->ev_stop, st), "timing event");
+    return SSD_OK;
+}
+
 ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen, const void* x,
                                const void* z, const float* dt_raw, const float* dt_bias,
                                const float* A, const void* B, const void* C, const float* D,
@@ -739,6 +947,7 @@ ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
     const Shape s = make_shape(&h, batch, seqlen);
     FwdArgs a;
     memset(&a, 0, sizeof a);
+    default_strides(a, s);
     a.x = x; a.z = z; a.B = B; a.C = C; a.conv_w = conv_w; a.conv_b = conv_b;
     a.dt_raw = dt_raw; a.dt_bias = dt_bias; a.A = A; a.D = D; a.seq_idx = seq_idx;
     a.init_ssm = (const float*)init_state;

@@ -39,7 +39,21 @@ struct FwdArgs {
     void* final_conv;        // or null
     const float *bn_w, *cn_w, *bn_bias, *cn_bias;  // B/C norm parameters (nullable)
     const int32_t* lengths;  // (batch) real tokens per row of a ragged batch, or null
+    // Row strides in elements of the token-major inputs (a packed in_proj output
+    // holds x, z, B, C and dt_raw as column blocks of one row): x, z, B and C,
+    // and dt_raw; dt_act: dt_raw has the activation dtype instead of fp32.
+    int64_t ld_x, ld_z, ld_bc, ld_dt;
+    int dt_act;
 };
+
+// Contiguous inputs: every row stride is the tensor's width.
+inline void default_strides(FwdArgs& a, const Shape& s)
+{
+    a.ld_x = a.ld_z = (int64_t)s.nheads * s.headdim;
+    a.ld_bc = (int64_t)s.ngroups * s.dstate;
+    a.ld_dt = s.nheads;
+    a.dt_act = 0;
+}
 
 // K1: conv + SiLU of every x|B|C channel into u (batch, seqlen, conv_dim) fp32.
 cudaError_t launch_conv_silu_all(const Shape& s, const FwdArgs& a, float* u, cudaStream_t st);
@@ -100,6 +114,36 @@ struct S6Args {
     float* fin;                         // or null
 };
 cudaError_t launch_s6_scan(const S6Args& s, cudaStream_t st);
+// Backward of a zero-state prefill (chunk_bwd.cu).  Forward quantities recomputed
+// by the staged kernels (u, dt, acs, cdecay, hin), the workspace buffers and the
+// caller's gradient outputs (fp32; a NULL weight-gradient pointer skips it).
+struct BwdBufs {
+    const float* u;        // (B, L, conv_dim) conv output, or null when dconv = 1
+    const float *dt, *acs; // (B, H, L)
+    const float* cdecay;   // (B, H, nc)
+    const float* hin;      // (B, nc, H, P, N) states entering each chunk
+    float* gs;             // (B, nc, H, P, N) gradient of each chunk state
+    const void* gout;      // (B, L, H*P) act dtype
+    float* gu;             // (B, L, conv_dim) gradient of the conv output
+    float *gbh, *gch;      // (B, L, H, N) per-head gradients of B^, C^
+    float *p_dtb, *p_A, *p_D;   // (B, nc, H) partial sums
+    float* p_conv;         // (B, nseg, conv_dim, 5) partial sums
+    float *p_nw, *p_nb;    // (B, nc, G, 2, N), (B, nc, 2, H, N) partial sums
+    // outputs
+    float *gx, *gz, *gB, *gC, *gdt_raw, *gA;
+    float *g_dt_bias, *g_D, *gconv_w, *gconv_b, *g_bnw, *g_cnw, *g_bnb, *g_cnb;
+};
+bool bwd_supported(const Shape& s);
+size_t bwd_chunk_smem_bytes(const Shape& s);
+// Enqueue the backward kernels after the forward recompute; *launches counts them.
+cudaError_t launch_backward(const Shape& s, const FwdArgs& a, const BwdBufs& w, int* launches,
+                            cudaStream_t st);
+// Gated RMSNorm of the scan output, in place: each group of gs consecutive channels
+// of every real token is scaled by weight / sqrt(mean(out^2) + eps) (weight null:
+// ones).  gs must divide H*P, be a multiple of 8 and at most 16384.
+bool gated_norm_group_ok(int d_inner, int gs);
+cudaError_t launch_gated_norm(const Shape& s, void* out, const float* weight, int gs, float eps,
+                              const int32_t* lengths, cudaStream_t st);
 // K6: one decode token per row, state updated in place.
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
                                cudaStream_t st);

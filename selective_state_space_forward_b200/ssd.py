@@ -31,7 +31,9 @@ DTYPES = {"f32": (0, torch.float32), "bf16": (1, torch.bfloat16)}
 EXPORTS = ("ssd_create", "ssd_destroy", "ssd_get_path", "ssd_set_bc_norm", "ssd_state_bytes",
            "ssd_state_conv_offset", "ssd_forward", "ssd_step", "ssd_stage_conv", "ssd_stage_dt",
            "ssd_set_timing_events", "ssd_launch_count", "ssd_check", "ssd_last_error",
-           "ssd_status_string", "ssd_forward_noalloc", "ssd_forward_ragged", "ssd_s6_forward")
+           "ssd_status_string", "ssd_forward_noalloc", "ssd_forward_ragged", "ssd_s6_forward",
+           "ssd_backward_workspace_bytes", "ssd_backward", "ssd_set_gated_norm",
+           "ssd_forward_packed")
 
 
 class SSDError(RuntimeError):
@@ -44,6 +46,13 @@ class Desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "nheads", "headdim", "dstate", "ngroups", "dconv", "chunk", "act_dtype", "a_mode",
         "bc_norm", "max_batch", "max_seqlen", "path", "validate_finite")]
+
+
+class Grads(ctypes.Structure):
+    """ssd_grads: device pointers of the backward's fp32 gradient outputs."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "x", "z", "B", "C", "dt_raw", "dt_bias", "A", "D", "conv_w", "conv_b", "B_norm_w",
+        "C_norm_w", "B_bias", "C_bias")]
 
 
 _lib = None
@@ -84,9 +93,15 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_status_string.argtypes = [ctypes.c_int]
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), i32, i32] + [vp] * 15 + [vp]
+    lib.ssd_set_gated_norm.argtypes = [vp, i32, vp, i32, ctypes.c_float]
+    lib.ssd_forward_packed.argtypes = [vp, i32, i32, vp, ctypes.c_int64] + [vp] * 9 + [vp]
+    lib.ssd_backward_workspace_bytes.argtypes = [vp, i32, i32]
+    lib.ssd_backward_workspace_bytes.restype = sz
+    lib.ssd_backward.argtypes = [vp, i32, i32] + [vp] * 13 + [ctypes.POINTER(Grads), vp, sz, vp]
     for f in ("ssd_create", "ssd_set_bc_norm", "ssd_forward", "ssd_step", "ssd_stage_conv",
               "ssd_stage_dt", "ssd_set_timing_events", "ssd_check", "ssd_forward_noalloc",
-              "ssd_forward_ragged", "ssd_s6_forward"):
+              "ssd_forward_ragged", "ssd_s6_forward", "ssd_backward", "ssd_set_gated_norm",
+              "ssd_forward_packed"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -280,6 +295,48 @@ class Handle:
             _ptr(final_state, torch.uint8, "final_state"), _stream(stream)))
         return out
 
+    def packed_width(self) -> int:
+        """Columns of a packed in_proj row: z, x, B, C, dt_raw."""
+        return 2 * self.nheads * self.headdim + 2 * self.ngroups * self.dstate + self.nheads
+
+    def forward_packed(self, zxbcdt, dt_bias, A, D, conv_w=None, conv_b=None, seq_idx=None,
+                       init_state=None, out=None, final_state=None, stream=None):
+        """ssd_forward_packed: zxbcdt is a (batch, seqlen, ld) activation tensor whose rows
+        hold [z | x | B | C | dt_raw] from column 0 (a view of a wider buffer is fine as
+        long as its last dimension is contiguous); returns `out`."""
+        at, f = self.torch_dtype, torch.float32
+        if not isinstance(zxbcdt, torch.Tensor) or zxbcdt.dim() != 3:
+            raise ValueError("zxbcdt must be (batch, seqlen, ld)")
+        batch, seqlen, width = zxbcdt.shape
+        if width < self.packed_width():
+            raise ValueError(f"zxbcdt rows hold {width} columns; {self.packed_width()} needed")
+        if zxbcdt.dtype != at or (zxbcdt.numel() and not zxbcdt.is_cuda):
+            raise TypeError(f"zxbcdt must be a CUDA {at} tensor")
+        if zxbcdt.stride(2) != 1 or zxbcdt.stride(0) != seqlen * zxbcdt.stride(1):
+            raise TypeError("zxbcdt must have contiguous rows of equal stride")
+        ld = zxbcdt.stride(1)
+        if out is None:
+            out = torch.empty(batch, seqlen, self.nheads * self.headdim, dtype=at,
+                              device=zxbcdt.device)
+        HP = self.nheads * self.headdim
+        _need(out, batch * seqlen * HP, "out")
+        _need(dt_bias, self.nheads, "dt_bias")
+        _need(D, self.nheads, "D")
+        _need(A, batch * seqlen * self.nheads if self.a_per_token else self.nheads, "A")
+        if self.dconv == 4:
+            _need(conv_w, self.conv_dim * 4, "conv_w")
+            _need(conv_b, self.conv_dim, "conv_b")
+        _need(seq_idx, batch * seqlen, "seq_idx")
+        _need(init_state, self.state_bytes(batch), "init_state")
+        _need(final_state, self.state_bytes(batch), "final_state")
+        _raise(self.lib, self.lib.ssd_forward_packed(
+            self._h, batch, seqlen, zxbcdt.data_ptr() or None, ld, _ptr(dt_bias, f, "dt_bias"),
+            _ptr(A, f, "A"), _ptr(D, f, "D"), _ptr(conv_w, at, "conv_w"),
+            _ptr(conv_b, at, "conv_b"), _ptr(seq_idx, torch.int32, "seq_idx"),
+            _ptr(init_state, torch.uint8, "init_state"), _ptr(out, at, "out"),
+            _ptr(final_state, torch.uint8, "final_state"), _stream(stream)))
+        return out
+
     def step(self, x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None, state=None,
              out=None, stream=None):
         """ssd_step: one token per row, `state` updated in place; returns `out`."""
@@ -333,6 +390,58 @@ class Handle:
             _ptr(A, f, "A"), _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(dt, f, "dt"),
             _ptr(acs, f, "acs"), _stream(stream)))
         return dt, acs
+
+    def set_gated_norm(self, weight=None, group_size: int = 0, eps: float = 1e-5,
+                       enable: bool = True):
+        """ssd_set_gated_norm: later forwards and steps write norm(y * silu(z)) * weight."""
+        self._gn_keep = weight
+        _raise(self.lib, self.lib.ssd_set_gated_norm(
+            self._h, int(bool(enable)), _ptr(weight, torch.float32, "weight"), int(group_size),
+            float(eps)))
+
+    def backward_workspace_bytes(self, batch: int, seqlen: int) -> int:
+        return int(self.lib.ssd_backward_workspace_bytes(self._h, batch, seqlen))
+
+    def backward(self, x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None, gout=None,
+                 seq_idx=None, lengths=None, workspace=None, grads=None, stream=None):
+        """ssd_backward of a zero-state prefill: returns a dict of fp32 gradients named like
+        the inputs (x, z, B, C, dt_raw, dt_bias, A, D, and conv_w, conv_b with the conv,
+        B_norm_w, C_norm_w, B_bias, C_bias with the B/C norm).  `grads` may hold
+        preallocated outputs; `workspace` a uint8 CUDA tensor of at least
+        backward_workspace_bytes(batch, seqlen) bytes."""
+        at, f = self.torch_dtype, torch.float32
+        batch, seqlen = _rows(x, self.nheads * self.headdim, "x")
+        check_forward_sizes(self.dims, batch, seqlen, self.state_bytes(batch), x=x, z=z,
+                            dt_raw=dt_raw, dt_bias=dt_bias, A=A, B=B, C=C, D=D, conv_w=conv_w,
+                            conv_b=conv_b, seq_idx=seq_idx, out=gout, lengths=lengths)
+        H, N, dev = self.nheads, self.dstate, x.device
+        need = {"x": (batch, seqlen, H * self.headdim), "z": (batch, seqlen, H * self.headdim),
+                "B": (batch, seqlen, self.ngroups * N), "C": (batch, seqlen, self.ngroups * N),
+                "dt_raw": (batch, seqlen, H), "dt_bias": (H,), "D": (H,),
+                "A": (batch, seqlen, H) if self.a_per_token else (H,)}
+        if self.dconv == 4:
+            need.update(conv_w=(self.conv_dim, 4), conv_b=(self.conv_dim,))
+        if self.bc_norm:
+            need.update(B_norm_w=(N,), C_norm_w=(N,), B_bias=(H, N), C_bias=(H, N))
+        g = dict(grads or {})
+        for k, shape in need.items():
+            if g.get(k) is None:
+                g[k] = torch.empty(shape, dtype=f, device=dev)
+            else:
+                _need(g[k], int(torch.Size(shape).numel()), "grads." + k)
+        ws_bytes = self.backward_workspace_bytes(batch, seqlen)
+        if workspace is None:
+            workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        _need(workspace, ws_bytes, "workspace")
+        gr = Grads(**{k: _ptr(v, f, "grads." + k) for k, v in g.items()})
+        _raise(self.lib, self.lib.ssd_backward(
+            self._h, batch, seqlen, _ptr(lengths, torch.int32, "lengths"), _ptr(x, at, "x"),
+            _ptr(z, at, "z"), _ptr(dt_raw, f, "dt_raw"), _ptr(dt_bias, f, "dt_bias"),
+            _ptr(A, f, "A"), _ptr(B, at, "B"), _ptr(C, at, "C"), _ptr(D, f, "D"),
+            _ptr(conv_w, at, "conv_w"), _ptr(conv_b, at, "conv_b"),
+            _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(gout, at, "gout"), ctypes.byref(gr),
+            _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)))
+        return g
 
     def set_timing_events(self, start=None, stop=None):
         """Bracket the main kernel of later calls with these torch.cuda.Events."""

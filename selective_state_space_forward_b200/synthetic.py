@@ -168,6 +168,13 @@ def make_inputs(w: Workload, seed: int | None = None) -> dict:
     return out
 
 
+def make_output_grad(w: Workload, seed: int) -> np.ndarray:
+    """A seeded gradient of the loss with respect to `out` for the backward:
+    N(0, 1) of shape (batch, seqlen, H*P), rounded to the activation dtype."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return _act(w, rng.standard_normal((w.batch, w.seqlen, w.nheads * w.headdim)))
+
+
 def make_step_inputs(w: Workload, step: int, seed: int | None = None) -> dict:
     """Fresh draws for decode step `step` (same distributions, one token per row):
     x, z (batch, H*P); B, C (batch, G*N); dt_raw (batch, H); A (batch, H) when
