@@ -511,6 +511,8 @@ def bench_backward(args, torch, peaks, wname="mini_k3_mixer"):
     torch.cuda.synchronize()
     ms = _event_ms(torch, call, max(5, min(args.steps, 20)))
     k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k0.record()        # torch times only events it has recorded once itself
+    k1.record()
     h.set_timing_events(k0, k1)
     call()
     torch.cuda.synchronize()
@@ -574,60 +576,51 @@ def bench_packed_norm(args, torch, peaks, wname="mini_k3_mixer"):
 
 # Mamba-1 selective scan (S6) at the Falcon-Mamba-7B mixer shape.
 S6_SHAPE = dict(batch=2, seqlen=4096, d_inner=8192, dstate=16)
-# MUFU (transcendental) issue rate assumed for the roofline: 16 results per clock per SM.
-MUFU_PER_SM_CLK = 16
 
 
 def bench_s6(args, torch, peaks, sm_mhz):
-    """ssd_s6_forward over synthetic Falcon-Mamba-7B mixer inputs (bf16 u, z, B, C; fp32
-    dt, A_log, D, states), each call timed alone with CUDA events; the inputs (674 MB) are
-    larger than L2.  Rooflines: HBM bytes, and the MUFU pipe, which takes the dstate
-    exponentials of every (token, channel) plus the softplus and the gate's tanh."""
+    """ssd_s6_forward over the Falcon-Mamba-7B mixer shape (bf16 u, z, B, C; fp32
+    dt, A_log, D, states) drawn by the seeded generator the parity tests use,
+    each call timed alone with CUDA events; the inputs (674 MB) are larger than
+    L2.  Rooflines: HBM bytes, and the MUFU pipe at its rate measured on this
+    GPU by a one-kernel probe (ssd_ex2_throughput), which takes the dstate
+    exponentials of every (token, channel)."""
     from selective_state_space_forward_b200 import ssd
+    from selective_state_space_forward_b200.synthetic import make_s6_inputs
     Bb, L, DI, N = (S6_SHAPE[k] for k in ("batch", "seqlen", "d_inner", "dstate"))
-    g = torch.Generator(device="cuda").manual_seed(9)
-    bf = torch.bfloat16
-
-    def rnd(*shape, dtype=torch.float32):
-        return torch.randn(*shape, generator=g, device="cuda").to(dtype)
-
-    u, z = rnd(Bb, L, DI, dtype=bf), rnd(Bb, L, DI, dtype=bf)
-    delta = rnd(Bb, L, DI) - 2.0
-    Bm, Cm = rnd(Bb, L, N, dtype=bf), rnd(Bb, L, N, dtype=bf)
-    A_log = torch.log(torch.rand(DI, N, generator=g, device="cuda") * (N - 1) + 1.0)
-    dbias = torch.rand(DI, generator=g, device="cuda") * -2.0
-    D = torch.rand(DI, generator=g, device="cuda")
-    state = torch.zeros(Bb, DI, N, device="cuda")
-    out = torch.empty_like(u)
+    inp = make_s6_inputs(Bb, L, DI, N, seed=9)
+    dev = {k: (None if v is None else torch.from_numpy(v).to(
+        torch.bfloat16 if k in ("u", "z", "B", "C") else torch.float32).cuda())
+        for k, v in inp.items()}
+    state = dev["init"].clone()
+    out = torch.empty_like(dev["u"])
 
     def call():
-        ssd.s6_forward(u, delta, dbias, A_log, Bm, Cm, D, z=z, init_state=state, out=out,
+        ssd.s6_forward(dev["u"], dev["delta"], dev["delta_bias"], dev["A_log"], dev["B"],
+                       dev["C"], dev["D"], z=dev["z"], init_state=state, out=out,
                        final_state=state)
 
     for _ in range(3):
         call()
-    ts = []
-    for _ in range(max(5, min(args.steps, 20))):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        call()
-        e1.record()
-        torch.cuda.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    ms = sorted(ts)[len(ts) // 2]
+    torch.cuda.synchronize()
+    ms = _event_ms(torch, call, max(5, min(args.steps, 20)))
     tc = Bb * L * DI
     nbytes = tc * (2 + 4 + 2 + 2) + 2 * Bb * L * N * 2 + 2 * Bb * DI * N * 4
-    mufu = tc * (N + 3)
+    exps = tc * N                                   # the state decays
+    rate = ssd.ex2_throughput()                     # measured exp2 results/s
     mhz = sm_mhz or 1965
-    mufu_peak = 148 * MUFU_PER_SM_CLK * mhz * 1e6
     return {"workload": "falcon_mamba_7b_mixer: Mamba-1 selective scan, batch 2 x 4096 tokens, "
                         "d_inner 8192, d_state 16, bf16 u/z/B/C, fp32 dt/A/D/state",
             "ms_per_call": round(ms, 4), "tokens_per_s": Bb * L / (ms * 1e-3),
-            "roofline": {"bound": "alu", "unit": "Gop/s (MUFU)", "achieved": round(mufu / (ms * 1e-3) / 1e9, 1),
-                         "peak": round(mufu_peak / 1e9, 1), "frac": round(mufu / (ms * 1e-3) / mufu_peak, 4),
-                         "peak_source": f"148 SMs x {MUFU_PER_SM_CLK} MUFU results/clk x {mhz} MHz"},
+            "roofline": {"bound": "alu", "unit": "G exp2/s (MUFU)",
+                         "achieved": round(exps / (ms * 1e-3) / 1e9, 1),
+                         "peak": round(rate / 1e9, 1), "frac": round(exps / (ms * 1e-3) / rate, 4),
+                         "peak_source": "measured by ssd_ex2_throughput on this GPU "
+                                        f"({rate / 148 / (mhz * 1e6):.2f} results/clk/SM at "
+                                        f"{mhz} MHz)"},
             "hbm": {"algorithmic_bytes": nbytes, "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
                     "frac_of_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "inputs": "make_s6_inputs(seed 9), the parity tests' generator",
             "l2": "inputs larger than L2 (674 MB), no flush"}
 
 

@@ -232,6 +232,18 @@ ssd_status ssd_stage_dt(ssd_handle* h, int32_t batch, int32_t seqlen, const floa
  * hook off.  The events stay owned by the caller. */
 ssd_status ssd_set_timing_events(ssd_handle* h, void* start, void* stop);
 
+/* Testing hook for the failure path of the FUSED kernel, whose CTAs hand each
+ * segment's leaving state to the next segment through a flag in device memory
+ * and wait for it with a bounded spin.  wait_limit_ns sets the bound of every
+ * wait of that kernel (0: the default of 1 s; otherwise at least 100000 ns),
+ * and withhold_stream >= 0 makes the kernel never publish the first hand-off
+ * of that (row * H + head) stream, so the wait for it runs out: the kernel then
+ * raises the timeout bit of the device status word, lets its own copies and
+ * tensor-core work finish, and exits; ssd_check reports SSD_ERR_DEVICE and the
+ * outputs of that call are invalid.  -1 publishes every hand-off.  Nothing
+ * faults or hangs, and the next call on the handle is unaffected. */
+ssd_status ssd_set_wait_test(ssd_handle* h, uint64_t wait_limit_ns, int32_t withhold_stream);
+
 /* Number of kernels this handle has launched since ssd_create. */
 uint64_t ssd_launch_count(const ssd_handle* h);
 
@@ -372,6 +384,12 @@ ssd_status ssd_s6_forward(int32_t batch, int32_t seqlen, int32_t d_inner, int32_
                           const float* delta_bias, const float* A_log, const void* B,
                           const void* C, const float* D, const void* z, const float* init_state,
                           void* out, float* final_state, struct CUstream_st* stream);
+
+/* Measurement aid: the device's throughput of the hardware base-2 exponential
+ * (the MUFU pipe), in results per second, from one timed kernel of independent
+ * ex2 chains on `stream` (the call waits for it).  The Mamba-1 scan takes one
+ * exponential per state and token, so this rate is its compute roofline. */
+ssd_status ssd_ex2_throughput(double* results_per_second, struct CUstream_st* stream);
 
 /* The calling thread's last error message ("" when none). */
 const char* ssd_last_error(void);

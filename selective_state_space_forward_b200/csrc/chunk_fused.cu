@@ -82,6 +82,8 @@ struct FusedParams {
     float* hseg;              // (streams, nseg, 64, N) segment leaving states
     unsigned* flags;          // (streams, nseg)
     int* status;
+    uint64_t wait_ns;         // limit of every bounded wait
+    int withhold;             // testing: this stream's first hand-off is never published (-1: none)
     // B/C RMSNorm + per-head bias (NORM kernels only)
     const float* rinv;        // (B, L, 2G): 1/rms of B (g) and C (G + g) per token
     const float *bn_w, *cn_w; // (N) or null (ones)
@@ -319,7 +321,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         int q = 0;
         for (StepIter it(p, nc); it.valid(); it.next(), q++) {
             const int st = q % NST;
-            if (q >= NST && !tc::mbar_wait(&empty[st], par(q / NST - 1), s_abort, p.status, kStatusTimeout))
+            if (q >= NST && !tc::mbar_wait(&empty[st], par(q / NST - 1), s_abort, p.status, kStatusTimeout, p.wait_ns))
                 break;
             const int b = it.b, h = it.h, g = h / (H / p.ngroups);
             const int t0 = it.c * 64;
@@ -419,7 +421,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
         // an aborting CTA lets its last loads land before the shared memory is released
         for (int k2 = max(0, q - NST); k2 < q; k2++)
-            tc::mbar_drain(&full[k2 % NST], par(k2 / NST), p.status, kStatusTimeout);
+            tc::mbar_drain(&full[k2 % NST], par(k2 / NST), p.status, kStatusTimeout, p.wait_ns);
     } else if (warp < kGroupWarps) {
         // ------------------------------------------------------------ group A: conv, mask
         // Warps 0-7.  Per step: conv -> Xb, Xs; [thread 0: S = B^T Xs]; mask from
@@ -488,13 +490,13 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         };
         if (NORM) {
             StepIter it0(p, nc);
-            tc::mbar_wait(&full[0], 0, s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(&full[0], 0, s_abort, p.status, kStatusTimeout, p.wait_ns);
             normalise(0, it0.h);
             tc::fence_async_smem();
             bar_group(kBarA);
             if (issuer) tc::mbar_arrive(&norm_done[0]);
         }
-        if (issuer && tc::mbar_wait(&full[0], 0, s_abort, p.status, kStatusTimeout)) {
+        if (issuer && tc::mbar_wait(&full[0], 0, s_abort, p.status, kStatusTimeout, p.wait_ns)) {
             tc::tc_fence_after();
             issue_cb(0);
         }
@@ -519,10 +521,10 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
             // On abort the waits return at once; every thread still runs the same
             // sequence of group barriers and leaves at the end of the iteration.
-            tc::mbar_wait(&full[st], par(q / NST), s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(&full[st], par(q / NST), s_abort, p.status, kStatusTimeout, p.wait_ns);
             // the operand buffers [i] and Ydiag columns [i] are free once group B
             // has finished step q-2
-            if (q >= 2) tc::mbar_wait(&epi_done[i], par((q >> 1) - 1), s_abort, p.status, kStatusTimeout);
+            if (q >= 2) tc::mbar_wait(&epi_done[i], par((q >> 1) - 1), s_abort, p.status, kStatusTimeout, p.wait_ns);
             const uint8_t* stg = sm + st * LY::kStage;
             const ChunkScalars* cs = &scal[st];
             const uint32_t m0 = cs->m0, m1 = cs->m1, pre = cs->pre;
@@ -625,7 +627,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             // S_c^T[n][p] = B^T Xs into S[i] (A = the B tile as MN-major over n, K = s);
             // S[i] last held S(q-2), which group B has read once it arrived on s_free[i]
             if (issuer && (q < 2 || tc::mbar_wait(&s_free[i], par((q >> 1) - 1), s_abort, p.status,
-                                                   kStatusTimeout))) {
+                                                   kStatusTimeout, p.wait_ns))) {
                 tc::tc_fence_after();
                 const uint32_t a_b = tc::smem_u32(stg + 2 * kTile);
                 const uint32_t a_xs = tc::smem_u32(xs);
@@ -637,7 +639,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
 
             // ---- mask: M[t][s] from the C B^T accumulator
-            tc::mbar_wait(cb_done, par(q), s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(cb_done, par(q), s_abort, p.status, kStatusTimeout, p.wait_ns);
             tc::tc_fence_after();
             {
                 const int t = r16;
@@ -705,7 +707,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if (NORM && it.valid()) {
                 // the next step's B and C tiles, before its C B^T and Yoff read them
                 const int q1 = q + 1;
-                tc::mbar_wait(&full[q1 % NST], par(q1 / NST), s_abort, p.status, kStatusTimeout);
+                tc::mbar_wait(&full[q1 % NST], par(q1 / NST), s_abort, p.status, kStatusTimeout, p.wait_ns);
                 normalise(q1 % NST, it.h);
             }
             tc::fence_async_smem();
@@ -727,7 +729,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 if (it.valid()) {
                     const int q1 = q + 1;
                     if (NORM) tc::mbar_arrive(&norm_done[q1 % NST]);
-                    if (tc::mbar_wait(&full[q1 % NST], par(q1 / NST), s_abort, p.status, kStatusTimeout)) {
+                    if (tc::mbar_wait(&full[q1 % NST], par(q1 / NST), s_abort, p.status, kStatusTimeout, p.wait_ns)) {
                         tc::tc_fence_after();
                         issue_cb(q1 % NST);
                     }
@@ -737,7 +739,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
         if (issuer) {
             tc::mma_commit(drain_a);
-            tc::mbar_drain(drain_a, 0, p.status, kStatusTimeout);
+            tc::mbar_drain(drain_a, 0, p.status, kStatusTimeout, p.wait_ns);
         }
     } else if (warp < 2 * kGroupWarps) {
         // ------------------------------------------------------------ group B: state, epilogue
@@ -781,7 +783,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 cur_h = h;
                 Dh = p.D[h];
             }
-            tc::mbar_wait(&full[st], par(q / NST), s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(&full[st], par(q / NST), s_abort, p.status, kStatusTimeout, p.wait_ns);
             const uint8_t* stg = sm + st * LY::kStage;
             const ChunkScalars* cs = &scal[st];
             const float carry = cs->carry;
@@ -800,7 +802,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                         for (;;) {
                             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(fl) : "memory");
                             if (v == p.epoch || *s_abort) break;
-                            if (tc::global_ns() - tw > tc::kWaitLimitNs) {
+                            if (tc::global_ns() - tw > p.wait_ns) {
                                 *s_abort = 1;
                                 atomicOr(p.status, kStatusTimeout);
                                 break;
@@ -815,7 +817,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 for (int jj = 0; jj < HR; jj++) hs[jj] = src ? __ldcg(src + (int64_t)(pcol + jj) * NS + nrow) : 0.f;
             } else {
                 // h_c = k_{c-1} h_{c-1} + S_{c-1}
-                tc::mbar_wait(&s_done[i ^ 1], par((q - 1) >> 1), s_abort, p.status, kStatusTimeout);
+                tc::mbar_wait(&s_done[i ^ 1], par((q - 1) >> 1), s_abort, p.status, kStatusTimeout, p.wait_ns);
                 tc::tc_fence_after();
                 uint32_t r[HR];
                 load_S(i ^ 1, r);
@@ -844,7 +846,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 // S[i^1] may be overwritten by S(q+1) now
                 if (q >= 1) tc::mbar_arrive(&s_free[i ^ 1]);
                 // NORM: group A has normalised this step's C tile
-                if (NORM) tc::mbar_wait(&norm_done[st], par(q / NST), s_abort, p.status, kStatusTimeout);
+                if (NORM) tc::mbar_wait(&norm_done[st], par(q / NST), s_abort, p.status, kStatusTimeout, p.wait_ns);
                 // Yoff = C h^T (K = n; h^T is MN-major: rows n, 64 p per row)
                 const uint32_t a_c = tc::smem_u32(stg + 2 * kTile + LY::kBC);
 #pragma unroll
@@ -857,8 +859,8 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
 
             // ---- epilogue: out = (Ydiag + f Yoff + D u) SiLU(z)
-            tc::mbar_wait(&y_done[i], par(q >> 1), s_abort, p.status, kStatusTimeout);
-            tc::mbar_wait(yo_done, par(q), s_abort, p.status, kStatusTimeout);
+            tc::mbar_wait(&y_done[i], par(q >> 1), s_abort, p.status, kStatusTimeout, p.wait_ns);
+            tc::mbar_wait(yo_done, par(q), s_abort, p.status, kStatusTimeout, p.wait_ns);
             tc::tc_fence_after();
             uint8_t* outt = sm + LY::kOut + i * kTile;
             {
@@ -893,7 +895,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             }
             // ---- leaving the segment: h_out = k_c h_c + S_c -> the next segment or the caller
             if (last) {
-                tc::mbar_wait(&s_done[i], par(q >> 1), s_abort, p.status, kStatusTimeout);
+                tc::mbar_wait(&s_done[i], par(q >> 1), s_abort, p.status, kStatusTimeout, p.wait_ns);
                 tc::tc_fence_after();
                 uint32_t r[HR];
                 load_S(i, r);
@@ -908,7 +910,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 }
                 if (!stream_end) {
                     bar_group(kBarB);
-                    if (issuer) {
+                    if (issuer && !(str == p.withhold && seg_k == 0)) {
                         __threadfence();
                         asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.flags + str * p.nseg + seg_k),
                                      "r"(p.epoch) : "memory");
@@ -930,7 +932,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
         if (issuer) {
             tc::mma_commit(drain_b);
-            tc::mbar_drain(drain_b, 0, p.status, kStatusTimeout);
+            tc::mbar_drain(drain_b, 0, p.status, kStatusTimeout, p.wait_ns);
             tc::bulk_wait0();
         }
     }
@@ -1094,6 +1096,8 @@ cudaError_t launch_chunk_fused(const Shape& s, const FwdArgs& a, const void* ubc
     fp.hseg = fw.hseg;
     fp.flags = fw.flags;
     fp.status = status;
+    fp.wait_ns = fw.wait_ns ? fw.wait_ns : tc::kWaitLimitNs;
+    fp.withhold = fw.withhold;
     fp.rinv = rinv;
     fp.bn_w = a.bn_w;
     fp.cn_w = a.cn_w;

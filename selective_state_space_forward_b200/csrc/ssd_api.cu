@@ -461,6 +461,8 @@ ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
     h->device = dev;
     h->fw.sm_count = sms;
     h->fw.epoch = 0;
+    h->fw.wait_ns = 0;
+    h->fw.withhold = -1;
     cudaError_t e = cudaMalloc(&h->ws, off);
     if (e != cudaSuccess) {
         delete h;
@@ -707,6 +709,20 @@ ssd_status ssd_set_timing_events(ssd_handle* h, void* start, void* stop)
 
 uint64_t ssd_launch_count(const ssd_handle* h) { return h ? h->launches : 0; }
 
+ssd_status ssd_set_wait_test(ssd_handle* h, uint64_t wait_limit_ns, int32_t withhold_stream)
+{
+    g_err.clear();
+    if (!h) return fail(SSD_ERR_INVALID_ARG, "handle is NULL");
+    if (withhold_stream < -1)
+        return fail(SSD_ERR_INVALID_ARG, "withhold_stream must be -1 or a stream index (got %d)",
+                    withhold_stream);
+    if (wait_limit_ns != 0 && wait_limit_ns < 100000)
+        return fail(SSD_ERR_INVALID_ARG, "wait_limit_ns must be 0 (the default) or at least 100000");
+    h->fw.wait_ns = wait_limit_ns;
+    h->fw.withhold = withhold_stream;
+    return SSD_OK;
+}
+
 ssd_status ssd_check(ssd_handle* h, struct CUstream_st* stream)
 {
     g_err.clear();
@@ -937,6 +953,8 @@ ssd_status ssd_forward_noalloc(const ssd_desc* d, int32_t batch, int32_t seqlen,
     fw.epoch = dev.epoch;
     fw.sm_count = dev.sm_count;
     fw.max_items = items;
+    fw.wait_ns = 0;
+    fw.withhold = -1;
     size_t off = kNoAllocFlagBytes + items * slot;   // slot is a multiple of 256 bytes
     float* dt = (float*)(p + off);
     off += dt_bytes;

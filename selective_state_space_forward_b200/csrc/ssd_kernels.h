@@ -87,6 +87,8 @@ struct FusedWork {
     unsigned epoch;     // distinct per call (never 0)
     int sm_count;
     size_t max_items;   // hand-off slots in hseg/flags; 0: fused_flag_count(streams, sm_count)
+    uint64_t wait_ns;   // limit of the kernel's bounded waits; 0: the default (1 s)
+    int withhold;       // testing: stream whose first hand-off is never published; -1: none
 };
 bool fused_path_available();
 size_t fused_handoff_floats(int max_streams, int dstate, int sm_count);

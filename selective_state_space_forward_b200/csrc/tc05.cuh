@@ -78,10 +78,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 }
 
 // Wait until the barrier completes the phase with this parity.  Gives up when
-// *abort is set by another thread or after kWaitLimitNs, then sets *abort and
-// the status bit; returns false in both cases.
+// *abort is set by another thread or after limit_ns, then sets *abort and the
+// status bit; returns false in both cases.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* status, int status_bit)
+                                          int* status, int status_bit,
+                                          uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
@@ -89,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 7) == 0) {
             if (*abort) return false;
-            if (global_ns() - t0 > kWaitLimitNs) {
+            if (global_ns() - t0 > limit_ns) {
                 *abort = 1;
                 atomicOr(status, status_bit);
                 return false;
@@ -100,13 +101,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Teardown wait: like mbar_wait but it does not stop at the abort flag, so an
 // aborting CTA still lets its own copies and MMAs land before it exits.
-__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* status, int status_bit)
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int* status, int status_bit,
+                                           uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; i++) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 7) == 0 && global_ns() - t0 > kWaitLimitNs) {
+        if ((i & 7) == 0 && global_ns() - t0 > limit_ns) {
             atomicOr(status, status_bit);
             return false;
         }

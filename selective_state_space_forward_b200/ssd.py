@@ -33,7 +33,7 @@ EXPORTS = ("ssd_create", "ssd_destroy", "ssd_get_path", "ssd_set_bc_norm", "ssd_
            "ssd_set_timing_events", "ssd_launch_count", "ssd_check", "ssd_last_error",
            "ssd_status_string", "ssd_forward_noalloc", "ssd_forward_ragged", "ssd_s6_forward",
            "ssd_backward_workspace_bytes", "ssd_backward", "ssd_set_gated_norm",
-           "ssd_forward_packed")
+           "ssd_forward_packed", "ssd_ex2_throughput", "ssd_set_wait_test")
 
 
 class SSDError(RuntimeError):
@@ -94,6 +94,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), i32, i32] + [vp] * 15 + [vp]
     lib.ssd_set_gated_norm.argtypes = [vp, i32, vp, i32, ctypes.c_float]
+    lib.ssd_ex2_throughput.argtypes = [ctypes.POINTER(ctypes.c_double), vp]
+    lib.ssd_set_wait_test.argtypes = [vp, ctypes.c_uint64, i32]
     lib.ssd_forward_packed.argtypes = [vp, i32, i32, vp, ctypes.c_int64] + [vp] * 9 + [vp]
     lib.ssd_backward_workspace_bytes.argtypes = [vp, i32, i32]
     lib.ssd_backward_workspace_bytes.restype = sz
@@ -101,7 +103,7 @@ def load_library(path: str = LIB_PATH):
     for f in ("ssd_create", "ssd_set_bc_norm", "ssd_forward", "ssd_step", "ssd_stage_conv",
               "ssd_stage_dt", "ssd_set_timing_events", "ssd_check", "ssd_forward_noalloc",
               "ssd_forward_ragged", "ssd_s6_forward", "ssd_backward", "ssd_set_gated_norm",
-              "ssd_forward_packed"):
+              "ssd_forward_packed", "ssd_ex2_throughput", "ssd_set_wait_test"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -449,6 +451,11 @@ class Handle:
             self._h, start.cuda_event if start is not None else None,
             stop.cuda_event if stop is not None else None))
 
+    def set_wait_test(self, wait_limit_ns: int = 0, withhold_stream: int = -1):
+        """ssd_set_wait_test: bound the fused kernel's waits and withhold one hand-off."""
+        _raise(self.lib, self.lib.ssd_set_wait_test(self._h, int(wait_limit_ns),
+                                                    int(withhold_stream)))
+
     def launch_count(self) -> int:
         return int(self.lib.ssd_launch_count(self._h))
 
@@ -492,6 +499,14 @@ def forward_noalloc(x, z, dt_raw, dt_bias, A, B, C, D, conv_w=None, conv_b=None,
         _ptr(final_state, torch.uint8, "final_state"), _ptr(status, torch.int32, "status"),
         _stream(stream)))
     return out
+
+
+def ex2_throughput(stream=None, lib=None) -> float:
+    """ssd_ex2_throughput: measured hardware exp2 results per second on this device."""
+    lib = lib or load_library()
+    v = ctypes.c_double(0.0)
+    _raise(lib, lib.ssd_ex2_throughput(ctypes.byref(v), _stream(stream)))
+    return v.value
 
 
 def s6_forward(u, delta, delta_bias, A_log, B, C, D, z=None, init_state=None, out=None,

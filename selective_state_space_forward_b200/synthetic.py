@@ -175,6 +175,26 @@ def make_output_grad(w: Workload, seed: int) -> np.ndarray:
     return _act(w, rng.standard_normal((w.batch, w.seqlen, w.nheads * w.headdim)))
 
 
+def make_s6_inputs(batch: int, seqlen: int, d_inner: int, dstate: int, seed: int,
+                   bf16: bool = True, gate: bool = True, init: bool = True) -> dict:
+    """Seeded inputs of the Mamba-1 selective scan (S6): u, z, B, C ~ N(0, 1) in the
+    activation dtype; delta ~ N(-2, 1); A_log = log U[1, dstate] per (channel,
+    state); delta_bias ~ U[-2, 0]; D ~ U[0, 1]; initial state ~ N(0, 0.1).  z and
+    the initial state are None when not asked for."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    act = round_bf16 if bf16 else (lambda a: np.asarray(a, dtype=np.float32))
+    f = np.float32
+    B, L, DI, N = batch, seqlen, d_inner, dstate
+    return dict(u=act(rng.standard_normal((B, L, DI))),
+                delta=(rng.standard_normal((B, L, DI)) - 2.0).astype(f),
+                z=act(rng.standard_normal((B, L, DI))) if gate else None,
+                B=act(rng.standard_normal((B, L, N))), C=act(rng.standard_normal((B, L, N))),
+                A_log=np.log(rng.uniform(1.0, N, (DI, N))).astype(f),
+                delta_bias=rng.uniform(-2.0, 0.0, DI).astype(f),
+                D=rng.uniform(0.0, 1.0, DI).astype(f),
+                init=(0.1 * rng.standard_normal((B, DI, N))).astype(f) if init else None)
+
+
 def make_step_inputs(w: Workload, step: int, seed: int | None = None) -> dict:
     """Fresh draws for decode step `step` (same distributions, one token per row):
     x, z (batch, H*P); B, C (batch, G*N); dt_raw (batch, H); A (batch, H) when

@@ -10,23 +10,13 @@ import torch
 import oracle
 from gpu_util import assert_close
 from selective_state_space_forward_b200 import ssd
-from selective_state_space_forward_b200.synthetic import round_bf16
+from selective_state_space_forward_b200.synthetic import make_s6_inputs
 
 pytestmark = pytest.mark.gpu
 
 
 def _inputs(B, L, DI, N, seed, bf16=True, gate=True, init=True):
-    rng = np.random.Generator(np.random.PCG64(seed))
-    act = (lambda a: round_bf16(a)) if bf16 else (lambda a: a.astype(np.float32))
-    f = np.float32
-    return dict(u=act(rng.standard_normal((B, L, DI))),
-                delta=(rng.standard_normal((B, L, DI)) - 2.0).astype(f),
-                z=act(rng.standard_normal((B, L, DI))) if gate else None,
-                B=act(rng.standard_normal((B, L, N))), C=act(rng.standard_normal((B, L, N))),
-                A_log=np.log(rng.uniform(1.0, N, (DI, N))).astype(f),
-                delta_bias=rng.uniform(-2.0, 0.0, DI).astype(f),
-                D=rng.uniform(0.0, 1.0, DI).astype(f),
-                init=(0.1 * rng.standard_normal((B, DI, N))).astype(f) if init else None)
+    return make_s6_inputs(B, L, DI, N, seed, bf16=bf16, gate=gate, init=init)
 
 
 def _gpu(inp, bf16=True):
