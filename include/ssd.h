@@ -124,8 +124,8 @@ ssd_status ssd_set_bc_norm(ssd_handle* h, const float* B_norm_w, const float* C_
  * rewrites out in place as out * weight / sqrt(mean(out^2) + eps), the mean
  * taken over each group of group_size consecutive channels of a token
  * (group_size 0 = H*P, one norm per token; otherwise it must divide H*P, be a
- * multiple of 8 and be at most 16384).  weight: (H*P) fp32 device pointer that
- * stays valid while calls run, or NULL (ones).  eps in [0, 1]; the Mamba3Block
+ * multiple of 8 and be at most 16384).  weight: (H*P) fp32 device pointer,
+ * 16-byte aligned, that stays valid while calls run, or NULL (ones).  eps in [0, 1]; the Mamba3Block
  * norms use 1e-5.  Padding tokens of a ragged batch stay +0.0.  enable = 0
  * turns the norm off (the other arguments are then ignored).  The norm adds one
  * read and one write of out; validate_finite checks the normed out. */

@@ -317,44 +317,60 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
+        // Software-pipelined by one step: the global loads of step q+1's per-token
+        // values are issued, then step q's scalars are computed from the values
+        // loaded one iteration earlier, and only then does the warp wait for step
+        // q's ring slot.  A freed slot is refilled by the TMA issue and a few
+        // shared-memory stores.
         const uint32_t tx = (uint32_t)(2 * kTile + 2 * LY::kBC);
-        int q = 0;
-        for (StepIter it(p, nc); it.valid(); it.next(), q++) {
-            const int st = q % NST;
-            if (q >= NST && !tc::mbar_wait(&empty[st], par(q / NST - 1), s_abort, p.status, kStatusTimeout, p.wait_ns))
-                break;
-            const int b = it.b, h = it.h, g = h / (H / p.ngroups);
-            const int t0 = it.c * 64;
+        struct Raw {
+            float dt[2], ac[2], rb[2], rc[2];
+            int32_t sq[2], sqm[2];    // seq_idx at t and t-1
+            int32_t ps, psm;          // lanes 0, 1: seq_idx at t0-2+lane and one before
+            int32_t len;              // lengths[b] (ragged batch)
+        };
+        auto load_raw = [&](const StepIter& s, Raw& r) {
+            const int b = s.b, h = s.h, g = h / (H / p.ngroups);
+            const int t0 = s.c * 64;
             const int64_t bh = (int64_t)b * H + h;
-            uint8_t* stg = sm + st * LY::kStage;
-            if (lane == 0) {
-                tc::mbar_arrive_expect_tx(&full[st], tx);
-                tc::tma_load_3d(stg, &tm_x, &full[st], h * 64, t0, b);
-                tc::tma_load_3d(stg + kTile, &tm_z, &full[st], h * 64, t0, b);
-#pragma unroll
-                for (int jj = 0; jj < NS / 64; jj++) {
-                    const int bx = g * NS + 64 * jj;
-                    const int cx = (CONV ? p.ngroups * NS : 0) + g * NS + 64 * jj;
-                    tc::tma_load_3d(stg + 2 * kTile + jj * kTile, &tm_b, &full[st], bx, t0, b);
-                    tc::tma_load_3d(stg + 2 * kTile + LY::kBC + jj * kTile, &tm_c, &full[st], cx, t0, b);
-                }
-            }
             const int32_t* seq_row = p.seq ? p.seq + (int64_t)b * L : nullptr;
-            // ragged batch: padding after the row's real tokens has dt = 0 (K2) and no boundary
-            const int Lb = RAG ? row_length(p.lengths, b, L) : L;
             const float* dt_row = p.dt + bh * L;
             const float* acs_row = p.acs + bh * L;
-            ChunkScalars* cs = &scal[st];
-            const int Lc = min(64, L - t0);
-            float dtv[2], acv[2];
-            int bdv[2];
+            r.len = RAG ? p.lengths[b] : L;
 #pragma unroll
             for (int hf = 0; hf < 2; hf++) {
                 const int t = t0 + hf * 32 + lane;
                 const bool ok = t < L;
-                dtv[hf] = ok ? dt_row[t] : 0.0f;
-                acv[hf] = ok ? acs_row[t] : 0.0f;
-                bdv[hf] = t < Lb ? is_boundary(seq_row, t) : 0;
+                r.dt[hf] = ok ? dt_row[t] : 0.0f;
+                r.ac[hf] = ok ? acs_row[t] : 0.0f;
+                r.sq[hf] = (seq_row && ok) ? seq_row[t] : 0;
+                r.sqm[hf] = (seq_row && ok && t > 0) ? seq_row[t - 1] : 0;
+                if (NORM) {
+                    const int64_t tok = ((int64_t)b * L + t) * (2 * p.ngroups);
+                    r.rb[hf] = ok ? p.rinv[tok + g] : 0.0f;
+                    r.rc[hf] = ok ? p.rinv[tok + p.ngroups + g] : 0.0f;
+                }
+            }
+            const int tt = t0 - 2 + lane;
+            const bool okp = seq_row && lane < 2 && tt >= 1 && tt < L;
+            r.ps = okp ? seq_row[tt] : 0;
+            r.psm = okp ? seq_row[tt - 1] : 0;
+        };
+        // the scalars of one step, as each lane stores them
+        struct Vals {
+            float dt[2], wd[2], f[2], a2[2], g[2], rb[2], rc[2], a2ref[2], carry;
+            int seg[2];
+            uint32_t m0, m1, pre, fast, nvalid;
+        };
+        auto compute = [&](const StepIter& s, const Raw& r, Vals& v) {
+            const int t0 = s.c * 64;
+            const int Lb = RAG ? min(max((int)r.len, 0), L) : L;
+            const int Lc = min(64, L - t0);
+            int bdv[2];
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+                const int t = t0 + hf * 32 + lane;
+                bdv[hf] = (p.seq && t > 0 && t < Lb) ? (r.sq[hf] != r.sqm[hf]) : 0;
             }
             const uint32_t m0 = __ballot_sync(0xffffffffu, bdv[0]);
             const uint32_t m1 = __ballot_sync(0xffffffffu, bdv[1]);
@@ -362,62 +378,108 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             const int seg1 = __popc(m0) + __popc(m1 & mask_le(lane));
             const int last = Lc - 1;
             const int seg_last = __shfl_sync(0xffffffffu, last < 32 ? seg0 : seg1, last & 31);
-            const float acs_last = __shfl_sync(0xffffffffu, last < 32 ? acv[0] : acv[1], last & 31);
+            const float acs_last = __shfl_sync(0xffffffffu, last < 32 ? r.ac[0] : r.ac[1], last & 31);
             const int segv[2] = {seg0, seg1};
-            // the 16-token block of token r ends at min(r | 15, Lc - 1)
-            float a2ref[2];
 #pragma unroll
             for (int hf = 0; hf < 2; hf++) {
                 const int rref = min((hf * 32 + lane) | 15, last);
-                const float v0 = __shfl_sync(0xffffffffu, acv[0], rref & 31);
-                const float v1 = __shfl_sync(0xffffffffu, acv[1], rref & 31);
-                a2ref[hf] = (rref < 32 ? v0 : v1) * kLog2e;
+                const float v0 = __shfl_sync(0xffffffffu, r.ac[0], rref & 31);
+                const float v1 = __shfl_sync(0xffffffffu, r.ac[1], rref & 31);
+                v.a2ref[hf] = (rref < 32 ? v0 : v1) * kLog2e;
             }
 #pragma unroll
             for (int hf = 0; hf < 2; hf++) {
-                const int r = hf * 32 + lane;
-                const bool ok = r < Lc;
-                const float a2 = acv[hf] * kLog2e;
-                cs->dt[r] = dtv[hf];
-                cs->wd[r] = (ok && segv[hf] == seg_last) ? __expf(acs_last - acv[hf]) * dtv[hf] : 0.0f;
-                cs->f[r] = (ok && segv[hf] == 0) ? __expf(acv[hf]) : 0.0f;
-                cs->a2[r] = a2;
-                cs->g[r] = ok ? dtv[hf] * ex2(fminf(a2ref[hf] - a2, 0.0f)) : 0.0f;
-                cs->seg[r] = (uint8_t)segv[hf];
-                if (NORM) {
-                    const int64_t tok = ((int64_t)b * L + (t0 + r)) * (2 * p.ngroups);
-                    cs->rb[r] = ok ? p.rinv[tok + g] : 0.0f;
-                    cs->rc[r] = ok ? p.rinv[tok + p.ngroups + g] : 0.0f;
-                }
+                const int rr = hf * 32 + lane;
+                const bool ok = rr < Lc;
+                const float a2 = r.ac[hf] * kLog2e;
+                v.dt[hf] = r.dt[hf];
+                v.wd[hf] = (ok && segv[hf] == seg_last) ? __expf(acs_last - r.ac[hf]) * r.dt[hf] : 0.0f;
+                v.f[hf] = (ok && segv[hf] == 0) ? __expf(r.ac[hf]) : 0.0f;
+                v.a2[hf] = a2;
+                v.g[hf] = ok ? r.dt[hf] * ex2(fminf(v.a2ref[hf] - a2, 0.0f)) : 0.0f;
+                v.seg[hf] = segv[hf];
+                v.rb[hf] = ok ? r.rb[hf] : 0.0f;
+                v.rc[hf] = ok ? r.rc[hf] : 0.0f;
             }
             // block b may use the factored mask when the chunk holds no boundary and the
             // decay across the block stays within kMaskBlockRange
-            const float a2first0 = __shfl_sync(0xffffffffu, acv[0], lane & 16) * kLog2e;
-            const float a2first1 = __shfl_sync(0xffffffffu, acv[1], lane & 16) * kLog2e;
-            const bool blk_ok0 = a2first0 - a2ref[0] <= kMaskBlockRange;
-            const bool blk_ok1 = a2first1 - a2ref[1] <= kMaskBlockRange;
-            const uint32_t okb0 = __ballot_sync(0xffffffffu, blk_ok0);
-            const uint32_t okb1 = __ballot_sync(0xffffffffu, blk_ok1);
+            const float a2first0 = __shfl_sync(0xffffffffu, r.ac[0], lane & 16) * kLog2e;
+            const float a2first1 = __shfl_sync(0xffffffffu, r.ac[1], lane & 16) * kLog2e;
+            const uint32_t okb0 = __ballot_sync(0xffffffffu, a2first0 - v.a2ref[0] <= kMaskBlockRange);
+            const uint32_t okb1 = __ballot_sync(0xffffffffu, a2first1 - v.a2ref[1] <= kMaskBlockRange);
+            const int tt = t0 - 2 + lane;
+            const int pb = (lane < 2 && p.seq && tt >= 1 && tt < Lb) ? (r.ps != r.psm) : 0;
+            v.pre = __ballot_sync(0xffffffffu, pb) & 3u;        // bit 0: t0-2, bit 1: t0-1
+            v.nvalid = (uint32_t)min(max(Lb - t0, 0), 64);
+            v.carry = (m0 | m1) ? kChunkReset : __expf(acs_last);
+            v.m0 = m0;
+            v.m1 = m1;
+            // lanes 0 and 16 hold blocks 0, 1 (first half) and 2, 3 (second half)
+            const uint32_t fb = ((okb0 & 1u) ? 1u : 0u) | ((okb0 >> 16) & 1u) << 1 |
+                                ((okb1 & 1u) ? 1u : 0u) << 2 | ((okb1 >> 16) & 1u) << 3;
+            v.fast = (m0 | m1) ? 0u : fb;
+        };
+        auto store = [&](ChunkScalars* cs, const Vals& v) {
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+                const int rr = hf * 32 + lane;
+                cs->dt[rr] = v.dt[hf];
+                cs->wd[rr] = v.wd[hf];
+                cs->f[rr] = v.f[hf];
+                cs->a2[rr] = v.a2[hf];
+                cs->g[rr] = v.g[hf];
+                cs->seg[rr] = (uint8_t)v.seg[hf];
+                if (NORM) {
+                    cs->rb[rr] = v.rb[hf];
+                    cs->rc[rr] = v.rc[hf];
+                }
+            }
             if (lane == 0) {
-                uint32_t pre = 0;
-                if (t0 - 2 >= 1 && t0 - 2 < Lb && is_boundary(seq_row, t0 - 2)) pre |= 1u;
-                if (t0 - 1 >= 1 && t0 - 1 < Lb && is_boundary(seq_row, t0 - 1)) pre |= 2u;
-                if (RAG) cs->nvalid = (uint32_t)min(max(Lb - t0, 0), 64);
-                cs->carry = (m0 | m1) ? kChunkReset : __expf(acs_last);
-                cs->m0 = m0;
-                cs->m1 = m1;
-                cs->pre = pre;
-                // lanes 0 and 16 hold blocks 0, 1 (first half) and 2, 3 (second half)
-                const uint32_t fb = ((okb0 & 1u) ? 1u : 0u) | ((okb0 >> 16) & 1u) << 1 |
-                                    ((okb1 & 1u) ? 1u : 0u) << 2 | ((okb1 >> 16) & 1u) << 3;
-                cs->fast = (m0 | m1) ? 0u : fb;
+                if (RAG) cs->nvalid = v.nvalid;
+                cs->carry = v.carry;
+                cs->m0 = v.m0;
+                cs->m1 = v.m1;
+                cs->pre = v.pre;
+                cs->fast = v.fast;
             }
             if (lane == 0 || lane == 16) {
-                cs->a2ref[lane >> 4] = a2ref[0];
-                cs->a2ref[2 + (lane >> 4)] = a2ref[1];
+                cs->a2ref[lane >> 4] = v.a2ref[0];
+                cs->a2ref[2 + (lane >> 4)] = v.a2ref[1];
             }
+        };
+        int q = 0;
+        StepIter it(p, nc);
+        Raw cur, nxt;
+        if (it.valid()) load_raw(it, cur);
+        for (; it.valid(); q++) {
+            const int st = q % NST;
+            StepIter nx = it;
+            nx.next();
+            if (nx.valid()) load_raw(nx, nxt);          // in flight while this step is finished
+            Vals v;
+            compute(it, cur, v);
+            if (q >= NST && !tc::mbar_wait(&empty[st], par(q / NST - 1), s_abort, p.status, kStatusTimeout, p.wait_ns))
+                break;
+            const int g = it.h / (H / p.ngroups);
+            const int t0 = it.c * 64;
+            uint8_t* stg = sm + st * LY::kStage;
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(&full[st], tx);
+                tc::tma_load_3d(stg, &tm_x, &full[st], it.h * 64, t0, it.b);
+                tc::tma_load_3d(stg + kTile, &tm_z, &full[st], it.h * 64, t0, it.b);
+#pragma unroll
+                for (int jj = 0; jj < NS / 64; jj++) {
+                    const int bx = g * NS + 64 * jj;
+                    const int cx = (CONV ? p.ngroups * NS : 0) + g * NS + 64 * jj;
+                    tc::tma_load_3d(stg + 2 * kTile + jj * kTile, &tm_b, &full[st], bx, t0, it.b);
+                    tc::tma_load_3d(stg + 2 * kTile + LY::kBC + jj * kTile, &tm_c, &full[st], cx, t0, it.b);
+                }
+            }
+            store(&scal[st], v);
             __syncwarp();
             tc::mbar_arrive(&full[st]);
+            it = nx;
+            cur = nxt;
         }
         // an aborting CTA lets its last loads land before the shared memory is released
         for (int k2 = max(0, q - NST); k2 < q; k2++)

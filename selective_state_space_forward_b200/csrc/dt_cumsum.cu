@@ -16,10 +16,6 @@
 // chunk's last -- and the reset marker -1 otherwise: the state entering such
 // a chunk does not reach its end.
 //
-// One warp per (row, head, chunk): lane l owns tokens l and l+32 of the chunk;
-// two segmented shuffle scans give the inclusive sums.  Warps are ordered
-// head-fastest, so the warps of one block read neighbouring dt_raw words of
-// the same token rows (dt_raw is (batch, seqlen, H)).
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
 
@@ -42,6 +38,14 @@ __device__ __forceinline__ float warp_seg_scan(float v, int& start, int lane)
     return v;
 }
 
+// One block per (row, chunk), 256 threads.  The chunk's dt_raw (and per-token A)
+// rows are read coalesced -- consecutive threads take consecutive heads of a
+// token row -- for a block of kHeadBlk heads at a time, turned into dt and dA in
+// shared memory, and then each warp scans whole heads: lane l owns tokens l and
+// l+32 of the chunk, and the two segmented shuffle scans give the inclusive sums.
+// dt and acs are written head-major, 64 consecutive floats per head.
+constexpr int kHeadBlk = 64;
+
 __global__ void __launch_bounds__(256)
 dt_cumsum_kernel(Shape s, const void* __restrict__ dt_raw, int64_t ld_dt, int dt_bf16,
                  const float* __restrict__ dt_bias,
@@ -49,68 +53,68 @@ dt_cumsum_kernel(Shape s, const void* __restrict__ dt_raw, int64_t ld_dt, int dt
                  const int32_t* __restrict__ lengths, float* __restrict__ dt_out,
                  float* __restrict__ acs_out, float* __restrict__ cdecay)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    __shared__ float s_dt[kChunk][kHeadBlk + 1], s_da[kChunk][kHeadBlk + 1];
+    __shared__ int s_bd[kChunk];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = s.nheads, nc = s.nchunks(), L = s.seqlen;
-    if (warp >= (int64_t)s.batch * nc * H) return;
-    const int h = (int)(warp % H);
-    const int c = (int)((warp / H) % nc);
-    const int b = (int)(warp / ((int64_t)H * nc));
-    const int t0 = c * kChunk;
+    const int c = blockIdx.x % nc, b = blockIdx.x / nc;
+    const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
     const int Lb = row_length(lengths, b, L);   // padding: dt = 0, no boundary
-    const float bias = dt_bias[h];
-    const float a_head = s.a_per_token ? 0.0f : A[h];
-
     const int32_t* seq_row = seq ? seq + (int64_t)b * L : nullptr;
-    float dtv[2], dA[2];
-    int bd[2];
-#pragma unroll
-    for (int half = 0; half < 2; half++) {
-        const int t = t0 + half * 32 + lane;
-        dtv[half] = 0.0f;
-        dA[half] = 0.0f;
-        bd[half] = 0;
-        if (t < Lb) {
-            const int64_t i = ((int64_t)b * L + t) * H + h;
-            const int64_t id = ((int64_t)b * L + t) * ld_dt + h;
-            const float raw = dt_bf16 ? to_f(((const bf16*)dt_raw)[id]) : ((const float*)dt_raw)[id];
-            dtv[half] = softplus_f(raw + bias);
-            const float av = s.a_per_token ? fminf(A[i], -kAFloor) : a_head;
-            dA[half] = dtv[half] * av;
-            bd[half] = is_boundary(seq_row, t);
+    if (tid < kChunk) s_bd[tid] = (tid < Lc && t0 + tid < Lb) ? is_boundary(seq_row, t0 + tid) : 0;
+    const int last = Lc - 1;
+    for (int h0 = 0; h0 < H; h0 += kHeadBlk) {
+        const int nh = min(kHeadBlk, H - h0);
+        __syncthreads();                        // the previous head block has been scanned
+        for (int e = tid; e < kChunk * kHeadBlk; e += blockDim.x) {
+            const int r = e / kHeadBlk, hh = e % kHeadBlk;
+            const int t = t0 + r, h = h0 + hh;
+            float dtv = 0.0f, dA = 0.0f;
+            if (hh < nh && r < Lc && t < Lb) {
+                const int64_t tok = (int64_t)b * L + t;
+                const float raw = dt_bf16 ? to_f(((const bf16*)dt_raw)[tok * ld_dt + h])
+                                          : ((const float*)dt_raw)[tok * ld_dt + h];
+                dtv = softplus_f(raw + dt_bias[h]);
+                const float av = s.a_per_token ? fminf(A[tok * H + h], -kAFloor) : A[h];
+                dA = dtv * av;
+            }
+            s_dt[r][hh] = dtv;
+            s_da[r][hh] = dA;
         }
-    }
-    const int any_bd = __any_sync(0xffffffffu, bd[0] | bd[1]);
-    int f0 = bd[0] | (lane == 0);   // the chunk start opens a segment
-    int f1 = bd[1];
-    const float s0 = warp_seg_scan(dA[0], f0, lane);
-    float s1 = warp_seg_scan(dA[1], f1, lane);
-    const float tail0 = __shfl_sync(0xffffffffu, s0, 31);
-    if (!f1) s1 = tail0 + s1;       // no segment start in tokens 32 .. lane+32
-
-    const int64_t row = ((int64_t)b * H + h) * L;
-    if (t0 + lane < L) {
-        dt_out[row + t0 + lane] = dtv[0];
-        acs_out[row + t0 + lane] = s0;
-    }
-    if (t0 + 32 + lane < L) {
-        dt_out[row + t0 + 32 + lane] = dtv[1];
-        acs_out[row + t0 + 32 + lane] = s1;
-    }
-    if (cdecay != nullptr) {
-        const int last = (L - t0 < kChunk ? L - t0 : kChunk) - 1;   // chunk-local index
-        const float acs_last = __shfl_sync(0xffffffffu, last < 32 ? s0 : s1, last & 31);
-        if (lane == 0) cdecay[((int64_t)b * H + h) * nc + c] = any_bd ? kChunkReset : expf(acs_last);
+        __syncthreads();
+        for (int hh = warp; hh < nh; hh += (int)(blockDim.x >> 5)) {
+            const int h = h0 + hh;
+            const int bd0 = s_bd[lane], bd1 = s_bd[lane + 32];
+            const int any_bd = __any_sync(0xffffffffu, bd0 | bd1);
+            int f0 = bd0 | (lane == 0);         // the chunk start opens a segment
+            int f1 = bd1;
+            const float s0 = warp_seg_scan(s_da[lane][hh], f0, lane);
+            float s1 = warp_seg_scan(s_da[lane + 32][hh], f1, lane);
+            const float tail0 = __shfl_sync(0xffffffffu, s0, 31);
+            if (!f1) s1 = tail0 + s1;           // no segment start in tokens 32 .. lane+32
+            const int64_t row = ((int64_t)b * H + h) * L;
+            if (lane < Lc) {
+                dt_out[row + t0 + lane] = s_dt[lane][hh];
+                acs_out[row + t0 + lane] = s0;
+            }
+            if (lane + 32 < Lc) {
+                dt_out[row + t0 + 32 + lane] = s_dt[lane + 32][hh];
+                acs_out[row + t0 + 32 + lane] = s1;
+            }
+            if (cdecay != nullptr) {
+                const float acs_last = __shfl_sync(0xffffffffu, last < 32 ? s0 : s1, last & 31);
+                if (lane == 0) cdecay[((int64_t)b * H + h) * nc + c] = any_bd ? kChunkReset : expf(acs_last);
+            }
+        }
     }
 }
 
 cudaError_t launch_dt_cumsum(const Shape& s, const FwdArgs& a, float* dt, float* acs,
                              float* cdecay, cudaStream_t st)
 {
-    const int64_t warps = (int64_t)s.batch * s.nchunks() * s.nheads;
-    const int64_t blocks = (warps * 32 + 255) / 256;
-    dt_cumsum_kernel<<<(unsigned)blocks, 256, 0, st>>>(s, a.dt_raw, a.ld_dt, a.dt_act, a.dt_bias, a.A, a.seq_idx,
-                                                       a.lengths, dt, acs, cdecay);
+    const int64_t blocks = (int64_t)s.batch * s.nchunks();
+    dt_cumsum_kernel<<<(unsigned)blocks, 256, 0, st>>>(s, a.dt_raw, a.ld_dt, a.dt_act, a.dt_bias, a.A,
+                                                       a.seq_idx, a.lengths, dt, acs, cdecay);
     return cudaGetLastError();
 }
 

@@ -8,8 +8,9 @@
 // consecutive channels (gs = d_inner: one norm per token; upstream's grouped
 // variant uses d_inner / ngroups).
 //
-// One block per (token, group): each thread holds up to kVecPerThread 8-channel
-// vectors of the group in registers, the sum of squares is reduced in a fixed
+// Groups of up to 2048 channels take one warp each (gated_norm_warp_kernel);
+// wider ones one block per (token, group): each thread holds up to kVecPerThread
+// 8-channel vectors of the group in registers, the sum of squares is reduced in a fixed
 // order (warp shuffles, then the warps in turn), and every vector is scaled
 // and written back.  Tokens past a ragged row's length are left untouched, so
 // their +0.0 padding stays +0.0.
@@ -65,6 +66,53 @@ gated_norm_kernel(Shape s, void* out_, const float* __restrict__ weight, int gs,
     }
 }
 
+// Groups of at most 2048 channels: one warp per (token, group), eight warps per
+// block; each lane holds up to eight 8-channel vectors, the warp reduces by xor
+// shuffles (a fixed order) and writes the scaled group back.
+template <typename T>
+__global__ void __launch_bounds__(256)
+gated_norm_warp_kernel(Shape s, void* out_, const float* __restrict__ weight, int gs, float eps,
+                       const int32_t* __restrict__ lengths)
+{
+    const int HP = s.nheads * s.headdim, L = s.seqlen, ngrp = HP / gs;
+    const int lane = threadIdx.x & 31;
+    const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (wid >= (int64_t)s.batch * L * ngrp) return;
+    const int64_t tok = wid / ngrp;
+    const int grp = (int)(wid % ngrp);
+    const int b = (int)(tok / L), t = (int)(tok % L);
+    if (t >= row_length(lengths, b, L)) return;          // padding stays +0.0
+    T* row = (T*)out_ + tok * HP + (int64_t)grp * gs;
+    const float* wr = weight ? weight + (int64_t)grp * gs : nullptr;
+    const int nvec = gs / 8;
+    float v[kVecPerThread][8];
+    float ss = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kVecPerThread; k++) {
+        const int i = lane + 32 * k;
+        if (i < nvec) {
+            load8(row + (int64_t)i * 8, v[k]);
+#pragma unroll
+            for (int j = 0; j < 8; j++) ss = fmaf(v[k][j], v[k][j], ss);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = rsqrtf(ss / gs + eps);
+#pragma unroll
+    for (int k = 0; k < kVecPerThread; k++) {
+        const int i = lane + 32 * k;
+        if (i < nvec) {
+            float wv[8];
+            if (wr) load8(wr + (int64_t)i * 8, wv);
+            float o[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) o[j] = v[k][j] * r * (wr ? wv[j] : 1.0f);
+            store8(row + (int64_t)i * 8, o);
+        }
+    }
+}
+
 bool gated_norm_group_ok(int d_inner, int gs)
 {
     return gs >= 8 && gs % 8 == 0 && d_inner % gs == 0 && gs / 8 <= 256 * kVecPerThread;
@@ -76,6 +124,15 @@ cudaError_t launch_gated_norm(const Shape& s, void* out, const float* weight, in
     const int HP = s.nheads * s.headdim;
     if (!gated_norm_group_ok(HP, gs)) return cudaErrorInvalidValue;
     const int nvec = gs / 8;
+    if (nvec <= 32 * kVecPerThread) {
+        const int64_t warps = (int64_t)s.batch * s.seqlen * (HP / gs);
+        const unsigned blocks = (unsigned)((warps + 7) / 8);
+        if (s.act_bf16)
+            gated_norm_warp_kernel<bf16><<<blocks, 256, 0, st>>>(s, out, weight, gs, eps, lengths);
+        else
+            gated_norm_warp_kernel<float><<<blocks, 256, 0, st>>>(s, out, weight, gs, eps, lengths);
+        return cudaGetLastError();
+    }
     int threads = (nvec + kVecPerThread - 1) / kVecPerThread;
     threads = ((threads + 31) / 32) * 32;
     if (threads > 256) threads = 256;

@@ -533,7 +533,7 @@ ssd_status ssd_set_gated_norm(ssd_handle* h, int32_t enable, const float* weight
                     "group_size %d must divide H*P = %d, be a multiple of 8 and at most 16384",
                     group_size, HP);
     if (!(eps >= 0.0f) || eps > 1.0f) return fail(SSD_ERR_INVALID_ARG, "eps must lie in [0, 1] (got %g)", (double)eps);
-    SSD_TRY(check_ptr(weight, "weight", 4, false));
+    SSD_TRY(check_ptr(weight, "weight", 16, false));
     h->gn_on = 1;
     h->gn_w = weight;
     h->gn_group = gs;
