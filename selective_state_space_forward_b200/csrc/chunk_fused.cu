@@ -458,7 +458,7 @@ ssd_chunk_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             if (nx.valid()) load_raw(nx, nxt);          // in flight while this step is finished
             Vals v;
             compute(it, cur, v);
-            if (q >= NST && !tc::mbar_wait(&empty[st], par(q / NST - 1), s_abort, p.status, kStatusTimeout, p.wait_ns))
+            if (q >= NST && !tc::mbar_wait_sleep(&empty[st], par(q / NST - 1), s_abort, p.status, kStatusTimeout, p.wait_ns))
                 break;
             const int g = it.h / (H / p.ngroups);
             const int t0 = it.c * 64;

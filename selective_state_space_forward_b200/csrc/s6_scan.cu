@@ -11,10 +11,13 @@
 // N/4 of its states and decay rates (pre-scaled by log2 e) in registers.  The
 // row is walked in chunks of 64 tokens (32 at d_state 32):
 //   stage   every thread turns its share of the chunk's (token, channel) inputs
-//           into dt = softplus(delta + bias), dt u, D u and SiLU(z) in shared
-//           memory, beside the chunk's B and C (shared by every channel);
-//   scan    each quartet walks the chunk's tokens reading shared memory only:
-//           its lanes update their states and sum C . h over two xor-shuffles;
+//           into {dt, dt u} = {softplus(delta + bias), dt u}, D u and SiLU(z) in
+//           shared memory, beside the chunk's B and C rows (shared by every
+//           channel); tokens past the row's end get dt = 0, which leaves h as it is;
+//   scan    each quartet walks the chunk eight tokens at a time from shared
+//           memory: the state updates of the eight tokens are independent of the
+//           C . h sums, and the eight partial sums of the quartet's lanes are
+//           reduced by a reduce-scatter (six shuffles, each lane finishing two);
 //   write   the chunk's outputs leave as coalesced rows of the block's channels.
 // The next chunk's raw inputs are loaded into registers before the scan starts,
 // so their memory latency overlaps the scan.  The bound is the N exponentials
@@ -27,8 +30,36 @@ namespace ssd {
 constexpr int kS6Threads = 128;
 constexpr int kS6Ch = 32;                         // channels per block
 constexpr int kS6Lanes = 4;                       // lanes per channel
-// tokens per chunk: 64, or 32 at d_state 32 (static shared memory stays under 48 KB)
+constexpr int kS6Group = 8;                       // tokens per unrolled scan group
+// tokens per chunk: 64, or 32 at d_state 32 (static shared memory stays within 48 KB)
 template <int N> constexpr int s6_chunk() { return N == 32 ? 32 : 64; }
+
+__device__ __forceinline__ uint64_t s6_p2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void s6_split(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t s6_fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t s6_mul2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// SiLU for the gate: the hardware tanh form for bf16 outputs, the IEEE form for fp32.
+template <typename T> __device__ __forceinline__ float s6_gate(float v) { return silu_t(v); }
+template <> __device__ __forceinline__ float s6_gate<float>(float v) { return silu_f(v); }
 
 template <typename T, int N>
 __global__ void __launch_bounds__(kS6Threads)
@@ -36,14 +67,16 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
                const float* __restrict__ delta_bias, const float* __restrict__ A_log,
                const T* __restrict__ Bm, const T* __restrict__ Cm, const float* __restrict__ D,
                const T* __restrict__ z, const float* __restrict__ init, T* __restrict__ out,
-               float* __restrict__ fin)
+               float* __restrict__ fin, int bc_vec)
 {
     constexpr int SPL = N / kS6Lanes;             // states per lane
+    static_assert(SPL % 2 == 0, "d_state 8, 16 or 32");
     constexpr int kS6T = s6_chunk<N>();
     constexpr int kS6PerThread = kS6T * kS6Ch / kS6Threads;   // staged (token, channel) pairs
     __shared__ __align__(16) float sb[kS6T][N], sc[kS6T][N];
-    __shared__ float s_dt[kS6T][kS6Ch], s_du[kS6T][kS6Ch], s_dx[kS6T][kS6Ch], s_g[kS6T][kS6Ch];
-    __shared__ float s_y[kS6T][kS6Ch];
+    __shared__ __align__(8) float2 s_dd[kS6T][kS6Ch];          // {dt, dt u}
+    __shared__ float s_dx[kS6T][kS6Ch], s_g[kS6T][kS6Ch];
+    __shared__ float s_y[kS6T][kS6Ch];     // row r's channel c at column (c + 8 ((r >> 1) & 3)) mod 32
     const int tid = threadIdx.x;
     const int d0 = blockIdx.x * kS6Ch;
     const int b = blockIdx.y;
@@ -56,13 +89,19 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
     const int dsr = d0 + cs;
     const bool live_s = dsr < DI;
 
-    float a2[SPL], h[SPL];
+    uint64_t a2[SPL / 2], h[SPL / 2];             // state pairs (j, j+1)
 #pragma unroll
-    for (int j = 0; j < SPL; j++) {
-        const int n = q * SPL + j;
-        const float al = live_q ? fminf(fmaxf(A_log[(int64_t)dq * N + n], -10.0f), 5.0f) : 0.0f;
-        a2[j] = -expf(al) * 1.4426950408889634f;        // A[d,n] log2(e)
-        h[j] = (live_q && init) ? init[((int64_t)b * DI + dq) * N + n] : 0.0f;
+    for (int j = 0; j < SPL; j += 2) {
+        float av[2], hv[2];
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int n = q * SPL + j + e;
+            const float al = live_q ? fminf(fmaxf(A_log[(int64_t)dq * N + n], -10.0f), 5.0f) : 0.0f;
+            av[e] = -expf(al) * 1.4426950408889634f;    // A[d,n] log2(e)
+            hv[e] = (live_q && init) ? init[((int64_t)b * DI + dq) * N + n] : 0.0f;
+        }
+        a2[j / 2] = s6_p2(av[0], av[1]);
+        h[j / 2] = s6_p2(hv[0], hv[1]);
     }
     const float bias = live_s ? delta_bias[dsr] : 0.0f;
     const float Dd = live_s ? D[dsr] : 0.0f;
@@ -84,50 +123,97 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
     for (int t0 = 0; t0 < L; t0 += kS6T) {
         const int Lc = min(kS6T, L - t0);
         __syncthreads();                     // the previous chunk's shared data is used
-        for (int i = tid; i < Lc * N; i += kS6Threads) {
-            const int r = i / N, n = i % N;
-            const int64_t o = ((int64_t)b * L + t0 + r) * N + n;
-            sb[r][n] = to_f(Bm[o]);
-            sc[r][n] = to_f(Cm[o]);
+        if (bc_vec) {
+            // eight elements per load (rows start 16-byte aligned)
+            for (int i = tid; i < kS6T * N / 8; i += kS6Threads) {
+                const int r = (i * 8) / N, n0 = (i * 8) % N;
+                float vb[8], vc[8];
+                if (r < Lc) {
+                    const int64_t o = ((int64_t)b * L + t0 + r) * N + n0;
+                    load8(Bm + o, vb);
+                    load8(Cm + o, vc);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; e++) vb[e] = vc[e] = 0.0f;
+                }
+                *reinterpret_cast<float4*>(&sb[r][n0]) = make_float4(vb[0], vb[1], vb[2], vb[3]);
+                *reinterpret_cast<float4*>(&sb[r][n0 + 4]) = make_float4(vb[4], vb[5], vb[6], vb[7]);
+                *reinterpret_cast<float4*>(&sc[r][n0]) = make_float4(vc[0], vc[1], vc[2], vc[3]);
+                *reinterpret_cast<float4*>(&sc[r][n0 + 4]) = make_float4(vc[4], vc[5], vc[6], vc[7]);
+            }
+        } else {
+            for (int i = tid; i < kS6T * N; i += kS6Threads) {
+                const int r = i / N, n = i % N;
+                const int64_t o = ((int64_t)b * L + t0 + r) * N + n;
+                sb[r][n] = r < Lc ? to_f(Bm[o]) : 0.0f;
+                sc[r][n] = r < Lc ? to_f(Cm[o]) : 0.0f;
+            }
         }
 #pragma unroll
         for (int k = 0; k < kS6PerThread; k++) {
             const int r = ts + k * (kS6Threads / kS6Ch);
-            const float dt = softplus_f(rd[k] + bias);
-            s_dt[r][cs] = dt;
-            s_du[r][cs] = dt * ru[k];
+            const bool ok = r < Lc;                 // past the row's end: dt = 0, h unchanged
+            const float dt = ok ? softplus_f(rd[k] + bias) : 0.0f;
+            s_dd[r][cs] = make_float2(dt, dt * ru[k]);
             s_dx[r][cs] = Dd * ru[k];
-            s_g[r][cs] = z ? silu_f(rz[k]) : 1.0f;
+            s_g[r][cs] = z ? s6_gate<T>(rz[k]) : 1.0f;
         }
         __syncthreads();
         if (t0 + kS6T < L) fetch(t0 + kS6T);   // in flight during the scan
-        for (int r = 0; r < Lc; r++) {
-            const float dt = s_dt[r][cq], du = s_du[r][cq];
-            float bv[SPL], cv[SPL];
-            if constexpr (SPL % 4 == 0) {
+        const int b0 = q & 1, b1 = (q >> 1) & 1;
+        for (int r0 = 0; r0 < Lc; r0 += kS6Group) {
+            float yv[kS6Group];
 #pragma unroll
-                for (int j = 0; j < SPL; j += 4) {
-                    const float4 b4 = *reinterpret_cast<const float4*>(&sb[r][q * SPL + j]);
-                    const float4 c4 = *reinterpret_cast<const float4*>(&sc[r][q * SPL + j]);
-                    bv[j] = b4.x; bv[j + 1] = b4.y; bv[j + 2] = b4.z; bv[j + 3] = b4.w;
-                    cv[j] = c4.x; cv[j + 1] = c4.y; cv[j + 2] = c4.z; cv[j + 3] = c4.w;
+            for (int k = 0; k < kS6Group; k++) {
+                const int r = r0 + k;
+                const float2 dd = s_dd[r][cq];
+                const uint64_t dtp = s6_p2(dd.x, dd.x), dup = s6_p2(dd.y, dd.y);
+                uint64_t bv[SPL / 2], cv[SPL / 2];
+                if constexpr (SPL % 4 == 0) {
+#pragma unroll
+                    for (int j = 0; j < SPL; j += 4) {
+                        const float4 b4 = *reinterpret_cast<const float4*>(&sb[r][q * SPL + j]);
+                        const float4 c4 = *reinterpret_cast<const float4*>(&sc[r][q * SPL + j]);
+                        bv[j / 2] = s6_p2(b4.x, b4.y); bv[j / 2 + 1] = s6_p2(b4.z, b4.w);
+                        cv[j / 2] = s6_p2(c4.x, c4.y); cv[j / 2 + 1] = s6_p2(c4.z, c4.w);
+                    }
+                } else {
+                    const float2 b2 = *reinterpret_cast<const float2*>(&sb[r][q * SPL]);
+                    const float2 c2 = *reinterpret_cast<const float2*>(&sc[r][q * SPL]);
+                    bv[0] = s6_p2(b2.x, b2.y);
+                    cv[0] = s6_p2(c2.x, c2.y);
                 }
-            } else {
-                static_assert(SPL == 2, "d_state 8, 16 or 32");
-                const float2 b2 = *reinterpret_cast<const float2*>(&sb[r][q * SPL]);
-                const float2 c2 = *reinterpret_cast<const float2*>(&sc[r][q * SPL]);
-                bv[0] = b2.x; bv[1] = b2.y;
-                cv[0] = c2.x; cv[1] = c2.y;
-            }
-            float y = 0.0f;
+                uint64_t y2 = 0;                   // two fp32 zeros
 #pragma unroll
-            for (int j = 0; j < SPL; j++) {
-                h[j] = fmaf(ex2(dt * a2[j]), h[j], du * bv[j]);
-                y = fmaf(cv[j], h[j], y);
+                for (int j = 0; j < SPL / 2; j++) {
+                    float x0, x1;
+                    s6_split(s6_mul2(dtp, a2[j]), x0, x1);
+                    h[j] = s6_fma2(s6_p2(ex2(x0), ex2(x1)), h[j], s6_mul2(dup, bv[j]));
+                    y2 = s6_fma2(cv[j], h[j], y2);
+                }
+                float ylo, yhi;
+                s6_split(y2, ylo, yhi);
+                yv[k] = ylo + yhi;
             }
-            y += __shfl_xor_sync(0xffffffffu, y, 1);
-            y += __shfl_xor_sync(0xffffffffu, y, 2);
-            if (q == 0) s_y[r][cq] = y;
+            // reduce-scatter over the quartet: lane (b0, b1) finishes tokens
+            // r0 + 4 b0 + 2 b1 and the one after it
+            float z1[4], z2[2];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float send = b0 ? yv[i] : yv[4 + i];
+                const float keep = b0 ? yv[4 + i] : yv[i];
+                z1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                const float send = b1 ? z1[i] : z1[2 + i];
+                const float keep = b1 ? z1[2 + i] : z1[i];
+                z2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+            const int rb = r0 + 4 * b0 + 2 * b1;
+            // the four lanes of a quartet store to four different banks
+            s_y[rb][(cq + 8 * ((rb >> 1) & 3)) & 31] = z2[0];
+            s_y[rb + 1][(cq + 8 * ((rb >> 1) & 3)) & 31] = z2[1];
         }
         __syncthreads();
 #pragma unroll
@@ -135,13 +221,18 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
             const int r = ts + k * (kS6Threads / kS6Ch);
             if (r < Lc && live_s) {
                 const int64_t o = ((int64_t)b * L + t0 + r) * DI + dsr;
-                out[o] = from_f<T>((s_y[r][cs] + s_dx[r][cs]) * s_g[r][cs]);
+                out[o] = from_f<T>((s_y[r][(cs + 8 * ((r >> 1) & 3)) & 31] + s_dx[r][cs]) * s_g[r][cs]);
             }
         }
     }
     if (live_q && fin) {
 #pragma unroll
-        for (int j = 0; j < SPL; j++) fin[((int64_t)b * DI + dq) * N + q * SPL + j] = h[j];
+        for (int j = 0; j < SPL; j += 2) {
+            float h0, h1;
+            s6_split(h[j / 2], h0, h1);
+            fin[((int64_t)b * DI + dq) * N + q * SPL + j] = h0;
+            fin[((int64_t)b * DI + dq) * N + q * SPL + j + 1] = h1;
+        }
     }
 }
 
@@ -149,10 +240,12 @@ template <typename T>
 static cudaError_t launch_s6_t(const S6Args& s, cudaStream_t st)
 {
     const dim3 grid((unsigned)((s.d_inner + kS6Ch - 1) / kS6Ch), (unsigned)s.batch);
+    // B and C rows are read eight elements at a time when both start 16-byte aligned
+    const int vec = ((reinterpret_cast<uintptr_t>(s.B) | reinterpret_cast<uintptr_t>(s.C)) & 15u) == 0;
 #define SSD_S6(NN)                                                                                  \
     s6_scan_kernel<T, NN><<<grid, kS6Threads, 0, st>>>(                                             \
         s.batch, s.seqlen, s.d_inner, (const T*)s.u, s.delta, s.delta_bias, s.A_log, (const T*)s.B, \
-        (const T*)s.C, s.D, (const T*)s.z, s.init, (T*)s.out, s.fin)
+        (const T*)s.C, s.D, (const T*)s.z, s.init, (T*)s.out, s.fin, vec)
     switch (s.dstate) {
     case 8: SSD_S6(8); break;
     case 16: SSD_S6(16); break;

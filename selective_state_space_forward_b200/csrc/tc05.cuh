@@ -63,16 +63,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
         : "memory");
 }
 
-// try_wait suspends the thread in hardware (up to the hint, in ns) until the
-// phase completes, so a waiting warp does not spin through issue slots.
+// test_wait returns at once: the compute roles poll, which wakes them sooner
+// after a phase completes than a suspended try_wait does.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
@@ -88,6 +88,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; i++) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 7) == 0) {
+            if (*abort) return false;
+            if (global_ns() - t0 > limit_ns) {
+                *abort = 1;
+                atomicOr(status, status_bit);
+                return false;
+            }
+        }
+    }
+}
+
+
+// Sleeping variant: try_wait suspends the thread in hardware (up to the hint, in
+// ns) until the phase completes, so a long wait off the critical path (the
+// producer's wait for a free ring slot) does not take issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                int* status, int status_bit, uint64_t limit_ns)
+{
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; i++) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if ((i & 7) == 0) {
             if (*abort) return false;
             if (global_ns() - t0 > limit_ns) {
