@@ -68,18 +68,18 @@ __device__ float block_sum(float v, float* red)
 // ---------------------------------------------------------------------------------
 // gHout_c[p,n] = sum_t f_t gy_t[p] C^_t[n]: the gradient of the state entering
 // chunk c through the chunk's own outputs.  Written into gs.
-template <typename T>
+template <typename T, int TCN>
 __global__ void __launch_bounds__(kBwdThreads)
 bwd_state_out_kernel(Shape s, FwdArgs a, BwdBufs w)
 {
     extern __shared__ float sm[];
     const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
-    const int HP = H * P;
+    const int HP = H * P, NB = N + 1, XS = P + 1;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
-    float* cs = sm;                    // [64][N]
-    float* gf = cs + kChunk * N;       // [64][P]  f_t gy_t
-    float* ft = gf + kChunk * P;       // [64]
+    float* cs = sm;                    // [64][NB]
+    float* gf = cs + kChunk * NB;      // [64][XS]  f_t gy_t
+    float* ft = gf + kChunk * XS;      // [64]
     int* seg = (int*)(ft + kChunk);    // [64]
     int* flag = seg + kChunk;          // [64]
 
@@ -90,7 +90,7 @@ bwd_state_out_kernel(Shape s, FwdArgs a, BwdBufs w)
         const int64_t o = ((int64_t)b * H + h) * L + t0 + r;
         ft[r] = (r < Lc && t0 + r < Lb && seg[r] == 0) ? expf(w.acs[o]) : 0.0f;
     }
-    load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 1, cs, N);
+    load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 1, cs, NB);
     __syncthreads();
     for (int e = threadIdx.x; e < kChunk * P; e += blockDim.x) {
         const int t = e / P, p = e % P;
@@ -99,16 +99,22 @@ bwd_state_out_kernel(Shape s, FwdArgs a, BwdBufs w)
             const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
             v = ft[t] * to_f(((const T*)w.gout)[o]) * silu_f(to_f(((const T*)a.z)[o]));
         }
-        gf[t * P + p] = v;
+        gf[t * XS + p] = v;
     }
     __syncthreads();
+    // [p][n] = sum_{t < Lc} gf[t][p] C^[t][n]
+    const int it = threadIdx.x >> 4, jt = threadIdx.x & 15;
+    float acc[4][TCN];
+    tile_zero(acc);
+    tile_mm<TCN>(acc, gf, 1, XS, P, cs, NB, 1, N, Lc, it, jt);
     float* dst = w.gs + (((int64_t)b * nc + c) * H + h) * P * N;
-    for (int e = threadIdx.x; e < P * N; e += blockDim.x) {
-        const int p = e / N, n = e % N;
-        float acc = 0.0f;
-        for (int t = 0; t < Lc; t++) acc += gf[t * P + p] * cs[t * N + n];
-        dst[e] = acc;
-    }
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+        for (int cc = 0; cc < TCN; cc++) {
+            const int pp = it + 16 * rr, n = jt + 16 * cc;
+            if (pp < P && n < N) dst[pp * N + n] = acc[rr][cc];
+        }
 }
 
 // Reverse state scan, one thread per state element: on entry gs holds gHout_c,
@@ -123,36 +129,55 @@ bwd_state_scan_kernel(Shape s, const float* __restrict__ cdecay, float* __restri
     const int h = (int)((gid / PN) % H);
     const int b = (int)(gid / ((int64_t)PN * H));
     const float* kd = cdecay + ((int64_t)b * H + h) * nc;
+    float* sp = gs + ((int64_t)b * nc * H + h) * PN + e;        // chunk c at sp + c * cs
+    const int64_t cs = (int64_t)H * PN;
+    // the next kAhead chunks (walking backwards) are in flight while the chain advances
+    constexpr int kAhead = 8;
+    float pre[kAhead], kpre[kAhead];
+#pragma unroll
+    for (int i = 0; i < kAhead; i++) {
+        const int c = nc - 1 - i;
+        pre[i] = c >= 0 ? sp[c * cs] : 0.0f;
+        kpre[i] = c >= 0 ? kd[c] : 0.0f;
+    }
     float g = 0.0f;                       // gHin_{c+1}
-    for (int c = nc - 1; c >= 0; c--) {
-        float* sp = gs + (((int64_t)b * nc + c) * H + h) * PN + e;
-        const float gout_c = *sp;
-        *sp = g;
-        const float k = kd[c];
-        g = (k == kChunkReset) ? gout_c : gout_c + k * g;
+    for (int j0 = 0; j0 < nc; j0 += kAhead) {
+#pragma unroll
+        for (int i = 0; i < kAhead; i++) {
+            const int c = nc - 1 - (j0 + i);
+            if (c >= 0) {
+                const float gout_c = pre[i], k = kpre[i];
+                if (c - kAhead >= 0) {
+                    pre[i] = sp[(c - kAhead) * cs];
+                    kpre[i] = kd[c - kAhead];
+                }
+                sp[c * cs] = g;
+                g = (k == kChunkReset) ? gout_c : gout_c + k * g;
+            }
+        }
     }
 }
 
 // ---------------------------------------------------------------------------------
-// The per-(chunk, head) gradients.  256 threads; P <= 64 and N <= 128.
-constexpr int kMaxXe = kChunk * 64 / kBwdThreads;     // x elements per thread
-constexpr int kMaxBe = kChunk * 128 / kBwdThreads;    // B elements per thread
-
-template <typename T>
-__global__ void __launch_bounds__(kBwdThreads)
+// The per-(chunk, head) gradients.  256 threads; P <= 64 and N <= 128 (TCN = 4
+// column tiles of 16 for N <= 64, else 8).  Every contraction is a register-tiled
+// product (tile_mm) over the chunk's operands in shared memory.
+template <typename T, int TCN>
+__global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
 {
     extern __shared__ float sm[];
     const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
-    const int HP = H * P, NB = N + 1, cd = s.conv_dim();
+    const int HP = H * P, NB = N + 1, XS = P + 1, cd = s.conv_dim();
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, L - t0), last = Lc - 1;
     const int tid = threadIdx.x;
-    float* cs = sm;                    // [64][N]   C^
-    float* bs = cs + kChunk * N;       // [64][NB]  B^
-    float* xs = bs + kChunk * NB;      // [64][P]   x (conv output)
-    float* gy = xs + kChunk * P;       // [64][P]   gradient of y
-    float* hb = gy + kChunk * P;       // [P][NB]   Hin_c, then gS_c
+    const int it = tid >> 4, jt = tid & 15;    // tile_mm thread coordinates
+    float* cs = sm;                    // [64][NB]  C^
+    float* bs = cs + kChunk * NB;      // [64][NB]  B^
+    float* xs = bs + kChunk * NB;      // [64][XS]  x (conv output)
+    float* gy = xs + kChunk * XS;      // [64][XS]  gradient of y
+    float* hb = gy + kChunk * XS;      // [P][NB]   Hin_c, then gS_c
     float* cbe = hb + P * NB;          // [64][65]  (C^_t . B^_s) E[t,s] on the mask
     float* gm = cbe + kChunk * 65;     // [64][65]  scratch; gM; then gM E dt_s
     float* ac = gm + kChunk * 65;      // [64] acs
@@ -181,53 +206,62 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
         ft[tid] = (tid < Lc && seg[tid] == 0) ? expf(ac[tid]) : 0.0f;
         ws[tid] = (tid < Lc && seg[tid] == seg[last]) ? expf(ac[last] - ac[tid]) * dv[tid] : 0.0f;
     }
-    load_x_rows<T>(s, a, w.u, b, h, t0, Lc, xs, P);
-    load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 1, cs, N);
+    load_x_rows<T>(s, a, w.u, b, h, t0, Lc, xs, XS);
+    load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 1, cs, NB);
     load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 0, bs, NB);
     const float* hp = w.hin + (((int64_t)b * nc + c) * H + h) * P * N;
     for (int e = tid; e < P * N; e += blockDim.x) hb[(e / N) * NB + e % N] = hp[e];
     __syncthreads();
 
-    // (C^_t . B^_s) E[t,s]
-    for (int e = tid; e < kChunk * kChunk; e += blockDim.x) {
-        const int t = e / kChunk, r = e % kChunk;
-        float v = 0.0f;
-        if (r <= t && t < Lc && seg[r] == seg[t]) {
-            float dot = 0.0f;
-            for (int n = 0; n < N; n++) dot += cs[t * N + n] * bs[r * NB + n];
-            v = dot * expf(ac[t] - ac[r]);
-        }
-        cbe[t * 65 + r] = v;
+    // (C^_t . B^_s) E[t,s] on the causal same-segment mask
+    {
+        float acc[4][4];
+        tile_zero(acc);
+        tile_mm<4>(acc, cs, NB, 1, kChunk, bs, 1, NB, kChunk, N, it, jt);
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int t = it + 16 * rr, r = jt + 16 * cc;
+                cbe[t * 65 + r] = (r <= t && t < Lc && seg[r] == seg[t]) ? acc[rr][cc] * expf(ac[t] - ac[r]) : 0.0f;
+            }
     }
     __syncthreads();
 
     // y recomputed; gy, gz; the carried-state term's share of gacs; gD
     const float Dh = a.D[h];
     float dpart = 0.0f;
-    for (int e = tid; e < kChunk * P; e += blockDim.x) {
-        const int t = e / P, p = e % P;
-        float gyv = 0.0f, prod = 0.0f;
-        if (t < Lc) {
-            const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
-            if (t0 + t < Lb) {
-                float y = 0.0f;
-                for (int r = 0; r <= t; r++) y += cbe[t * 65 + r] * dv[r] * xs[r * P + p];
-                float off = 0.0f;
-                if (ft[t] != 0.0f)
-                    for (int n = 0; n < N; n++) off += cs[t * N + n] * hb[p * NB + n];
-                y += ft[t] * off + Dh * xs[t * P + p];
-                const float zv = to_f(((const T*)a.z)[o]);
-                const float go = to_f(((const T*)w.gout)[o]);
-                gyv = go * silu_f(zv);
-                w.gz[o] = go * y * silu_grad_f(zv);
-                prod = ft[t] * gyv * off;
-                dpart += gyv * xs[t * P + p];
-            } else {
-                w.gz[o] = 0.0f;
+    {
+        float ys[4][4], off[4][4];
+        tile_zero(ys);
+        tile_zero(off);
+        tile_mm<4>(ys, cbe, 65, 1, kChunk, xs, XS, 1, P, kChunk, it, jt, dv);   // sum_s M[t,s] x_s
+        tile_mm<4>(off, cs, NB, 1, kChunk, hb, 1, NB, P, N, it, jt);           // C^_t . Hin[p]
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int t = it + 16 * rr, p = jt + 16 * cc;
+                if (p >= P) continue;
+                float gyv = 0.0f, prod = 0.0f;
+                if (t < Lc) {
+                    const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
+                    if (t0 + t < Lb) {
+                        const float offv = ft[t] != 0.0f ? off[rr][cc] : 0.0f;
+                        const float y = ys[rr][cc] + ft[t] * offv + Dh * xs[t * XS + p];
+                        const float zv = to_f(((const T*)a.z)[o]);
+                        const float go = to_f(((const T*)w.gout)[o]);
+                        gyv = go * silu_f(zv);
+                        w.gz[o] = go * y * silu_grad_f(zv);
+                        prod = ft[t] * gyv * offv;
+                        dpart += gyv * xs[t * XS + p];
+                    } else {
+                        w.gz[o] = 0.0f;
+                    }
+                }
+                gy[t * XS + p] = gyv;
+                gm[t * 65 + p] = prod;
             }
-        }
-        gy[t * P + p] = gyv;
-        gm[t * 65 + p] = prod;
     }
     __syncthreads();
     if (tid < kChunk) {
@@ -239,12 +273,17 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     __syncthreads();
 
     // gM[t,s] = gy_t . x_s on the mask
-    for (int e = tid; e < kChunk * kChunk; e += blockDim.x) {
-        const int t = e / kChunk, r = e % kChunk;
-        float v = 0.0f;
-        if (r <= t && t < Lc && seg[r] == seg[t])
-            for (int p = 0; p < P; p++) v += gy[t * P + p] * xs[r * P + p];
-        gm[t * 65 + r] = v;
+    {
+        float acc[4][4];
+        tile_zero(acc);
+        tile_mm<4>(acc, gy, XS, 1, kChunk, xs, 1, XS, kChunk, P, it, jt);
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int t = it + 16 * rr, r = jt + 16 * cc;
+                gm[t * 65 + r] = (r <= t && t < Lc && seg[r] == seg[t]) ? acc[rr][cc] : 0.0f;
+            }
     }
     __syncthreads();
     // acs through E: + row sums, - column sums of gM M; dt through M
@@ -275,45 +314,37 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     __syncthreads();
 
     // gx (intra-chunk and D), kept in registers until the chunk-state part is added
-    float gx_r[kMaxXe];
+    float gx[4][4];
+    tile_zero(gx);
+    tile_mm<4>(gx, cbe, 1, 65, kChunk, gy, XS, 1, P, kChunk, it, jt);        // sum_t M[t,s] gy_t
 #pragma unroll
-    for (int k = 0; k < kMaxXe; k++) {
-        const int e = tid + k * kBwdThreads;
-        float v = 0.0f;
-        if (e < kChunk * P) {
-            const int r = e / P, p = e % P;
-            if (r < Lc) {
-                for (int t = r; t < Lc; t++) v += cbe[t * 65 + r] * gy[t * P + p];
-                v = v * dv[r] + Dh * gy[r * P + p];
-            }
+    for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+        for (int cc = 0; cc < 4; cc++) {
+            const int r = it + 16 * rr, p = min(jt + 16 * cc, P - 1);
+            gx[rr][cc] = r < Lc ? gx[rr][cc] * dv[r] + Dh * gy[r * XS + p] : 0.0f;
         }
-        gx_r[k] = v;
-    }
     // gC^ (complete), written per head
-    for (int e = tid; e < kChunk * N; e += blockDim.x) {
-        const int t = e / N, n = e % N;
-        if (t >= Lc) continue;
-        float v = 0.0f;
-        for (int r = 0; r <= t; r++) v += gm[t * 65 + r] * bs[r * NB + n];
-        if (ft[t] != 0.0f) {
-            float o = 0.0f;
-            for (int p = 0; p < P; p++) o += gy[t * P + p] * hb[p * NB + n];
-            v += ft[t] * o;
-        }
-        w.gch[(((int64_t)b * L + t0 + t) * H + h) * N + n] = v;
+    {
+        float acc[4][TCN], acc2[4][TCN];
+        tile_zero(acc);
+        tile_zero(acc2);
+        tile_mm<TCN>(acc, gm, 65, 1, kChunk, bs, NB, 1, N, kChunk, it, jt);   // sum_s gM E dt_s B^_s
+        tile_mm<TCN>(acc2, gy, XS, 1, kChunk, hb, NB, 1, N, P, it, jt);      // gy_t . Hin[:, n]
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < TCN; cc++) {
+                const int t = it + 16 * rr, n = jt + 16 * cc;
+                if (t < Lc && n < N)
+                    w.gch[(((int64_t)b * L + t0 + t) * H + h) * N + n] =
+                        acc[rr][cc] + (ft[t] != 0.0f ? ft[t] * acc2[rr][cc] : 0.0f);
+            }
     }
     // gB^ (intra-chunk part)
-    float gb_r[kMaxBe];
-#pragma unroll
-    for (int k = 0; k < kMaxBe; k++) {
-        const int e = tid + k * kBwdThreads;
-        float v = 0.0f;
-        if (e < kChunk * N) {
-            const int r = e / N, n = e % N;
-            for (int t = r; t < Lc; t++) v += gm[t * 65 + r] * cs[t * N + n];
-        }
-        gb_r[k] = v;
-    }
+    float gb[4][TCN];
+    tile_zero(gb);
+    tile_mm<TCN>(gb, gm, 1, 65, kChunk, cs, NB, 1, N, kChunk, it, jt);       // sum_t gM E dt_s C^_t
     __syncthreads();
 
     // gS_c replaces Hin_c; gk = <gS_c, Hin_c> is the carry's gradient
@@ -329,37 +360,40 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     __syncthreads();
 
     // chunk state: gXs = gS B^_s -> gx += w_s gXs; gw_s = gXs . x_s; gB^_s += w_s x_s gS
+    {
+        float g7[4][4];
+        tile_zero(g7);
+        tile_mm<4>(g7, bs, NB, 1, kChunk, hb, 1, NB, P, N, it, jt);
 #pragma unroll
-    for (int k = 0; k < kMaxXe; k++) {
-        const int e = tid + k * kBwdThreads;
-        if (e < kChunk * P) {
-            const int r = e / P, p = e % P;
-            float g = 0.0f;
-            for (int n = 0; n < N; n++) g += hb[p * NB + n] * bs[r * NB + n];
-            gx_r[k] += ws[r] * g;
-            gm[r * 65 + p] = g * xs[r * P + p];
-        }
-    }
+        for (int rr = 0; rr < 4; rr++)
 #pragma unroll
-    for (int k = 0; k < kMaxBe; k++) {
-        const int e = tid + k * kBwdThreads;
-        if (e < kChunk * N) {
-            const int r = e / N, n = e % N;
-            if (r < Lc) {
-                float g = 0.0f;
-                for (int p = 0; p < P; p++) g += xs[r * P + p] * hb[p * NB + n];
-                w.gbh[(((int64_t)b * L + t0 + r) * H + h) * N + n] = gb_r[k] + ws[r] * g;
+            for (int cc = 0; cc < 4; cc++) {
+                const int r = it + 16 * rr, p = jt + 16 * cc;
+                if (p >= P) continue;
+                gx[rr][cc] += ws[r] * g7[rr][cc];
+                gm[r * 65 + p] = g7[rr][cc] * xs[r * XS + p];
             }
-        }
+    }
+    {
+        float g8[4][TCN];
+        tile_zero(g8);
+        tile_mm<TCN>(g8, xs, XS, 1, kChunk, hb, NB, 1, N, P, it, jt);
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < TCN; cc++) {
+                const int r = it + 16 * rr, n = jt + 16 * cc;
+                if (r < Lc && n < N)
+                    w.gbh[(((int64_t)b * L + t0 + r) * H + h) * N + n] = gb[rr][cc] + ws[r] * g8[rr][cc];
+            }
     }
 #pragma unroll
-    for (int k = 0; k < kMaxXe; k++) {
-        const int e = tid + k * kBwdThreads;
-        if (e < kChunk * P) {
-            const int r = e / P, p = e % P;
-            if (r < Lc) w.gu[((int64_t)b * L + t0 + r) * cd + h * P + p] = gx_r[k];
+    for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+        for (int cc = 0; cc < 4; cc++) {
+            const int r = it + 16 * rr, p = jt + 16 * cc;
+            if (r < Lc && p < P) w.gu[((int64_t)b * L + t0 + r) * cd + h * P + p] = gx[rr][cc];
         }
-    }
     __syncthreads();
     if (tid < kChunk) {
         float acc = 0.0f;
@@ -619,14 +653,14 @@ bwd_conv_reduce_kernel(const float* __restrict__ in, int64_t R, int cd, float* _
 
 size_t bwd_chunk_smem_bytes(const Shape& s)
 {
-    const size_t P = s.headdim, N = s.dstate, NB = N + 1;
-    return sizeof(float) * (kChunk * N + kChunk * NB + 2 * kChunk * P + P * NB + 2 * kChunk * 65 +
+    const size_t P = s.headdim, N = s.dstate, NB = N + 1, XS = P + 1;
+    return sizeof(float) * (2 * kChunk * NB + 2 * kChunk * XS + P * NB + 2 * kChunk * 65 +
                             8 * kChunk + 32) + sizeof(int) * 2 * kChunk;
 }
 
 static size_t state_out_smem_bytes(const Shape& s)
 {
-    return sizeof(float) * (kChunk * (size_t)s.dstate + kChunk * (size_t)s.headdim + kChunk) +
+    return sizeof(float) * (kChunk * ((size_t)s.dstate + 1) + kChunk * ((size_t)s.headdim + 1) + kChunk) +
            sizeof(int) * 2 * kChunk;
 }
 
@@ -648,8 +682,9 @@ static cudaError_t launch_bwd_t(const Shape& s, const FwdArgs& a, const BwdBufs&
     cudaError_t e;
     const dim3 cgrid(s.nchunks(), s.nheads, s.batch);
     const size_t so = state_out_smem_bytes(s);
-    if ((e = set_smem(bwd_state_out_kernel<T>, so)) != cudaSuccess) return e;
-    bwd_state_out_kernel<T><<<cgrid, kBwdThreads, so, st>>>(s, a, w);
+    auto k_out = s.dstate > 64 ? bwd_state_out_kernel<T, 8> : bwd_state_out_kernel<T, 4>;
+    if ((e = set_smem(k_out, so)) != cudaSuccess) return e;
+    k_out<<<cgrid, kBwdThreads, so, st>>>(s, a, w);
     ++*launches;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -659,8 +694,9 @@ static cudaError_t launch_bwd_t(const Shape& s, const FwdArgs& a, const BwdBufs&
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     const size_t sc = bwd_chunk_smem_bytes(s);
-    if ((e = set_smem(bwd_chunk_kernel<T>, sc)) != cudaSuccess) return e;
-    bwd_chunk_kernel<T><<<cgrid, kBwdThreads, sc, st>>>(s, a, w);
+    auto k_chunk = s.dstate > 64 ? bwd_chunk_kernel<T, 8> : bwd_chunk_kernel<T, 4>;
+    if ((e = set_smem(k_chunk, sc)) != cudaSuccess) return e;
+    k_chunk<<<cgrid, kBwdThreads, sc, st>>>(s, a, w);
     ++*launches;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 

@@ -35,11 +35,12 @@ chunk_state_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float*
 {
     extern __shared__ float sm[];
     const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
+    const int XS = P + 1, NB = N + 1;  // padded row strides (bank spread)
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
-    float* xs = sm;                    // [64][P], pre-scaled by the token weight
-    float* bs = xs + kChunk * P;       // [64][N]
-    float* wv = bs + kChunk * N;       // [64]
+    float* xs = sm;                    // [64][XS], pre-scaled by the token weight
+    float* bs = xs + kChunk * XS;      // [64][NB]
+    float* wv = bs + kChunk * NB;      // [64]
     int* seg = (int*)(wv + kChunk);    // [64]
     int* flag = seg + kChunk;          // [64]
 
@@ -51,19 +52,28 @@ chunk_state_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float*
         const int r = threadIdx.x;
         wv[r] = (r < Lc && seg[r] == seg[Lc - 1]) ? expf(acr[Lc - 1] - acr[r]) * dtr[r] : 0.0f;
     }
-    load_x_rows<T>(s, a, u, b, h, t0, Lc, xs, P);
-    load_bc_rows<T>(s, a, u, b, h, t0, Lc, 0, bs, N);
+    load_x_rows<T>(s, a, u, b, h, t0, Lc, xs, XS);
+    load_bc_rows<T>(s, a, u, b, h, t0, Lc, 0, bs, NB);
     __syncthreads();
-    for (int i = threadIdx.x; i < kChunk * P; i += blockDim.x) xs[i] *= wv[i / P];
+    for (int i = threadIdx.x; i < kChunk * P; i += blockDim.x) xs[(i / P) * XS + i % P] *= wv[i / P];
     __syncthreads();
 
+    // S[p][n] = sum_{r < Lc} xs[r][p] B[r][n], in 64 x 128 output blocks
     float* dst = states + (((int64_t)b * nc + c) * H + h) * P * N;
-    for (int e = threadIdx.x; e < P * N; e += blockDim.x) {
-        const int p = e / N, n = e % N;
-        float acc = 0.0f;
-        for (int r = 0; r < Lc; r++) acc += xs[r * P + p] * bs[r * N + n];
-        dst[e] = acc;
-    }
+    const int it = threadIdx.x >> 4, jt = threadIdx.x & 15;
+    for (int p0 = 0; p0 < P; p0 += 64)
+        for (int n0 = 0; n0 < N; n0 += 128) {
+            float acc[4][8];
+            tile_zero(acc);
+            tile_mm<8>(acc, xs + p0, 1, XS, P - p0, bs + n0, NB, 1, N - n0, Lc, it, jt);
+#pragma unroll
+            for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+                for (int cc = 0; cc < 8; cc++) {
+                    const int pp = p0 + it + 16 * rr, n = n0 + jt + 16 * cc;
+                    if (pp < P && n < N) dst[pp * N + n] = acc[rr][cc];
+                }
+        }
 }
 
 // One thread per state element (row, head, p, n), walking the chunks in order.
@@ -80,12 +90,31 @@ state_passing_kernel(Shape s, const float* __restrict__ cdecay, float* __restric
     const int b = (int)(gid / ((int64_t)PN * H));
     float hv = init ? init[gid] : 0.0f;
     const float* kd = cdecay + ((int64_t)b * H + h) * nc;
-    for (int c = 0; c < nc; c++) {
-        float* sp = states + (((int64_t)b * nc + c) * H + h) * PN + e;
-        const float sc = *sp;
-        *sp = hv;
-        const float k = kd[c];
-        hv = (k == kChunkReset) ? sc : k * hv + sc;   // select: a reset drops hv exactly
+    float* sp = states + ((int64_t)b * nc * H + h) * PN + e;     // chunk c at sp + c * cs
+    const int64_t cs = (int64_t)H * PN;
+    // the chunk states and carries of the next kAhead chunks are in flight while
+    // the chain advances (each thread's loads are independent of its chain)
+    constexpr int kAhead = 8;
+    float pre[kAhead], kpre[kAhead];
+#pragma unroll
+    for (int i = 0; i < kAhead; i++) {
+        pre[i] = i < nc ? sp[i * cs] : 0.0f;
+        kpre[i] = i < nc ? kd[i] : 0.0f;
+    }
+    for (int c0 = 0; c0 < nc; c0 += kAhead) {
+#pragma unroll
+        for (int i = 0; i < kAhead; i++) {
+            const int c = c0 + i;
+            if (c < nc) {
+                const float sc = pre[i], k = kpre[i];
+                if (c + kAhead < nc) {
+                    pre[i] = sp[(c + kAhead) * cs];
+                    kpre[i] = kd[c + kAhead];
+                }
+                sp[c * cs] = hv;
+                hv = (k == kChunkReset) ? sc : k * hv + sc;   // select: a reset drops hv exactly
+            }
+        }
     }
     if (fin) fin[gid] = hv;
 }
@@ -162,7 +191,7 @@ chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float
 
 size_t chunk_state_smem_bytes(const Shape& s)
 {
-    return sizeof(float) * ((size_t)kChunk * s.headdim + (size_t)kChunk * s.dstate + kChunk) +
+    return sizeof(float) * ((size_t)kChunk * (s.headdim + 1) + (size_t)kChunk * (s.dstate + 1) + kChunk) +
            sizeof(int) * 2 * kChunk;
 }
 

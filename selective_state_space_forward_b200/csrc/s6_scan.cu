@@ -9,15 +9,15 @@
 // A is diagonal, so channels never mix.  A block of 128 threads takes 32
 // channels of one row; the 4 lanes of a quartet share a channel and each keeps
 // N/4 of its states and decay rates (pre-scaled by log2 e) in registers.  The
-// row is walked in chunks of 64 tokens (32 at d_state 32):
+// row is walked in chunks of 32 tokens:
 //   stage   every thread turns its share of the chunk's (token, channel) inputs
 //           into {dt, dt u} = {softplus(delta + bias), dt u}, D u and SiLU(z) in
 //           shared memory, beside the chunk's B and C rows (shared by every
 //           channel); tokens past the row's end get dt = 0, which leaves h as it is;
-//   scan    each quartet walks the chunk eight tokens at a time from shared
-//           memory: the state updates of the eight tokens are independent of the
-//           C . h sums, and the eight partial sums of the quartet's lanes are
-//           reduced by a reduce-scatter (six shuffles, each lane finishing two);
+//   scan    each quartet walks the chunk four tokens at a time from shared
+//           memory: the state updates of the four tokens are independent of the
+//           C . h sums, and the four partial sums of the quartet's lanes are
+//           reduced by a reduce-scatter (three shuffles, each lane finishing one);
 //   write   the chunk's outputs leave as coalesced rows of the block's channels.
 // The next chunk's raw inputs are loaded into registers before the scan starts,
 // so their memory latency overlaps the scan.  The bound is the N exponentials
@@ -30,9 +30,9 @@ namespace ssd {
 constexpr int kS6Threads = 128;
 constexpr int kS6Ch = 32;                         // channels per block
 constexpr int kS6Lanes = 4;                       // lanes per channel
-constexpr int kS6Group = 8;                       // tokens per unrolled scan group
-// tokens per chunk: 64, or 32 at d_state 32 (static shared memory stays within 48 KB)
-template <int N> constexpr int s6_chunk() { return N == 32 ? 32 : 64; }
+constexpr int kS6Group = 4;                       // tokens per unrolled scan group
+// tokens per chunk: 32 (the next chunk's raw inputs wait in registers)
+template <int N> constexpr int s6_chunk() { return 32; }
 
 __device__ __forceinline__ uint64_t s6_p2(float lo, float hi)
 {
@@ -62,7 +62,7 @@ template <typename T> __device__ __forceinline__ float s6_gate(float v) { return
 template <> __device__ __forceinline__ float s6_gate<float>(float v) { return silu_f(v); }
 
 template <typename T, int N>
-__global__ void __launch_bounds__(kS6Threads)
+__global__ void __launch_bounds__(kS6Threads, 4)
 s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* __restrict__ delta,
                const float* __restrict__ delta_bias, const float* __restrict__ A_log,
                const T* __restrict__ Bm, const T* __restrict__ Cm, const float* __restrict__ D,
@@ -76,7 +76,7 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
     __shared__ __align__(16) float sb[kS6T][N], sc[kS6T][N];
     __shared__ __align__(8) float2 s_dd[kS6T][kS6Ch];          // {dt, dt u}
     __shared__ float s_dx[kS6T][kS6Ch], s_g[kS6T][kS6Ch];
-    __shared__ float s_y[kS6T][kS6Ch];     // row r's channel c at column (c + 8 ((r >> 1) & 3)) mod 32
+    __shared__ float s_y[kS6T][kS6Ch];     // row r's channel c at column (c + 8 (r & 3)) mod 32
     const int tid = threadIdx.x;
     const int d0 = blockIdx.x * kS6Ch;
     const int b = blockIdx.y;
@@ -195,25 +195,20 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
                 s6_split(y2, ylo, yhi);
                 yv[k] = ylo + yhi;
             }
-            // reduce-scatter over the quartet: lane (b0, b1) finishes tokens
-            // r0 + 4 b0 + 2 b1 and the one after it
-            float z1[4], z2[2];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float send = b0 ? yv[i] : yv[4 + i];
-                const float keep = b0 ? yv[4 + i] : yv[i];
-                z1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-            }
+            // reduce-scatter over the quartet: lane (b0, b1) finishes token r0 + 2 b0 + b1
+            float z1[2];
 #pragma unroll
             for (int i = 0; i < 2; i++) {
-                const float send = b1 ? z1[i] : z1[2 + i];
-                const float keep = b1 ? z1[2 + i] : z1[i];
-                z2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                const float send = b0 ? yv[i] : yv[2 + i];
+                const float keep = b0 ? yv[2 + i] : yv[i];
+                z1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
             }
-            const int rb = r0 + 4 * b0 + 2 * b1;
+            const float send = b1 ? z1[0] : z1[1];
+            const float keep = b1 ? z1[1] : z1[0];
+            const float z2 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            const int rb = r0 + 2 * b0 + b1;
             // the four lanes of a quartet store to four different banks
-            s_y[rb][(cq + 8 * ((rb >> 1) & 3)) & 31] = z2[0];
-            s_y[rb + 1][(cq + 8 * ((rb >> 1) & 3)) & 31] = z2[1];
+            s_y[rb][(cq + 8 * (rb & 3)) & 31] = z2;
         }
         __syncthreads();
 #pragma unroll
@@ -221,7 +216,7 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
             const int r = ts + k * (kS6Threads / kS6Ch);
             if (r < Lc && live_s) {
                 const int64_t o = ((int64_t)b * L + t0 + r) * DI + dsr;
-                out[o] = from_f<T>((s_y[r][(cs + 8 * ((r >> 1) & 3)) & 31] + s_dx[r][cs]) * s_g[r][cs]);
+                out[o] = from_f<T>((s_y[r][(cs + 8 * (r & 3)) & 31] + s_dx[r][cs]) * s_g[r][cs]);
             }
         }
     }

@@ -1,6 +1,6 @@
-// staged_rows.cuh -- per-chunk loads shared by the staged forward kernels and the
-// backward kernels: chunk-local document segments and the (64-token) rows of
-// x, B and C a block works on, in fp32.
+// staged_rows.cuh -- per-chunk pieces shared by the staged forward kernels and the
+// backward kernels: chunk-local document segments, the (64-token) rows of x, B
+// and C a block works on, in fp32, and a register-tiled product over them.
 #pragma once
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
@@ -72,6 +72,49 @@ __device__ void load_bc_rows(const Shape& s, const FwdArgs& a, const float* u, i
             dst[r * ld + n] = dst[r * ld + n] * rs * (wn ? wn[n] : 1.0f) +
                               (bias ? bias[(int64_t)h * N + n] : 0.0f);
     }
+}
+
+// Register-tiled fp32 product over shared-memory operands.  Thread (it, jt) =
+// (tid / 16, tid % 16) accumulates
+//   acc[rr][cc] += sum_{k < K} A(i, k) B(k, j) [s_k],   i = it + 16 rr, j = jt + 16 cc,
+// with A(i, k) = A[i a_si + k a_sk] and B(k, j) = B[k b_sk + j b_sj], k in order
+// (so results repeat bit for bit); s_k scales A's column k when given.  Rows at or
+// past R and columns at or past C read the last valid row / column: the caller
+// discards those results.  The strides the kernels pass keep a warp's 16 columns
+// on 16 banks and its 2 rows on different banks.
+template <int TC>
+__device__ __forceinline__ void tile_mm(float (&acc)[4][TC], const float* A, int a_si, int a_sk, int R,
+                                        const float* B, int b_sk, int b_sj, int C, int K, int it, int jt,
+                                        const float* sk = nullptr)
+{
+    const float* ap[4];
+    const float* bp[TC];
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++) ap[rr] = A + min(it + 16 * rr, R - 1) * a_si;
+#pragma unroll
+    for (int cc = 0; cc < TC; cc++) bp[cc] = B + min(jt + 16 * cc, C - 1) * b_sj;
+#pragma unroll 4
+    for (int k = 0; k < K; k++) {
+        float av[4], bv[TC];
+        const float sc = sk ? sk[k] : 1.0f;
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++) av[rr] = sk ? ap[rr][k * a_sk] * sc : ap[rr][k * a_sk];
+#pragma unroll
+        for (int cc = 0; cc < TC; cc++) bv[cc] = bp[cc][k * b_sk];
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < TC; cc++) acc[rr][cc] = fmaf(av[rr], bv[cc], acc[rr][cc]);
+    }
+}
+
+template <int TC>
+__device__ __forceinline__ void tile_zero(float (&acc)[4][TC])
+{
+#pragma unroll
+    for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+        for (int cc = 0; cc < TC; cc++) acc[rr][cc] = 0.0f;
 }
 
 }  // namespace ssd
