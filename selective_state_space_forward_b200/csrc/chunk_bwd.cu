@@ -74,7 +74,7 @@ bwd_state_out_kernel(Shape s, FwdArgs a, BwdBufs w)
 {
     extern __shared__ float sm[];
     const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
-    const int HP = H * P, NB = N + 1, XS = P + 1;
+    const int HP = H * P, NB = N + kPad, XS = P + kPad;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
     float* cs = sm;                    // [64][NB]
@@ -102,17 +102,17 @@ bwd_state_out_kernel(Shape s, FwdArgs a, BwdBufs w)
         gf[t * XS + p] = v;
     }
     __syncthreads();
-    // [p][n] = sum_{t < Lc} gf[t][p] C^[t][n]
-    const int it = threadIdx.x >> 4, jt = threadIdx.x & 15;
+    // [p][n] = sum_t gf[t][p] C^[t][n] (rows past the chunk's end are zero in both)
+    const Prod<T, TCN> pr(threadIdx.x);
     float acc[4][TCN];
     tile_zero(acc);
-    tile_mm<TCN>(acc, gf, 1, XS, P, cs, NB, 1, N, Lc, it, jt);
+    pr.mm(acc, gf, 1, XS, P, cs, NB, 1, N, kChunk);
     float* dst = w.gs + (((int64_t)b * nc + c) * H + h) * P * N;
 #pragma unroll
     for (int rr = 0; rr < 4; rr++)
 #pragma unroll
         for (int cc = 0; cc < TCN; cc++) {
-            const int pp = it + 16 * rr, n = jt + 16 * cc;
+            const int pp = pr.row(rr, cc), n = pr.col(rr, cc);
             if (pp < P && n < N) dst[pp * N + n] = acc[rr][cc];
         }
 }
@@ -160,27 +160,29 @@ bwd_state_scan_kernel(Shape s, const float* __restrict__ cdecay, float* __restri
 
 // ---------------------------------------------------------------------------------
 // The per-(chunk, head) gradients.  256 threads; P <= 64 and N <= 128 (TCN = 4
-// column tiles of 16 for N <= 64, else 8).  Every contraction is a register-tiled
-// product (tile_mm) over the chunk's operands in shared memory.
+// column tiles for N <= 64, else 8).  Every contraction is a product of the
+// kernel's engine (Prod: tensor-core tf32 tiles for bf16, fp32 SIMT tiles for
+// fp32) over the chunk's operands in shared memory.
 template <typename T, int TCN>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
 {
     extern __shared__ float sm[];
     const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
-    const int HP = H * P, NB = N + 1, XS = P + 1, cd = s.conv_dim();
+    const int HP = H * P, NB = N + kPad, XS = P + kPad, cd = s.conv_dim();
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, L - t0), last = Lc - 1;
     const int tid = threadIdx.x;
-    const int it = tid >> 4, jt = tid & 15;    // tile_mm thread coordinates
+    const Prod<T, 4> p4(tid);                  // 64 x 64 products
+    const Prod<T, TCN> pn(tid);                // 64 x N products
     float* cs = sm;                    // [64][NB]  C^
     float* bs = cs + kChunk * NB;      // [64][NB]  B^
     float* xs = bs + kChunk * NB;      // [64][XS]  x (conv output)
     float* gy = xs + kChunk * XS;      // [64][XS]  gradient of y
     float* hb = gy + kChunk * XS;      // [P][NB]   Hin_c, then gS_c
-    float* cbe = hb + P * NB;          // [64][65]  (C^_t . B^_s) E[t,s] on the mask
-    float* gm = cbe + kChunk * 65;     // [64][65]  scratch; gM; then gM E dt_s
-    float* ac = gm + kChunk * 65;      // [64] acs
+    float* cbe = hb + P * NB;          // [64][kMS] (C^_t . B^_s) E[t,s] on the mask
+    float* gm = cbe + kChunk * kMS;    // [64][kMS] scratch; gM; then gM E dt_s
+    float* ac = gm + kChunk * kMS;     // [64] acs
     float* dv = ac + kChunk;           // [64] dt
     float* ft = dv + kChunk;           // [64] weight of the carried-state term
     float* ws = ft + kChunk;           // [64] chunk-state weight
@@ -217,13 +219,13 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     {
         float acc[4][4];
         tile_zero(acc);
-        tile_mm<4>(acc, cs, NB, 1, kChunk, bs, 1, NB, kChunk, N, it, jt);
+        p4.mm(acc, cs, NB, 1, kChunk, bs, 1, NB, kChunk, N);
 #pragma unroll
         for (int rr = 0; rr < 4; rr++)
 #pragma unroll
             for (int cc = 0; cc < 4; cc++) {
-                const int t = it + 16 * rr, r = jt + 16 * cc;
-                cbe[t * 65 + r] = (r <= t && t < Lc && seg[r] == seg[t]) ? acc[rr][cc] * expf(ac[t] - ac[r]) : 0.0f;
+                const int t = p4.row(rr, cc), r = p4.col(rr, cc);
+                cbe[t * kMS + r] = (r <= t && t < Lc && seg[r] == seg[t]) ? acc[rr][cc] * expf(ac[t] - ac[r]) : 0.0f;
             }
     }
     __syncthreads();
@@ -235,13 +237,13 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
         float ys[4][4], off[4][4];
         tile_zero(ys);
         tile_zero(off);
-        tile_mm<4>(ys, cbe, 65, 1, kChunk, xs, XS, 1, P, kChunk, it, jt, dv);   // sum_s M[t,s] x_s
-        tile_mm<4>(off, cs, NB, 1, kChunk, hb, 1, NB, P, N, it, jt);           // C^_t . Hin[p]
+        p4.mm(ys, cbe, kMS, 1, kChunk, xs, XS, 1, P, kChunk, dv);   // sum_s M[t,s] x_s
+        p4.mm(off, cs, NB, 1, kChunk, hb, 1, NB, P, N);           // C^_t . Hin[p]
 #pragma unroll
         for (int rr = 0; rr < 4; rr++)
 #pragma unroll
             for (int cc = 0; cc < 4; cc++) {
-                const int t = it + 16 * rr, p = jt + 16 * cc;
+                const int t = p4.row(rr, cc), p = p4.col(rr, cc);
                 if (p >= P) continue;
                 float gyv = 0.0f, prod = 0.0f;
                 if (t < Lc) {
@@ -260,13 +262,13 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
                     }
                 }
                 gy[t * XS + p] = gyv;
-                gm[t * 65 + p] = prod;
+                gm[t * kMS + p] = prod;
             }
     }
     __syncthreads();
     if (tid < kChunk) {
         float acc = 0.0f;
-        for (int p = 0; p < P; p++) acc += gm[tid * 65 + p];
+        for (int p = 0; p < P; p++) acc += gm[tid * kMS + p];
         gac[tid] += acc;
     }
     dpart = block_sum(dpart, red2);
@@ -276,13 +278,13 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     {
         float acc[4][4];
         tile_zero(acc);
-        tile_mm<4>(acc, gy, XS, 1, kChunk, xs, 1, XS, kChunk, P, it, jt);
+        p4.mm(acc, gy, XS, 1, kChunk, xs, 1, XS, kChunk, P);
 #pragma unroll
         for (int rr = 0; rr < 4; rr++)
 #pragma unroll
             for (int cc = 0; cc < 4; cc++) {
-                const int t = it + 16 * rr, r = jt + 16 * cc;
-                gm[t * 65 + r] = (r <= t && t < Lc && seg[r] == seg[t]) ? acc[rr][cc] : 0.0f;
+                const int t = p4.row(rr, cc), r = p4.col(rr, cc);
+                gm[t * kMS + r] = (r <= t && t < Lc && seg[r] == seg[t]) ? acc[rr][cc] : 0.0f;
             }
     }
     __syncthreads();
@@ -290,13 +292,13 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     if (tid < kChunk) {
         const int t = tid;
         float acc = 0.0f;
-        for (int r = 0; r <= t; r++) acc += gm[t * 65 + r] * cbe[t * 65 + r] * dv[r];
+        for (int r = 0; r <= t; r++) acc += gm[t * kMS + r] * cbe[t * kMS + r] * dv[r];
         gac[t] += acc;
     } else if (tid < 2 * kChunk) {
         const int r = tid - kChunk;
         float acc = 0.0f, gd = 0.0f;
         for (int t = r; t < kChunk; t++) {
-            const float g = gm[t * 65 + r] * cbe[t * 65 + r];
+            const float g = gm[t * kMS + r] * cbe[t * kMS + r];
             acc += g * dv[r];
             gd += g;
         }
@@ -308,20 +310,20 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     // gM -> gradient of (C^_t . B^_s): gM E dt_s
     for (int e = tid; e < kChunk * kChunk; e += blockDim.x) {
         const int t = e / kChunk, r = e % kChunk;
-        const float g = gm[t * 65 + r];
-        gm[t * 65 + r] = g != 0.0f ? g * expf(ac[t] - ac[r]) * dv[r] : 0.0f;
+        const float g = gm[t * kMS + r];
+        gm[t * kMS + r] = g != 0.0f ? g * expf(ac[t] - ac[r]) * dv[r] : 0.0f;
     }
     __syncthreads();
 
     // gx (intra-chunk and D), kept in registers until the chunk-state part is added
     float gx[4][4];
     tile_zero(gx);
-    tile_mm<4>(gx, cbe, 1, 65, kChunk, gy, XS, 1, P, kChunk, it, jt);        // sum_t M[t,s] gy_t
+    p4.mm(gx, cbe, 1, kMS, kChunk, gy, XS, 1, P, kChunk);        // sum_t M[t,s] gy_t
 #pragma unroll
     for (int rr = 0; rr < 4; rr++)
 #pragma unroll
         for (int cc = 0; cc < 4; cc++) {
-            const int r = it + 16 * rr, p = min(jt + 16 * cc, P - 1);
+            const int r = p4.row(rr, cc), p = min(p4.col(rr, cc), P - 1);
             gx[rr][cc] = r < Lc ? gx[rr][cc] * dv[r] + Dh * gy[r * XS + p] : 0.0f;
         }
     // gC^ (complete), written per head
@@ -329,13 +331,13 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
         float acc[4][TCN], acc2[4][TCN];
         tile_zero(acc);
         tile_zero(acc2);
-        tile_mm<TCN>(acc, gm, 65, 1, kChunk, bs, NB, 1, N, kChunk, it, jt);   // sum_s gM E dt_s B^_s
-        tile_mm<TCN>(acc2, gy, XS, 1, kChunk, hb, NB, 1, N, P, it, jt);      // gy_t . Hin[:, n]
+        pn.mm(acc, gm, kMS, 1, kChunk, bs, NB, 1, N, kChunk);   // sum_s gM E dt_s B^_s
+        pn.mm(acc2, gy, XS, 1, kChunk, hb, NB, 1, N, P);      // gy_t . Hin[:, n]
 #pragma unroll
         for (int rr = 0; rr < 4; rr++)
 #pragma unroll
             for (int cc = 0; cc < TCN; cc++) {
-                const int t = it + 16 * rr, n = jt + 16 * cc;
+                const int t = pn.row(rr, cc), n = pn.col(rr, cc);
                 if (t < Lc && n < N)
                     w.gch[(((int64_t)b * L + t0 + t) * H + h) * N + n] =
                         acc[rr][cc] + (ft[t] != 0.0f ? ft[t] * acc2[rr][cc] : 0.0f);
@@ -344,7 +346,7 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     // gB^ (intra-chunk part)
     float gb[4][TCN];
     tile_zero(gb);
-    tile_mm<TCN>(gb, gm, 1, 65, kChunk, cs, NB, 1, N, kChunk, it, jt);       // sum_t gM E dt_s C^_t
+    pn.mm(gb, gm, 1, kMS, kChunk, cs, NB, 1, N, kChunk);       // sum_t gM E dt_s C^_t
     __syncthreads();
 
     // gS_c replaces Hin_c; gk = <gS_c, Hin_c> is the carry's gradient
@@ -363,26 +365,26 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     {
         float g7[4][4];
         tile_zero(g7);
-        tile_mm<4>(g7, bs, NB, 1, kChunk, hb, 1, NB, P, N, it, jt);
+        p4.mm(g7, bs, NB, 1, kChunk, hb, 1, NB, P, N);
 #pragma unroll
         for (int rr = 0; rr < 4; rr++)
 #pragma unroll
             for (int cc = 0; cc < 4; cc++) {
-                const int r = it + 16 * rr, p = jt + 16 * cc;
+                const int r = p4.row(rr, cc), p = p4.col(rr, cc);
                 if (p >= P) continue;
                 gx[rr][cc] += ws[r] * g7[rr][cc];
-                gm[r * 65 + p] = g7[rr][cc] * xs[r * XS + p];
+                gm[r * kMS + p] = g7[rr][cc] * xs[r * XS + p];
             }
     }
     {
         float g8[4][TCN];
         tile_zero(g8);
-        tile_mm<TCN>(g8, xs, XS, 1, kChunk, hb, NB, 1, N, P, it, jt);
+        pn.mm(g8, xs, XS, 1, kChunk, hb, NB, 1, N, P);
 #pragma unroll
         for (int rr = 0; rr < 4; rr++)
 #pragma unroll
             for (int cc = 0; cc < TCN; cc++) {
-                const int r = it + 16 * rr, n = jt + 16 * cc;
+                const int r = pn.row(rr, cc), n = pn.col(rr, cc);
                 if (r < Lc && n < N)
                     w.gbh[(((int64_t)b * L + t0 + r) * H + h) * N + n] = gb[rr][cc] + ws[r] * g8[rr][cc];
             }
@@ -391,13 +393,13 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     for (int rr = 0; rr < 4; rr++)
 #pragma unroll
         for (int cc = 0; cc < 4; cc++) {
-            const int r = it + 16 * rr, p = jt + 16 * cc;
+            const int r = p4.row(rr, cc), p = p4.col(rr, cc);
             if (r < Lc && p < P) w.gu[((int64_t)b * L + t0 + r) * cd + h * P + p] = gx[rr][cc];
         }
     __syncthreads();
     if (tid < kChunk) {
         float acc = 0.0f;
-        for (int p = 0; p < P; p++) acc += gm[tid * 65 + p];
+        for (int p = 0; p < P; p++) acc += gm[tid * kMS + p];
         red[tid] = acc;                               // gradient of w_s
     }
     __syncthreads();
@@ -653,14 +655,14 @@ bwd_conv_reduce_kernel(const float* __restrict__ in, int64_t R, int cd, float* _
 
 size_t bwd_chunk_smem_bytes(const Shape& s)
 {
-    const size_t P = s.headdim, N = s.dstate, NB = N + 1, XS = P + 1;
-    return sizeof(float) * (2 * kChunk * NB + 2 * kChunk * XS + P * NB + 2 * kChunk * 65 +
+    const size_t P = s.headdim, N = s.dstate, NB = N + kPad, XS = P + kPad;
+    return sizeof(float) * (2 * kChunk * NB + 2 * kChunk * XS + P * NB + 2 * kChunk * kMS +
                             8 * kChunk + 32) + sizeof(int) * 2 * kChunk;
 }
 
 static size_t state_out_smem_bytes(const Shape& s)
 {
-    return sizeof(float) * (kChunk * ((size_t)s.dstate + 1) + kChunk * ((size_t)s.headdim + 1) + kChunk) +
+    return sizeof(float) * (kChunk * ((size_t)s.dstate + kPad) + kChunk * ((size_t)s.headdim + kPad) + kChunk) +
            sizeof(int) * 2 * kChunk;
 }
 

@@ -28,14 +28,14 @@
 
 namespace ssd {
 
-template <typename T>
+template <typename T, int TC>
 __global__ void __launch_bounds__(256)
 chunk_state_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float* __restrict__ dt,
                    const float* __restrict__ acs, float* __restrict__ states)
 {
     extern __shared__ float sm[];
     const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
-    const int XS = P + 1, NB = N + 1;  // padded row strides (bank spread)
+    const int XS = P + kPad, NB = N + kPad;  // padded row strides (bank spread)
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
     float* xs = sm;                    // [64][XS], pre-scaled by the token weight
@@ -58,19 +58,20 @@ chunk_state_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float*
     for (int i = threadIdx.x; i < kChunk * P; i += blockDim.x) xs[(i / P) * XS + i % P] *= wv[i / P];
     __syncthreads();
 
-    // S[p][n] = sum_{r < Lc} xs[r][p] B[r][n], in 64 x 128 output blocks
+    // S[p][n] = sum_r xs[r][p] B[r][n] in 64 x 16 TC output blocks (rows past the
+    // chunk's end are zero in both operands)
     float* dst = states + (((int64_t)b * nc + c) * H + h) * P * N;
-    const int it = threadIdx.x >> 4, jt = threadIdx.x & 15;
+    const Prod<T, TC> pr(threadIdx.x);
     for (int p0 = 0; p0 < P; p0 += 64)
-        for (int n0 = 0; n0 < N; n0 += 128) {
-            float acc[4][8];
+        for (int n0 = 0; n0 < N; n0 += 16 * TC) {
+            float acc[4][TC];
             tile_zero(acc);
-            tile_mm<8>(acc, xs + p0, 1, XS, P - p0, bs + n0, NB, 1, N - n0, Lc, it, jt);
+            pr.mm(acc, xs + p0, 1, XS, P - p0, bs + n0, NB, 1, N - n0, kChunk);
 #pragma unroll
             for (int rr = 0; rr < 4; rr++)
 #pragma unroll
-                for (int cc = 0; cc < 8; cc++) {
-                    const int pp = p0 + it + 16 * rr, n = n0 + jt + 16 * cc;
+                for (int cc = 0; cc < TC; cc++) {
+                    const int pp = p0 + pr.row(rr, cc), n = n0 + pr.col(rr, cc);
                     if (pp < P && n < N) dst[pp * N + n] = acc[rr][cc];
                 }
         }
@@ -191,7 +192,7 @@ chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float
 
 size_t chunk_state_smem_bytes(const Shape& s)
 {
-    return sizeof(float) * ((size_t)kChunk * (s.headdim + 1) + (size_t)kChunk * (s.dstate + 1) + kChunk) +
+    return sizeof(float) * ((size_t)kChunk * (s.headdim + kPad) + (size_t)kChunk * (s.dstate + kPad) + kChunk) +
            sizeof(int) * 2 * kChunk;
 }
 
@@ -207,18 +208,13 @@ cudaError_t launch_chunk_state(const Shape& s, const FwdArgs& a, const float* u,
 {
     const dim3 grid(s.nchunks(), s.nheads, s.batch);
     const size_t smem = chunk_state_smem_bytes(s);
-    cudaError_t e;
-    if (s.act_bf16) {
-        e = cudaFuncSetAttribute(chunk_state_kernel<bf16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        chunk_state_kernel<bf16><<<grid, 256, smem, st>>>(s, a, u, dt, acs, states);
-    } else {
-        e = cudaFuncSetAttribute(chunk_state_kernel<float>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        chunk_state_kernel<float><<<grid, 256, smem, st>>>(s, a, u, dt, acs, states);
-    }
+    // output blocks of 64 x 64 for d_state <= 64, else 64 x 128
+    void (*kern)(Shape, FwdArgs, const float*, const float*, const float*, float*) =
+        s.act_bf16 ? (s.dstate > 64 ? chunk_state_kernel<bf16, 8> : chunk_state_kernel<bf16, 4>)
+                   : (s.dstate > 64 ? chunk_state_kernel<float, 8> : chunk_state_kernel<float, 4>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 256, smem, st>>>(s, a, u, dt, acs, states);
     return cudaGetLastError();
 }
 

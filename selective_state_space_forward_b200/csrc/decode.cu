@@ -20,7 +20,7 @@
 
 namespace ssd {
 
-constexpr int kDecodeThreads = 256;
+constexpr int kDecodeThreads = 128;
 
 // Conv + SiLU of the new token, dt and decay per head, B/C norm: fills the
 // block's shared arrays ux[hpg*P], ub[N], uc[N], dts[hpg], dec[hpg] and, with
@@ -71,12 +71,12 @@ __device__ void decode_prologue(const Shape& s, const FwdArgs& a, T* hist, float
             *dst = raw;
         }
     }
-    if (tid < hpg) {
-        const int h = g * hpg + tid;
+    for (int i = tid; i < hpg; i += blockDim.x) {
+        const int h = g * hpg + i;
         const float dtv = softplus_f(a.dt_raw[(int64_t)b * H + h] + a.dt_bias[h]);
         const float av = s.a_per_token ? fminf(a.A[(int64_t)b * H + h], -kAFloor) : a.A[h];
-        dts[tid] = dtv;
-        dec[tid] = expf(dtv * av);
+        dts[i] = dtv;
+        dec[i] = expf(dtv * av);
     }
     __syncthreads();
     if (s.bc_norm) {

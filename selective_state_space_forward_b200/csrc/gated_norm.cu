@@ -8,7 +8,8 @@
 // consecutive channels (gs = d_inner: one norm per token; upstream's grouped
 // variant uses d_inner / ngroups).
 //
-// Groups of up to 2048 channels take one warp each (gated_norm_warp_kernel);
+// Groups of up to 2048 channels take one warp each (gated_norm_warp_kernel, its
+// register footprint sized to the group);
 // wider ones one block per (token, group): each thread holds up to kVecPerThread
 // 8-channel vectors of the group in registers, the sum of squares is reduced in a fixed
 // order (warp shuffles, then the warps in turn), and every vector is scaled
@@ -67,9 +68,11 @@ gated_norm_kernel(Shape s, void* out_, const float* __restrict__ weight, int gs,
 }
 
 // Groups of at most 2048 channels: one warp per (token, group), eight warps per
-// block; each lane holds up to eight 8-channel vectors, the warp reduces by xor
-// shuffles (a fixed order) and writes the scaled group back.
-template <typename T>
+// block; each lane holds VPL 8-channel vectors (VPL = the group's vectors / 32,
+// rounded up to a power of two, so a small group keeps few registers and many
+// warps in flight), the warp reduces by xor shuffles (a fixed order) and writes
+// the scaled group back.
+template <typename T, int VPL>
 __global__ void __launch_bounds__(256)
 gated_norm_warp_kernel(Shape s, void* out_, const float* __restrict__ weight, int gs, float eps,
                        const int32_t* __restrict__ lengths)
@@ -85,10 +88,10 @@ gated_norm_warp_kernel(Shape s, void* out_, const float* __restrict__ weight, in
     T* row = (T*)out_ + tok * HP + (int64_t)grp * gs;
     const float* wr = weight ? weight + (int64_t)grp * gs : nullptr;
     const int nvec = gs / 8;
-    float v[kVecPerThread][8];
+    float v[VPL][8];
     float ss = 0.0f;
 #pragma unroll
-    for (int k = 0; k < kVecPerThread; k++) {
+    for (int k = 0; k < VPL; k++) {
         const int i = lane + 32 * k;
         if (i < nvec) {
             load8(row + (int64_t)i * 8, v[k]);
@@ -100,7 +103,7 @@ gated_norm_warp_kernel(Shape s, void* out_, const float* __restrict__ weight, in
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float r = rsqrtf(ss / gs + eps);
 #pragma unroll
-    for (int k = 0; k < kVecPerThread; k++) {
+    for (int k = 0; k < VPL; k++) {
         const int i = lane + 32 * k;
         if (i < nvec) {
             float wv[8];
@@ -127,10 +130,24 @@ cudaError_t launch_gated_norm(const Shape& s, void* out, const float* weight, in
     if (nvec <= 32 * kVecPerThread) {
         const int64_t warps = (int64_t)s.batch * s.seqlen * (HP / gs);
         const unsigned blocks = (unsigned)((warps + 7) / 8);
-        if (s.act_bf16)
-            gated_norm_warp_kernel<bf16><<<blocks, 256, 0, st>>>(s, out, weight, gs, eps, lengths);
-        else
-            gated_norm_warp_kernel<float><<<blocks, 256, 0, st>>>(s, out, weight, gs, eps, lengths);
+        const int vpl = nvec <= 32 ? 1 : nvec <= 64 ? 2 : nvec <= 128 ? 4 : 8;
+#define SSD_GN(TT, VV) gated_norm_warp_kernel<TT, VV><<<blocks, 256, 0, st>>>(s, out, weight, gs, eps, lengths)
+        if (s.act_bf16) {
+            switch (vpl) {
+            case 1: SSD_GN(bf16, 1); break;
+            case 2: SSD_GN(bf16, 2); break;
+            case 4: SSD_GN(bf16, 4); break;
+            default: SSD_GN(bf16, 8); break;
+            }
+        } else {
+            switch (vpl) {
+            case 1: SSD_GN(float, 1); break;
+            case 2: SSD_GN(float, 2); break;
+            case 4: SSD_GN(float, 4); break;
+            default: SSD_GN(float, 8); break;
+            }
+        }
+#undef SSD_GN
         return cudaGetLastError();
     }
     int threads = (nvec + kVecPerThread - 1) / kVecPerThread;

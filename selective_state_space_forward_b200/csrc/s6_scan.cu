@@ -76,7 +76,7 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
     __shared__ __align__(16) float sb[kS6T][N], sc[kS6T][N];
     __shared__ __align__(8) float2 s_dd[kS6T][kS6Ch];          // {dt, dt u}
     __shared__ float s_dx[kS6T][kS6Ch], s_g[kS6T][kS6Ch];
-    __shared__ float s_y[kS6T][kS6Ch];     // row r's channel c at column (c + 8 (r & 3)) mod 32
+    __shared__ float s_y[kS6T][kS6Ch];     // row r's channel c at column (c + kS6Ch/4 (r & 3)) mod kS6Ch
     const int tid = threadIdx.x;
     const int d0 = blockIdx.x * kS6Ch;
     const int b = blockIdx.y;
@@ -208,7 +208,7 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
             const float z2 = keep + __shfl_xor_sync(0xffffffffu, send, 2);
             const int rb = r0 + 2 * b0 + b1;
             // the four lanes of a quartet store to four different banks
-            s_y[rb][(cq + 8 * (rb & 3)) & 31] = z2;
+            s_y[rb][(cq + (kS6Ch / 4) * (rb & 3)) % kS6Ch] = z2;
         }
         __syncthreads();
 #pragma unroll
@@ -216,7 +216,7 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
             const int r = ts + k * (kS6Threads / kS6Ch);
             if (r < Lc && live_s) {
                 const int64_t o = ((int64_t)b * L + t0 + r) * DI + dsr;
-                out[o] = from_f<T>((s_y[r][(cs + 8 * (r & 3)) & 31] + s_dx[r][cs]) * s_g[r][cs]);
+                out[o] = from_f<T>((s_y[r][(cs + (kS6Ch / 4) * (r & 3)) % kS6Ch] + s_dx[r][cs]) * s_g[r][cs]);
             }
         }
     }

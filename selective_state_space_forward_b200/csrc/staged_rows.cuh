@@ -108,6 +108,66 @@ __device__ __forceinline__ void tile_mm(float (&acc)[4][TC], const float* A, int
     }
 }
 
+// The same product on the tensor cores (mma.sync m16n8k8, tf32 operands rounded
+// to nearest, fp32 accumulation), for operands that tolerate tf32 rounding: a
+// warp w owns rows 16 (w % 4) .. +15 and columns 8 TC (w / 4) .. +8 TC - 1 of
+// the 64 x 16 TC output; accumulator element (rr, cc) is that of MmaMap below.
+// K must be a multiple of 8 (rows of zeros pad a short chunk).
+struct SimtMap {
+    int it, jt;
+    __device__ explicit SimtMap(int tid) : it(tid >> 4), jt(tid & 15) {}
+    __device__ int row(int rr, int) const { return it + 16 * rr; }
+    __device__ int col(int, int cc) const { return jt + 16 * cc; }
+};
+template <int TC>
+struct MmaMap {
+    int r0, c0;
+    __device__ explicit MmaMap(int tid)
+        : r0(16 * ((tid >> 5) & 3) + ((tid & 31) >> 2)), c0(8 * TC * (tid >> 7) + 2 * (tid & 3)) {}
+    __device__ int row(int rr, int) const { return r0 + 8 * (rr >> 1); }
+    __device__ int col(int rr, int cc) const { return c0 + 8 * cc + (rr & 1); }
+};
+
+__device__ __forceinline__ uint32_t to_tf32(float v)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
+    return r;
+}
+
+template <int TC>
+__device__ __forceinline__ void tile_mm_tc(float (&acc)[4][TC], const float* A, int a_si, int a_sk, int R,
+                                           const float* B, int b_sk, int b_sj, int C, int K, int tid,
+                                           const float* sk = nullptr)
+{
+    const int w = tid >> 5, g = (tid & 31) >> 2, t4 = tid & 3;
+    const int row0 = 16 * (w & 3), col0 = 8 * TC * (w >> 2);
+    const float* alo = A + min(row0 + g, R - 1) * a_si;
+    const float* ahi = A + min(row0 + g + 8, R - 1) * a_si;
+    const float* bp[TC];
+#pragma unroll
+    for (int cc = 0; cc < TC; cc++) bp[cc] = B + min(col0 + 8 * cc + g, C - 1) * b_sj;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const int ka = k0 + t4, kb = ka + 4;
+        float x0 = alo[ka * a_sk], x1 = ahi[ka * a_sk], x2 = alo[kb * a_sk], x3 = ahi[kb * a_sk];
+        if (sk) {
+            const float sa = sk[ka], sb = sk[kb];
+            x0 *= sa; x1 *= sa; x2 *= sb; x3 *= sb;
+        }
+        const uint32_t a0 = to_tf32(x0), a1 = to_tf32(x1), a2 = to_tf32(x2), a3 = to_tf32(x3);
+#pragma unroll
+        for (int cc = 0; cc < TC; cc++) {
+            const uint32_t b0 = to_tf32(bp[cc][ka * b_sk]), b1 = to_tf32(bp[cc][kb * b_sk]);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+                "{%8,%9}, {%0,%1,%2,%3};"
+                : "+f"(acc[0][cc]), "+f"(acc[1][cc]), "+f"(acc[2][cc]), "+f"(acc[3][cc])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+}
+
 template <int TC>
 __device__ __forceinline__ void tile_zero(float (&acc)[4][TC])
 {
@@ -116,5 +176,41 @@ __device__ __forceinline__ void tile_zero(float (&acc)[4][TC])
 #pragma unroll
         for (int cc = 0; cc < TC; cc++) acc[rr][cc] = 0.0f;
 }
+
+// The contraction engine of a kernel instance: the tensor cores (tf32 operands,
+// fp32 accumulation) for bf16 activations, whose inputs tf32 holds exactly;
+// fp32 SIMT for fp32 activations, whose 1e-5 tolerance tf32 rounding would miss.
+// Both give a thread the same 4 x TC accumulator; row() and col() name the output
+// element each entry holds.
+template <typename T, int TC>
+struct Prod {
+    SimtMap m;
+    __device__ explicit Prod(int tid) : m(tid) {}
+    __device__ void mm(float (&acc)[4][TC], const float* A, int a_si, int a_sk, int R, const float* B,
+                       int b_sk, int b_sj, int C, int K, const float* sk = nullptr) const
+    {
+        tile_mm<TC>(acc, A, a_si, a_sk, R, B, b_sk, b_sj, C, K, m.it, m.jt, sk);
+    }
+    __device__ int row(int rr, int cc) const { return m.row(rr, cc); }
+    __device__ int col(int rr, int cc) const { return m.col(rr, cc); }
+};
+template <int TC>
+struct Prod<bf16, TC> {
+    MmaMap<TC> m;
+    int tid;
+    __device__ explicit Prod(int t) : m(t), tid(t) {}
+    __device__ void mm(float (&acc)[4][TC], const float* A, int a_si, int a_sk, int R, const float* B,
+                       int b_sk, int b_sj, int C, int K, const float* sk = nullptr) const
+    {
+        tile_mm_tc<TC>(acc, A, a_si, a_sk, R, B, b_sk, b_sj, C, K, tid, sk);
+    }
+    __device__ int row(int rr, int cc) const { return m.row(rr, cc); }
+    __device__ int col(int rr, int cc) const { return m.col(rr, cc); }
+};
+
+// Row strides of the shared-memory operands: 4 floats of padding spread a warp's
+// fragment loads over the banks.
+constexpr int kPad = 4;
+constexpr int kMS = kChunk + kPad;     // [64][64] token x token arrays
 
 }  // namespace ssd
