@@ -19,9 +19,10 @@
 //           C . h sums, and the four partial sums of the quartet's lanes are
 //           reduced by a reduce-scatter (three shuffles, each lane finishing one);
 //   write   the chunk's outputs leave as coalesced rows of the block's channels.
-// The next chunk's raw inputs are loaded into registers before the scan starts,
-// so their memory latency overlaps the scan.  The bound is the N exponentials
-// per (token, channel) on the MUFU pipe.
+// The next chunk's raw inputs (u, delta, z, B, C rows) are copied into shared
+// memory with cp.async before the scan starts (into registers when the rows are
+// not 16-byte aligned), so their memory latency overlaps the scan.  The bound is
+// the N exponentials per (token, channel) on the MUFU pipe.
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
 
@@ -61,7 +62,18 @@ __device__ __forceinline__ uint64_t s6_mul2(uint64_t a, uint64_t b)
 template <typename T> __device__ __forceinline__ float s6_gate(float v) { return silu_t(v); }
 template <> __device__ __forceinline__ float s6_gate<float>(float v) { return silu_f(v); }
 
-template <typename T, int N>
+// 16-byte asynchronous copy global -> shared (cp.async); bytes past src_bytes
+// are zero-filled, and with src_bytes = 0 nothing is read.
+__device__ __forceinline__ void s6_cp16(void* dst, const void* src, int src_bytes)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void s6_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void s6_cp_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <typename T, int N, bool ASYNC>
 __global__ void __launch_bounds__(kS6Threads, 4)
 s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* __restrict__ delta,
                const float* __restrict__ delta_bias, const float* __restrict__ A_log,
@@ -77,6 +89,10 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
     __shared__ __align__(8) float2 s_dd[kS6T][kS6Ch];          // {dt, dt u}
     __shared__ float s_dx[kS6T][kS6Ch], s_g[kS6T][kS6Ch];
     __shared__ float s_y[kS6T][kS6Ch];     // row r's channel c at column (c + kS6Ch/4 (r & 3)) mod kS6Ch
+    // ASYNC: the next chunk's raw inputs, copied in while the current chunk is scanned
+    constexpr int kRawT = ASYNC ? kS6T : 1;
+    __shared__ __align__(16) T raw_u[kRawT][kS6Ch], raw_z[kRawT][kS6Ch], raw_b[kRawT][N], raw_c[kRawT][N];
+    __shared__ __align__(16) float raw_d[kRawT][kS6Ch];
     const int tid = threadIdx.x;
     const int d0 = blockIdx.x * kS6Ch;
     const int b = blockIdx.y;
@@ -119,11 +135,62 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
             rz[k] = (ok && z) ? to_f(z[o]) : 0.0f;
         }
     };
-    fetch(0);
+    // ASYNC: copy chunk t0's u, delta, z rows (the block's channels) and B, C rows
+    // into the raw buffers in 16-byte pieces; rows past L and channels past DI are
+    // zero-filled (the host takes this path when every piece is 16-byte aligned
+    // and whole: DI a multiple of 16 / sizeof(T))
+    auto fetch_async = [&](int t0) {
+        constexpr int kPu = kS6Ch * (int)sizeof(T) / 16;        // 16-byte pieces per token row of u, z
+        constexpr int kPd = kS6Ch * 4 / 16;                     // of delta
+        constexpr int kPb = N * (int)sizeof(T) / 16;            // of B, C
+        constexpr int kTask = kS6T * (2 * kPu + kPd + 2 * kPb);
+        for (int i = tid; i < kTask; i += kS6Threads) {
+            int j = i;
+            const int which = j < kS6T * kPu ? 0 : (j -= kS6T * kPu) < kS6T * kPu ? 1
+                            : (j -= kS6T * kPu) < kS6T * kPd ? 2 : (j -= kS6T * kPd) < kS6T * kPb ? 3
+                            : (j -= kS6T * kPb, 4);
+            const int per = which < 2 ? kPu : which == 2 ? kPd : kPb;
+            const int r = j / per, piece = j % per;
+            const int t = t0 + r;
+            const bool tok_ok = t < L;
+            const int64_t trow = (int64_t)b * L + (tok_ok ? t : 0);
+            if (which <= 2) {
+                const int elems = which < 2 ? 16 / (int)sizeof(T) : 4;
+                const int c0 = d0 + piece * elems;
+                const bool ok = tok_ok && c0 < DI;
+                const int64_t o = trow * DI + (ok ? c0 : 0);
+                if (which == 0) s6_cp16(&raw_u[r][piece * elems], u + o, ok ? 16 : 0);
+                else if (which == 1) s6_cp16(&raw_z[r][piece * elems], (z ? z : u) + o, ok && z ? 16 : 0);
+                else s6_cp16(&raw_d[r][piece * elems], delta + o, ok ? 16 : 0);
+            } else {
+                const int elems = 16 / (int)sizeof(T);
+                const int64_t o = trow * N + piece * elems;
+                s6_cp16(which == 3 ? &raw_b[r][piece * elems] : &raw_c[r][piece * elems],
+                        (which == 3 ? Bm : Cm) + o, tok_ok ? 16 : 0);
+            }
+        }
+        s6_cp_commit();
+    };
+    if (ASYNC) fetch_async(0);
+    else fetch(0);
     for (int t0 = 0; t0 < L; t0 += kS6T) {
         const int Lc = min(kS6T, L - t0);
-        __syncthreads();                     // the previous chunk's shared data is used
-        if (bc_vec) {
+        if (ASYNC) s6_cp_wait();             // this chunk's raw inputs have landed
+        __syncthreads();                     // ... for every thread; the previous chunk's shared data is used
+        if (ASYNC) {
+            for (int i = tid; i < kS6T * N; i += kS6Threads) {
+                const int r = i / N, n = i % N;
+                sb[r][n] = to_f(raw_b[r][n]);
+                sc[r][n] = to_f(raw_c[r][n]);
+            }
+#pragma unroll
+            for (int k = 0; k < kS6PerThread; k++) {
+                const int r = ts + k * (kS6Threads / kS6Ch);
+                ru[k] = to_f(raw_u[r][cs]);
+                rd[k] = raw_d[r][cs];
+                rz[k] = to_f(raw_z[r][cs]);
+            }
+        } else if (bc_vec) {
             // eight elements per load (rows start 16-byte aligned)
             for (int i = tid; i < kS6T * N / 8; i += kS6Threads) {
                 const int r = (i * 8) / N, n0 = (i * 8) % N;
@@ -159,7 +226,10 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
             s_g[r][cs] = z ? s6_gate<T>(rz[k]) : 1.0f;
         }
         __syncthreads();
-        if (t0 + kS6T < L) fetch(t0 + kS6T);   // in flight during the scan
+        if (t0 + kS6T < L) {                   // in flight during the scan
+            if (ASYNC) fetch_async(t0 + kS6T);
+            else fetch(t0 + kS6T);
+        }
         const int b0 = q & 1, b1 = (q >> 1) & 1;
         for (int r0 = 0; r0 < Lc; r0 += kS6Group) {
             float yv[kS6Group];
@@ -236,11 +306,20 @@ static cudaError_t launch_s6_t(const S6Args& s, cudaStream_t st)
 {
     const dim3 grid((unsigned)((s.d_inner + kS6Ch - 1) / kS6Ch), (unsigned)s.batch);
     // B and C rows are read eight elements at a time when both start 16-byte aligned
-    const int vec = ((reinterpret_cast<uintptr_t>(s.B) | reinterpret_cast<uintptr_t>(s.C)) & 15u) == 0;
-#define SSD_S6(NN)                                                                                  \
-    s6_scan_kernel<T, NN><<<grid, kS6Threads, 0, st>>>(                                             \
-        s.batch, s.seqlen, s.d_inner, (const T*)s.u, s.delta, s.delta_bias, s.A_log, (const T*)s.B, \
-        (const T*)s.C, s.D, (const T*)s.z, s.init, (T*)s.out, s.fin, vec)
+    const uintptr_t bc = reinterpret_cast<uintptr_t>(s.B) | reinterpret_cast<uintptr_t>(s.C);
+    const int vec = (bc & 15u) == 0;
+    // the asynchronous copies need every 16-byte piece of u, z, delta, B and C
+    // aligned and whole: aligned bases and d_inner a multiple of 16 / sizeof(T)
+    const uintptr_t all = bc | reinterpret_cast<uintptr_t>(s.u) | reinterpret_cast<uintptr_t>(s.z) |
+                          reinterpret_cast<uintptr_t>(s.delta);
+    const bool async = (all & 15u) == 0 && s.d_inner % (16 / (int)sizeof(T)) == 0 && s.d_inner % 4 == 0;
+#define SSD_S6(NN)                                                                                    \
+    (async ? s6_scan_kernel<T, NN, true><<<grid, kS6Threads, 0, st>>>(                                \
+                 s.batch, s.seqlen, s.d_inner, (const T*)s.u, s.delta, s.delta_bias, s.A_log,         \
+                 (const T*)s.B, (const T*)s.C, s.D, (const T*)s.z, s.init, (T*)s.out, s.fin, vec)     \
+           : s6_scan_kernel<T, NN, false><<<grid, kS6Threads, 0, st>>>(                               \
+                 s.batch, s.seqlen, s.d_inner, (const T*)s.u, s.delta, s.delta_bias, s.A_log,         \
+                 (const T*)s.B, (const T*)s.C, s.D, (const T*)s.z, s.init, (T*)s.out, s.fin, vec))
     switch (s.dstate) {
     case 8: SSD_S6(8); break;
     case 16: SSD_S6(16); break;
