@@ -62,6 +62,22 @@ __device__ __forceinline__ uint64_t s6_mul2(uint64_t a, uint64_t b)
 template <typename T> __device__ __forceinline__ float s6_gate(float v) { return silu_t(v); }
 template <> __device__ __forceinline__ float s6_gate<float>(float v) { return silu_f(v); }
 
+// softplus(v) = log(1 + e^v) for bf16 paths from the hardware exp2 and log2:
+// v above 15 gives v (e^-15 is below fp32's resolution of v); below -5 the
+// series e - e^2/2 + e^3/3 (e = e^v < 0.0068, the first dropped term e^4/4 is
+// below 2.1e-9 of the result); in between log2(1 + e) ln 2, with 1 + e >= 1.0067
+// so its rounding costs at most 2e-5 of the result.  fp32 paths keep softplus_f.
+template <typename T> __device__ __forceinline__ float s6_softplus(float v)
+{
+    const float e = ex2(v * 1.4426950408889634f);
+    if (v > 15.0f) return v;
+    if (v < -5.0f) return e * (1.0f - e * (0.5f - e * 0.33333334f));
+    float l;
+    asm("lg2.approx.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e));
+    return l * 0.6931471805599453f;
+}
+template <> __device__ __forceinline__ float s6_softplus<float>(float v) { return softplus_f(v); }
+
 // 16-byte asynchronous copy global -> shared (cp.async); bytes past src_bytes
 // are zero-filled, and with src_bytes = 0 nothing is read.
 __device__ __forceinline__ void s6_cp16(void* dst, const void* src, int src_bytes)
@@ -220,7 +236,7 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
         for (int k = 0; k < kS6PerThread; k++) {
             const int r = ts + k * (kS6Threads / kS6Ch);
             const bool ok = r < Lc;                 // past the row's end: dt = 0, h unchanged
-            const float dt = ok ? softplus_f(rd[k] + bias) : 0.0f;
+            const float dt = ok ? s6_softplus<T>(rd[k] + bias) : 0.0f;
             s_dd[r][cs] = make_float2(dt, dt * ru[k]);
             s_dx[r][cs] = Dd * ru[k];
             s_g[r][cs] = z ? s6_gate<T>(rz[k]) : 1.0f;
