@@ -528,8 +528,9 @@ def bench_backward(args, torch, peaks, wname="mini_k3_mixer"):
                          "achieved": round(nbytes / (ms * 1e-3) / 1e9, 1),
                          "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
                          "frac": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
-            "arithmetic": "fp32 SIMT (forward recompute on the staged kernels, then the "
-                          "backward kernels)",
+            "arithmetic": "forward recompute on the staged kernels, then the backward kernels; "
+                          "their contractions on the tensor cores (mma.sync tf32 operands, fp32 "
+                          "accumulation) for bf16 activations, fp32 SIMT for fp32",
             "workspace_bytes": ws.numel()}
 
 

@@ -211,8 +211,7 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     load_x_rows<T>(s, a, w.u, b, h, t0, Lc, xs, XS);
     load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 1, cs, NB);
     load_bc_rows<T>(s, a, w.u, b, h, t0, Lc, 0, bs, NB);
-    const float* hp = w.hin + (((int64_t)b * nc + c) * H + h) * P * N;
-    for (int e = tid; e < P * N; e += blockDim.x) hb[(e / N) * NB + e % N] = hp[e];
+    load_rows8(w.hin + (((int64_t)b * nc + c) * H + h) * P * N, N, N, P, hb, NB, P);
     __syncthreads();
 
     // (C^_t . B^_s) E[t,s] on the causal same-segment mask
@@ -237,6 +236,19 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
         float ys[4][4], off[4][4];
         tile_zero(ys);
         tile_zero(off);
+        // z and the output gradient of the thread's elements, requested before the
+        // products so their latency overlaps them (and before any store of gz)
+        float zr[4][4], gr[4][4];
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int t = p4.row(rr, cc), p = p4.col(rr, cc);
+                const bool ok = p < P && t < Lc && t0 + t < Lb;
+                const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
+                zr[rr][cc] = ok ? to_f(((const T*)a.z)[o]) : 0.0f;
+                gr[rr][cc] = ok ? to_f(((const T*)w.gout)[o]) : 0.0f;
+            }
         p4.mm(ys, cbe, kMS, 1, kChunk, xs, XS, 1, P, kChunk, dv);   // sum_s M[t,s] x_s
         p4.mm(off, cs, NB, 1, kChunk, hb, 1, NB, P, N);           // C^_t . Hin[p]
 #pragma unroll
@@ -251,8 +263,8 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
                     if (t0 + t < Lb) {
                         const float offv = ft[t] != 0.0f ? off[rr][cc] : 0.0f;
                         const float y = ys[rr][cc] + ft[t] * offv + Dh * xs[t * XS + p];
-                        const float zv = to_f(((const T*)a.z)[o]);
-                        const float go = to_f(((const T*)w.gout)[o]);
+                        const float zv = zr[rr][cc];
+                        const float go = gr[rr][cc];
                         gyv = go * silu_f(zv);
                         w.gz[o] = go * y * silu_grad_f(zv);
                         prod = ft[t] * gyv * offv;
@@ -352,11 +364,26 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
     // gS_c replaces Hin_c; gk = <gS_c, Hin_c> is the carry's gradient
     const float* gsp = w.gs + (((int64_t)b * nc + c) * H + h) * P * N;
     float gk = 0.0f;
-    for (int e = tid; e < P * N; e += blockDim.x) {
-        const int i = (e / N) * NB + e % N;
-        const float g = gsp[e];
-        gk += g * hb[i];
-        hb[i] = g;
+    {
+        // four consecutive elements per task (N is a multiple of 8), two tasks' loads in flight
+        const int ntask = P * N / 4;
+        for (int i0 = tid; i0 < ntask; i0 += 2 * blockDim.x) {
+            float4 g[2];
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                const int i = i0 + k * blockDim.x;
+                g[k] = i < ntask ? *reinterpret_cast<const float4*>(gsp + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                const int i = i0 + k * blockDim.x;
+                if (i < ntask) {
+                    float* hr = hb + ((4 * i) / N) * NB + (4 * i) % N;
+                    gk += g[k].x * hr[0] + g[k].y * hr[1] + g[k].z * hr[2] + g[k].w * hr[3];
+                    *reinterpret_cast<float4*>(hr) = g[k];
+                }
+            }
+        }
     }
     gk = block_sum(gk, red2);
     __syncthreads();

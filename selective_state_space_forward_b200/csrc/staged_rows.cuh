@@ -22,21 +22,80 @@ __device__ inline void chunk_segments(const int32_t* seq_row, int t0, int Lc, in
     __syncthreads();
 }
 
-// Load token rows [t0, t0+64) of the head's x (fp32 result, zero past the end).
+// Eight consecutive values as floats: two 16-byte loads (fp32) or one (bf16) when
+// the address is 16-byte aligned, else element by element.
+__device__ __forceinline__ void ld8(const float* p, bool vec, float (&v)[8])
+{
+    if (vec) {
+        const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; e++) v[e] = p[e];
+    }
+}
+__device__ __forceinline__ void ld8(const bf16* p, bool vec, float (&v)[8])
+{
+    if (vec) {
+        load8(p, v);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; e++) v[e] = __bfloat162float(p[e]);
+    }
+}
+__device__ __forceinline__ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Rows [t0, t0+64) of width W (a multiple of 8) from src (row r at src + r * ld_src)
+// into dst (row r at dst + r * ld_dst), zero past Lc.  Each task moves 8 values;
+// a thread issues the loads of two tasks before storing.  Loads and stores are
+// 16 bytes wide where both the base and the row stride keep 16-byte alignment.
+template <typename S>
+__device__ __forceinline__ void load_rows8(const S* src, int64_t ld_src, int W, int Lc, float* dst, int ld_dst,
+                                           int rows = kChunk)
+{
+    const int per = W / 8, ntask = rows * per;
+    const bool vec = aligned16(src) && (ld_src * (int64_t)sizeof(S)) % 16 == 0;
+    const bool vst = aligned16(dst) && ld_dst % 4 == 0;
+    for (int i0 = threadIdx.x; i0 < ntask; i0 += 2 * blockDim.x) {
+        float v[2][8];
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            const int i = i0 + k * blockDim.x;
+            const int r = i / per, c = (i % per) * 8;
+            if (i < ntask && r < Lc) {
+                ld8(src + r * ld_src + c, vec, v[k]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; e++) v[k][e] = 0.0f;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            const int i = i0 + k * blockDim.x;
+            if (i < ntask) {
+                float* d = dst + (i / per) * ld_dst + (i % per) * 8;
+                if (vst) {
+                    *reinterpret_cast<float4*>(d) = make_float4(v[k][0], v[k][1], v[k][2], v[k][3]);
+                    *reinterpret_cast<float4*>(d + 4) = make_float4(v[k][4], v[k][5], v[k][6], v[k][7]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; e++) d[e] = v[k][e];
+                }
+            }
+        }
+    }
+}
+
+// Load token rows [t0, t0+64) of the head's x (fp32 result, zero past the end);
+// ld is the destination row stride (a multiple of 4).
 template <typename T>
 __device__ void load_x_rows(const Shape& s, const FwdArgs& a, const float* u, int b, int h,
                             int t0, int Lc, float* xs, int ld)
 {
-    const int P = s.headdim, HP = s.nheads * P, cd = s.conv_dim();
-    for (int i = threadIdx.x; i < kChunk * P; i += blockDim.x) {
-        const int r = i / P, p = i % P;
-        float v = 0.0f;
-        if (r < Lc) {
-            const int64_t tok = (int64_t)b * s.seqlen + t0 + r;
-            v = u ? u[tok * cd + h * P + p] : to_f(((const T*)a.x)[tok * a.ld_x + h * P + p]);
-        }
-        xs[r * ld + p] = v;
-    }
+    const int P = s.headdim, cd = s.conv_dim();
+    const int64_t tok0 = (int64_t)b * s.seqlen + t0;
+    if (u) load_rows8(u + tok0 * cd + h * P, cd, P, Lc, xs, ld);
+    else load_rows8((const T*)a.x + tok0 * a.ld_x + h * P, a.ld_x, P, Lc, xs, ld);
 }
 
 // Load B (which = 0) or C (which = 1) rows of the head's group, then apply the
@@ -47,16 +106,9 @@ __device__ void load_bc_rows(const Shape& s, const FwdArgs& a, const float* u, i
 {
     const int N = s.dstate, GN = s.ngroups * N, HP = s.nheads * s.headdim, cd = s.conv_dim();
     const int g = h / (s.nheads / s.ngroups);
-    const T* raw = (const T*)(which ? a.C : a.B);
-    for (int i = threadIdx.x; i < kChunk * N; i += blockDim.x) {
-        const int r = i / N, n = i % N;
-        float v = 0.0f;
-        if (r < Lc) {
-            const int64_t tok = (int64_t)b * s.seqlen + t0 + r;
-            v = u ? u[tok * cd + HP + which * GN + g * N + n] : to_f(raw[tok * a.ld_bc + g * N + n]);
-        }
-        dst[r * ld + n] = v;
-    }
+    const int64_t tok0 = (int64_t)b * s.seqlen + t0;
+    if (u) load_rows8(u + tok0 * cd + HP + which * GN + g * N, cd, N, Lc, dst, ld);
+    else load_rows8((const T*)(which ? a.C : a.B) + tok0 * a.ld_bc + g * N, a.ld_bc, N, Lc, dst, ld);
     if (!s.bc_norm) return;
     __syncthreads();
     const float* wn = which ? a.cn_w : a.bn_w;
