@@ -435,22 +435,44 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
         gdv[tid] += red[tid] * expf(ac[last] - ac[tid]);
     }
     __syncthreads();
+    if (tid < kChunk) {
+        // gl = sum_r red[r] ws[r] (ws is zero past the chunk's end): per warp, then in order
+        float gl = red[tid] * ws[tid];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gl += __shfl_xor_sync(0xffffffffu, gl, o);
+        if ((tid & 31) == 0) red2[1 + (tid >> 5)] = gl;
+    }
+    __syncthreads();
     if (tid == 0) {
-        float gl = 0.0f;
-        for (int r = 0; r < Lc; r++) gl += red[r] * ws[r];
+        float gl = red2[1] + red2[2];
         const float kc = w.cdecay[bh * nc + c];
         if (kc != kChunkReset) gl += gk * kc;         // k_c = exp(acs_last)
         gac[last] += gl;
     }
     __syncthreads();
 
-    // dA = dt a feeds acs through the segmented in-chunk cumsum: gdA is its reverse
+    // dA = dt a feeds acs through the segmented in-chunk cumsum: gdA is its reverse,
+    // a suffix sum within each segment (warps 0 and 1, 32 tokens each, by shuffles;
+    // segment ids never decrease along the chunk, so equal ids mean one run)
+    if (tid < kChunk) {
+        const int j = tid, lane = tid & 31;
+        float v = j < Lc ? gac[j] : 0.0f;
+        const int sj = seg[j];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float vo = __shfl_down_sync(0xffffffffu, v, o);
+            const int so = __shfl_down_sync(0xffffffffu, sj, o);
+            if (lane + o < 32 && so == sj) v += vo;
+        }
+        if (j == 32) red2[0] = v;                     // suffix of the second half
+        red[j] = v;
+    }
+    __syncthreads();
     if (tid < kChunk) {
         float gv = 0.0f, ga = 0.0f;
         if (tid < Lc) {
             const int j = tid;
-            float gda = 0.0f;
-            for (int t = j; t < Lc && seg[t] == seg[j]; t++) gda += gac[t];
+            const float gda = red[j] + ((j < 32 && Lc > 32 && seg[32] == seg[j]) ? red2[0] : 0.0f);
             const int64_t tok = (int64_t)b * L + t0 + j;
             const bool real = t0 + j < Lb;
             float av;
@@ -469,19 +491,23 @@ bwd_chunk_kernel(Shape s, FwdArgs a, BwdBufs w)
             w.gdt_raw[tok * H + h] = gv;
             if (s.a_per_token && w.gA) w.gA[tok * H + h] = ga;
         }
-        red[tid] = gv;
-        gm[tid] = ga;
+        // per-chunk sums of the dt_bias and A gradients: each warp in a fixed order,
+        // then warp 0's before warp 1's
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gv += __shfl_xor_sync(0xffffffffu, gv, o);
+            ga += __shfl_xor_sync(0xffffffffu, ga, o);
+        }
+        if ((tid & 31) == 0) {
+            red2[3 + (tid >> 5)] = gv;
+            red2[5 + (tid >> 5)] = ga;
+        }
     }
     __syncthreads();
     if (tid == 0) {
-        float sdt = 0.0f, sa = 0.0f;
-        for (int j = 0; j < Lc; j++) {
-            sdt += red[j];
-            sa += gm[j];
-        }
         const int64_t pi = ((int64_t)b * nc + c) * H + h;
-        w.p_dtb[pi] = sdt;
-        w.p_A[pi] = sa;
+        w.p_dtb[pi] = red2[3] + red2[4];
+        w.p_A[pi] = red2[5] + red2[6];
         w.p_D[pi] = dpart;
     }
 }

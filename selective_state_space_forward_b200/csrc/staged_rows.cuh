@@ -9,15 +9,18 @@ namespace ssd {
 
 // Chunk-local segment ids: seg[t] = boundaries at positions t0 .. t0+t (padding
 // positions, at or after the row length Lb, hold none).
+// The inclusive prefix count runs on warps 0 and 1 by ballots.
 __device__ inline void chunk_segments(const int32_t* seq_row, int t0, int Lc, int Lb, int* seg, int* flag)
 {
     const int tid = threadIdx.x;
     if (tid < kChunk) flag[tid] = (tid < Lc && t0 + tid < Lb) ? is_boundary(seq_row, t0 + tid) : 0;
     __syncthreads();
     if (tid < kChunk) {
-        int acc = 0;
-        for (int j = 0; j <= tid; j++) acc += flag[j];
-        seg[tid] = acc;
+        const int lane = tid & 31;
+        const uint32_t m0 = __ballot_sync(0xffffffffu, flag[lane] != 0);
+        const uint32_t m1 = __ballot_sync(0xffffffffu, flag[32 + lane] != 0);
+        const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
+        seg[tid] = tid < 32 ? __popc(m0 & le) : __popc(m0) + __popc(m1 & le);
     }
     __syncthreads();
 }
