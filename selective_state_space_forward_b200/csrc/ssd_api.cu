@@ -66,6 +66,10 @@ struct ssd_handle {
     cudaEvent_t ev_start, ev_stop;   // measurement hook (caller-owned), or null
     uint64_t launches;               // kernels launched since ssd_create
     FusedWork fw;                    // fused path: segment hand-off buffers, epoch, SM count
+    // fused path: K2 runs on an auxiliary stream beside K1, forked from and joined
+    // back into the caller's stream with events
+    cudaStream_t aux;
+    cudaEvent_t ev_fork, ev_join;
 };
 
 namespace {
@@ -361,9 +365,19 @@ static ssd_status forward_impl(ssd_handle* h, int32_t batch, int32_t seqlen, con
         SSD_MAIN_LAUNCH(h, st, launch_chunk_output(s, a, h->u, h->dt, h->acs, h->states, st),
                         "chunk-output kernel");
     } else {
+        // K2 depends on nothing K1 writes: it runs on the auxiliary stream, which
+        // starts after everything already on the caller's stream (so the last call's
+        // fused kernel has read dt and acs) and which the caller's stream waits for
+        // before the fused kernel.  (The final conv history stays after the fused
+        // kernel: with the state updated in place it overwrites the history K1 and
+        // the fused kernel read.)
+        SSD_CUDA(cudaEventRecord(h->ev_fork, st), "cudaEventRecord(fork)");
+        SSD_CUDA(cudaStreamWaitEvent(h->aux, h->ev_fork, 0), "cudaStreamWaitEvent(fork)");
+        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, nullptr, h->aux), "dt/cumsum kernel");
+        SSD_CUDA(cudaEventRecord(h->ev_join, h->aux), "cudaEventRecord(join)");
         if (s.dconv == 4) SSD_LAUNCH(h, launch_conv_silu_bc(s, a, h->ubc, st), "B|C conv kernel");
-        SSD_LAUNCH(h, launch_dt_cumsum(s, a, h->dt, h->acs, nullptr, st), "dt/cumsum kernel");
         if (s.bc_norm) SSD_LAUNCH(h, launch_bc_rms(s, a, h->ubc, h->rinv, st), "B/C rms kernel");
+        SSD_CUDA(cudaStreamWaitEvent(st, h->ev_join, 0), "cudaStreamWaitEvent(join)");
         if (++h->fw.epoch == 0) h->fw.epoch = 1;      // flags hold the last call's epoch
         SSD_MAIN_LAUNCH(h, st,
                         launch_chunk_fused(s, a, h->ubc, h->dt, h->acs, h->rinv, h->status, h->fw, st),
@@ -468,6 +482,14 @@ ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
         delete h;
         return cuda_fail(e, "cudaMalloc(workspace)");
     }
+    e = cudaStreamCreateWithFlags(&h->aux, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+        cudaFree(h->ws);
+        delete h;
+        return cuda_fail(e, "cudaStreamCreate / cudaEventCreate");
+    }
     h->ws_bytes = off;
     h->u = (path == SSD_PATH_STAGED && dd.dconv == 4) ? (float*)(h->ws + o_u) : nullptr;
     h->dt = (float*)(h->ws + o_dt);
@@ -493,6 +515,12 @@ ssd_status ssd_create(const ssd_desc* d, ssd_handle** out)
 void ssd_destroy(ssd_handle* h)
 {
     if (!h) return;
+    if (h->aux) {
+        cudaStreamSynchronize(h->aux);
+        cudaStreamDestroy(h->aux);
+    }
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
     cudaFree(h->ws);
     delete h;
 }
