@@ -34,6 +34,12 @@
  *    pointers 4-byte aligned.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream).  A handle serves one stream at a time.
+ *  - Calls may be captured into a CUDA graph (stream capture).  A graph
+ *    replays every call with the argument values and the handle workspace of
+ *    its capture, so replays of a graph must not overlap on the GPU with
+ *    each other or with other calls on the same handle.  A captured fused
+ *    forward clears its segment hand-off flags inside the graph, so every
+ *    replay waits for its own hand-offs.
  *  - Arguments are validated on the host before anything is launched: a call
  *    that returns an error status launched nothing and touched no memory.
  *    ssd_last_error() then names the offending argument (the calling thread's

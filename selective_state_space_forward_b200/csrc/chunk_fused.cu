@@ -1099,6 +1099,17 @@ static cudaError_t launch_t(const Shape& s, FusedParams fp, const CUtensorMap* m
     choose_segments(streams, nc, grid, cap, fp.nseg, fp.cps);
     fp.nitems = streams * fp.nseg;
     if (grid > fp.nitems) grid = fp.nitems;
+    // A launch captured into a CUDA graph keeps this call's epoch for every
+    // replay, so the flags the previous replay published would already read
+    // "ready".  Captured, the flag words are cleared in the graph itself, just
+    // ahead of the kernel (zero is never an epoch).
+    cudaStreamCaptureStatus cap_status = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(st, &cap_status);
+    if (e != cudaSuccess) return e;
+    if (cap_status != cudaStreamCaptureStatusNone) {
+        e = cudaMemsetAsync(fp.flags, 0, (size_t)fp.nitems * sizeof(unsigned), st);
+        if (e != cudaSuccess) return e;
+    }
     // A cooperative launch makes co-residency of the whole grid a condition of
     // the launch: on a GPU shared with other work (another stream's kernels, a
     // reduced SM partition) it is refused with an error instead of starting CTAs
