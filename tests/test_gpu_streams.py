@@ -26,10 +26,9 @@ from selective_state_space_forward_b200.synthetic import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-# More (row, head) streams than the grid has CTAs (296 at dstate 64, two per
-# SM; 148 at dstate 128): the fused kernel then splits every stream into
-# several segments to balance the last round of items, so the hand-off flags
-# are in use.
+# More (row, head) streams than the persistent grid has CTAs (one per SM): the
+# fused kernel then splits every stream into several segments to balance the
+# last round of items, so the hand-off flags are in use.
 CASES = {
     "mini_k3_mixer": WORKLOADS["mini_k3_mixer"].with_(batch=10, seqlen=700, mean_doc_len=300),
     "mamba3_siso": WORKLOADS["mamba3_siso"].with_(batch=4, seqlen=900),
