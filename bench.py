@@ -456,6 +456,22 @@ def bench_decode(args, torch, peaks):
     times = sorted(a_.elapsed_time(b_) for a_, b_ in ev)
     med_ms = times[len(times) // 2]
     state_b = w.batch * w.nheads * w.headdim * w.dstate * 4
+    # Size-matched reference: torch's own copy of a buffer the size of the fp32
+    # state (the same bytes read and written as the state update), L2 evicted
+    # the same way.  At this size a copy does not reach the long-copy peak.
+    src = torch.rand(state_b // 4, device="cuda")
+    dst = torch.empty_like(src)
+    cev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(64)]
+    for a_, b_ in cev:
+        flush_sum = flush.sum(dtype=torch.int64)
+        a_.record(stream)
+        dst.copy_(src)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    del flush_sum, src, dst
+    ctimes = sorted(a_.elapsed_time(b_) for a_, b_ in cev)
+    copy_gbs = 2 * state_b / (ctimes[len(ctimes) // 2] * 1e-3) / 1e9
     conv_b = w.batch * 3 * w.conv_dim * 2
     io_b = w.batch * (3 * w.nheads * w.headdim * 2 + 2 * w.ngroups * w.dstate * 2 + w.nheads * 4)
     total = 2 * state_b + 2 * conv_b + io_b
@@ -465,6 +481,9 @@ def bench_decode(args, torch, peaks):
             "us_per_step_median": round(med_ms * 1e3, 2), "bytes_per_step": total,
             "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
             "peak_source": peaks["source"], "steps_timed": n, "l2": "evicted before each step by reading a 256 MB buffer",
+            "copy_reference": {"what": "torch copy of a buffer the size of the fp32 state, L2 evicted the same way",
+                               "bytes": 2 * state_b, "gbs": round(copy_gbs, 1),
+                               "decode_frac_of_it": round(gbs / copy_gbs, 4)},
             "traffic": measured_traffic(f"decode:{DECODE_WORKLOAD}", "decode")}
 
 

@@ -103,7 +103,7 @@ __device__ void decode_prologue(const Shape& s, const FwdArgs& a, T* hist, float
 }
 
 struct DecodeSmem {
-    float *ux, *ub, *uc, *dts, *dec, *bh, *ch;
+    float *ux, *ub, *uc, *dts, *dec, *bh, *ch, *gz, *ys;
     __device__ DecodeSmem(float* sm, const Shape& s)
     {
         const int hpg = s.nheads / s.ngroups;
@@ -115,8 +115,16 @@ struct DecodeSmem {
         dec = dts + hp4;
         bh = dec + hp4;
         ch = bh + (s.bc_norm ? hpg * s.dstate : 0);
+        gz = ch + (s.bc_norm ? hpg * s.dstate : 0);   // SiLU(z) of the block's rows
+        ys = gz + hpg * s.headdim;                     // C . h of the block's rows
     }
 };
+__host__ __device__ inline size_t decode_smem_floats(int hpg, int P, int N, bool bc_norm)
+{
+    const size_t hp4 = (size_t)((hpg + 3) & ~3);
+    return (size_t)hpg * P + 2 * (size_t)N + 2 * hp4 + (bc_norm ? 2 * (size_t)hpg * N : 0) +
+           2 * (size_t)hpg * P;
+}
 
 // Main kernel: N = 32 * NV.  Lane l8 of a row owns float4 q at floats
 // (q * 8 + l8) * 4 .. +3, so the 8 lanes of a row cover 32 consecutive floats
@@ -131,6 +139,9 @@ decode_step_vec(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ his
     const int g = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     DecodeSmem sv(sm, s);
+    // SiLU(z) of the block's rows, so the row loop's output needs no global load
+    for (int i = threadIdx.x; i < hpg * P; i += blockDim.x)
+        sv.gz[i] = silu_f(to_f(((const T*)a.z)[(int64_t)b * HP + (int64_t)g * hpg * P + i]));
     decode_prologue<T>(s, a, hist, sv.ux, sv.ub, sv.uc, sv.dts, sv.dec, sv.bh, sv.ch, g, b);
 
     const int sub = lane >> 3, l8 = lane & 7;
@@ -184,14 +195,16 @@ decode_step_vec(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ his
         y += __shfl_xor_sync(0xffffffffu, y, 1);
         y += __shfl_xor_sync(0xffffffffu, y, 2);
         y += __shfl_xor_sync(0xffffffffu, y, 4);
-        if (valid && l8 == 0) {
-            const int hh = g * hpg + hl, p = r % P;
-            const int64_t o = (int64_t)b * HP + hh * P + p;
-            const float zv = to_f(((const T*)a.z)[o]);
-            ((T*)a.out)[o] = from_f<T>((y + a.D[hh] * sv.ux[r]) * silu_f(zv));
-        }
+        if (valid && l8 == 0) sv.ys[r] = y;
 #pragma unroll
         for (int q = 0; q < NV; q++) cur[q] = nxt[q];
+    }
+    __syncthreads();
+    // the block's outputs, one coalesced row of hpg * P values
+    for (int i = threadIdx.x; i < nrows; i += blockDim.x) {
+        const int hh = g * hpg + i / P;
+        ((T*)a.out)[(int64_t)b * HP + (int64_t)g * hpg * P + i] =
+            from_f<T>((sv.ys[i] + a.D[hh] * sv.ux[i]) * sv.gz[i]);
     }
 }
 
@@ -235,9 +248,7 @@ static cudaError_t launch_decode_t(const Shape& s, const FwdArgs& a, float* ssm,
                                    cudaStream_t st)
 {
     const int hpg = s.nheads / s.ngroups;
-    const size_t hp4 = (size_t)((hpg + 3) & ~3);
-    const size_t smem = sizeof(float) * ((size_t)hpg * s.headdim + 2 * s.dstate + 2 * hp4 +
-                                         (s.bc_norm ? 2 * (size_t)hpg * s.dstate : 0));
+    const size_t smem = sizeof(float) * decode_smem_floats(hpg, s.headdim, s.dstate, s.bc_norm);
     const dim3 grid(s.ngroups, s.batch);
     void (*kern)(Shape, FwdArgs, float*, T*);
     switch (s.dstate) {

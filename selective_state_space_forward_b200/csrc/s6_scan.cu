@@ -6,8 +6,9 @@
 //   h[n] <- exp(dt_t A[d,n]) h[n] + dt_t u_t B_t[n];   y_t = C_t . h + D[d] u_t
 //   out_t = y_t SiLU(z_t)   (no z: y_t)
 //
-// A is diagonal, so channels never mix.  A block of 128 threads takes 32
-// channels of one row; the 4 lanes of a quartet share a channel and each keeps
+// A is diagonal, so channels never mix.  A block of 64 threads takes 16
+// channels of one row (up to 8 blocks per SM, so the blocks of a row spread
+// evenly over the SMs); the 4 lanes of a quartet share a channel and each keeps
 // N/4 of its states and decay rates (pre-scaled by log2 e) in registers.  The
 // row is walked in chunks of 32 tokens:
 //   stage   every thread turns its share of the chunk's (token, channel) inputs
@@ -21,15 +22,17 @@
 //   write   the chunk's outputs leave as coalesced rows of the block's channels.
 // The next chunk's raw inputs (u, delta, z, B, C rows) are copied into shared
 // memory with cp.async before the scan starts (into registers when the rows are
-// not 16-byte aligned), so their memory latency overlaps the scan.  The bound is
+// not 16-byte aligned), so their memory latency overlaps the scan; the copies
+// are issued kind by kind, so each piece's row and column follow from
+// compile-time piece counts.  The bound is
 // the N exponentials per (token, channel) on the MUFU pipe.
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
 
 namespace ssd {
 
-constexpr int kS6Threads = 128;
-constexpr int kS6Ch = 32;                         // channels per block
+constexpr int kS6Threads = 64;
+constexpr int kS6Ch = 16;                         // channels per block
 constexpr int kS6Lanes = 4;                       // lanes per channel
 constexpr int kS6Group = 4;                       // tokens per unrolled scan group
 // tokens per chunk: 32 (the next chunk's raw inputs wait in registers)
@@ -90,7 +93,7 @@ __device__ __forceinline__ void s6_cp_commit() { asm volatile("cp.async.commit_g
 __device__ __forceinline__ void s6_cp_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 template <typename T, int N, bool ASYNC>
-__global__ void __launch_bounds__(kS6Threads, 4)
+__global__ void __launch_bounds__(kS6Threads, 8)
 s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* __restrict__ delta,
                const float* __restrict__ delta_bias, const float* __restrict__ A_log,
                const T* __restrict__ Bm, const T* __restrict__ Cm, const float* __restrict__ D,
@@ -159,31 +162,26 @@ s6_scan_kernel(int batch, int L, int DI, const T* __restrict__ u, const float* _
         constexpr int kPu = kS6Ch * (int)sizeof(T) / 16;        // 16-byte pieces per token row of u, z
         constexpr int kPd = kS6Ch * 4 / 16;                     // of delta
         constexpr int kPb = N * (int)sizeof(T) / 16;            // of B, C
-        constexpr int kTask = kS6T * (2 * kPu + kPd + 2 * kPb);
-        for (int i = tid; i < kTask; i += kS6Threads) {
-            int j = i;
-            const int which = j < kS6T * kPu ? 0 : (j -= kS6T * kPu) < kS6T * kPu ? 1
-                            : (j -= kS6T * kPu) < kS6T * kPd ? 2 : (j -= kS6T * kPd) < kS6T * kPb ? 3
-                            : (j -= kS6T * kPb, 4);
-            const int per = which < 2 ? kPu : which == 2 ? kPd : kPb;
-            const int r = j / per, piece = j % per;
-            const int t = t0 + r;
-            const bool tok_ok = t < L;
-            const int64_t trow = (int64_t)b * L + (tok_ok ? t : 0);
-            if (which <= 2) {
-                const int elems = which < 2 ? 16 / (int)sizeof(T) : 4;
-                const int c0 = d0 + piece * elems;
-                const bool ok = tok_ok && c0 < DI;
-                const int64_t o = trow * DI + (ok ? c0 : 0);
-                if (which == 0) s6_cp16(&raw_u[r][piece * elems], u + o, ok ? 16 : 0);
-                else if (which == 1) s6_cp16(&raw_z[r][piece * elems], (z ? z : u) + o, ok && z ? 16 : 0);
-                else s6_cp16(&raw_d[r][piece * elems], delta + o, ok ? 16 : 0);
-            } else {
-                const int elems = 16 / (int)sizeof(T);
-                const int64_t o = trow * N + piece * elems;
-                s6_cp16(which == 3 ? &raw_b[r][piece * elems] : &raw_c[r][piece * elems],
-                        (which == 3 ? Bm : Cm) + o, tok_ok ? 16 : 0);
-            }
+        constexpr int kEu = 16 / (int)sizeof(T);                // elements per piece of u, z, B, C
+        for (int i = tid; i < kS6T * kPu; i += kS6Threads) {
+            const int r = i / kPu, piece = i % kPu, t = t0 + r, c0 = d0 + piece * kEu;
+            const bool ok = t < L && c0 < DI;
+            const int64_t o = ok ? ((int64_t)b * L + t) * DI + c0 : 0;
+            s6_cp16(&raw_u[r][piece * kEu], u + o, ok ? 16 : 0);
+            s6_cp16(&raw_z[r][piece * kEu], (z ? z : u) + o, ok && z ? 16 : 0);
+        }
+        for (int i = tid; i < kS6T * kPd; i += kS6Threads) {
+            const int r = i / kPd, piece = i % kPd, t = t0 + r, c0 = d0 + piece * 4;
+            const bool ok = t < L && c0 < DI;
+            const int64_t o = ok ? ((int64_t)b * L + t) * DI + c0 : 0;
+            s6_cp16(&raw_d[r][piece * 4], delta + o, ok ? 16 : 0);
+        }
+        for (int i = tid; i < kS6T * kPb; i += kS6Threads) {
+            const int r = i / kPb, piece = i % kPb, t = t0 + r;
+            const bool ok = t < L;
+            const int64_t o = ok ? ((int64_t)b * L + t) * N + piece * kEu : 0;
+            s6_cp16(&raw_b[r][piece * kEu], Bm + o, ok ? 16 : 0);
+            s6_cp16(&raw_c[r][piece * kEu], Cm + o, ok ? 16 : 0);
         }
         s6_cp_commit();
     };
