@@ -81,8 +81,14 @@ typedef enum { SSD_A_PER_HEAD = 0, SSD_A_PER_TOKEN = 1 } ssd_a_mode;
  *          d_state 64 or 128.  With bc_norm, each head's normalised B and C
  *          tiles are built in shared memory and never written to memory.
  *  STAGED: the five-stage pipeline conv -> dt/cumsum -> chunk states ->
- *          state passing -> chunk outputs, fp32 arithmetic throughout; any
- *          supported shape and both dtypes.
+ *          state passing -> chunk outputs, fp32 accumulation throughout (the
+ *          chunk-state and chunk-output contractions on the tensor cores with
+ *          tf32 operands for bf16 activations, as fp32 products for fp32
+ *          activations); any supported shape and both dtypes.  It writes
+ *          every chunk state to memory and reads it back, so it is several
+ *          times slower than FUSED on the shapes both serve (about 4.7x on a
+ *          32-head, d_state 64 layer; 6x at d_state 128): read ssd_get_path
+ *          after ssd_create when throughput matters.
  *  AUTO  : FUSED when the shape and dtype allow it, else STAGED. */
 typedef enum { SSD_PATH_AUTO = 0, SSD_PATH_FUSED = 1, SSD_PATH_STAGED = 2 } ssd_path;
 

@@ -1,5 +1,7 @@
 // chunk_staged.cu -- the staged path's K3 (chunk states), K4 (state passing)
-// and K5 (chunk outputs), in fp32 arithmetic.
+// and K5 (chunk outputs): fp32 accumulation throughout; the contractions of K3
+// and K5 run on the tensor cores (tf32 operands) for bf16 activations and as
+// register-tiled fp32 products for fp32 activations.
 //
 // The chunked evaluation of the selective scan (chunk 64; mojolearn
 // Mamba3Block, "chunk size 64"): within a chunk c of tokens t0 .. t0+Lc-1,
@@ -120,6 +122,12 @@ state_passing_kernel(Shape s, const float* __restrict__ cdecay, float* __restric
     if (fin) fin[gid] = hv;
 }
 
+// Per (chunk, head): the three contractions of the chunk output go through the
+// per-dtype product engine (tf32 tensor-core tiles for bf16 activations,
+// register-tiled fp32 for fp32), 64 x 64 output blocks:
+//   (C_t . B_s) on the causal same-segment mask, times exp(acs_t - acs_s);
+//   sum_s [that] dt_s x_s[p]           (dt_s scales the reduction index);
+//   C_t . Hin_c[p, :]                  (Hin_c takes B's tile once C B^T is done).
 template <typename T>
 __global__ void __launch_bounds__(256)
 chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float* __restrict__ dt,
@@ -127,19 +135,18 @@ chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float
 {
     extern __shared__ float sm[];
     const int P = s.headdim, N = s.dstate, H = s.nheads, L = s.seqlen, nc = s.nchunks();
-    const int HP = H * P;
+    const int HP = H * P, NB = N + kPad, XS = P + kPad;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk, Lc = min(kChunk, L - t0);
-    const int NB = N + 1;              // padded row stride (bank spread)
-    float* cs = sm;                    // [64][N]
-    float* bs = cs + kChunk * N;       // [64][N+1]
-    float* xs = bs + kChunk * NB;      // [64][P]
-    float* hs = xs + kChunk * P;       // [P][N+1]
-    float* cb = hs + P * NB;           // [64][65]
-    float* ac = cb + kChunk * 65;      // [64]
-    float* dv = ac + kChunk;           // [64]
-    int* seg = (int*)(dv + kChunk);    // [64]
-    int* flag = seg + kChunk;          // [64]
+    float* cs = sm;                             // [64][NB]          C
+    float* bs = cs + kChunk * NB;               // [max(64, P)][NB]  B, then Hin_c ([P][NB])
+    float* xs = bs + max(kChunk, P) * NB;       // [64][XS]          x
+    float* cbe = xs + kChunk * XS;              // [64][kMS]         (C_t . B_s) E[t,s] on the mask
+    float* ac = cbe + kChunk * kMS;             // [64]
+    float* dv = ac + kChunk;                    // [64]
+    float* ft = dv + kChunk;                    // [64] weight of the carried-state term
+    int* seg = (int*)(ft + kChunk);             // [64]
+    int* flag = seg + kChunk;                   // [64]
 
     const int Lb = row_length(a.lengths, b, L);
     chunk_segments(a.seq_idx ? a.seq_idx + (int64_t)b * L : nullptr, t0, Lc, Lb, seg, flag);
@@ -149,44 +156,56 @@ chunk_output_kernel(Shape s, FwdArgs a, const float* __restrict__ u, const float
         ac[r] = r < Lc ? acs[o] : 0.0f;
         dv[r] = r < Lc ? dt[o] : 0.0f;
     }
-    load_x_rows<T>(s, a, u, b, h, t0, Lc, xs, P);
-    load_bc_rows<T>(s, a, u, b, h, t0, Lc, 1, cs, N);
+    load_x_rows<T>(s, a, u, b, h, t0, Lc, xs, XS);
+    load_bc_rows<T>(s, a, u, b, h, t0, Lc, 1, cs, NB);
     load_bc_rows<T>(s, a, u, b, h, t0, Lc, 0, bs, NB);
-    const float* hp = hin + (((int64_t)b * nc + c) * H + h) * P * N;
-    for (int e = threadIdx.x; e < P * N; e += blockDim.x) hs[(e / N) * NB + e % N] = hp[e];
     __syncthreads();
-
-    for (int e = threadIdx.x; e < kChunk * kChunk; e += blockDim.x) {
-        const int t = e / kChunk, r = e % kChunk;
-        float v = 0.0f;
-        if (r <= t && t < Lc && seg[r] == seg[t]) {
-            float dot = 0.0f;
-            for (int n = 0; n < N; n++) dot += cs[t * N + n] * bs[r * NB + n];
-            v = dot * expf(ac[t] - ac[r]) * dv[r];
-        }
-        cb[t * 65 + r] = v;
+    if (threadIdx.x < kChunk) {
+        const int r = threadIdx.x;
+        ft[r] = (r < Lc && seg[r] == 0) ? expf(ac[r]) : 0.0f;
     }
+
+    const Prod<T, 4> p4(threadIdx.x);
+    {
+        float acc[4][4];
+        tile_zero(acc);
+        p4.mm(acc, cs, NB, 1, kChunk, bs, 1, NB, kChunk, N);
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int t = p4.row(rr, cc), r = p4.col(rr, cc);
+                cbe[t * kMS + r] = (r <= t && t < Lc && seg[r] == seg[t]) ? acc[rr][cc] * expf(ac[t] - ac[r]) : 0.0f;
+            }
+    }
+    __syncthreads();                            // B's tile has been read
+    load_rows8(hin + (((int64_t)b * nc + c) * H + h) * P * N, N, N, P, bs, NB, P);
     __syncthreads();
 
     const float Dh = a.D[h];
-    for (int e = threadIdx.x; e < kChunk * P; e += blockDim.x) {
-        const int t = e / P, p = e % P;
-        if (t >= Lc) continue;
-        if (t0 + t >= Lb) {   // padding of a ragged row
-            ((T*)a.out)[((int64_t)b * L + t0 + t) * HP + h * P + p] = from_f<T>(0.0f);
-            continue;
-        }
-        float y = 0.0f;
-        for (int r = 0; r <= t; r++) y += cb[t * 65 + r] * xs[r * P + p];
-        if (seg[t] == 0) {
-            float off = 0.0f;
-            for (int n = 0; n < N; n++) off += cs[t * N + n] * hs[p * NB + n];
-            y += expf(ac[t]) * off;
-        }
-        y += Dh * xs[t * P + p];
-        const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
-        const float zv = to_f(((const T*)a.z)[((int64_t)b * L + t0 + t) * a.ld_z + h * P + p]);
-        ((T*)a.out)[o] = from_f<T>(y * silu_f(zv));
+    for (int p0 = 0; p0 < P; p0 += 64) {
+        float ys[4][4], off[4][4];
+        tile_zero(ys);
+        tile_zero(off);
+        p4.mm(ys, cbe, kMS, 1, kChunk, xs + p0, XS, 1, P - p0, kChunk, dv);   // sum_s M[t,s] x_s
+        p4.mm(off, cs, NB, 1, kChunk, bs + p0 * NB, 1, NB, P - p0, N);        // C_t . Hin[p]
+#pragma unroll
+        for (int rr = 0; rr < 4; rr++)
+#pragma unroll
+            for (int cc = 0; cc < 4; cc++) {
+                const int t = p4.row(rr, cc), p = p0 + p4.col(rr, cc);
+                if (t >= Lc || p >= P) continue;
+                const int64_t o = ((int64_t)b * L + t0 + t) * HP + h * P + p;
+                if (t0 + t >= Lb) {   // padding of a ragged row
+                    ((T*)a.out)[o] = from_f<T>(0.0f);
+                    continue;
+                }
+                float y = ys[rr][cc];
+                if (seg[t] == 0) y += ft[t] * off[rr][cc];
+                y += Dh * xs[t * XS + p];
+                const float zv = to_f(((const T*)a.z)[((int64_t)b * L + t0 + t) * a.ld_z + h * P + p]);
+                ((T*)a.out)[o] = from_f<T>(y * silu_f(zv));
+            }
     }
 }
 
@@ -198,9 +217,10 @@ size_t chunk_state_smem_bytes(const Shape& s)
 
 size_t chunk_output_smem_bytes(const Shape& s)
 {
-    const size_t N = s.dstate, P = s.headdim;
-    return sizeof(float) * (kChunk * N + kChunk * (N + 1) + kChunk * P + P * (N + 1) +
-                            kChunk * 65 + 2 * kChunk) + sizeof(int) * 2 * kChunk;
+    const size_t N = s.dstate, P = s.headdim, NB = N + kPad, XS = P + kPad;
+    const size_t rows_b = P > (size_t)kChunk ? P : (size_t)kChunk;
+    return sizeof(float) * (kChunk * NB + rows_b * NB + kChunk * XS + kChunk * kMS + 3 * kChunk) +
+           sizeof(int) * 2 * kChunk;
 }
 
 cudaError_t launch_chunk_state(const Shape& s, const FwdArgs& a, const float* u,
