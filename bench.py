@@ -125,7 +125,7 @@ def kernel_source_hash(path_kind: str) -> str:
     """Hash of the sources that make up the dominant kernel of a path."""
     files = {"fused": ["chunk_fused.cu", "ssd_device.cuh", "tc05.cuh"],
              "staged": ["chunk_staged.cu", "staged_rows.cuh", "ssd_device.cuh"],
-             "decode": ["decode.cu", "ssd_device.cuh"]}[path_kind]
+             "decode": ["decode.cu", "ssd_device.cuh", "tc05.cuh"]}[path_kind]
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, "selective_state_space_forward_b200", "csrc", f), "rb") as fh:

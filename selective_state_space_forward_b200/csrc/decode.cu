@@ -11,16 +11,22 @@
 // One block per (row, B/C group): the group's B|C conv channels and its heads'
 // x channels are convolved once, so each conv-history column has exactly one
 // reader/writer.  The state is 95% of the bytes and is read and written once:
-// in the main kernel 8 lanes share a state row (each lane a float4 per 32
-// floats of the row, so a row is read in full 128-byte pieces), a warp walks 4
-// rows at a time, the next rows' loads are issued before the current rows are
-// computed, and the row's C.h sum is reduced over its 8 lanes.
+// the block's state is one contiguous run, moved through shared memory by 1-D
+// bulk copies (the first pieces requested before the conv prologue), updated
+// there in place with 8 lanes per row, and the row's C.h sum is reduced over
+// its 8 lanes.  d_state other than 32/64/128/256 takes a warp-per-row kernel.
 #include "ssd_device.cuh"
 #include "ssd_kernels.h"
+#include "tc05.cuh"
 
 namespace ssd {
 
 constexpr int kDecodeThreads = 128;
+// The bulk kernel moves the block's state through a ring of kDecRing pieces of
+// kDecPiece bytes in shared memory (16 KB: nine 128-thread blocks fit per SM,
+// as many as the registers allow).
+constexpr int kDecPiece = 8192;
+constexpr int kDecRing = 2;
 
 // Conv + SiLU of the new token, dt and decay per head, B/C norm: fills the
 // block's shared arrays ux[hpg*P], ub[N], uc[N], dts[hpg], dec[hpg] and, with
@@ -126,23 +132,67 @@ __host__ __device__ inline size_t decode_smem_floats(int hpg, int P, int N, bool
            2 * (size_t)hpg * P;
 }
 
-// Main kernel: N = 32 * NV.  Lane l8 of a row owns float4 q at floats
-// (q * 8 + l8) * 4 .. +3, so the 8 lanes of a row cover 32 consecutive floats
-// per q.
+// 1-D bulk copies (no tensor map): global -> shared completing on an mbarrier,
+// and shared -> global in a bulk group.  Addresses 16-byte aligned, sizes
+// multiples of 16.
+__device__ __forceinline__ void dec_bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void dec_bulk_store(void* dst, const void* src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst), "r"(tc::smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk kernel: N = 32 * NV.  The block's state (hpg * P rows of N fp32, one
+// contiguous run) goes through shared memory in pieces of kDecPiece bytes:
+// thread 0 requests the first kDecRing pieces before the conv prologue, so
+// their DRAM latency overlaps it; every piece is updated in place by the
+// block (8 lanes per row, lane l8 owning float4 q at (q * 8 + l8) * 4, so the
+// 8 lanes cover 32 consecutive floats per q) and written back by one bulk
+// store, and its slot is
+// refilled once that store has read it.  Every wait is bounded: on timeout the
+// block raises kStatusTimeout, stops updating, lets its copies land and exits.
 template <typename T, int NV>
 __global__ void __launch_bounds__(kDecodeThreads)
-decode_step_vec(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ hist)
+decode_step_bulk(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ hist, int* status,
+                 uint64_t wait_ns)
 {
-    extern __shared__ float sm[];
-    const int H = s.nheads, P = s.headdim, N = s.dstate;
-    const int hpg = H / s.ngroups, HP = H * P;
+    extern __shared__ __align__(128) float sm[];
+    constexpr int N = 32 * NV;
+    constexpr int kRows = kDecPiece / (N * 4);      // state rows per piece
+    static_assert(kRows >= 1, "a piece holds at least one state row");
+    const int H = s.nheads, P = s.headdim;
+    const int hpg = H / s.ngroups;
     const int g = blockIdx.x, b = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    DecodeSmem sv(sm, s);
-    // SiLU(z) of the block's rows, so the row loop's output needs no global load
-    for (int i = threadIdx.x; i < hpg * P; i += blockDim.x)
-        sv.gz[i] = silu_f(to_f(((const T*)a.z)[(int64_t)b * HP + (int64_t)g * hpg * P + i]));
-    decode_prologue<T>(s, a, hist, sv.ux, sv.ub, sv.uc, sv.dts, sv.dec, sv.bh, sv.ch, g, b);
+    float* ring = sm;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + kDecRing * kDecPiece / 4);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(full + kDecRing);
+    DecodeSmem sv(sm + kDecRing * kDecPiece / 4 + 4 * kDecRing, s);   // past the barriers and the flag
+    const int nrows = hpg * P;
+    const int npieces = (nrows + kRows - 1) / kRows;
+    float* base = ssm + ((int64_t)b * H + (int64_t)g * hpg) * P * N;
+    auto piece_bytes = [&](int k) { return (uint32_t)(min(kRows, nrows - k * kRows) * N * 4); };
+    auto issue_load = [&](int k) {
+        uint64_t* bar = &full[k % kDecRing];
+        tc::mbar_arrive_expect_tx(bar, piece_bytes(k));
+        dec_bulk_load(ring + (k % kDecRing) * (kDecPiece / 4), base + (int64_t)k * kRows * N, piece_bytes(k), bar);
+    };
+    if (threadIdx.x == 0) {
+        *s_abort = 0;
+        for (int i = 0; i < kDecRing; i++) tc::mbar_init(&full[i], 1);
+        tc::fence_mbar_init();
+        for (int k = 0; k < min(kDecRing, npieces); k++) issue_load(k);
+    }
+    // SiLU(z) of the block's rows, so the outputs need no global load
+    for (int i = threadIdx.x; i < nrows; i += blockDim.x)
+        sv.gz[i] = silu_f(to_f(((const T*)a.z)[(int64_t)b * H * P + (int64_t)g * hpg * P + i]));
+    decode_prologue<T>(s, a, hist, sv.ux, sv.ub, sv.uc, sv.dts, sv.dec, sv.bh, sv.ch, g, b);   // ends in a barrier
 
     const int sub = lane >> 3, l8 = lane & 7;
     float4 Bq[NV], Cq[NV];
@@ -153,57 +203,73 @@ decode_step_vec(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ his
             Cq[q] = *reinterpret_cast<const float4*>(sv.uc + (q * 8 + l8) * 4);
         }
     }
-    const int nrows = hpg * P;
-    const int step = nw * 4;
-    float* base = ssm + ((int64_t)b * H + (int64_t)g * hpg) * P * N;   // row r at base + r*N
-    auto load_row = [&](int r, float4 (&v)[NV]) {
-        if (r < nrows) {
+    int loaded = min(kDecRing, npieces);          // pieces requested so far (thread 0's count)
+    int k = 0;
+    for (; k < npieces; k++) {
+        float* slot = ring + (k % kDecRing) * (kDecPiece / 4);
+        // every thread waits on the piece; the block then leaves together if any gave up
+        const bool ok = tc::mbar_wait(&full[k % kDecRing], (uint32_t)(k / kDecRing) & 1u, s_abort, status,
+                                      kStatusTimeout, wait_ns);
+        if (__syncthreads_or(!ok)) break;
+        const int r0 = k * kRows, rows = min(kRows, nrows - r0);
+        // a warp takes 4 rows per pass (the loop test is the same for its 32 lanes)
+        for (int rr = warp * 4 + sub; rr - sub < rows; rr += nw * 4) {
+            const bool valid = rr < rows;
+            const int r = r0 + (valid ? rr : 0);
+            const int hl = r / P;
+            const float xdt = sv.dts[hl] * sv.ux[r];
+            const float d = sv.dec[hl];
+            float* row = slot + (valid ? rr : 0) * N;
+            float y = 0.f;
 #pragma unroll
-            for (int q = 0; q < NV; q++)
-                v[q] = *reinterpret_cast<const float4*>(base + (int64_t)r * N + (q * 8 + l8) * 4);
-        }
-    };
-    int r = warp * 4 + sub;
-    float4 cur[NV], nxt[NV];
-    load_row(r, cur);
-    for (; r - sub < nrows; r += step) {
-        load_row(r + step, nxt);
-        const bool valid = r < nrows;
-        const int hl = valid ? r / P : 0;
-        const float xdt = valid ? sv.dts[hl] * sv.ux[r] : 0.f;
-        const float d = sv.dec[hl];
-        float y = 0.f;
-#pragma unroll
-        for (int q = 0; q < NV; q++) {
-            float4 bv = Bq[q], cv = Cq[q];
-            if (s.bc_norm) {
-                bv = *reinterpret_cast<const float4*>(sv.bh + hl * N + (q * 8 + l8) * 4);
-                cv = *reinterpret_cast<const float4*>(sv.ch + hl * N + (q * 8 + l8) * 4);
+            for (int q = 0; q < NV; q++) {
+                float4 bv = Bq[q], cv = Cq[q];
+                if (s.bc_norm) {
+                    bv = *reinterpret_cast<const float4*>(sv.bh + hl * N + (q * 8 + l8) * 4);
+                    cv = *reinterpret_cast<const float4*>(sv.ch + hl * N + (q * 8 + l8) * 4);
+                }
+                float4* hp = reinterpret_cast<float4*>(row + (q * 8 + l8) * 4);
+                const float4 hc = *hp;
+                float4 hv;
+                hv.x = fmaf(d, hc.x, xdt * bv.x);
+                hv.y = fmaf(d, hc.y, xdt * bv.y);
+                hv.z = fmaf(d, hc.z, xdt * bv.z);
+                hv.w = fmaf(d, hc.w, xdt * bv.w);
+                y = fmaf(cv.x, hv.x, y);
+                y = fmaf(cv.y, hv.y, y);
+                y = fmaf(cv.z, hv.z, y);
+                y = fmaf(cv.w, hv.w, y);
+                if (valid) *hp = hv;
             }
-            float4 hv;
-            hv.x = fmaf(d, cur[q].x, xdt * bv.x);
-            hv.y = fmaf(d, cur[q].y, xdt * bv.y);
-            hv.z = fmaf(d, cur[q].z, xdt * bv.z);
-            hv.w = fmaf(d, cur[q].w, xdt * bv.w);
-            y = fmaf(cv.x, hv.x, y);
-            y = fmaf(cv.y, hv.y, y);
-            y = fmaf(cv.z, hv.z, y);
-            y = fmaf(cv.w, hv.w, y);
-            if (valid)
-                *reinterpret_cast<float4*>(base + (int64_t)r * N + (q * 8 + l8) * 4) = hv;
+            y += __shfl_xor_sync(0xffffffffu, y, 1);
+            y += __shfl_xor_sync(0xffffffffu, y, 2);
+            y += __shfl_xor_sync(0xffffffffu, y, 4);
+            if (valid && l8 == 0) sv.ys[r] = y;
         }
-        y += __shfl_xor_sync(0xffffffffu, y, 1);
-        y += __shfl_xor_sync(0xffffffffu, y, 2);
-        y += __shfl_xor_sync(0xffffffffu, y, 4);
-        if (valid && l8 == 0) sv.ys[r] = y;
-#pragma unroll
-        for (int q = 0; q < NV; q++) cur[q] = nxt[q];
+        tc::fence_async_smem();                   // the updated rows, to the bulk store
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            dec_bulk_store(base + (int64_t)r0 * N, slot, piece_bytes(k));
+            tc::bulk_commit();
+            if (loaded < npieces) {
+                tc::bulk_wait_read0();            // the store has read the slot
+                issue_load(loaded);
+                loaded++;
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        // an aborted block lets every requested piece land before it exits
+        for (int j = k; j < loaded; j++)
+            tc::mbar_drain(&full[j % kDecRing], (uint32_t)(j / kDecRing) & 1u, status, kStatusTimeout, wait_ns);
+        tc::bulk_wait0();
     }
     __syncthreads();
+    if (*s_abort) return;
     // the block's outputs, one coalesced row of hpg * P values
     for (int i = threadIdx.x; i < nrows; i += blockDim.x) {
         const int hh = g * hpg + i / P;
-        ((T*)a.out)[(int64_t)b * HP + (int64_t)g * hpg * P + i] =
+        ((T*)a.out)[(int64_t)b * H * P + (int64_t)g * hpg * P + i] =
             from_f<T>((sv.ys[i] + a.D[hh] * sv.ux[i]) * sv.gz[i]);
     }
 }
@@ -245,30 +311,37 @@ decode_step_any(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ his
 
 template <typename T>
 static cudaError_t launch_decode_t(const Shape& s, const FwdArgs& a, float* ssm, void* hist,
-                                   cudaStream_t st)
+                                   int* status, cudaStream_t st)
 {
     const int hpg = s.nheads / s.ngroups;
     const size_t smem = sizeof(float) * decode_smem_floats(hpg, s.headdim, s.dstate, s.bc_norm);
     const dim3 grid(s.ngroups, s.batch);
-    void (*kern)(Shape, FwdArgs, float*, T*);
-    switch (s.dstate) {
-    case 32: kern = decode_step_vec<T, 1>; break;
-    case 64: kern = decode_step_vec<T, 2>; break;
-    case 128: kern = decode_step_vec<T, 4>; break;
-    case 256: kern = decode_step_vec<T, 8>; break;
-    default: kern = decode_step_any<T>; break;
+    if (s.dstate == 32 || s.dstate == 64 || s.dstate == 128 || s.dstate == 256) {
+        // the bulk kernel: the ring, its barriers and the abort flag ahead of the arrays
+        void (*kern)(Shape, FwdArgs, float*, T*, int*, uint64_t);
+        switch (s.dstate) {
+        case 32: kern = decode_step_bulk<T, 1>; break;
+        case 64: kern = decode_step_bulk<T, 2>; break;
+        case 128: kern = decode_step_bulk<T, 4>; break;
+        default: kern = decode_step_bulk<T, 8>; break;
+        }
+        const size_t bsmem = smem + (size_t)kDecRing * kDecPiece + 16 * (size_t)kDecRing;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsmem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kDecodeThreads, bsmem, st>>>(s, a, ssm, (T*)hist, status, tc::kWaitLimitNs);
+        return cudaGetLastError();
     }
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(decode_step_any<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kDecodeThreads, smem, st>>>(s, a, ssm, (T*)hist);
+    decode_step_any<T><<<grid, kDecodeThreads, smem, st>>>(s, a, ssm, (T*)hist);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
-                               cudaStream_t st)
+                               int* status, cudaStream_t st)
 {
-    return s.act_bf16 ? launch_decode_t<bf16>(s, a, ssm, conv_hist, st)
-                      : launch_decode_t<float>(s, a, ssm, conv_hist, st);
+    return s.act_bf16 ? launch_decode_t<bf16>(s, a, ssm, conv_hist, status, st)
+                      : launch_decode_t<float>(s, a, ssm, conv_hist, status, st);
 }
 
 }  // namespace ssd

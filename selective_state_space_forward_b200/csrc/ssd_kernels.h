@@ -146,8 +146,9 @@ cudaError_t launch_backward(const Shape& s, const FwdArgs& a, const BwdBufs& w, 
 bool gated_norm_group_ok(int d_inner, int gs);
 cudaError_t launch_gated_norm(const Shape& s, void* out, const float* weight, int gs, float eps,
                               const int32_t* lengths, cudaStream_t st);
-// K6: one decode token per row, state updated in place.
+// K6: one decode token per row, state updated in place.  status: the handle's
+// device status word (kStatusTimeout when a bounded wait of the kernel gave up).
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
-                               cudaStream_t st);
+                               int* status, cudaStream_t st);
 
 }  // namespace ssd
