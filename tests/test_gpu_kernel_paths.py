@@ -1,7 +1,10 @@
 """GPU checks of kernel paths that the main parity tests reach only on some shapes.
 
 - The decode step with more heads per B/C group than a block has threads (its
-  per-head dt and decay loop), against the oracle's sequential recurrence.
+  per-head dt and decay loop), against the oracle's sequential recurrence; and
+  on shapes whose state pieces (8 KB of a block's state each) end part-way:
+  fewer rows than a piece holds, rows that fill only some of a block's warps,
+  d_state 32 to 256.
 - The S6 scan's two ways of bringing a chunk's raw inputs on chip: asynchronous
   copies into shared memory (16-byte aligned rows) and loads into registers (any
   other rows).  They compute the same values in the same order, so the outputs
@@ -48,6 +51,45 @@ def test_decode_more_heads_per_group_than_threads():
     fs, fc = state_to_numpy(h, state, w.batch)
     assert_close(fs, ssm, "bf16", "state after the steps")
     assert np.array_equal(fc, conv)
+
+
+def _decode_steps(w, steps=3):
+    inp = make_inputs(w)
+    h = make_handle(w, "auto")
+    dev = to_device(inp, w)
+    _, _, _, state = run_forward(h, w, dev, None)
+    r = oracle.forward(w.dims(), inp)
+    ssm, conv = r["final_ssm"].astype(np.float32), r["final_conv"].astype(np.float32)
+    at = torch.bfloat16
+    for step in range(steps):
+        si = make_step_inputs(w, step)
+        out = h.step(*(torch.from_numpy(si[k]).to(at).cuda() for k in ("x", "z")),
+                     torch.from_numpy(si["dt_raw"]).cuda(), dev["dt_bias"], dev["A"],
+                     torch.from_numpy(si["B"]).to(at).cuda(), torch.from_numpy(si["C"]).to(at).cuda(),
+                     dev["D"], dev["conv_w"], dev["conv_b"], state=state)
+        torch.cuda.synchronize()
+        h.check()
+        tok = dict(inp)
+        tok.update({k: v[:, None] for k, v in si.items()})
+        ro = oracle.step(w.dims(), tok, ssm, conv)
+        assert_close(out.double().cpu().numpy(), ro["out"][:, 0], "bf16", f"step {step}")
+        ssm = ro["final_ssm"].astype(np.float32)
+        conv = ro["final_conv"].astype(np.float32)
+    fs, fc = state_to_numpy(h, state, w.batch)
+    assert_close(fs, ssm, "bf16", "state after the steps")
+    assert np.array_equal(fc, conv)
+
+
+@pytest.mark.parametrize("nheads,headdim,dstate,ngroups", [
+    (3, 8, 64, 1),      # 24 rows: one piece of 32 rows' room, the last 8 rows on two warps
+    (2, 8, 256, 1),     # 8 rows per piece: two pieces, one warp each
+    (6, 24, 128, 2),    # 72 rows per group: 16 rows per piece, a last piece of 8
+    (5, 8, 32, 5),      # one head per group, 8 rows of 64 per piece
+])
+def test_decode_partial_state_pieces(nheads, headdim, dstate, ngroups):
+    w = WORKLOADS["mini_k3_mixer"].with_(batch=3, seqlen=70, nheads=nheads, headdim=headdim,
+                                         dstate=dstate, ngroups=ngroups, documents="none")
+    _decode_steps(w)
 
 
 def _s6_dev(inp):
