@@ -252,8 +252,13 @@ ssd_status ssd_set_timing_events(ssd_handle* h, void* start, void* stop);
  * of that (row * H + head) stream, so the wait for it runs out: the kernel then
  * raises the timeout bit of the device status word, lets its own copies and
  * tensor-core work finish, and exits; ssd_check reports SSD_ERR_DEVICE and the
- * outputs of that call are invalid.  -1 publishes every hand-off.  Nothing
- * faults or hangs, and the next call on the handle is unaffected. */
+ * outputs of that call are invalid.  -1 publishes every hand-off.  For
+ * ssd_step the same two settings apply to the decode kernel, whose blocks wait
+ * for bulk copies of their state: withhold_stream >= 0 makes the block of
+ * (row * G + group) never request its first state piece, so its wait runs out;
+ * that step's outputs, and that block's state and conv history, are then
+ * invalid.  Nothing faults or hangs, and the next call on the handle is
+ * unaffected. */
 ssd_status ssd_set_wait_test(ssd_handle* h, uint64_t wait_limit_ns, int32_t withhold_stream);
 
 /* Number of kernels this handle has launched since ssd_create. */

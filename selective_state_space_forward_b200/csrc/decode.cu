@@ -155,12 +155,14 @@ __device__ __forceinline__ void dec_bulk_store(void* dst, const void* src, uint3
 // block (8 lanes per row, lane l8 owning float4 q at (q * 8 + l8) * 4, so the
 // 8 lanes cover 32 consecutive floats per q) and written back by one bulk
 // store, and its slot is
-// refilled once that store has read it.  Every wait is bounded: on timeout the
-// block raises kStatusTimeout, stops updating, lets its copies land and exits.
+// refilled once that store has read it.  Every wait is bounded (wait_ns): on
+// timeout the block raises kStatusTimeout, stops updating, lets its copies land
+// and exits.  withhold >= 0 (testing): that block never requests its first
+// piece, so its first wait runs out.
 template <typename T, int NV>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_step_bulk(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ hist, int* status,
-                 uint64_t wait_ns)
+                 uint64_t wait_ns, int withhold)
 {
     extern __shared__ __align__(128) float sm[];
     constexpr int N = 32 * NV;
@@ -187,7 +189,9 @@ decode_step_bulk(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ hi
         *s_abort = 0;
         for (int i = 0; i < kDecRing; i++) tc::mbar_init(&full[i], 1);
         tc::fence_mbar_init();
-        for (int k = 0; k < min(kDecRing, npieces); k++) issue_load(k);
+        // testing hook: block `withhold` never requests its first piece, so its wait runs out
+        const bool held = withhold == (int)(blockIdx.y * gridDim.x + blockIdx.x);
+        for (int k = held ? 1 : 0; k < min(kDecRing, npieces); k++) issue_load(k);
     }
     // SiLU(z) of the block's rows, so the outputs need no global load
     for (int i = threadIdx.x; i < nrows; i += blockDim.x)
@@ -311,14 +315,14 @@ decode_step_any(Shape s, FwdArgs a, float* __restrict__ ssm, T* __restrict__ his
 
 template <typename T>
 static cudaError_t launch_decode_t(const Shape& s, const FwdArgs& a, float* ssm, void* hist,
-                                   int* status, cudaStream_t st)
+                                   int* status, uint64_t wait_ns, int withhold, cudaStream_t st)
 {
     const int hpg = s.nheads / s.ngroups;
     const size_t smem = sizeof(float) * decode_smem_floats(hpg, s.headdim, s.dstate, s.bc_norm);
     const dim3 grid(s.ngroups, s.batch);
     if (s.dstate == 32 || s.dstate == 64 || s.dstate == 128 || s.dstate == 256) {
         // the bulk kernel: the ring, its barriers and the abort flag ahead of the arrays
-        void (*kern)(Shape, FwdArgs, float*, T*, int*, uint64_t);
+        void (*kern)(Shape, FwdArgs, float*, T*, int*, uint64_t, int);
         switch (s.dstate) {
         case 32: kern = decode_step_bulk<T, 1>; break;
         case 64: kern = decode_step_bulk<T, 2>; break;
@@ -328,7 +332,8 @@ static cudaError_t launch_decode_t(const Shape& s, const FwdArgs& a, float* ssm,
         const size_t bsmem = smem + (size_t)kDecRing * kDecPiece + 16 * (size_t)kDecRing;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsmem);
         if (e != cudaSuccess) return e;
-        kern<<<grid, kDecodeThreads, bsmem, st>>>(s, a, ssm, (T*)hist, status, tc::kWaitLimitNs);
+        kern<<<grid, kDecodeThreads, bsmem, st>>>(s, a, ssm, (T*)hist, status,
+                                                  wait_ns ? wait_ns : tc::kWaitLimitNs, withhold);
         return cudaGetLastError();
     }
     cudaError_t e = cudaFuncSetAttribute(decode_step_any<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -338,10 +343,10 @@ static cudaError_t launch_decode_t(const Shape& s, const FwdArgs& a, float* ssm,
 }
 
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
-                               int* status, cudaStream_t st)
+                               int* status, uint64_t wait_ns, int withhold, cudaStream_t st)
 {
-    return s.act_bf16 ? launch_decode_t<bf16>(s, a, ssm, conv_hist, status, st)
-                      : launch_decode_t<float>(s, a, ssm, conv_hist, status, st);
+    return s.act_bf16 ? launch_decode_t<bf16>(s, a, ssm, conv_hist, status, wait_ns, withhold, st)
+                      : launch_decode_t<float>(s, a, ssm, conv_hist, status, wait_ns, withhold, st);
 }
 
 }  // namespace ssd

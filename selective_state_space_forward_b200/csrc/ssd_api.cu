@@ -656,7 +656,8 @@ ssd_status ssd_step(ssd_handle* h, int32_t batch, const void* x, const void* z,
     a.bn_w = h->bn_w; a.cn_w = h->cn_w; a.bn_bias = h->bn_bias; a.cn_bias = h->cn_bias;
     void* hist = s.dconv == 4 ? (char*)state + conv_offset(h->d, batch) : nullptr;
     SSD_MAIN_LAUNCH(h, (cudaStream_t)stream,
-                    launch_decode_step(s, a, (float*)state, hist, h->status, (cudaStream_t)stream),
+                    launch_decode_step(s, a, (float*)state, hist, h->status, h->fw.wait_ns, h->fw.withhold,
+                                       (cudaStream_t)stream),
                     "decode kernel");
     if (h->gn_on)
         SSD_LAUNCH(h, launch_gated_norm(s, out, h->gn_w, h->gn_group, h->gn_eps, nullptr,

@@ -147,8 +147,10 @@ bool gated_norm_group_ok(int d_inner, int gs);
 cudaError_t launch_gated_norm(const Shape& s, void* out, const float* weight, int gs, float eps,
                               const int32_t* lengths, cudaStream_t st);
 // K6: one decode token per row, state updated in place.  status: the handle's
-// device status word (kStatusTimeout when a bounded wait of the kernel gave up).
+// device status word (kStatusTimeout when a bounded wait of the kernel gave up);
+// wait_ns: the bound of its waits (0: the default); withhold: testing, the
+// (row * G + group) block that never requests its first state piece (-1: none).
 cudaError_t launch_decode_step(const Shape& s, const FwdArgs& a, float* ssm, void* conv_hist,
-                               int* status, cudaStream_t st);
+                               int* status, uint64_t wait_ns, int withhold, cudaStream_t st);
 
 }  // namespace ssd
