@@ -5,6 +5,9 @@
   on shapes whose state pieces (8 KB of a block's state each) end part-way:
   fewer rows than a piece holds, rows that fill only some of a block's warps,
   d_state 32 to 256.
+- The staged path's chunk-output kernel on heads wider than one 64-column
+  output block (headdim 128, and 72 with a part block) and a d_state that is
+  not a power of two, element by element against the oracle.
 - The S6 scan's two ways of bringing a chunk's raw inputs on chip: asynchronous
   copies into shared memory (16-byte aligned rows) and loads into registers (any
   other rows).  They compute the same values in the same order, so the outputs
@@ -90,6 +93,19 @@ def test_decode_partial_state_pieces(nheads, headdim, dstate, ngroups):
     w = WORKLOADS["mini_k3_mixer"].with_(batch=3, seqlen=70, nheads=nheads, headdim=headdim,
                                          dstate=dstate, ngroups=ngroups, documents="none")
     _decode_steps(w)
+
+
+@pytest.mark.parametrize("headdim,dstate", [(128, 128), (72, 200)])
+def test_staged_wide_heads(headdim, dstate):
+    w = WORKLOADS["mini_k3_mixer"].with_(batch=2, seqlen=150, nheads=2, headdim=headdim, dstate=dstate,
+                                         ngroups=1, mean_doc_len=60)
+    inp = make_inputs(w)
+    res = oracle.forward(w.dims(), inp)
+    h = make_handle(w, "staged")
+    out, fs, fc, _ = run_forward(h, w, to_device(inp, w), None)
+    assert_close(out, res["out"], "bf16", f"staged P={headdim} N={dstate} out")
+    assert_close(fs, res["final_ssm"], "bf16", f"staged P={headdim} N={dstate} final state")
+    assert np.array_equal(fc, res["final_conv"])
 
 
 def _s6_dev(inp):
